@@ -1,0 +1,165 @@
+"""fp64 CPU oracle for paged attention (ctypes front end of oracle/pa_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU-baseline leg are
+the only callers. The CUDA library neither imports nor links it, and this module imports
+nothing from the CUDA package.
+
+Every function returns float64 tensors. Inputs are CPU torch tensors holding the exact
+values the GPU sees (fp32, bf16 or fp16); the C code widens them to double.
+
+Pins (tests/test_oracle_pins.py): brute force against torch's fp64 SDPA/logsumexp on tiny
+dense cases, closed forms (single key, constant V, Q = 0 -> exp(lse) counts the visible keys,
+W = 1 -> own value row, position probe), invariances (page permutation, split == unsplit,
+chunked == one-shot prefill, window >= context == no window, GQA == MHA on a repeated cache,
+MLA == single-head GQA on a concatenated key), and compile-time mutants of this file that the
+pins must reject.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+from . import build as _build
+
+_DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+
+
+class Oracle:
+    """One loaded copy of the oracle library (the real one, or a test mutant)."""
+
+    def __init__(self, path: Optional[str] = None):
+        if path is None:
+            path = _build.build()
+        self.path = path
+        lib = ctypes.CDLL(path)
+        lib.pao_paged_attention.restype = ctypes.c_int
+        lib.pao_paged_attention.argtypes = [_P, _P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I,
+                                            _I, _I, _I, _I, ctypes.c_double, ctypes.c_int, _I, _P,
+                                            _P, _P, _P, _P, ctypes.c_int]
+        lib.pao_mla_attention.restype = ctypes.c_int
+        lib.pao_mla_attention.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I,
+                                          _I, _I, _I, ctypes.c_double, ctypes.c_int, _I, _P, _P,
+                                          _P, _P, _P, ctypes.c_int]
+        lib.pao_lse_combine.restype = None
+        lib.pao_lse_combine.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _I, _P, _P]
+        self.lib = lib
+
+    # -- helpers ---------------------------------------------------------------------------
+    @staticmethod
+    def _c(t: torch.Tensor, dtype=None) -> torch.Tensor:
+        t = t.detach().cpu()
+        if dtype is not None:
+            t = t.to(dtype)
+        return t.contiguous()
+
+    @staticmethod
+    def _want(num_rows: int, rows: Optional[Sequence[int]]):
+        if rows is None:
+            return None
+        w = torch.zeros(num_rows, dtype=torch.uint8)
+        w[torch.as_tensor(rows, dtype=torch.int64)] = 1
+        return w
+
+    @staticmethod
+    def _threads(nthreads: Optional[int]) -> int:
+        return nthreads if nthreads else (os.cpu_count() or 1)
+
+    # -- paged GQA attention ---------------------------------------------------------------
+    def attention(self, q, k_cache, v_cache, seq_lens, query_offsets, block_tables, page_size,
+                  scale, causal=True, window=0, key_begin=None, key_end=None, rows=None,
+                  nthreads=None):
+        """out [Nq, Hq, Dv] float64, lse [Nq, Hq] float64 (rows not asked for stay NaN)."""
+        dt = q.dtype
+        assert k_cache.dtype == dt and v_cache.dtype == dt and dt in _DT
+        q, k_cache, v_cache = self._c(q), self._c(k_cache), self._c(v_cache)
+        nq, hq, d = q.shape
+        num_pages, ps, hkv, _ = k_cache.shape
+        dv = v_cache.shape[3]
+        assert ps == page_size
+        sl = self._c(seq_lens, torch.int32)
+        qo = self._c(query_offsets, torch.int32)
+        bt = self._c(block_tables, torch.int32)
+        kb = self._c(key_begin, torch.int32) if key_begin is not None else None
+        ke = self._c(key_end, torch.int32) if key_end is not None else None
+        want = self._want(nq * hq, rows)
+        out = torch.full((nq, hq, dv), float("nan"), dtype=torch.float64)
+        lse = torch.full((nq, hq), float("nan"), dtype=torch.float64)
+        rc = self.lib.pao_paged_attention(
+            q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), _DT[dt], sl.data_ptr(),
+            qo.data_ptr(), sl.numel(), bt.data_ptr(), bt.shape[1] if bt.dim() == 2 else 0,
+            page_size, num_pages, hq, hkv, d, dv, float(scale), int(bool(causal)), int(window),
+            kb.data_ptr() if kb is not None else None, ke.data_ptr() if ke is not None else None,
+            want.data_ptr() if want is not None else None, out.data_ptr(), lse.data_ptr(),
+            self._threads(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle rejected the schedule (code {rc})")
+        return out, lse
+
+    # -- MLA absorbed-latent attention ------------------------------------------------------
+    def mla(self, q_latent, q_rope, latent_cache, rope_cache, seq_lens, query_offsets,
+            block_tables, page_size, scale, causal=True, window=0, key_begin=None, key_end=None,
+            rows=None, nthreads=None):
+        dt = q_latent.dtype
+        q_latent, q_rope = self._c(q_latent), self._c(q_rope)
+        latent_cache, rope_cache = self._c(latent_cache), self._c(rope_cache)
+        nq, h, r = q_latent.shape
+        pr = q_rope.shape[2]
+        num_pages, ps = latent_cache.shape[0], latent_cache.shape[1]
+        assert ps == page_size and latent_cache.shape[2] == 1
+        sl = self._c(seq_lens, torch.int32)
+        qo = self._c(query_offsets, torch.int32)
+        bt = self._c(block_tables, torch.int32)
+        kb = self._c(key_begin, torch.int32) if key_begin is not None else None
+        ke = self._c(key_end, torch.int32) if key_end is not None else None
+        want = self._want(nq * h, rows)
+        out = torch.full((nq, h, r), float("nan"), dtype=torch.float64)
+        lse = torch.full((nq, h), float("nan"), dtype=torch.float64)
+        rc = self.lib.pao_mla_attention(
+            q_latent.data_ptr(), q_rope.data_ptr(), latent_cache.data_ptr(), rope_cache.data_ptr(),
+            _DT[dt], sl.data_ptr(), qo.data_ptr(), sl.numel(), bt.data_ptr(), bt.shape[1],
+            page_size, num_pages, h, r, pr, float(scale), int(bool(causal)), int(window),
+            kb.data_ptr() if kb is not None else None, ke.data_ptr() if ke is not None else None,
+            want.data_ptr() if want is not None else None, out.data_ptr(), lse.data_ptr(),
+            self._threads(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle rejected the schedule (code {rc})")
+        return out, lse
+
+    # -- merge of partial results -------------------------------------------------------------
+    def lse_combine(self, o_parts: torch.Tensor, lse_parts: torch.Tensor):
+        """o_parts [nparts, rows, dv], lse_parts [nparts, rows] -> (out [rows, dv], lse [rows])."""
+        o_parts = self._c(o_parts, torch.float64)
+        lse_parts = self._c(lse_parts, torch.float64)
+        nparts, rows, dv = o_parts.shape
+        out = torch.empty((rows, dv), dtype=torch.float64)
+        lse = torch.empty(rows, dtype=torch.float64)
+        self.lib.pao_lse_combine(o_parts.data_ptr(), lse_parts.data_ptr(), nparts, rows, dv,
+                                 out.data_ptr(), lse.data_ptr())
+        return out, lse
+
+    # -- workload conveniences ----------------------------------------------------------------
+    def run(self, wl, rows=None, nthreads=None, key_begin=None, key_end=None):
+        """Run the oracle on a workload object (GQA or MLA) from the seeded input module."""
+        s = wl.sched
+        if wl.kind == "mla":
+            return self.mla(wl.q_latent, wl.q_rope, wl.latent_cache, wl.rope_cache, s.seq_lens,
+                            s.query_offsets, s.block_tables, s.page_size, wl.scale, wl.causal,
+                            wl.window, key_begin, key_end, rows, nthreads)
+        return self.attention(wl.q, wl.k_cache, wl.v_cache, s.seq_lens, s.query_offsets,
+                              s.block_tables, s.page_size, wl.scale, wl.causal, wl.window,
+                              key_begin, key_end, rows, nthreads)
+
+
+_default: Optional[Oracle] = None
+
+
+def get() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

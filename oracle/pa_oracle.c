@@ -1,0 +1,352 @@
+/*
+ * pa_oracle.c -- fp64 CPU oracle for paged attention.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg call this code. It shares nothing with the CUDA library: no header, no
+ * helper, no table. It is deliberately plain and slow.
+ *
+ * What it computes is the dense definition of attention from boostr's
+ * `standard_attention_fwd` (flash_standard.rs): scores = Q.K^T * scale, an additive 0/-inf
+ * mask, lse = logsumexp(scores) over the key axis, out = softmax(scores).V, with GQA query
+ * head h reading KV head h / (Hq/Hkv) (`expand_kv`, repeat_interleave on the head axis).
+ * The paged part follows ruDNN's `DevicePlan::attention` contract: K/V live in a paged cache
+ * [pages, page_size, Hkv, D] reached through each sequence's block table; the oracle first
+ * materialises each sequence's K/V contiguously (key t sits in page block_table[s][t / ps],
+ * slot t % ps), then runs the dense definition on it.
+ *
+ * Readings where the pages leave a step open (each is listed in the design notes):
+ *  - causal masking uses absolute, right-aligned positions: query j of a sequence with n
+ *    queries and L keys (L includes the sequence's own new keys) sits at p = L - n + j
+ *    (ruDNN "absolute positions ... including prefill chunks"; alice-llm "right-aligned
+ *    causal mask"). Key t is masked when t > p.
+ *  - the sliding window masks key t when t + window <= p (boostr `build_attention_mask`),
+ *    window 0 meaning no window; it applies whether or not the mask is causal.
+ *  - a row with no visible key gets out = 0 and lse = -inf.
+ *  - lse is the natural-log logsumexp of the scaled, masked scores.
+ * MLA (ruDNN `DevicePlan::mla`): score = scale * (q_lat . latent_t + q_rope . rope_t); the
+ * latent is both key and value, so out has the latent width R.
+ *
+ * Inputs are the exact stored values (fp32, bf16 or fp16 bit patterns) widened to double.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define PAO_F32 0
+#define PAO_BF16 1
+#define PAO_F16 2
+
+/* Exact widening of one stored element to double. */
+static double pao_load(const void* base, int dtype, int64_t i) {
+    if (dtype == PAO_F32) {
+        return (double)((const float*)base)[i];
+    }
+    uint16_t h = ((const uint16_t*)base)[i];
+    if (dtype == PAO_BF16) {
+        uint32_t bits = (uint32_t)h << 16; /* bf16 is the top half of an IEEE binary32 */
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        return (double)f;
+    }
+    /* IEEE binary16: 1 sign, 5 exponent (bias 15), 10 fraction bits */
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int frac = h & 0x3ff;
+    double v;
+    if (e == 0) {
+        v = ldexp((double)frac, -24); /* subnormal: frac * 2^-14 * 2^-10 */
+    } else if (e == 31) {
+        v = frac ? NAN : INFINITY;
+    } else {
+        v = ldexp((double)(1024 + frac), e - 25); /* (1 + frac/1024) * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+typedef struct {
+    /* operands */
+    const void* q;      /* [Nq, Hq, D]   (GQA)  or absorbed q [Nq, H, R]  (MLA) */
+    const void* k;      /* [P, ps, Hkv, D]      or latent   [P, ps, 1, R] */
+    const void* v;      /* [P, ps, Hkv, Dv]     or unused (MLA: V is the latent) */
+    const void* qr;     /* MLA only: position q [Nq, H, Pr] */
+    const void* kr;     /* MLA only: rope cache [P, ps, 1, Pr] */
+    int dtype;
+    int mla;
+    /* schedule */
+    const int32_t* seq_lens;
+    const int32_t* query_offsets;
+    int32_t num_seqs;
+    const int32_t* block_tables;
+    int32_t table_width, page_size, num_pages;
+    /* geometry */
+    int32_t hq, hkv, d, dv, pr;
+    double scale;
+    int causal;
+    int32_t window;
+    const int32_t* key_begin; /* optional [S]: keys t < key_begin[s] are dropped */
+    const int32_t* key_end;   /* optional [S]: keys t >= key_end[s] are dropped */
+    const uint8_t* want;      /* optional [Nq*Hq]: compute only rows with want != 0 */
+    double* out;              /* [Nq, Hq, Dv] */
+    double* lse;              /* [Nq, Hq] */
+    /* work distribution over (sequence, kv head) */
+    int64_t next_item;
+    pthread_mutex_t lock;
+    int error;
+} pao_job;
+
+/* Is key t visible to a query at absolute position p? */
+static int pao_visible(const pao_job* J, int32_t s, int64_t t, int64_t p) {
+#ifdef PAO_MUTANT_CAUSAL_STRICT
+    if (J->causal && t >= p) return 0;
+#else
+    if (J->causal && t > p) return 0;
+#endif
+#ifdef PAO_MUTANT_WINDOW_WIDE
+    if (J->window > 0 && t + J->window < p) return 0;
+#else
+    if (J->window > 0 && t + J->window <= p) return 0;
+#endif
+    if (J->key_begin && t < J->key_begin[s]) return 0;
+    if (J->key_end && t >= J->key_end[s]) return 0;
+    return 1;
+}
+
+static void pao_run_item(pao_job* J, int32_t s, int32_t kvh, double* kbuf, double* vbuf,
+                         double* krbuf, double* xbuf, double* qbuf) {
+    const int64_t L = J->seq_lens[s];
+    const int64_t q0 = J->query_offsets[s];
+    const int64_t n = J->query_offsets[s + 1] - q0;
+    const int32_t ps = J->page_size;
+    const int32_t G = J->hq / J->hkv;
+    const int32_t kd = J->d;            /* width of the key rows */
+    const int32_t vd = J->dv;           /* width of the value rows */
+    const int32_t kheads = J->mla ? 1 : J->hkv;
+    if (n == 0) return;
+
+    /* 1. materialise this sequence's keys/values for this KV head contiguously */
+    for (int64_t t = 0; t < L; ++t) {
+#ifdef PAO_MUTANT_IDENTITY_TABLE
+        int64_t page = t / ps; /* wrong: ignores the block table */
+        int64_t slot = t % ps;
+#else
+        int64_t page = J->block_tables[(int64_t)s * J->table_width + t / ps];
+        int64_t slot = t % ps;
+#endif
+        int64_t row = (page * ps + slot) * kheads + (J->mla ? 0 : kvh);
+        for (int32_t c = 0; c < kd; ++c) kbuf[t * kd + c] = pao_load(J->k, J->dtype, row * kd + c);
+        if (J->mla) {
+            for (int32_t c = 0; c < J->pr; ++c)
+                krbuf[t * J->pr + c] = pao_load(J->kr, J->dtype, (page * ps + slot) * J->pr + c);
+        } else {
+            for (int32_t c = 0; c < vd; ++c) vbuf[t * vd + c] = pao_load(J->v, J->dtype, row * vd + c);
+        }
+    }
+    const double* V = J->mla ? kbuf : vbuf; /* MLA: the latent is both key and value */
+
+    /* 2. dense masked softmax for every query head of the group and every query */
+    for (int32_t g = 0; g < G; ++g) {
+#ifdef PAO_MUTANT_GQA_MODULO
+        const int32_t h = g * J->hkv + kvh; /* wrong map: h % Hkv == kvh */
+#else
+        const int32_t h = kvh * G + g;
+#endif
+        for (int64_t j = 0; j < n; ++j) {
+            const int64_t qi = q0 + j;
+            const int64_t r = qi * J->hq + h;
+            if (J->want && !J->want[r]) continue;
+#ifdef PAO_MUTANT_LEFT_ALIGNED
+            const int64_t p = j;
+#else
+            const int64_t p = L - n + j;
+#endif
+            for (int32_t c = 0; c < kd; ++c) qbuf[c] = pao_load(J->q, J->dtype, r * kd + c);
+            for (int32_t c = 0; c < J->pr; ++c) qbuf[kd + c] = pao_load(J->qr, J->dtype, r * J->pr + c);
+            double m = -INFINITY;
+            for (int64_t t = 0; t < L; ++t) {
+                if (!pao_visible(J, s, t, p)) { xbuf[t] = -INFINITY; continue; }
+                double acc = 0.0;
+                for (int32_t c = 0; c < kd; ++c) acc += qbuf[c] * kbuf[t * kd + c];
+#ifndef PAO_MUTANT_DROP_ROPE
+                if (J->mla)
+                    for (int32_t c = 0; c < J->pr; ++c) acc += qbuf[kd + c] * krbuf[t * J->pr + c];
+#endif
+#ifdef PAO_MUTANT_SCALE_DROPPED
+                xbuf[t] = acc;
+#else
+                xbuf[t] = J->scale * acc;
+#endif
+                if (xbuf[t] > m) m = xbuf[t];
+            }
+            double* o = J->out + r * vd;
+            for (int32_t c = 0; c < vd; ++c) o[c] = 0.0;
+            if (m == -INFINITY) { J->lse[r] = -INFINITY; continue; }
+            double sum = 0.0;
+            for (int64_t t = 0; t < L; ++t)
+                if (xbuf[t] != -INFINITY) sum += exp(xbuf[t] - m);
+#ifdef PAO_MUTANT_LSE_NO_MAX
+            const double lse = log(sum);
+#else
+            const double lse = m + log(sum);
+#endif
+            J->lse[r] = lse;
+            for (int64_t t = 0; t < L; ++t) {
+                if (xbuf[t] == -INFINITY) continue;
+#ifdef PAO_MUTANT_UNNORMALISED
+                const double w = exp(xbuf[t] - m);
+#else
+                const double w = exp(xbuf[t] - lse);
+#endif
+                for (int32_t c = 0; c < vd; ++c) o[c] += w * V[t * vd + c];
+            }
+        }
+    }
+}
+
+static void* pao_worker(void* arg) {
+    pao_job* J = (pao_job*)arg;
+    int64_t maxL = 0;
+    for (int32_t s = 0; s < J->num_seqs; ++s)
+        if (J->seq_lens[s] > maxL) maxL = J->seq_lens[s];
+    const int64_t rows = maxL > 0 ? maxL : 1;
+    double* kbuf = (double*)malloc(sizeof(double) * rows * (size_t)J->d);
+    double* vbuf = J->mla ? NULL : (double*)malloc(sizeof(double) * rows * (size_t)J->dv);
+    double* krbuf = J->mla ? (double*)malloc(sizeof(double) * rows * (size_t)(J->pr > 0 ? J->pr : 1)) : NULL;
+    double* xbuf = (double*)malloc(sizeof(double) * rows);
+    double* qbuf = (double*)malloc(sizeof(double) * (size_t)(J->d + J->pr));
+    if (!kbuf || (!J->mla && !vbuf) || (J->mla && !krbuf) || !xbuf || !qbuf) {
+        pthread_mutex_lock(&J->lock);
+        J->error = 1;
+        pthread_mutex_unlock(&J->lock);
+    } else {
+        const int32_t kheads = J->mla ? 1 : J->hkv;
+        for (;;) {
+            pthread_mutex_lock(&J->lock);
+            int64_t it = J->next_item++;
+            pthread_mutex_unlock(&J->lock);
+            if (it >= (int64_t)J->num_seqs * kheads) break;
+            pao_run_item(J, (int32_t)(it / kheads), (int32_t)(it % kheads), kbuf, vbuf, krbuf, xbuf, qbuf);
+        }
+    }
+    free(kbuf);
+    free(vbuf);
+    free(krbuf);
+    free(xbuf);
+    free(qbuf);
+    return NULL;
+}
+
+static int pao_check_schedule(const pao_job* J) {
+    if (J->num_seqs < 0 || J->page_size <= 0 || J->table_width < 0) return -1;
+    if (J->query_offsets[0] != 0) return -1;
+    for (int32_t s = 0; s < J->num_seqs; ++s) {
+        int64_t L = J->seq_lens[s];
+        int64_t n = (int64_t)J->query_offsets[s + 1] - J->query_offsets[s];
+        if (L < 0 || n < 0 || n > L) return -1;
+        int64_t used = (L + J->page_size - 1) / J->page_size;
+        if (used > J->table_width) return -1;
+        for (int64_t b = 0; b < used; ++b) {
+            int32_t page = J->block_tables[(int64_t)s * J->table_width + b];
+            if (page < 0 || page >= J->num_pages) return -2;
+        }
+    }
+    return 0;
+}
+
+static int pao_run(pao_job* J, int nthreads) {
+    int rc = pao_check_schedule(J);
+    if (rc) return rc;
+    J->next_item = 0;
+    J->error = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, pao_worker, J) == 0) ++started;
+        else break;
+    }
+    if (started == 0) pao_worker(J);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&J->lock);
+    return J->error ? -3 : 0;
+}
+
+/*
+ * Paged GQA attention. Returns 0 on success, -1 on a malformed schedule, -2 on a block-table
+ * entry outside the pool, -3 on an allocation failure.
+ */
+int pao_paged_attention(const void* q, const void* k_cache, const void* v_cache, int dtype,
+                        const int32_t* seq_lens, const int32_t* query_offsets, int32_t num_seqs,
+                        const int32_t* block_tables, int32_t table_width, int32_t page_size,
+                        int32_t num_pages, int32_t hq, int32_t hkv, int32_t d, int32_t dv,
+                        double scale, int causal, int32_t window, const int32_t* key_begin,
+                        const int32_t* key_end, const uint8_t* want_rows, double* out, double* lse,
+                        int nthreads) {
+    if (hq <= 0 || hkv <= 0 || hq % hkv || d <= 0 || dv <= 0 || window < 0) return -1;
+    pao_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k_cache; J.v = v_cache; J.dtype = dtype; J.mla = 0;
+    J.seq_lens = seq_lens; J.query_offsets = query_offsets; J.num_seqs = num_seqs;
+    J.block_tables = block_tables; J.table_width = table_width; J.page_size = page_size;
+    J.num_pages = num_pages; J.hq = hq; J.hkv = hkv; J.d = d; J.dv = dv; J.pr = 0;
+    J.scale = scale; J.causal = causal; J.window = window;
+    J.key_begin = key_begin; J.key_end = key_end; J.want = want_rows; J.out = out; J.lse = lse;
+    return pao_run(&J, nthreads);
+}
+
+/* MLA absorbed-latent attention: one shared latent head; V is the latent itself. */
+int pao_mla_attention(const void* q_latent, const void* q_rope, const void* latent_cache,
+                      const void* rope_cache, int dtype, const int32_t* seq_lens,
+                      const int32_t* query_offsets, int32_t num_seqs, const int32_t* block_tables,
+                      int32_t table_width, int32_t page_size, int32_t num_pages, int32_t heads,
+                      int32_t latent_dim, int32_t rope_dim, double scale, int causal,
+                      int32_t window, const int32_t* key_begin, const int32_t* key_end,
+                      const uint8_t* want_rows, double* out, double* lse, int nthreads) {
+    if (heads <= 0 || latent_dim <= 0 || rope_dim < 0 || window < 0) return -1;
+    pao_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q_latent; J.k = latent_cache; J.v = NULL; J.qr = q_rope; J.kr = rope_cache;
+    J.dtype = dtype; J.mla = 1;
+    J.seq_lens = seq_lens; J.query_offsets = query_offsets; J.num_seqs = num_seqs;
+    J.block_tables = block_tables; J.table_width = table_width; J.page_size = page_size;
+    J.num_pages = num_pages; J.hq = heads; J.hkv = 1; J.d = latent_dim; J.dv = latent_dim;
+    J.pr = rope_dim; J.scale = scale; J.causal = causal; J.window = window;
+    J.key_begin = key_begin; J.key_end = key_end; J.want = want_rows; J.out = out; J.lse = lse;
+    return pao_run(&J, nthreads);
+}
+
+/*
+ * Merge of partial results over disjoint key subsets (ruDNN "merge FP32 statistics";
+ * alice-llm `lse_combine`). Part i of row r holds the normalised output o_i and its
+ * logsumexp lse_i over its keys. The merged logsumexp is the logsumexp of the lse_i, and the
+ * merged output weights each o_i by exp(lse_i - lse). Parts with lse_i = -inf have no keys
+ * and weight 0; a row whose parts are all empty gets out = 0, lse = -inf.
+ * Layout: o_parts [nparts, rows, dv], lse_parts [nparts, rows].
+ */
+void pao_lse_combine(const double* o_parts, const double* lse_parts, int64_t nparts, int64_t rows,
+                     int32_t dv, double* out, double* lse) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double m = -INFINITY;
+        for (int64_t i = 0; i < nparts; ++i)
+            if (lse_parts[i * rows + r] > m) m = lse_parts[i * rows + r];
+        double* o = out + r * dv;
+        for (int32_t c = 0; c < dv; ++c) o[c] = 0.0;
+        if (m == -INFINITY) { lse[r] = -INFINITY; continue; }
+        double sum = 0.0;
+        for (int64_t i = 0; i < nparts; ++i) {
+            double li = lse_parts[i * rows + r];
+            if (li != -INFINITY) sum += exp(li - m);
+        }
+        const double total = m + log(sum);
+        lse[r] = total;
+        for (int64_t i = 0; i < nparts; ++i) {
+            double li = lse_parts[i * rows + r];
+            if (li == -INFINITY) continue;
+            const double w = exp(li - total);
+            for (int32_t c = 0; c < dv; ++c) o[c] += w * o_parts[(i * rows + r) * dv + c];
+        }
+    }
+}

@@ -1,0 +1,334 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the oracle itself.
+
+Each pin takes an `Oracle` (the real one, or a compile-time mutant) and raises AssertionError
+when the oracle disagrees with the fact it checks. Sources of truth:
+  * torch's fp64 scaled_dot_product_attention / logsumexp on a densely gathered copy
+    (boostr `standard_attention_fwd` says every fused kernel must match the dense result);
+  * closed forms: a single key returns its value row and lse = scale * q.k; a constant value
+    per KV head comes back unchanged for every query head of its group; with Q = 0 every
+    visible key weighs the same, so exp(lse) is the visible-key count (closed form from the
+    query's absolute position, the causal flag and the window) and out is their mean value;
+    V[t] = t makes out the mean visible position; q = a large multiple of K[t*] selects t*;
+  * invariances the definition implies: relabelling the page pool, splitting the keys and
+    merging the parts (ruDNN "merge FP32 statistics"; alice-llm `lse_combine`), splitting a
+    prefill chunk in two, a window wider than the context, GQA on a repeated cache, MLA as
+    single-head attention on the concatenated key;
+  * exact widening of bf16/fp16 inputs (same values given as fp32 give identical results).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+from paged_kv_attention_39_b200 import workloads as W
+
+
+def _dense_kv(cache: torch.Tensor, bt: torch.Tensor, s: int, L: int, ps: int) -> torch.Tensor:
+    """Gather sequence s's first L rows as [L, heads, dim] via torch indexing."""
+    t = torch.arange(L)
+    pages = bt[s, (t // ps)].long()
+    return cache[pages, t % ps].double()
+
+
+def _counts(L: int, n: int, causal: bool, window: int):
+    """Closed-form visible range [lo, hi] per query of a sequence (right-aligned positions)."""
+    res = []
+    for j in range(n):
+        p = L - n + j
+        hi = p if causal else L - 1
+        lo = max(0, p - window + 1) if window > 0 else 0
+        res.append((lo, hi))
+    return res
+
+
+def _small_cases():
+    """Tiny GQA workloads spanning decode, prefill chunks, windows, page sizes and dtypes."""
+    return [
+        W.make_gqa("t1", 1, [5, 17, 33], [1, 3, 33], 4, 2, 8, 8, 4, torch.float32, causal=True),
+        W.make_gqa("t2", 2, [40, 9], [7, 9], 6, 3, 16, 8, 8, torch.float32, causal=True, window=5),
+        W.make_gqa("t3", 3, [30, 12, 1], [4, 12, 1], 4, 1, 8, 12, 16, torch.bfloat16, causal=False),
+        W.make_gqa("t4", 4, [23, 64], [23, 2], 8, 8, 8, 8, 4, torch.float16, causal=False, window=7),
+        W.make_gqa("t5", 5, [50], [20], 4, 2, 8, 8, 16, torch.float32, causal=True, window=1),
+    ]
+
+
+def pin_sdpa_bruteforce(orc):
+    for wl in _small_cases():
+        s_ = wl.sched
+        out, lse = orc.run(wl)
+        G = wl.num_q_heads // wl.num_kv_heads
+        for s in range(s_.num_seqs):
+            L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+            if n == 0:
+                continue
+            K = _dense_kv(wl.k_cache, s_.block_tables, s, L, s_.page_size).repeat_interleave(G, dim=1)
+            V = _dense_kv(wl.v_cache, s_.block_tables, s, L, s_.page_size).repeat_interleave(G, dim=1)
+            Q = wl.q[q0:q0 + n].double()
+            pos = torch.arange(L - n, L).view(n, 1)
+            t = torch.arange(L).view(1, L)
+            keep = torch.ones(n, L, dtype=torch.bool)
+            if wl.causal:
+                keep &= t <= pos
+            if wl.window > 0:
+                keep &= t + wl.window > pos
+            qh, kh, vh = Q.transpose(0, 1), K.transpose(0, 1), V.transpose(0, 1)
+            ref = F.scaled_dot_product_attention(qh, kh, vh, attn_mask=keep, scale=wl.scale)
+            sc = (qh @ kh.transpose(1, 2)) * wl.scale
+            ref_lse = torch.logsumexp(sc.masked_fill(~keep, float("-inf")), dim=-1)
+            got = out[q0:q0 + n].transpose(0, 1)
+            assert torch.allclose(got, ref, rtol=1e-11, atol=1e-12), (wl.name, s, (got - ref).abs().max())
+            assert torch.allclose(lse[q0:q0 + n].transpose(0, 1), ref_lse, rtol=1e-12, atol=1e-12), (wl.name, s)
+
+
+def alice_fixture():
+    """alice-llm `fixture_gqa`: tq=3, hq=4, hkv=2, head_dim=8, seq_len=12, values sin/cos of
+    the flat index; dense [seq, hkv, d] K/V placed in pages of 4 with an identity table."""
+    tq, hq, hkv, d, L, ps = 3, 4, 2, 8, 12, 4
+    q = torch.tensor([math.sin(i * 0.05) for i in range(tq * hq * d)], dtype=torch.float32).view(tq, hq, d)
+    k = torch.tensor([math.cos(i * 0.07) for i in range(L * hkv * d)], dtype=torch.float32).view(L // ps, ps, hkv, d)
+    v = torch.tensor([math.sin(i * 0.03) for i in range(L * hkv * d)], dtype=torch.float32).view(L // ps, ps, hkv, d)
+    sl = torch.tensor([L], dtype=torch.int32)
+    qo = torch.tensor([0, tq], dtype=torch.int32)
+    bt = torch.arange(L // ps, dtype=torch.int32).view(1, -1)
+    return q, k, v, sl, qo, bt, ps, 1.0 / math.sqrt(d)
+
+
+def pin_alice_fixture_dense(orc):
+    q, k, v, sl, qo, bt, ps, scale = alice_fixture()
+    out, lse = orc.attention(q, k, v, sl, qo, bt, ps, scale, causal=False, window=0)
+    G = 2
+    K = k.reshape(-1, 2, 8).double().repeat_interleave(G, 1).transpose(0, 1)
+    V = v.reshape(-1, 2, 8).double().repeat_interleave(G, 1).transpose(0, 1)
+    Q = q.double().transpose(0, 1)
+    ref = F.scaled_dot_product_attention(Q, K, V, scale=scale).transpose(0, 1)
+    rel = ((out - ref).abs() / ref.abs().clamp_min(1e-6)).max()
+    assert rel < 1e-12, rel
+
+
+def pin_single_key(orc):
+    for dt in (torch.float32, torch.bfloat16):
+        wl = W.make_gqa("one", 7, [1, 1, 1], [1, 1, 1], 6, 2, 16, 8, 4, dt, causal=True)
+        out, lse = orc.run(wl)
+        s_ = wl.sched
+        G = 3
+        for s in range(3):
+            page = int(s_.block_tables[s, 0])
+            for h in range(6):
+                kv = h // G
+                assert torch.equal(out[s, h], wl.v_cache[page, 0, kv].double())
+                qk = math.fsum(float(a) * float(b) for a, b in zip(wl.q[s, h].double(), wl.k_cache[page, 0, kv].double()))
+                assert abs(float(lse[s, h]) - wl.scale * qk) <= 1e-12 * max(1.0, abs(wl.scale * qk))
+
+
+def pin_constant_v_per_kv_head(orc):
+    wl = W.make_gqa("cv", 8, [19, 40, 7], [3, 1, 7], 8, 2, 8, 6, 8, torch.float32, causal=True, window=9)
+    c = torch.randn(2, 6, generator=torch.Generator().manual_seed(1))
+    wl.v_cache[:] = c.view(1, 1, 2, 6)
+    out, _ = orc.run(wl)
+    G = 4
+    for h in range(8):
+        ref = c[h // G].double().view(1, 6)
+        assert torch.allclose(out[:, h], ref.expand_as(out[:, h]), rtol=0, atol=1e-14), h
+
+
+def pin_q_zero_counts_and_mean(orc):
+    cases = [
+        W.make_gqa("z1", 9, [37, 100, 64, 5], [1, 1, 13, 5], 4, 2, 8, 8, 16, torch.float32, causal=True),
+        W.make_gqa("z2", 10, [37, 100, 64], [1, 9, 13], 4, 2, 8, 8, 16, torch.float32, causal=True, window=6),
+        W.make_gqa("z3", 11, [37, 60], [2, 9], 4, 4, 8, 8, 8, torch.float32, causal=False, window=11),
+        W.make_gqa("z4", 12, [37, 60], [2, 9], 2, 1, 8, 8, 8, torch.float32, causal=False),
+    ]
+    for wl in cases:
+        wl.q.zero_()
+        out, lse = orc.run(wl)
+        s_ = wl.sched
+        G = wl.num_q_heads // wl.num_kv_heads
+        for s in range(s_.num_seqs):
+            L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+            V = _dense_kv(wl.v_cache, s_.block_tables, s, L, s_.page_size)
+            for j, (lo, hi) in enumerate(_counts(L, n, wl.causal, wl.window)):
+                cnt = hi - lo + 1
+                for h in range(wl.num_q_heads):
+                    got = float(lse[q0 + j, h])
+                    assert round(math.exp(got)) == cnt, (wl.name, s, j, h, math.exp(got), cnt)
+                    assert abs(got - math.log(cnt)) <= 1e-12
+                    ref = V[lo:hi + 1, h // G].mean(0)
+                    assert torch.allclose(out[q0 + j, h], ref, rtol=1e-12, atol=1e-13), (wl.name, s, j, h)
+
+
+def pin_position_probe(orc):
+    """V[t, :, 0] = t (exact in fp32), Q = 0: out[..., 0] is the mean visible position."""
+    wl = W.make_gqa("pp", 13, [100, 37, 250], [1, 5, 30], 4, 2, 8, 8, 16, torch.float32, causal=True, window=40)
+    wl.q.zero_()
+    s_ = wl.sched
+    for s in range(s_.num_seqs):
+        L = int(s_.seq_lens[s])
+        t = torch.arange(L)
+        wl.v_cache[s_.block_tables[s, t // s_.page_size].long(), t % s_.page_size, :, 0] = t.float().view(-1, 1)
+    out, _ = orc.run(wl)
+    for s in range(s_.num_seqs):
+        L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+        for j, (lo, hi) in enumerate(_counts(L, n, True, 40)):
+            assert torch.allclose(out[q0 + j, :, 0], torch.full((4,), (lo + hi) / 2.0, dtype=torch.float64),
+                                  rtol=0, atol=1e-10), (s, j)
+
+
+def select_target_queries(wl, seed: int, margin: float = 80.0):
+    """Rewrite Q so that each (query, head) row puts all its weight on one visible key t*.
+
+    q = alpha * K[t*] with t* a visible key whose self-score beats every other visible key's
+    score by a positive gap, and alpha chosen so the scaled gap is `margin`: every other
+    weight is below exp(-margin). Returns {(query, head): (sequence, t*)}.
+    """
+    s_ = wl.sched
+    g = torch.Generator().manual_seed(seed)
+    G = wl.num_q_heads // wl.num_kv_heads
+    target = {}
+    for s in range(s_.num_seqs):
+        L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+        K = _dense_kv(wl.k_cache, s_.block_tables, s, L, s_.page_size)
+        for j, (lo, hi) in enumerate(_counts(L, n, wl.causal, wl.window)):
+            for h in range(wl.num_q_heads):
+                Kh = K[lo:hi + 1, h // G]
+                cand = torch.randperm(hi - lo + 1, generator=g)[:8].tolist() + [int(Kh.norm(dim=1).argmax())]
+                for c in cand:
+                    dots = Kh @ Kh[c]
+                    own = float(dots[c])
+                    dots[c] = float("-inf")
+                    gap = own - (float(dots.max()) if hi > lo else own - 1.0)
+                    if gap > 1e-3 * max(own, 1e-30):
+                        break
+                alpha = margin / (wl.scale * gap)
+                wl.q[q0 + j, h] = (alpha * Kh[c]).to(wl.q.dtype)
+                target[(q0 + j, h)] = (s, lo + c)
+    return target
+
+
+def pin_large_score_selects_target(orc):
+    """q = alpha * K[t*] for a visible t*: every other weight underflows, out == V[t*]."""
+    wl = W.make_gqa("ls", 14, [70, 33, 129], [1, 6, 2], 4, 2, 16, 8, 8, torch.float32, causal=True, window=50)
+    s_ = wl.sched
+    target = select_target_queries(wl, 3)
+    out, _ = orc.run(wl)
+    G = 2
+    for (qi, h), (s, ts) in target.items():
+        V = _dense_kv(wl.v_cache, s_.block_tables, s, int(s_.seq_lens[s]), s_.page_size)
+        assert torch.allclose(out[qi, h], V[ts, h // G], rtol=0, atol=1e-12), (qi, h, s, ts)
+
+
+def pin_page_permutation_invariance(orc):
+    wl = W.make_gqa("perm", 15, [45, 90, 3], [2, 1, 3], 4, 2, 8, 8, 8, torch.bfloat16, causal=True, window=20)
+    out, lse = orc.run(wl)
+    P = wl.sched.num_pages
+    pi = torch.randperm(P, generator=torch.Generator().manual_seed(4))
+    k2 = torch.empty_like(wl.k_cache); k2[pi] = wl.k_cache
+    v2 = torch.empty_like(wl.v_cache); v2[pi] = wl.v_cache
+    bt = wl.sched.block_tables.clone()
+    m = bt >= 0
+    bt[m] = pi[bt[m].long()].to(torch.int32)
+    out2, lse2 = orc.attention(wl.q, k2, v2, wl.sched.seq_lens, wl.sched.query_offsets, bt,
+                               wl.sched.page_size, wl.scale, wl.causal, wl.window)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def pin_split_equals_unsplit(orc):
+    wl = W.make_gqa("split", 16, [77, 130, 20], [1, 4, 20], 4, 2, 8, 8, 16, torch.float32, causal=True, window=60)
+    out, lse = orc.run(wl)
+    L = wl.sched.seq_lens
+    nparts = 5
+    o_parts, l_parts = [], []
+    for i in range(nparts):
+        kb = (L.long() * i // nparts).to(torch.int32)
+        ke = (L.long() * (i + 1) // nparts).to(torch.int32)
+        o, l = orc.run(wl, key_begin=kb, key_end=ke)
+        o_parts.append(o.reshape(-1, o.shape[-1])); l_parts.append(l.reshape(-1))
+    mo, ml = orc.lse_combine(torch.stack(o_parts), torch.stack(l_parts))
+    assert torch.allclose(mo.view_as(out), out, rtol=1e-12, atol=1e-13)
+    assert torch.allclose(ml.view_as(lse), lse, rtol=1e-12, atol=1e-13)
+
+
+def pin_chunked_equals_oneshot(orc):
+    hist, nA, nB = 45, 13, 22
+    for causal, window in ((True, 0), (True, 17)):
+        wl = W.make_gqa("chunk", 17, [hist + nA + nB], [nA + nB], 4, 2, 8, 8, 8, torch.float32, causal=causal, window=window)
+        s_ = wl.sched
+        out, lse = orc.run(wl)
+        oa, la = orc.attention(wl.q[:nA], wl.k_cache, wl.v_cache, torch.tensor([hist + nA]),
+                               torch.tensor([0, nA]), s_.block_tables, s_.page_size, wl.scale, causal, window)
+        ob, lb = orc.attention(wl.q[nA:], wl.k_cache, wl.v_cache, torch.tensor([hist + nA + nB]),
+                               torch.tensor([0, nB]), s_.block_tables, s_.page_size, wl.scale, causal, window)
+        assert torch.equal(torch.cat([oa, ob]), out) and torch.equal(torch.cat([la, lb]), lse)
+
+
+def pin_window_cases(orc):
+    wl = W.make_gqa("win", 18, [60, 31], [5, 31], 4, 2, 8, 8, 8, torch.float32, causal=True)
+    out0, lse0 = orc.run(wl)
+    big, lbig = orc.attention(wl.q, wl.k_cache, wl.v_cache, wl.sched.seq_lens, wl.sched.query_offsets,
+                              wl.sched.block_tables, 8, wl.scale, True, 61)
+    assert torch.equal(out0, big) and torch.equal(lse0, lbig)
+    one, _ = orc.attention(wl.q, wl.k_cache, wl.v_cache, wl.sched.seq_lens, wl.sched.query_offsets,
+                           wl.sched.block_tables, 8, wl.scale, True, 1)
+    s_ = wl.sched
+    for s in range(2):
+        L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+        V = _dense_kv(wl.v_cache, s_.block_tables, s, L, 8)
+        for j in range(n):
+            p = L - n + j
+            for h in range(4):
+                assert torch.equal(one[q0 + j, h], V[p, h // 2])
+
+
+def pin_gqa_equals_mha_repeated(orc):
+    wl = W.make_gqa("rep", 19, [33, 70], [3, 1], 8, 2, 8, 8, 8, torch.bfloat16, causal=True, window=25)
+    out, lse = orc.run(wl)
+    k = wl.k_cache.repeat_interleave(4, dim=2)
+    v = wl.v_cache.repeat_interleave(4, dim=2)
+    out2, lse2 = orc.attention(wl.q, k, v, wl.sched.seq_lens, wl.sched.query_offsets, wl.sched.block_tables,
+                               8, wl.scale, True, 25)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def pin_mla_equals_gqa_concat(orc):
+    wl = W.make_mla("mla", 20, [40, 9, 77], [1, 9, 3], 8, 32, 8, 8, torch.float32, causal=True, window=30)
+    out, lse = orc.run(wl)
+    q = torch.cat([wl.q_latent, wl.q_rope], dim=-1)
+    k = torch.cat([wl.latent_cache, wl.rope_cache], dim=-1)
+    out2, lse2 = orc.attention(q, k, wl.latent_cache, wl.sched.seq_lens, wl.sched.query_offsets,
+                               wl.sched.block_tables, 8, wl.scale, True, 30)
+    assert torch.allclose(out, out2, rtol=1e-12, atol=1e-13)
+    assert torch.allclose(lse, lse2, rtol=1e-12, atol=1e-13)
+
+
+def pin_half_precision_widening(orc):
+    for dt in (torch.bfloat16, torch.float16):
+        wl = W.make_gqa("wid", 21, [29, 50], [2, 1], 4, 2, 16, 8, 8, dt, causal=True)
+        out, lse = orc.run(wl)
+        out2, lse2 = orc.attention(wl.q.float(), wl.k_cache.float(), wl.v_cache.float(), wl.sched.seq_lens,
+                                   wl.sched.query_offsets, wl.sched.block_tables, 8, wl.scale, True, 0)
+        assert torch.equal(out, out2) and torch.equal(lse, lse2)
+    # every fp16 bit pattern (finite ones) widens to the value torch assigns it
+    bits = torch.from_numpy(np.arange(1 << 16, dtype=np.uint16).view(np.float16).copy())
+    finite = bits[torch.isfinite(bits)]
+    n = finite.numel() // 8 * 8
+    vals = finite[:n].view(-1, 1, 1, 8)  # pages of one slot, one head, eight dims
+    P = vals.shape[0]
+    q = torch.zeros(1, 1, 8, dtype=torch.float16)
+    q[0, 0, 0] = 1.0
+    sl = torch.tensor([1], dtype=torch.int32)
+    qo = torch.tensor([0, 1], dtype=torch.int32)
+    for page in (0, P // 3, P - 1):
+        bt = torch.tensor([[page]], dtype=torch.int32)
+        o, _ = orc.attention(q, vals, vals, sl, qo, bt, 1, 1.0, True, 0)
+        assert torch.equal(o[0, 0], vals[page, 0, 0].double())
+
+
+ALL_PINS = [
+    pin_sdpa_bruteforce, pin_alice_fixture_dense, pin_single_key, pin_constant_v_per_kv_head,
+    pin_q_zero_counts_and_mean, pin_position_probe, pin_large_score_selects_target,
+    pin_page_permutation_invariance, pin_split_equals_unsplit, pin_chunked_equals_oneshot,
+    pin_window_cases, pin_gqa_equals_mha_repeated, pin_mla_equals_gqa_concat,
+    pin_half_precision_widening,
+]
