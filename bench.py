@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the paged-KV attention library on B200.
+
+Headline: the paged GQA bf16 decode workload (batch 64 per GPU, context lengths uniform in
+[512, 8192], Hq 32, Hkv 8, D 128, pages of 16 shuffled over a shared pool, N(0,1) inputs
+rounded to bf16, scale 1/sqrt(128), causal). One step = one pa_forward over the whole batch
+(split-KV decode kernel + merge kernel). Metric: algorithmic KV bytes per second (each
+visible K/V row read once per sequence) -- GB/s.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch (seed + rank) on its own GPU: weak scaling, no
+collective on the data path. Rank 0 prints one JSON line.
+
+The reference arm (--impl reference) times the fp64 CPU oracle on the host cores, one bounded
+sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "decode KV GB/s & prefill TFLOPS, paged GQA attention (% of B200 roofline)"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def allreduce_max(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_sum(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(ws: int) -> None:
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.15)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_traffic(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            d = json.load(f)[key]
+        src = open(os.path.join(ROOT, "paged_kv_attention_39_b200", "csrc", kernel_file), "rb").read()
+        if d.get("source_sha256") != hashlib.sha256(src).hexdigest():
+            return None
+        return d
+    except Exception:
+        return None
+
+
+def time_forward(pa, plan, args_fn, steps, warmup, trace=True, sampler=None, ws=1):
+    """W untimed calls, then K calls bracketed by barrier + synchronize; per-call trace events."""
+    for _ in range(warmup):
+        args_fn(None)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)] if trace else None
+    trs = [pa.trace_events(e) for e in evs] if trace else None
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+    start.record()
+    for i in range(steps):
+        args_fn(trs[i] if trace else None)
+    end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    barrier(ws)
+    ms = start.elapsed_time(end) / steps
+    kern = comb = None
+    if trace:
+        kern = statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+        comb = statistics.fmean(e[1].elapsed_time(e[2]) for e in evs)
+    return ms, kern, comb, clocks
+
+
+def run_ours(args, ws, rank, local):
+    import paged_kv_attention_39_b200 as pa
+    from paged_kv_attention_39_b200 import workloads as W
+
+    pa.load_library()
+    hbm, tf_burst, tf_sust, peak_src = peaks()
+    dev = torch.device("cuda", local)
+    wl = W.c2_bf16_decode(args.seed + rank)
+    kv_bytes = W.algorithmic_kv_bytes(wl)
+    q = wl.q.to(dev)
+    k = wl.k_cache.to(dev)
+    v = wl.v_cache.to(dev)
+    nq, hq, d = q.shape
+    out = torch.empty(nq, hq, d, dtype=q.dtype, device=dev)
+    lse = torch.empty(nq, hq, dtype=torch.float32, device=dev)
+    plan = pa.plan_for(wl, device=local)
+    pa.pa_plan_prepare(plan, q.dtype, hq, wl.num_kv_heads, d, d, wl.causal, wl.window)
+
+    def step(tr):
+        pa.pa_forward(plan, q, k, v, out, lse, wl.scale, wl.causal, wl.window, trace=tr)
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    ms, kern_ms, comb_ms, clocks = time_forward(pa, plan, step, args.steps, args.warmup, True, sampler, ws)
+    launches_per_step = pa.pa_plan_get_info(plan)["last_launches"]
+    ms_max = allreduce_max(ms, ws)
+    total_bytes = allreduce_sum(kv_bytes, ws)
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+    achieved = kv_bytes / (kern_ms * 1e-3) / 1e9
+    traffic = kernel_traffic("decode.cu", "decode_mma_kernel")
+
+    # ---- end to end through the public API with host buffers -------------------------------
+    q_host = wl.q.pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 200))
+    e2e_times = []
+    uploaded = 0
+    for i in range((args.warmup if e2e_steps else 0) + e2e_steps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        q.copy_(q_host, non_blocking=True)
+        p2 = pa.plan_for(wl, device=local)
+        pa.pa_forward(p2, q, k, v, out, lse, wl.scale, wl.causal, wl.window)
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+        e1.record()
+        uploaded = pa.pa_plan_get_info(p2)["uploaded_bytes"]
+        p2.close()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            e2e_times.append(e0.elapsed_time(e1))
+    e2e_ms = allreduce_max(statistics.fmean(e2e_times) if e2e_times else float("nan"), ws)
+    e2e_val = total_bytes / (e2e_ms * 1e-3) / 1e9
+    plan.close()
+
+    extra = {}
+    if not args.no_extra and rank == 0:
+        extra = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src)
+
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) rounded to bf16; shuffled page pool)",
+        "config": {
+            "workload": f"paged GQA bf16 decode: batch {wl.sched.num_seqs}/GPU, context U[512,8192], "
+                        "Hq 32, Hkv 8, D 128, page 16, causal",
+            "kv_bytes_per_gpu_step": kv_bytes,
+            "tokens_per_gpu_step": int(wl.sched.seq_lens.sum()),
+            "l2": "inputs larger than L2 (%.2f GB of visible K/V vs 126 MB L2); no flush" % (kv_bytes / 1e9),
+            "parallelism": f"replicas x{ws} (independent batches, no collective)",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "decode_mma_kernel",
+            "achieved": round(achieved, 1),
+            "peak": hbm,
+            "peak_source": f"hbm_gbs {peak_src}",
+            "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "frac_note": f"of {peak_src}",
+            "kernel_ms": round(kern_ms, 5),
+            "merge_ms": round(comb_ms, 5),
+            "traffic": (traffic["dram_bytes_per_launch"] * kv_bytes / traffic["kv_bytes_per_launch"]) if traffic else None,
+            "traffic_source": traffic.get("source") if traffic else None,
+            "frac_of_8tbs": round(achieved / 8000.0, 4),
+        },
+        "e2e": {
+            "value": round(e2e_val, 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size() + uploaded),
+            "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size() + lse_host.numel() * 4),
+            "ms_per_step": round(e2e_ms, 4),
+            "includes": "H2D of Q from pinned memory, pa_plan_create (schedule upload) + work-list upload, "
+                        "pa_forward, D2H of out and lse into pinned memory",
+        },
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if extra:
+        result["extra"] = extra
+    if rank == 0 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, kv_bytes)
+    return result
+
+
+def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src):
+    """The other configurations, timed the same way (few steps): context for the headline."""
+    res = {}
+    cfgs = [("bf16_chunked_prefill", W.c3_chunked_prefill), ("bf16_window_mixed", W.c4_window_mixed),
+            ("bf16_mla_decode", W.c5_mla_decode)]
+    for name, fn in cfgs:
+        try:
+            wl = fn(args.seed)
+            flops = W.algorithmic_flops(wl)
+            kvb = W.algorithmic_kv_bytes(wl)
+            plan = pa.plan_for(wl, device=dev.index)
+            if wl.kind == "mla":
+                ql, qr = wl.q_latent.to(dev), wl.q_rope.to(dev)
+                lat, rope = wl.latent_cache.to(dev), wl.rope_cache.to(dev)
+                out = torch.empty(ql.shape, dtype=ql.dtype, device=dev)
+                lse = torch.empty(ql.shape[:2], dtype=torch.float32, device=dev)
+
+                def step(tr):
+                    pa.pa_mla_forward(plan, ql, qr, lat, rope, out, lse, wl.scale, wl.causal, wl.window, trace=tr)
+            else:
+                q, k, v = wl.q.to(dev), wl.k_cache.to(dev), wl.v_cache.to(dev)
+                out = torch.empty(q.shape[0], q.shape[1], wl.v_head_dim, dtype=q.dtype, device=dev)
+                lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+
+                def step(tr):
+                    pa.pa_forward(plan, q, k, v, out, lse, wl.scale, wl.causal, wl.window, trace=tr)
+            ms, kern, comb, _ = time_forward(pa, plan, step, args.extra_steps, 3, True, None, 1)
+            res[name] = {
+                "ms_per_step": round(ms, 4),
+                "attention_kernels_ms": round(kern, 4),
+                "merge_ms": round(comb, 4),
+                "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                "kv_gbs": round(kvb / (ms * 1e-3) / 1e9, 1),
+                "frac_tensor_of_%s" % peak_src: round(flops / (ms * 1e-3) / 1e12 / tf_burst, 4),
+                "frac_hbm_of_%s" % peak_src: round(kvb / (ms * 1e-3) / 1e9 / hbm, 4),
+                "algorithmic_gflop": round(flops / 1e9, 2),
+                "algorithmic_kv_mb": round(kvb / 1e6, 1),
+                "launches": pa.pa_plan_get_info(plan)["last_launches"],
+            }
+            plan.close()
+            del wl
+        except Exception as e:  # a failing extra must not hide the headline
+            res[name] = {"error": str(e)[:300]}
+    return res
+
+
+def cpu_baseline(wl, kv_bytes, budget_s: float = 10.0):
+    """The fp64 oracle, as it stands, on the host cores: whole workload, repeated ~budget_s."""
+    import oracle
+    from paged_kv_attention_39_b200 import workloads as W  # noqa: F401
+    orc = oracle.get()
+    cores = os.cpu_count() or 1
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orc.run(wl, nthreads=cores)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(kv_bytes * reps / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"the full headline workload (one GPU's batch), {reps} run(s) in {dt:.1f} s"}
+
+
+def run_reference(args, ws, rank):
+    """The oracle arm: each step runs the fp64 CPU oracle on a bounded sample of the workload."""
+    import oracle
+    from paged_kv_attention_39_b200 import workloads as W
+    if rank != 0:
+        return None
+    orc = oracle.get()
+    cores = os.cpu_count() or 1
+    wl = W.c2_bf16_decode(args.seed)
+    s = wl.sched
+    # a sample of whole sequences sized so that warmup + steps fit about two minutes
+    t0 = time.perf_counter()
+    orc.run(wl, nthreads=cores, rows=list(range(0, wl.num_q_heads)))  # one sequence's rows
+    one = max(time.perf_counter() - t0, 1e-4)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    nseq = int(max(1, min(s.num_seqs, budget / one)))
+    rows = list(range(0, nseq * wl.num_q_heads))
+    sub_bytes = 0
+    per_tok = wl.num_kv_heads * (wl.head_dim + wl.v_head_dim) * 2
+    for i in range(nseq):
+        sub_bytes += int(s.seq_lens[i]) * per_tok
+    for _ in range(args.warmup):
+        orc.run(wl, nthreads=cores, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.run(wl, nthreads=cores, rows=rows)
+    dt = (time.perf_counter() - t0) / args.steps
+    val = sub_bytes / dt / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) rounded to bf16; shuffled page pool)",
+        "config": {"workload": "paged GQA bf16 decode: batch 64, context U[512,8192], Hq 32, Hkv 8, D 128, "
+                               "page 16, causal", "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {nseq} sequence(s) of the batch per step, all heads"},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-extra", action="store_true", help="skip the other configurations")
+    ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = dist_setup()
+    if args.impl == "reference":
+        res = run_reference(args, ws, rank)
+    else:
+        res = run_ours(args, ws, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

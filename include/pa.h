@@ -1,0 +1,215 @@
+/*
+ * pa.h -- C ABI of the paged-KV attention library (libpa.so), CUDA sm_100a (B200).
+ *
+ * The library computes attention over a paged KV cache for packed decode and chunked
+ * prefill, returning the output and a float32 logsumexp:
+ *
+ *     out[q, h, :] = softmax_t( scale * Q[q, h, :] . K_s[t, h / G, :] + mask(q, t) ) . V_s[t, h / G, :]
+ *     lse[q, h]    = ln sum_t exp( scale * Q[q, h, :] . K_s[t, h / G, :] )   over visible t
+ *
+ * This is the dense definition of boostr's `standard_attention_fwd` (flash_standard.rs:
+ * scores, additive 0/-inf mask, logsumexp cast to F32, softmax times V; query head h reads
+ * KV head h / G with G = Hq / Hkv as in `expand_kv`), evaluated over ruDNN's paged layout
+ * (paged_attention/mod.rs, `DevicePlan::attention`): packed Q [queries, Hq, D], K cache
+ * [pages, page_size, Hkv, D], V cache [pages, page_size, Hkv, Dv], with key t of sequence s
+ * in page block_tables[s][t / page_size], slot t % page_size. Neither padded KV gathers nor
+ * per-head KV copies are made.
+ *
+ * Positions and mask. Sequence s has L_s keys (its own new keys included: they are already
+ * in the cache) and n_s queries; query j of s sits at absolute position p = L_s - n_s + j
+ * (right-aligned: ruDNN "absolute positions ... including prefill chunks", alice-llm
+ * "right-aligned causal mask"). Key t is visible to it iff
+ *     (!causal || t <= p)  &&  (window == 0 || t + window > p)
+ * (boostr `build_attention_mask`: causal masks j > i, a window masks j + window <= i,
+ * window 0 is unlimited). A row with no visible key yields out = 0 and lse = -inf.
+ *
+ * Ownership. Every data pointer is caller-owned device memory on the plan's device,
+ * contiguous in the stated layout. The library never synchronises the host with the GPU
+ * inside pa_forward / pa_mla_forward and never reads device data back (ruDNN: "no CPU
+ * synchronization or host readback").
+ *
+ * Errors. Every entry point validates all of its arguments before it launches or allocates
+ * anything (ruDNN: validate every supplied output before any allocation, clear or launch);
+ * on error nothing is launched, a pa_status other than PA_OK is returned, and
+ * pa_last_error_message() describes the failure (a thread-local string).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes (ruDNN's PagedAttentionError becomes a code plus a message). */
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad flag, non-finite or non-positive scale */
+    PA_ERR_SHAPE = 2,            /* head counts/dims inconsistent (e.g. Hq % Hkv != 0) */
+    PA_ERR_DTYPE = 3,            /* unknown element type */
+    PA_ERR_BOUNDS = 4,           /* page id outside the pool, table too narrow, size overflow */
+    PA_ERR_ALIAS = 5,            /* out or lse overlaps an input or each other */
+    PA_ERR_UNSUPPORTED = 6,      /* valid but not implemented (e.g. head_dim > 1024) */
+    PA_ERR_CUDA = 7              /* a CUDA runtime call or kernel launch failed */
+} pa_status;
+
+/* Element type of Q, K, V and out (ruDNN accepts F32, F16, BF16). lse is always float32. */
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+
+/* A cudaStream_t. NULL is the legacy default stream. */
+typedef void* pa_stream;
+
+/* Opaque, immutable schedule: per-sequence lengths, query offsets and block tables on the
+ * device, plus the plan-owned float32 split workspace. */
+typedef struct pa_plan pa_plan;
+
+/*
+ * pa_plan_create -- validate a batch schedule and upload it once (ruDNN `DevicePlan::upload`:
+ * "creating a new plan is one small upload"; immutable, reusable while the schedule is
+ * unchanged).
+ *
+ *   seq_lens       [num_seqs] host int32: L_s >= 0, keys of sequence s incl. its new ones.
+ *   query_offsets  [num_seqs + 1] host int32: prefix sums of n_s, query_offsets[0] == 0,
+ *                  0 <= n_s <= L_s. Queries of s are rows query_offsets[s] .. [s+1]-1 of Q.
+ *   block_tables   [num_seqs, table_width] host int32, row-major. Entries 0 .. ceil(L_s /
+ *                  page_size) - 1 of row s must lie in [0, num_pages); later entries are never
+ *                  read and may hold anything (e.g. -1).
+ *   page_size      > 0 tokens per page; num_pages >= 0 pages in the pool.
+ *   device         CUDA device ordinal, or -1 for a host-only plan: it validates and keeps
+ *                  the schedule but owns no device memory, and every forward call on it fails
+ *                  with PA_ERR_INVALID_ARGUMENT after validating its own arguments.
+ *   upload_stream  stream of the single host-to-device copy (the plan keeps its host copy
+ *                  alive, so the caller may free its arrays on return).
+ *   out_plan       receives the plan; set to NULL on error.
+ *
+ * Errors: PA_ERR_INVALID_ARGUMENT (null pointers, negative sizes, n_s > L_s, offsets not
+ * starting at 0 or decreasing), PA_ERR_BOUNDS (table too narrow, page id outside the pool),
+ * PA_ERR_CUDA (allocation or copy failed).
+ */
+pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, int32_t num_seqs,
+                         const int32_t* block_tables, int32_t table_width, int32_t page_size,
+                         int32_t num_pages, int device, pa_stream upload_stream,
+                         pa_plan** out_plan);
+
+/* Free the plan's device memory, stream-ordered on the stream of its last call (or its upload
+ * stream): work already queued there may still use it, work on other streams must be done.
+ * The host does not wait. NULL is a no-op. */
+pa_status pa_plan_destroy(pa_plan* plan);
+
+/* Read-only facts about a plan. */
+typedef struct pa_plan_info {
+    int32_t num_seqs;
+    int32_t num_queries;     /* query_offsets[num_seqs] */
+    int32_t table_width;
+    int32_t page_size;
+    int32_t num_pages;
+    int32_t device;          /* -1 for a host-only plan */
+    int32_t last_launches;   /* kernels the last successful forward call launched */
+    int64_t workspace_bytes; /* current size of the plan-owned split workspace */
+    int64_t uploaded_bytes;  /* host-to-device bytes the plan has copied (schedule, work lists) */
+} pa_plan_info;
+pa_status pa_plan_get_info(const pa_plan* plan, pa_plan_info* info);
+
+/* Path selection (testing and tuning). */
+typedef enum pa_path {
+    PA_PATH_AUTO = 0, /* tensor-core kernels where the shape allows, CUDA-core kernel elsewhere */
+    PA_PATH_SIMT = 1  /* the CUDA-core kernel for every row (any dtype and head size) */
+} pa_path;
+
+typedef struct pa_forward_options {
+    int32_t kv_chunk; /* keys per split-KV part on the decode paths: 0 = automatic,
+                         -1 = never split, > 0 = that many keys per part */
+    int32_t path;     /* a pa_path */
+    void** trace_events; /* NULL, or three cudaEvent_t recorded on the call's stream: before
+                            the attention kernels, between them and the merge kernel, and
+                            after the merge kernel (kernel timing without a profiler) */
+} pa_forward_options;
+
+/*
+ * pa_forward -- paged GQA/MHA attention for every query row of the plan, on `stream`.
+ *
+ *   q          [N_q, num_q_heads, head_dim]             dtype, N_q = plan's num_queries
+ *   k_cache    [num_pages, page_size, num_kv_heads, head_dim]    dtype
+ *   v_cache    [num_pages, page_size, num_kv_heads, v_head_dim]  dtype
+ *   scale      finite, > 0 (the caller's choice, e.g. 1/sqrt(head_dim))
+ *   causal     0 or 1; window >= 0 (0 = no window)
+ *   out        [N_q, num_q_heads, v_head_dim] dtype (written; must not overlap any input)
+ *   lse        [N_q, num_q_heads] float32 (written; natural log; must not overlap anything)
+ *
+ * Shapes: num_kv_heads >= 1, num_q_heads % num_kv_heads == 0, 1 <= head_dim, v_head_dim
+ * <= 1024 (ruDNN's limit). N_q == 0 returns PA_OK without launching anything.
+ * Long contexts are split over several CTAs whose float32 partial results (o_i, lse_i) go to
+ * the plan-owned workspace and are merged by a second kernel (ruDNN "split the visible
+ * history over multiple planes and merge FP32 statistics"). The workspace grows on demand
+ * with stream-ordered allocation on `stream`; calls on one plan must therefore be ordered
+ * (one stream, or explicit events). The first call with a new head configuration builds and
+ * uploads that configuration's work list once (also available as pa_plan_prepare); make it
+ * before capturing the stream into a CUDA graph.
+ * Inputs must be finite; non-finite values propagate (ruDNN contract).
+ */
+pa_status pa_forward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                     pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads,
+                     int32_t head_dim, int32_t v_head_dim, float scale, int causal,
+                     int32_t window, void* out, float* lse, pa_stream stream);
+
+/* pa_forward with options (NULL = defaults). */
+pa_status pa_forward_ex(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                        pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads,
+                        int32_t head_dim, int32_t v_head_dim, float scale, int causal,
+                        int32_t window, void* out, float* lse, pa_stream stream,
+                        const pa_forward_options* opts);
+
+/*
+ * pa_mla_forward -- MLA absorbed-latent attention (ruDNN `DevicePlan::mla`).
+ *
+ *   q_latent      [N_q, num_heads, latent_dim]   absorbed queries
+ *   q_rope        [N_q, num_heads, rope_dim]     position queries
+ *   latent_cache  [num_pages, page_size, 1, latent_dim]  one shared latent head
+ *   rope_cache    [num_pages, page_size, 1, rope_dim]
+ *   out           [N_q, num_heads, latent_dim]   compressed context (the latent is both key
+ *                 and value; the caller applies the value/output projection afterwards)
+ *   lse           [N_q, num_heads] float32
+ *
+ * score(q, h, t) = scale * (q_latent[q,h,:] . latent[t,:] + q_rope[q,h,:] . rope[t,:]);
+ * `scale` comes from the original model's QK dimensions, not the latent rank (ruDNN).
+ * Shapes: 1 <= latent_dim <= 1024, 1 <= rope_dim <= 256 (ruDNN's positional limit).
+ * Same masking, ownership, workspace and error rules as pa_forward.
+ */
+pa_status pa_mla_forward(pa_plan* plan, const void* q_latent, const void* q_rope,
+                         const void* latent_cache, const void* rope_cache, pa_dtype dtype,
+                         int32_t num_heads, int32_t latent_dim, int32_t rope_dim, float scale,
+                         int causal, int32_t window, void* out, float* lse, pa_stream stream);
+
+pa_status pa_mla_forward_ex(pa_plan* plan, const void* q_latent, const void* q_rope,
+                            const void* latent_cache, const void* rope_cache, pa_dtype dtype,
+                            int32_t num_heads, int32_t latent_dim, int32_t rope_dim, float scale,
+                            int causal, int32_t window, void* out, float* lse, pa_stream stream,
+                            const pa_forward_options* opts);
+
+/*
+ * pa_plan_prepare -- build and upload the work list of one head configuration ahead of the
+ * first forward call (pa_forward does it implicitly). `mla` selects pa_mla_forward's
+ * configuration (num_kv_heads is then 1 and v_head_dim == head_dim == latent_dim).
+ * Uses `stream` for the one upload and the workspace allocation.
+ */
+pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_heads,
+                          int32_t num_kv_heads, int32_t head_dim, int32_t v_head_dim,
+                          int causal, int32_t window, pa_stream stream,
+                          const pa_forward_options* opts);
+
+/* Human-readable name of a status code (static string). */
+const char* pa_status_string(pa_status status);
+
+/* Message of the last failing call on this thread ("" if none); valid until the next call. */
+const char* pa_last_error_message(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -124,6 +124,13 @@ static void pao_run_item(pao_job* J, int32_t s, int32_t kvh, double* kbuf, doubl
     const int32_t vd = J->dv;           /* width of the value rows */
     const int32_t kheads = J->mla ? 1 : J->hkv;
     if (n == 0) return;
+    if (J->want) { /* skip the gather when no row of this (sequence, kv head) is asked for */
+        int any = 0;
+        for (int32_t g = 0; g < G && !any; ++g)
+            for (int64_t j = 0; j < n && !any; ++j)
+                any = J->want[(q0 + j) * J->hq + (J->mla ? g : kvh * G + g)] != 0;
+        if (!any) return;
+    }
 
     /* 1. materialise this sequence's keys/values for this KV head contiguously */
     for (int64_t t = 0; t < L; ++t) {

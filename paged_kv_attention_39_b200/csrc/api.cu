@@ -1,0 +1,607 @@
+// Host side of libpa.so: the C ABI, argument validation, the plan (schedule upload and
+// split workspace) and kernel dispatch.
+//
+// Validation follows ruDNN's paged_attention/mod.rs (`check_tensor`, `bounded`,
+// `execute_attention_into`): every argument is checked before anything is launched or
+// allocated, and an empty batch returns success without a launch.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <memory>
+#include <mutex>
+#include <vector>
+
+#include "pa_internal.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+pa_status fail(pa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+pa_status ok() {
+    g_msg[0] = '\0';
+    return PA_OK;
+}
+
+#define PA_CUDA_TRY(expr)                                                                    \
+    do {                                                                                     \
+        cudaError_t e_ = (expr);                                                             \
+        if (e_ != cudaSuccess)                                                               \
+            return fail(PA_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));        \
+    } while (0)
+
+size_t dtype_size(pa_dtype dt) { return dt == PA_F32 ? 4 : 2; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t* r) { return !__builtin_mul_overflow(a, b, r); }
+
+// Product of non-negative dims; false on overflow of int64.
+bool product(std::initializer_list<int64_t> dims, int64_t* r) {
+    int64_t acc = 1;
+    for (int64_t d : dims) {
+        if (d < 0 || !mul_ok(acc, d, &acc)) return false;
+    }
+    *r = acc;
+    return true;
+}
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+constexpr int kMaxSplits = 1024;           // parts one sequence's keys may be cut into
+constexpr int kTargetCtasPerSm = 8;        // automatic split size aims at this many CTAs/SM
+
+struct SchedKey {
+    int mla, dtype, hq, hkv, d, dv, causal, window, path, kv_chunk;
+    bool operator==(const SchedKey& o) const { return std::memcmp(this, &o, sizeof o) == 0; }
+};
+
+struct Schedule {
+    SchedKey key;
+    std::vector<char> host;  // uploaded blob, kept alive for the asynchronous copy
+    void* dev = nullptr;
+    const pa::KvUnit* tc_units = nullptr;     // tensor-core decode kernel
+    const pa::KvUnit* simt_units = nullptr;   // CUDA-core kernel
+    const pa::CombineUnit* cunits = nullptr;
+    int32_t n_tc = 0, n_simt = 0, n_comb = 0;
+    int32_t tc_rows_max = 0;
+    int64_t slots = 0;  // workspace parts
+    int32_t kv_chunk = 0;
+};
+
+}  // namespace
+
+struct pa_plan {
+    int device = -1;
+    int num_sms = 148;
+    int32_t S = 0, Nq = 0, table_width = 0, page_size = 0, num_pages = 0;
+    std::vector<pa::SeqInfo> seqs;
+    std::vector<int32_t> bt;
+    void* d_meta = nullptr;
+    std::vector<char> meta_host;
+    pa::SeqInfo* d_seqs = nullptr;
+    int32_t* d_bt = nullptr;
+    std::vector<std::unique_ptr<Schedule>> scheds;  // most recent last
+    float* ws = nullptr;
+    size_t ws_bytes = 0;
+    cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
+    int32_t last_launches = 0;
+    int64_t uploaded_bytes = 0;
+    std::mutex mu;
+};
+
+namespace {
+
+// ---------------------------------------------------------------------------------------
+// Schedule construction
+// ---------------------------------------------------------------------------------------
+
+// Keys [lo, hi) that queries j0 .. j1-1 of a sequence can see (union over those queries).
+void visible_union(int32_t L, int32_t n, int32_t j0, int32_t j1, bool causal, int32_t window,
+                   int32_t* lo, int32_t* hi) {
+    const int64_t p_first = (int64_t)L - n + j0;
+    const int64_t p_last = (int64_t)L - n + j1 - 1;
+    int64_t a = window > 0 ? std::max<int64_t>(0, p_first - window + 1) : 0;
+    int64_t b = causal ? std::min<int64_t>(L, p_last + 1) : L;
+    if (b < a) b = a;
+    *lo = (int32_t)a;
+    *hi = (int32_t)b;
+}
+
+int32_t ceil_div(int64_t a, int64_t b) { return (int32_t)((a + b - 1) / b); }
+
+pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedule** out) {
+    for (auto& s : P->scheds)
+        if (s->key == k) { *out = s.get(); return PA_OK; }
+
+    auto S = std::make_unique<Schedule>();
+    S->key = k;
+    const int32_t G = k.hq / k.hkv;
+    const bool tc_decode = !k.mla && k.path == PA_PATH_AUTO && k.dtype != PA_F32 &&
+                           k.d == k.dv && (k.d == 64 || k.d == 128);
+
+    struct Block { int32_t seq, j0, j1, lo, hi; bool tc; };
+    std::vector<Block> blocks;
+    int64_t total = 0;  // keys x kv heads, over all blocks
+    for (int32_t s = 0; s < P->S; ++s) {
+        const pa::SeqInfo& si = P->seqs[s];
+        if (si.n == 0) continue;
+        const bool tc = tc_decode && (int64_t)si.n * G <= pa::kDecodeMaxRows;
+        // CUDA-core blocks take few queries so that long prefill chunks spread over CTAs.
+        const int32_t qb = tc ? si.n : std::max<int32_t>(1, 16 / std::min<int32_t>(G, 16));
+        for (int32_t j0 = 0; j0 < si.n; j0 += qb) {
+            Block b{s, j0, std::min(si.n, j0 + qb), 0, 0, tc};
+            visible_union(si.L, si.n, b.j0, b.j1, k.causal, k.window, &b.lo, &b.hi);
+            total += (int64_t)(b.hi - b.lo) * (k.mla ? 1 : k.hkv);
+            blocks.push_back(b);
+        }
+    }
+    int64_t chunk;
+    if (k.kv_chunk > 0) chunk = k.kv_chunk;
+    else if (k.kv_chunk < 0) chunk = INT32_MAX;
+    else {
+        const int64_t target = (int64_t)P->num_sms * kTargetCtasPerSm;
+        chunk = (total + target - 1) / std::max<int64_t>(1, target);
+        chunk = ((chunk + 63) / 64) * 64;
+        chunk = std::max<int64_t>(chunk, 256);
+    }
+
+    std::vector<pa::KvUnit> tcu, simtu;
+    std::vector<pa::CombineUnit> cu;
+    int64_t slots = 0;
+    for (const Block& b : blocks) {
+        const int64_t len = b.hi - b.lo;
+        int64_t c = chunk;
+        int32_t nsplit = len <= 0 ? 1 : ceil_div(len, c);
+        if (nsplit > kMaxSplits) { c = (len + kMaxSplits - 1) / kMaxSplits; nsplit = ceil_div(len, c); }
+        const int32_t base = nsplit > 1 ? (int32_t)slots : -1;
+        if (nsplit > 1) {
+            for (int32_t j = b.j0; j < b.j1; ++j)
+                cu.push_back({P->seqs[b.seq].q_start + j, base + (j - b.j0) * nsplit, nsplit, 0});
+            slots += (int64_t)(b.j1 - b.j0) * nsplit;
+        }
+        for (int32_t i = 0; i < nsplit; ++i) {
+            pa::KvUnit u;
+            u.seq = b.seq;
+            u.t0 = (int32_t)std::min<int64_t>(b.hi, b.lo + i * c);
+            u.t1 = (int32_t)std::min<int64_t>(b.hi, b.lo + (i + 1) * c);
+            u.split = i;
+            u.nsplit = nsplit;
+            u.part_base = base;
+            u.j0 = b.j0;
+            u.j1 = b.j1;
+            (b.tc ? tcu : simtu).push_back(u);
+            if (b.tc) S->tc_rows_max = std::max<int32_t>(S->tc_rows_max, (b.j1 - b.j0) * G);
+        }
+    }
+    // Longest units first: the block scheduler hands them out in index order.
+    auto longer = [](const pa::KvUnit& a, const pa::KvUnit& b) {
+        return (int64_t)(a.t1 - a.t0) * (a.j1 - a.j0) > (int64_t)(b.t1 - b.t0) * (b.j1 - b.j0);
+    };
+    std::stable_sort(tcu.begin(), tcu.end(), longer);
+    std::stable_sort(simtu.begin(), simtu.end(), longer);
+    if (slots > INT32_MAX) return fail(PA_ERR_BOUNDS, "split workspace needs too many parts");
+
+    // One blob: [tc units][simt units][combine units], 256-byte aligned sections.
+    auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t o_tc = 0;
+    const size_t o_simt = align(o_tc + tcu.size() * sizeof(pa::KvUnit));
+    const size_t o_c = align(o_simt + simtu.size() * sizeof(pa::KvUnit));
+    const size_t bytes = align(o_c + cu.size() * sizeof(pa::CombineUnit));
+    S->host.assign(std::max<size_t>(bytes, 256), 0);
+    if (!tcu.empty()) std::memcpy(S->host.data() + o_tc, tcu.data(), tcu.size() * sizeof(pa::KvUnit));
+    if (!simtu.empty()) std::memcpy(S->host.data() + o_simt, simtu.data(), simtu.size() * sizeof(pa::KvUnit));
+    if (!cu.empty()) std::memcpy(S->host.data() + o_c, cu.data(), cu.size() * sizeof(pa::CombineUnit));
+    PA_CUDA_TRY(cudaMallocAsync(&S->dev, S->host.size(), st));
+    cudaError_t e = cudaMemcpyAsync(S->dev, S->host.data(), S->host.size(), cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(S->dev, st);
+        return fail(PA_ERR_CUDA, "schedule upload failed: %s", cudaGetErrorString(e));
+    }
+    P->uploaded_bytes += (int64_t)S->host.size();
+    char* base = (char*)S->dev;
+    S->tc_units = (const pa::KvUnit*)(base + o_tc);
+    S->simt_units = (const pa::KvUnit*)(base + o_simt);
+    S->cunits = (const pa::CombineUnit*)(base + o_c);
+    S->n_tc = (int32_t)tcu.size();
+    S->n_simt = (int32_t)simtu.size();
+    S->n_comb = (int32_t)cu.size();
+    S->slots = slots;
+    S->kv_chunk = (int32_t)std::min<int64_t>(chunk, INT32_MAX);
+
+    if (P->scheds.size() >= 8) {  // keep the plan's footprint bounded
+        // The host blob must outlive its copy: retire it only after the stream drains.
+        cudaStreamSynchronize(st);
+        cudaFreeAsync(P->scheds.front()->dev, st);
+        P->scheds.erase(P->scheds.begin());
+    }
+    P->scheds.push_back(std::move(S));
+    *out = P->scheds.back().get();
+    return PA_OK;
+}
+
+pa_status ensure_workspace(pa_plan* P, size_t bytes, cudaStream_t st) {
+    if (bytes <= P->ws_bytes) return PA_OK;
+    if (P->ws) {
+        PA_CUDA_TRY(cudaFreeAsync(P->ws, st));
+        P->ws = nullptr;
+        P->ws_bytes = 0;
+    }
+    void* p = nullptr;
+    PA_CUDA_TRY(cudaMallocAsync(&p, bytes, st));
+    P->ws = (float*)p;
+    P->ws_bytes = bytes;
+    return PA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Shared validation of a forward call
+// ---------------------------------------------------------------------------------------
+
+struct Call {
+    bool mla;
+    const void *q, *k, *v, *qr, *kr;
+    pa_dtype dtype;
+    int32_t hq, hkv, d, dv, pr;
+    float scale;
+    int causal;
+    int32_t window;
+    void* out;
+    float* lse;
+    pa_forward_options opts;
+};
+
+pa_status validate(pa_plan* P, const Call& c) {
+    if (!P) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    if (c.dtype != PA_F32 && c.dtype != PA_BF16 && c.dtype != PA_F16)
+        return fail(PA_ERR_DTYPE, "unknown dtype %d", (int)c.dtype);
+    if (c.hq <= 0 || c.hkv <= 0 || c.hq % c.hkv != 0)
+        return fail(PA_ERR_SHAPE, "query heads (%d) must be a positive multiple of kv heads (%d)", c.hq, c.hkv);
+    if (c.d <= 0 || c.dv <= 0)
+        return fail(PA_ERR_SHAPE, "head dims must be positive (d=%d, dv=%d)", c.d, c.dv);
+    if (c.d > 1024 || c.dv > 1024)
+        return fail(PA_ERR_UNSUPPORTED, "head dims above 1024 are not supported (d=%d, dv=%d)", c.d, c.dv);
+    if (c.mla && (c.pr <= 0 || c.pr > 256))
+        return fail(PA_ERR_SHAPE, "MLA rope dim must be in 1..256 (got %d)", c.pr);
+    if (!std::isfinite(c.scale) || !(c.scale > 0.0f))
+        return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and > 0");
+    if (c.causal != 0 && c.causal != 1) return fail(PA_ERR_INVALID_ARGUMENT, "causal must be 0 or 1");
+    if (c.window < 0) return fail(PA_ERR_INVALID_ARGUMENT, "window must be >= 0");
+    if (c.opts.path != PA_PATH_AUTO && c.opts.path != PA_PATH_SIMT)
+        return fail(PA_ERR_INVALID_ARGUMENT, "unknown path %d", c.opts.path);
+    if (c.opts.kv_chunk < -1) return fail(PA_ERR_INVALID_ARGUMENT, "kv_chunk must be -1, 0 or > 0");
+
+    const int64_t es = (int64_t)dtype_size(c.dtype);
+    int64_t nq = P->Nq, pages = P->num_pages, ps = P->page_size;
+    int64_t n_q, n_k, n_v, n_o, n_l, n_qr = 0, n_kr = 0;
+    if (!product({nq, c.hq, c.d, es}, &n_q) || !product({pages, ps, c.hkv, c.d, es}, &n_k) ||
+        !product({pages, ps, c.hkv, c.dv, es}, &n_v) || !product({nq, c.hq, c.dv, es}, &n_o) ||
+        !product({nq, c.hq, 4}, &n_l) ||
+        (c.mla && (!product({nq, c.hq, c.pr, es}, &n_qr) || !product({pages, ps, c.pr, es}, &n_kr))))
+        return fail(PA_ERR_BOUNDS, "tensor size overflows 64-bit byte counts");
+    if (nq == 0) return PA_OK;  // nothing is read or written
+    if (!c.q || !c.out || !c.lse || (n_k > 0 && (!c.k || !c.v)) || (c.mla && (!c.qr || (n_kr > 0 && !c.kr))))
+        return fail(PA_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    for (const void* ptr : {c.q, c.k, c.v, c.qr, c.kr, (const void*)c.out, (const void*)c.lse})
+        if ((uintptr_t)ptr % 16 != 0)
+            return fail(PA_ERR_INVALID_ARGUMENT, "device pointers must be 16-byte aligned");
+    auto R = [](const void* p, int64_t n) { return Range{(uintptr_t)p, (uintptr_t)p + (uintptr_t)n}; };
+    Range ro = R(c.out, n_o), rl = R(c.lse, n_l);
+    Range ins[5] = {R(c.q, n_q), R(c.k, n_k), R(c.v, n_v), R(c.qr, n_qr), R(c.kr, n_kr)};
+    if (overlap(ro, rl)) return fail(PA_ERR_ALIAS, "out and lse overlap");
+    for (const Range& r : ins)
+        if (overlap(ro, r) || overlap(rl, r)) return fail(PA_ERR_ALIAS, "out or lse overlaps an input");
+    return PA_OK;
+}
+
+pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
+    pa_status vs = validate(P, c);
+    if (vs != PA_OK) return vs;
+    if (P->Nq == 0) return ok();
+    if (P->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to run on");
+    int cur = -1;
+    PA_CUDA_TRY(cudaGetDevice(&cur));
+    if (cur != P->device)
+        return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, P->device);
+
+    std::lock_guard<std::mutex> lock(P->mu);
+    P->last_stream = st;
+    SchedKey key{};
+    key.mla = c.mla;
+    key.dtype = c.dtype;
+    key.hq = c.hq;
+    key.hkv = c.hkv;
+    key.d = c.d;
+    key.dv = c.dv;
+    key.causal = c.causal;
+    key.window = c.window;
+    key.path = c.opts.path;
+    key.kv_chunk = c.opts.kv_chunk;
+    Schedule* S = nullptr;
+    pa_status bs = build_schedule(P, key, st, &S);
+    if (bs != PA_OK) return bs;
+    if (S->slots > 0) {
+        const size_t need = (size_t)S->slots * c.hq * (c.dv + 1) * sizeof(float);
+        pa_status ws = ensure_workspace(P, need, st);
+        if (ws != PA_OK) return ws;
+    }
+
+    pa::AttnParams p{};
+    p.q = c.q; p.k = c.k; p.v = c.v; p.qr = c.qr; p.kr = c.kr;
+    p.out = c.out; p.lse = c.lse;
+    p.ws_o = P->ws;
+    p.ws_lse = P->ws ? P->ws + (size_t)S->slots * c.hq * c.dv : nullptr;
+    p.seqs = P->d_seqs;
+    p.block_tables = P->d_bt;
+    p.cunits = S->cunits;
+    p.num_cunits = S->n_comb;
+    p.table_width = P->table_width;
+    p.page_size = P->page_size;
+    p.hq = c.hq; p.hkv = c.hkv; p.group = c.hq / c.hkv;
+    p.d = c.d; p.dv = c.dv; p.pr = c.mla ? c.pr : 0;
+    p.scale = c.scale;
+    p.scale_log2 = (float)((double)c.scale * 1.4426950408889634);
+    p.causal = c.causal; p.window = c.window;
+
+    cudaEvent_t* ev = (cudaEvent_t*)c.opts.trace_events;
+    cudaError_t e;
+    int launches = 0;
+    if (ev) PA_CUDA_TRY(cudaEventRecord(ev[0], st));
+    if (S->n_tc > 0) {
+        ++launches;
+        p.units = S->tc_units;
+        p.num_units = S->n_tc;
+        e = pa::launch_decode_mma(p, c.dtype, S->tc_rows_max, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode kernel launch failed: %s", cudaGetErrorString(e));
+    }
+    if (S->n_simt > 0) {
+        ++launches;
+        p.units = S->simt_units;
+        p.num_units = S->n_simt;
+        e = pa::launch_simt(p, c.dtype, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "CUDA-core kernel launch failed: %s", cudaGetErrorString(e));
+    }
+    if (ev) PA_CUDA_TRY(cudaEventRecord(ev[1], st));
+    if (S->n_comb > 0) {
+        ++launches;
+        e = pa::launch_combine(p, c.dtype, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine kernel launch failed: %s", cudaGetErrorString(e));
+    }
+    if (ev) PA_CUDA_TRY(cudaEventRecord(ev[2], st));
+    P->last_launches = launches;
+    return ok();
+}
+
+pa_forward_options default_opts(const pa_forward_options* o) {
+    pa_forward_options d{0, PA_PATH_AUTO, nullptr};
+    return o ? *o : d;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------------------
+
+extern "C" {
+
+pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, int32_t num_seqs,
+                         const int32_t* block_tables, int32_t table_width, int32_t page_size,
+                         int32_t num_pages, int device, pa_stream upload_stream, pa_plan** out_plan) {
+    if (!out_plan) return fail(PA_ERR_INVALID_ARGUMENT, "out_plan is NULL");
+    *out_plan = nullptr;
+    if (num_seqs < 0) return fail(PA_ERR_INVALID_ARGUMENT, "num_seqs must be >= 0");
+    if (page_size <= 0) return fail(PA_ERR_INVALID_ARGUMENT, "page_size must be > 0");
+    if (num_pages < 0 || table_width < 0)
+        return fail(PA_ERR_INVALID_ARGUMENT, "num_pages and table_width must be >= 0");
+    if (device < -1) return fail(PA_ERR_INVALID_ARGUMENT, "device must be >= -1");
+    if (!query_offsets) return fail(PA_ERR_INVALID_ARGUMENT, "query_offsets is NULL");
+    if (num_seqs > 0 && !seq_lens) return fail(PA_ERR_INVALID_ARGUMENT, "seq_lens is NULL");
+    if (query_offsets[0] != 0) return fail(PA_ERR_INVALID_ARGUMENT, "query_offsets[0] must be 0");
+    int64_t bt_elems = 0;
+    if (!product({num_seqs, table_width}, &bt_elems) || bt_elems > INT32_MAX)
+        return fail(PA_ERR_BOUNDS, "block table too large");
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        const int64_t L = seq_lens[s];
+        const int64_t n = (int64_t)query_offsets[s + 1] - query_offsets[s];
+        if (L < 0) return fail(PA_ERR_INVALID_ARGUMENT, "seq_lens[%d] = %lld < 0", s, (long long)L);
+        if (n < 0) return fail(PA_ERR_INVALID_ARGUMENT, "query_offsets decrease at sequence %d", s);
+        if (n > L) return fail(PA_ERR_INVALID_ARGUMENT, "sequence %d has %lld queries but only %lld keys", s, (long long)n, (long long)L);
+        const int64_t used = (L + page_size - 1) / page_size;
+        if (used > table_width)
+            return fail(PA_ERR_BOUNDS, "sequence %d needs %lld pages but table_width is %d", s, (long long)used, table_width);
+        if (used > 0 && !block_tables) return fail(PA_ERR_INVALID_ARGUMENT, "block_tables is NULL");
+        for (int64_t b = 0; b < used; ++b) {
+            const int32_t pg = block_tables[(int64_t)s * table_width + b];
+            if (pg < 0 || pg >= num_pages)
+                return fail(PA_ERR_BOUNDS, "block_tables[%d][%lld] = %d is outside the pool [0, %d)", s, (long long)b, pg, num_pages);
+        }
+    }
+    const int64_t nq = query_offsets[num_seqs];
+    if (nq > INT32_MAX) return fail(PA_ERR_BOUNDS, "too many queries");
+
+    auto P = std::make_unique<pa_plan>();
+    P->device = device;
+    P->S = num_seqs;
+    P->Nq = (int32_t)nq;
+    P->table_width = table_width;
+    P->page_size = page_size;
+    P->num_pages = num_pages;
+    P->seqs.resize(num_seqs);
+    for (int32_t s = 0; s < num_seqs; ++s)
+        P->seqs[s] = {seq_lens[s], query_offsets[s], query_offsets[s + 1] - query_offsets[s], 0};
+    if (bt_elems > 0) {
+        if (!block_tables) return fail(PA_ERR_INVALID_ARGUMENT, "block_tables is NULL");
+        P->bt.assign(block_tables, block_tables + bt_elems);
+    }
+
+    if (device >= 0) {
+        int cur = -1;
+        PA_CUDA_TRY(cudaGetDevice(&cur));
+        if (cur != device) return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not %d", cur, device);
+        PA_CUDA_TRY(cudaDeviceGetAttribute(&P->num_sms, cudaDevAttrMultiProcessorCount, device));
+        const size_t seq_bytes = ((sizeof(pa::SeqInfo) * num_seqs + 255) / 256) * 256;
+        const size_t bt_bytes = sizeof(int32_t) * (size_t)bt_elems;
+        const size_t total = std::max<size_t>(seq_bytes + bt_bytes, 256);
+        std::vector<char>& blob = P->meta_host;  // kept alive for the asynchronous copy
+        blob.assign(total, 0);
+        if (num_seqs) std::memcpy(blob.data(), P->seqs.data(), sizeof(pa::SeqInfo) * num_seqs);
+        if (bt_elems) std::memcpy(blob.data() + seq_bytes, P->bt.data(), bt_bytes);
+        PA_CUDA_TRY(cudaMallocAsync(&P->d_meta, total, (cudaStream_t)upload_stream));
+        cudaError_t e = cudaMemcpyAsync(P->d_meta, blob.data(), total, cudaMemcpyHostToDevice,
+                                        (cudaStream_t)upload_stream);
+        P->last_stream = (cudaStream_t)upload_stream;
+        P->uploaded_bytes = (int64_t)total;
+        if (e != cudaSuccess) {
+            cudaFreeAsync(P->d_meta, (cudaStream_t)upload_stream);
+            return fail(PA_ERR_CUDA, "plan upload failed: %s", cudaGetErrorString(e));
+        }
+        P->d_seqs = (pa::SeqInfo*)P->d_meta;
+        P->d_bt = (int32_t*)((char*)P->d_meta + seq_bytes);
+    }
+    *out_plan = P.release();
+    return ok();
+}
+
+pa_status pa_plan_destroy(pa_plan* plan) {
+    if (!plan) return ok();
+    if (plan->device >= 0) {
+        // Stream-ordered frees after the plan's last queued use. The host blobs of pending
+        // uploads must outlive those copies, so the plan object is deleted by a host callback
+        // once the stream reaches this point.
+        cudaStream_t st = plan->last_stream;
+        if (plan->ws) cudaFreeAsync(plan->ws, st);
+        for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
+        if (plan->d_meta) cudaFreeAsync(plan->d_meta, st);
+        cudaError_t e = cudaLaunchHostFunc(st, [](void* ud) { delete static_cast<pa_plan*>(ud); }, plan);
+        if (e != cudaSuccess) {
+            cudaStreamSynchronize(st);
+            delete plan;
+            return fail(PA_ERR_CUDA, "plan release failed: %s", cudaGetErrorString(e));
+        }
+        return ok();
+    }
+    delete plan;
+    return ok();
+}
+
+pa_status pa_plan_get_info(const pa_plan* plan, pa_plan_info* info) {
+    if (!plan || !info) return fail(PA_ERR_INVALID_ARGUMENT, "plan or info is NULL");
+    info->num_seqs = plan->S;
+    info->num_queries = plan->Nq;
+    info->table_width = plan->table_width;
+    info->page_size = plan->page_size;
+    info->num_pages = plan->num_pages;
+    info->device = plan->device;
+    info->last_launches = plan->last_launches;
+    info->workspace_bytes = (int64_t)plan->ws_bytes;
+    info->uploaded_bytes = plan->uploaded_bytes;
+    return ok();
+}
+
+pa_status pa_forward_ex(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                        pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t v_head_dim, float scale, int causal, int32_t window, void* out,
+                        float* lse, pa_stream stream, const pa_forward_options* opts) {
+    Call c{};
+    c.mla = false;
+    c.q = q; c.k = k_cache; c.v = v_cache;
+    c.dtype = dtype;
+    c.hq = num_q_heads; c.hkv = num_kv_heads; c.d = head_dim; c.dv = v_head_dim;
+    c.scale = scale; c.causal = causal; c.window = window;
+    c.out = out; c.lse = lse;
+    c.opts = default_opts(opts);
+    return run_forward(plan, c, (cudaStream_t)stream);
+}
+
+pa_status pa_forward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                     pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t v_head_dim, float scale, int causal, int32_t window, void* out,
+                     float* lse, pa_stream stream) {
+    return pa_forward_ex(plan, q, k_cache, v_cache, dtype, num_q_heads, num_kv_heads, head_dim,
+                         v_head_dim, scale, causal, window, out, lse, stream, nullptr);
+}
+
+pa_status pa_mla_forward_ex(pa_plan* plan, const void* q_latent, const void* q_rope,
+                            const void* latent_cache, const void* rope_cache, pa_dtype dtype,
+                            int32_t num_heads, int32_t latent_dim, int32_t rope_dim, float scale,
+                            int causal, int32_t window, void* out, float* lse, pa_stream stream,
+                            const pa_forward_options* opts) {
+    Call c{};
+    c.mla = true;
+    c.q = q_latent; c.k = latent_cache; c.v = latent_cache; c.qr = q_rope; c.kr = rope_cache;
+    c.dtype = dtype;
+    c.hq = num_heads; c.hkv = 1; c.d = latent_dim; c.dv = latent_dim; c.pr = rope_dim;
+    c.scale = scale; c.causal = causal; c.window = window;
+    c.out = out; c.lse = lse;
+    c.opts = default_opts(opts);
+    return run_forward(plan, c, (cudaStream_t)stream);
+}
+
+pa_status pa_mla_forward(pa_plan* plan, const void* q_latent, const void* q_rope,
+                         const void* latent_cache, const void* rope_cache, pa_dtype dtype,
+                         int32_t num_heads, int32_t latent_dim, int32_t rope_dim, float scale,
+                         int causal, int32_t window, void* out, float* lse, pa_stream stream) {
+    return pa_mla_forward_ex(plan, q_latent, q_rope, latent_cache, rope_cache, dtype, num_heads,
+                             latent_dim, rope_dim, scale, causal, window, out, lse, stream, nullptr);
+}
+
+pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_heads,
+                          int32_t num_kv_heads, int32_t head_dim, int32_t v_head_dim, int causal,
+                          int32_t window, pa_stream stream, const pa_forward_options* opts) {
+    if (!plan) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    if (plan->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to prepare");
+    pa_forward_options o = default_opts(opts);
+    SchedKey key{};
+    key.mla = mla ? 1 : 0;
+    key.dtype = dtype;
+    key.hq = num_q_heads;
+    key.hkv = mla ? 1 : num_kv_heads;
+    key.d = head_dim;
+    key.dv = mla ? head_dim : v_head_dim;
+    key.causal = causal;
+    key.window = window;
+    key.path = o.path;
+    key.kv_chunk = o.kv_chunk;
+    if (key.hq <= 0 || key.hkv <= 0 || key.hq % key.hkv || key.d <= 0 || key.dv <= 0)
+        return fail(PA_ERR_SHAPE, "inconsistent head configuration");
+    std::lock_guard<std::mutex> lock(plan->mu);
+    Schedule* S = nullptr;
+    pa_status st = build_schedule(plan, key, (cudaStream_t)stream, &S);
+    if (st != PA_OK) return st;
+    if (S->slots > 0) {
+        st = ensure_workspace(plan, (size_t)S->slots * key.hq * (key.dv + 1) * sizeof(float), (cudaStream_t)stream);
+        if (st != PA_OK) return st;
+    }
+    return ok();
+}
+
+const char* pa_status_string(pa_status s) {
+    switch (s) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARGUMENT: return "PA_ERR_INVALID_ARGUMENT";
+        case PA_ERR_SHAPE: return "PA_ERR_SHAPE";
+        case PA_ERR_DTYPE: return "PA_ERR_DTYPE";
+        case PA_ERR_BOUNDS: return "PA_ERR_BOUNDS";
+        case PA_ERR_ALIAS: return "PA_ERR_ALIAS";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+    }
+    return "PA_ERR_UNKNOWN";
+}
+
+const char* pa_last_error_message(void) { return g_msg; }
+
+const char* pa_version(void) { return "0.1.0"; }
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// Internal types shared by the host plan code and the kernels of libpa.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+// Per-sequence facts on the device (16 bytes).
+struct SeqInfo {
+    int32_t L;        // keys in the cache, including the sequence's own new keys
+    int32_t q_start;  // first packed query row
+    int32_t n;        // number of queries
+    int32_t pad;
+};
+
+// One unit of key-split work on the decode-style kernels: queries j0 .. j1-1 of sequence
+// `seq` against keys [t0, t1) (the union of what those queries can see, cut into parts), for
+// the KV head given by blockIdx.y. nsplit == 1 means the unit writes final results;
+// otherwise query j's part `split` goes to workspace slot
+// part_base + (j - j0) * nsplit + split.
+struct KvUnit {
+    int32_t seq, t0, t1, split;
+    int32_t nsplit, part_base, j0, j1;
+};
+
+// One query row set to merge: query `query`, parts part_base .. part_base + nsplit - 1.
+struct CombineUnit {
+    int32_t query, part_base, nsplit, pad;
+};
+
+// One prefill tile: queries [j0, j0 + qpt) of sequence `seq` (qpt = 128 / G rows), keys
+// [t0, t1), KV head kvh.
+struct PrefillUnit {
+    int32_t seq, j0, t0, t1;
+    int32_t kvh, pad0, pad1, pad2;
+};
+
+// Everything a kernel needs; passed by value.
+struct AttnParams {
+    const void* q;    // [Nq, Hq, D]   (MLA: absorbed q [Nq, H, R])
+    const void* k;    // [P, ps, Hkv, D] (MLA: latent [P, ps, 1, R])
+    const void* v;    // [P, ps, Hkv, Dv] (MLA: same as k)
+    const void* qr;   // MLA only: position q [Nq, H, Pr]
+    const void* kr;   // MLA only: rope cache [P, ps, 1, Pr]
+    void* out;        // [Nq, Hq, Dv]
+    float* lse;       // [Nq, Hq]
+    float* ws_o;      // [slots, Hq, Dv] float32 split partials (normalised)
+    float* ws_lse;    // [slots, Hq] float32 (natural log)
+    const SeqInfo* seqs;
+    const int32_t* block_tables;
+    const KvUnit* units;
+    const CombineUnit* cunits;
+    const PrefillUnit* punits;
+    int32_t num_units, num_cunits, num_punits;
+    int32_t table_width, page_size;
+    int32_t hq, hkv, group, d, dv, pr;
+    float scale;       // softmax scale
+    float scale_log2;  // scale * log2(e): scores in base-2 units
+    int32_t causal, window;
+};
+
+// Kernel launchers (one per .cu file). Each returns the launch's cudaError_t.
+cudaError_t launch_simt(const AttnParams& p, pa_dtype dt, cudaStream_t st);
+cudaError_t launch_decode_mma(const AttnParams& p, pa_dtype dt, int rows_max, cudaStream_t st);
+cudaError_t launch_combine(const AttnParams& p, pa_dtype dt, cudaStream_t st);
+
+// Largest row count (queries x group heads per KV head) the tensor-core decode kernel takes.
+constexpr int kDecodeMaxRows = 16;
+
+}  // namespace pa

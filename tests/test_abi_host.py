@@ -1,0 +1,169 @@
+"""C ABI on the host (no GPU): the library loads, exports what include/pa.h declares, and
+rejects bad arguments with the documented status before touching a device.
+
+ruDNN's paged_attention/mod.rs validates every operand (`check_tensor`, `bounded`,
+`execute_attention_into`) before any allocation or launch; these tests pin the same order
+through host-only plans (device -1), which own no device memory.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import paged_kv_attention_39_b200 as pa
+from paged_kv_attention_39_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_attention_39_b200 import build
+    build.build()
+    return pa.load_library()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:pa_status|const char\s*\*)\s*(pa_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(pa.SYMBOLS) == names
+
+
+def test_status_strings(lib):
+    for i, name in enumerate(pa.STATUS):
+        assert pa.pa_status_string(i) == name
+    assert pa.pa_version().count(".") == 2
+
+
+def host_plan(**kw):
+    wl = W.make_gqa("h", 1, [37, 100], [1, 5], 4, 2, 64, 64, 16, torch.bfloat16)
+    s = wl.sched
+    args = dict(seq_lens=s.seq_lens, query_offsets=s.query_offsets, block_tables=s.block_tables,
+                page_size=s.page_size, num_pages=s.num_pages, device=-1)
+    args.update(kw)
+    return wl, pa.pa_plan_create(**args)
+
+
+def expect(status_name, fn, *a, **k):
+    with pytest.raises(pa.PaError) as ei:
+        fn(*a, **k)
+    assert ei.value.name == status_name, str(ei.value)
+
+
+def test_plan_create_validation(lib):
+    wl, plan = host_plan()
+    info = pa.pa_plan_get_info(plan)
+    assert info["num_queries"] == 6 and info["device"] == -1 and info["workspace_bytes"] == 0
+    s = wl.sched
+    bad = s.block_tables.clone(); bad[1, 3] = s.num_pages
+    expect("PA_ERR_BOUNDS", pa.pa_plan_create, s.seq_lens, s.query_offsets, bad, 16, s.num_pages, device=-1)
+    bad = s.block_tables.clone(); bad[0, 0] = -1
+    expect("PA_ERR_BOUNDS", pa.pa_plan_create, s.seq_lens, s.query_offsets, bad, 16, s.num_pages, device=-1)
+    expect("PA_ERR_BOUNDS", pa.pa_plan_create, s.seq_lens, s.query_offsets, s.block_tables[:, :2], 16,
+           s.num_pages, device=-1)  # table too narrow for 37 keys in pages of 16
+    expect("PA_ERR_INVALID_ARGUMENT", pa.pa_plan_create, [3, 100], [0, 5, 6], s.block_tables, 16,
+           s.num_pages, device=-1)  # 5 queries but only 3 keys
+    expect("PA_ERR_INVALID_ARGUMENT", pa.pa_plan_create, s.seq_lens, [1, 2, 3], s.block_tables, 16,
+           s.num_pages, device=-1)
+    expect("PA_ERR_INVALID_ARGUMENT", pa.pa_plan_create, s.seq_lens, [0, 3, 2], s.block_tables, 16,
+           s.num_pages, device=-1)
+    expect("PA_ERR_INVALID_ARGUMENT", pa.pa_plan_create, s.seq_lens, s.query_offsets, s.block_tables, 0,
+           s.num_pages, device=-1)
+    expect("PA_ERR_INVALID_ARGUMENT", pa.pa_plan_create, [-1, 100], [0, 0, 1], s.block_tables, 16,
+           s.num_pages, device=-1)
+    # entries past the used count are never read, so they may hold anything
+    odd = s.block_tables.clone(); odd[0, 3:] = 123456
+    pa.pa_plan_create(s.seq_lens, s.query_offsets, odd, 16, s.num_pages, device=-1).close()
+    # an empty batch is a valid plan
+    pa.pa_plan_create([], [0], torch.zeros(0, 0, dtype=torch.int32), 16, 0, device=-1).close()
+
+
+def fake_ptrs(wl):
+    """Disjoint, 256-byte aligned fake addresses standing in for device buffers."""
+    base = 1 << 40
+    sizes = [wl.q.numel() * 2, wl.k_cache.numel() * 2, wl.v_cache.numel() * 2,
+             wl.q.shape[0] * wl.q.shape[1] * wl.v_head_dim * 2, wl.q.shape[0] * wl.q.shape[1] * 4]
+    out = []
+    for sz in sizes:
+        out.append(base)
+        base += (sz + 4095) // 4096 * 4096 + 4096
+    return out
+
+
+def call(lib, plan, ptrs, hq=4, hkv=2, d=64, dv=64, scale=0.125, causal=1, window=0, dtype=1, opts=None):
+    q, k, v, o, l = ptrs
+    st = lib.pa_forward_ex(plan.handle, q, k, v, dtype, hq, hkv, d, dv, ctypes.c_float(scale), causal,
+                           window, o, l, None, opts)
+    return pa.STATUS[st], pa.pa_last_error_message()
+
+
+def test_forward_validation_order(lib):
+    wl, plan = host_plan()
+    p = fake_ptrs(wl)
+    assert call(lib, plan, p)[0] == "PA_ERR_INVALID_ARGUMENT"  # all valid -> host-only plan refusal
+    assert "host-only" in call(lib, plan, p)[1]
+    assert call(lib, plan, p, hq=6, hkv=4)[0] == "PA_ERR_SHAPE"
+    assert call(lib, plan, p, hq=0)[0] == "PA_ERR_SHAPE"
+    assert call(lib, plan, p, d=0)[0] == "PA_ERR_SHAPE"
+    assert call(lib, plan, p, d=2048)[0] == "PA_ERR_UNSUPPORTED"
+    assert call(lib, plan, p, scale=0.0)[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, scale=float("nan"))[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, scale=-1.0)[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, window=-3)[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, causal=2)[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, dtype=7)[0] == "PA_ERR_DTYPE"
+    q, k, v, o, l = p
+    assert call(lib, plan, [q, k, v, q, l])[0] == "PA_ERR_ALIAS"          # out over q
+    assert call(lib, plan, [q, k, v, o, k + 64])[0] == "PA_ERR_ALIAS"     # lse inside K
+    assert call(lib, plan, [q, k, v, o, o + 32])[0] == "PA_ERR_ALIAS"     # lse inside out
+    assert call(lib, plan, [q, k, v, o + 8, l])[0] == "PA_ERR_INVALID_ARGUMENT"  # misaligned
+    assert call(lib, plan, [q, k, None, o, l])[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, opts=ctypes.byref(pa._Options(-5, 0, None)))[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert call(lib, plan, p, opts=ctypes.byref(pa._Options(0, 9, None)))[0] == "PA_ERR_INVALID_ARGUMENT"
+    assert lib.pa_forward_ex(None, q, k, v, 1, 4, 2, 64, 64, ctypes.c_float(1.0), 1, 0, o, l, None, None) == 1
+
+
+def test_mla_validation(lib):
+    wl, plan = host_plan()
+    q, k, v, o, l = fake_ptrs(wl)
+    def mla(pr=64, r=512, h=4, scale=0.1):
+        st = lib.pa_mla_forward_ex(plan.handle, q, k + (1 << 30), k, v, 1, h, r, pr, ctypes.c_float(scale), 1, 0,
+                                   o + (1 << 31), l + (1 << 32), None, None)
+        return pa.STATUS[st]
+    assert mla() == "PA_ERR_INVALID_ARGUMENT"  # host-only plan
+    assert mla(pr=0) == "PA_ERR_SHAPE"
+    assert mla(pr=300) == "PA_ERR_SHAPE"
+    assert mla(r=1500) == "PA_ERR_UNSUPPORTED"
+
+
+def test_empty_batch_is_ok_without_launch(lib):
+    plan = pa.pa_plan_create([5], [0, 0], torch.zeros(1, 1, dtype=torch.int32), 16, 1, device=-1)
+    st = lib.pa_forward_ex(plan.handle, None, None, None, 1, 4, 2, 64, 64, ctypes.c_float(1.0), 1, 0,
+                           None, None, None, None)
+    assert pa.STATUS[st] == "PA_OK"
+
+
+def test_binding_functions_compile_their_calls():
+    """Every binding wrapper resolves the globals it loads (a typo would only show on a GPU)."""
+    import builtins
+    import dis
+    for name in ("pa_plan_prepare", "pa_forward", "pa_mla_forward", "pa_plan_create", "pa_plan_get_info",
+                 "plan_for", "trace_events"):
+        fn = getattr(pa, name)
+        for ins in dis.get_instructions(fn):
+            if ins.opname == "LOAD_GLOBAL":
+                g = ins.argval
+                assert hasattr(pa, g) or hasattr(builtins, g), (name, g)
+    # host-only plan: pa_plan_prepare reaches the library and is refused there
+    plan = pa.pa_plan_create([5], [0, 1], torch.zeros(1, 1, dtype=torch.int32), 16, 1, device=-1)
+    with pytest.raises(pa.PaError):
+        pa.pa_plan_prepare(plan, torch.bfloat16, 4, 2, 64, 64)

@@ -1,0 +1,174 @@
+"""GPU parity of the decode paths (CUDA-core kernel, tensor-core split-KV kernel, combine)
+against the fp64 oracle, element by element on seeded inputs, through the C ABI."""
+import math
+
+import pytest
+import torch
+
+import oracle_pins
+import paged_kv_attention_39_b200 as pa
+from gpu_helpers import check, run, run_gqa, sample_rows, visible_count
+from paged_kv_attention_39_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+SIMT = pa.PA_PATH_SIMT
+
+
+@pytest.mark.parametrize("seed", range(10))
+@pytest.mark.parametrize("kv_chunk", [0, -1, 16, 23, 64])
+def test_tiny_fp32_decode(orc, seed, kv_chunk):
+    """2 sequences (37 and 100 keys), Hq 4, Hkv 2, D 64, pages of 16 shuffled in a 16-page pool
+    with 6 NaN pages; forced splits cut 100 keys into 1..7 parts."""
+    wl = W.c1_tiny_fp32_decode(seed)
+    ref = orc.run(wl)
+    out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+    check(wl, out, lse, *ref, tag=f"seed {seed} chunk {kv_chunk}")
+
+
+def small_decode(seed, dtype=torch.bfloat16, hq=32, hkv=8, d=128, batch=8, lmin=17, lmax=600, ps=16,
+                 window=0, qn=1):
+    lens = W._uniform_ints(seed, 99, batch, lmin, lmax)
+    return W.make_gqa("small_decode", seed, lens, [qn] * batch, hq, hkv, d, d, ps, dtype, window=window)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("kv_chunk", [0, -1, 48, 100])
+def test_small_decode_tensor_core(orc, dtype, d, kv_chunk):
+    wl = small_decode(1, dtype=dtype, d=d)
+    ref = orc.run(wl)
+    out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+    check(wl, out, lse, *ref, tag=f"{dtype} d{d} chunk {kv_chunk}")
+
+
+@pytest.mark.parametrize("hq,hkv,qn", [(8, 8, 1), (16, 2, 1), (16, 1, 1), (8, 2, 3), (4, 2, 8), (6, 2, 5)])
+def test_decode_groups_and_multi_query(orc, hq, hkv, qn):
+    """G from 1 to 16 and several queries per sequence (speculative-decode shapes): up to 16
+    rows share one KV head; per-element causal masks at right-aligned positions."""
+    wl = small_decode(2, hq=hq, hkv=hkv, qn=qn, window=0, lmin=qn, lmax=300)
+    ref = orc.run(wl)
+    for kv_chunk in (0, 32):
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+        check(wl, out, lse, *ref, tag=f"G{hq // hkv} n{qn} chunk {kv_chunk}")
+
+
+@pytest.mark.parametrize("window", [1, 7, 100, 5000])
+def test_decode_window(orc, window):
+    wl = small_decode(3, window=window, qn=2, hq=16, hkv=4, lmin=2, lmax=900)
+    ref = orc.run(wl)
+    for path in (pa.PA_PATH_AUTO, SIMT):
+        out, lse = run_gqa(wl, kv_chunk=64, path=path)
+        check(wl, out, lse, *ref, tag=f"window {window} path {path}")
+
+
+def test_simt_path_matches_oracle_bf16(orc):
+    wl = small_decode(4, d=128)
+    ref = orc.run(wl)
+    out, lse = run_gqa(wl, path=SIMT)
+    check(wl, out, lse, *ref, tag="simt bf16")
+
+
+def test_non_causal_and_edges(orc):
+    """L = 1, a sequence with no queries between two others, non-causal scores."""
+    wl = W.make_gqa("edges", 5, [1, 40, 300, 2], [1, 0, 1, 2], 8, 2, 128, 128, 16, torch.bfloat16,
+                    causal=False, window=0)
+    ref = orc.run(wl)
+    for kv_chunk in (0, 16):
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+        check(wl, out, lse, *ref, tag=f"edges {kv_chunk}")
+
+
+def test_empty_batch():
+    wl = W.make_gqa("empty", 6, [10, 20], [0, 0], 8, 2, 128, 128, 16, torch.bfloat16)
+    plan = pa.plan_for(wl)
+    q = torch.empty(0, 8, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(0, 8, 128, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(0, 8, dtype=torch.float32, device="cuda")
+    pa.pa_forward(plan, q, wl.k_cache.cuda(), wl.v_cache.cuda(), out, lse, wl.scale)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("path", [pa.PA_PATH_AUTO, SIMT])
+@pytest.mark.parametrize("kv_chunk", [0, 32])
+def test_mask_bit_exact_by_counts(path, kv_chunk):
+    """Q = 0 gives every visible key weight 1, so exp(lse) counts the visible keys exactly:
+    the closed-form count for each row's absolute position, causal flag and window."""
+    for window, causal in ((0, True), (37, True), (5, False)):
+        wl = W.make_gqa("mask", 7, [1, 57, 130, 333], [1, 3, 1, 4], 8, 2, 128, 128, 16, torch.bfloat16,
+                        causal=causal, window=window)
+        wl.q.zero_()
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk, path=path)
+        s = wl.sched
+        for si in range(s.num_seqs):
+            L = int(s.seq_lens[si]); q0 = int(s.query_offsets[si]); n = int(s.query_offsets[si + 1]) - q0
+            for j in range(n):
+                cnt, _, _ = visible_count(L, n, j, causal, window)
+                got = torch.exp(lse[q0 + j].double()).round().long()
+                assert bool((got == cnt).all()), (window, causal, si, j, got.tolist(), cnt)
+
+
+@pytest.mark.parametrize("dtype,path", [(torch.float32, pa.PA_PATH_AUTO), (torch.bfloat16, pa.PA_PATH_AUTO),
+                                        (torch.bfloat16, SIMT), (torch.float16, pa.PA_PATH_AUTO)])
+def test_block_table_indexing_bit_exact(dtype, path):
+    """Each row's query is a large multiple of one visible key: its output must be exactly that
+    key's value row, read through the shuffled block table (NaN pages all around)."""
+    wl = W.make_gqa("idx", 8, [70, 33, 129, 500], [1, 2, 1, 1], 8, 2, 128, 128, 16, torch.float32,
+                    causal=True, window=300)
+    target = oracle_pins.select_target_queries(wl, 5, margin=120.0)
+    wl.q = wl.q.to(dtype); wl.k_cache = wl.k_cache.to(dtype); wl.v_cache = wl.v_cache.to(dtype)
+    # recheck after rounding to dtype that the target still dominates by a wide margin
+    out, lse = run_gqa(wl, kv_chunk=48, path=path)
+    s = wl.sched
+    for (qi, h), (si, ts) in target.items():
+        page = int(s.block_tables[si, ts // s.page_size])
+        want = wl.v_cache[page, ts % s.page_size, h // 4]
+        assert torch.equal(out[qi, h], want), (qi, h, si, ts)
+
+
+def test_page_permutation_invariance():
+    wl = small_decode(9, lmin=100, lmax=700)
+    out, lse = run_gqa(wl, kv_chunk=64)
+    P = wl.sched.num_pages
+    pi = torch.randperm(P, generator=torch.Generator().manual_seed(2))
+    k2 = torch.empty_like(wl.k_cache); k2[pi] = wl.k_cache
+    v2 = torch.empty_like(wl.v_cache); v2[pi] = wl.v_cache
+    bt = wl.sched.block_tables.clone(); m = bt >= 0
+    bt[m] = pi[bt[m].long()].to(torch.int32)
+    wl.k_cache, wl.v_cache = k2, v2
+    wl.sched.block_tables = bt
+    out2, lse2 = run_gqa(wl, kv_chunk=64)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_split_equals_unsplit_within_tolerance(orc):
+    wl = small_decode(10, lmin=500, lmax=3000)
+    ref = orc.run(wl)
+    base, lbase = run_gqa(wl, kv_chunk=-1)
+    for kv_chunk in (16, 112, 1000):
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+        check(wl, out, lse, *ref, tag=f"chunk {kv_chunk}")
+        assert float((out.float() - base.float()).abs().max()) < 1e-2
+        assert float((lse - lbase).abs().max()) < 1e-3
+
+
+def test_plan_reuse_and_workspace_growth(orc):
+    wl = small_decode(11, lmin=400, lmax=2000)
+    ref = orc.run(wl)
+    plan = pa.plan_for(wl)
+    for kv_chunk in (256, 64, 16, 64):
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk, plan=plan)
+        check(wl, out, lse, *ref, tag=f"reuse {kv_chunk}")
+    assert pa.pa_plan_get_info(plan)["workspace_bytes"] > 0
+    plan.close()
+
+
+@pytest.mark.slow
+def test_full_size_bf16_decode_sampled(orc):
+    """The full decode workload (batch 64, context U[512, 8192], Hq 32, Hkv 8, D 128, pages of
+    16) in the benchmark's launch configuration, checked on sampled rows."""
+    wl = W.c2_bf16_decode(0)
+    rows = sample_rows(wl, 192, seed=1)
+    ref = orc.run(wl, rows=rows)
+    out, lse = run_gqa(wl)
+    check(wl, out, lse, *ref, rows=rows, tag="full decode")
