@@ -199,6 +199,13 @@ pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_
                           int causal, int32_t window, pa_stream stream,
                           const pa_forward_options* opts);
 
+/*
+ * pa_plan_device_status -- diagnostic read of the plan's device error word (synchronous copy:
+ * not for the hot path). 0 means no kernel reported a failure; a non-zero code means a kernel
+ * gave up a bounded wait in its pipeline (the results of that call are undefined).
+ */
+pa_status pa_plan_device_status(const pa_plan* plan, int32_t* code);
+
 /* Human-readable name of a status code (static string). */
 const char* pa_status_string(pa_status status);
 

@@ -29,8 +29,8 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
           "PA_ERR_ALIAS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA"]
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
-           "pa_forward_ex", "pa_mla_forward", "pa_mla_forward_ex", "pa_status_string",
-           "pa_last_error_message", "pa_version"]
+           "pa_forward_ex", "pa_mla_forward", "pa_mla_forward_ex", "pa_plan_device_status",
+           "pa_status_string", "pa_last_error_message", "pa_version"]
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -87,6 +87,8 @@ def load_library(path: Optional[str] = None):
     lib.pa_mla_forward.argtypes = mla
     lib.pa_mla_forward_ex.restype = ctypes.c_int
     lib.pa_mla_forward_ex.argtypes = mla + [ctypes.POINTER(_Options)]
+    lib.pa_plan_device_status.restype = ctypes.c_int
+    lib.pa_plan_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_status_string.argtypes = [ctypes.c_int]
     lib.pa_last_error_message.restype = ctypes.c_char_p
@@ -182,6 +184,13 @@ def pa_plan_get_info(plan: Plan) -> dict:
     return {k: getattr(info, k) for k, _ in _Info._fields_}
 
 
+def pa_plan_device_status(plan: Plan) -> int:
+    """Diagnostic: the plan's device error word (0 = no kernel reported a failure)."""
+    code = ctypes.c_int32(0)
+    _check(load_library().pa_plan_device_status(plan.handle, ctypes.byref(code)))
+    return int(code.value)
+
+
 def _opts(kv_chunk: int, path: int, trace=None):
     """Options struct; `trace` is a ctypes array of three cudaEvent_t handles, or None."""
     ev = ctypes.cast(trace, ctypes.c_void_p) if trace is not None else None
@@ -189,7 +198,14 @@ def _opts(kv_chunk: int, path: int, trace=None):
 
 
 def trace_events(events):
-    """Three torch.cuda.Event objects -> the array pa_forward_options.trace_events takes."""
+    """Three torch.cuda.Event objects -> the array pa_forward_options.trace_events takes.
+
+    torch creates the CUDA event behind an Event lazily, on its first record: record each one
+    once here so that the handles exist.
+    """
+    for e in events:
+        if not e.cuda_event:
+            e.record()
     return (ctypes.c_void_p * 3)(*[int(e.cuda_event) for e in events])
 
 

@@ -73,7 +73,8 @@ struct Schedule {
     const pa::KvUnit* tc_units = nullptr;     // tensor-core decode kernel
     const pa::KvUnit* simt_units = nullptr;   // CUDA-core kernel
     const pa::CombineUnit* cunits = nullptr;
-    int32_t n_tc = 0, n_simt = 0, n_comb = 0;
+    const pa::PrefillUnit* punits = nullptr;  // tensor-core prefill kernel
+    int32_t n_tc = 0, n_simt = 0, n_comb = 0, n_pre = 0;
     int32_t tc_rows_max = 0;
     int64_t slots = 0;  // workspace parts
     int32_t kv_chunk = 0;
@@ -91,6 +92,7 @@ struct pa_plan {
     std::vector<char> meta_host;
     pa::SeqInfo* d_seqs = nullptr;
     int32_t* d_bt = nullptr;
+    int* d_err = nullptr;  // kernels' error word (bounded waits that ran out)
     std::vector<std::unique_ptr<Schedule>> scheds;  // most recent last
     float* ws = nullptr;
     size_t ws_bytes = 0;
@@ -129,6 +131,10 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     const int32_t G = k.hq / k.hkv;
     const bool tc_decode = !k.mla && k.path == PA_PATH_AUTO && k.dtype != PA_F32 &&
                            k.d == k.dv && (k.d == 64 || k.d == 128);
+    const bool tc_prefill = !k.mla && k.path == PA_PATH_AUTO &&
+                            pa::prefill_tc_supported((pa_dtype)k.dtype, k.d, k.dv, G, P->page_size);
+    std::vector<pa::PrefillUnit> pu;
+    std::vector<int64_t> pu_cost;
 
     struct Block { int32_t seq, j0, j1, lo, hi; bool tc; };
     std::vector<Block> blocks;
@@ -137,6 +143,25 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
         const pa::SeqInfo& si = P->seqs[s];
         if (si.n == 0) continue;
         const bool tc = tc_decode && (int64_t)si.n * G <= pa::kDecodeMaxRows;
+        if (!tc && tc_prefill) {
+            // 128-row tiles: 128 / G queries times the G heads of one KV head
+            const int32_t qpt = 128 / G;
+            for (int32_t j0 = 0; j0 < si.n; j0 += qpt) {
+                int32_t lo, hi;
+                visible_union(si.L, si.n, j0, std::min(si.n, j0 + qpt), k.causal, k.window, &lo, &hi);
+                for (int32_t h = 0; h < k.hkv; ++h) {
+                    pa::PrefillUnit u{};
+                    u.seq = s;
+                    u.j0 = j0;
+                    u.t0 = lo;
+                    u.t1 = hi;
+                    u.kvh = h;
+                    pu.push_back(u);
+                    pu_cost.push_back((int64_t)(hi - lo) + 128);
+                }
+            }
+            continue;
+        }
         // CUDA-core blocks take few queries so that long prefill chunks spread over CTAs.
         const int32_t qb = tc ? si.n : std::max<int32_t>(1, 16 / std::min<int32_t>(G, 16));
         for (int32_t j0 = 0; j0 < si.n; j0 += qb) {
@@ -190,6 +215,15 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     };
     std::stable_sort(tcu.begin(), tcu.end(), longer);
     std::stable_sort(simtu.begin(), simtu.end(), longer);
+    {
+        std::vector<size_t> order(pu.size());
+        for (size_t i = 0; i < order.size(); ++i) order[i] = i;
+        std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return pu_cost[a] > pu_cost[b]; });
+        std::vector<pa::PrefillUnit> sorted;
+        sorted.reserve(pu.size());
+        for (size_t i : order) sorted.push_back(pu[i]);
+        pu.swap(sorted);
+    }
     if (slots > INT32_MAX) return fail(PA_ERR_BOUNDS, "split workspace needs too many parts");
 
     // One blob: [tc units][simt units][combine units], 256-byte aligned sections.
@@ -197,11 +231,13 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     const size_t o_tc = 0;
     const size_t o_simt = align(o_tc + tcu.size() * sizeof(pa::KvUnit));
     const size_t o_c = align(o_simt + simtu.size() * sizeof(pa::KvUnit));
-    const size_t bytes = align(o_c + cu.size() * sizeof(pa::CombineUnit));
+    const size_t o_p = align(o_c + cu.size() * sizeof(pa::CombineUnit));
+    const size_t bytes = align(o_p + pu.size() * sizeof(pa::PrefillUnit));
     S->host.assign(std::max<size_t>(bytes, 256), 0);
     if (!tcu.empty()) std::memcpy(S->host.data() + o_tc, tcu.data(), tcu.size() * sizeof(pa::KvUnit));
     if (!simtu.empty()) std::memcpy(S->host.data() + o_simt, simtu.data(), simtu.size() * sizeof(pa::KvUnit));
     if (!cu.empty()) std::memcpy(S->host.data() + o_c, cu.data(), cu.size() * sizeof(pa::CombineUnit));
+    if (!pu.empty()) std::memcpy(S->host.data() + o_p, pu.data(), pu.size() * sizeof(pa::PrefillUnit));
     PA_CUDA_TRY(cudaMallocAsync(&S->dev, S->host.size(), st));
     cudaError_t e = cudaMemcpyAsync(S->dev, S->host.data(), S->host.size(), cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) {
@@ -213,6 +249,8 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     S->tc_units = (const pa::KvUnit*)(base + o_tc);
     S->simt_units = (const pa::KvUnit*)(base + o_simt);
     S->cunits = (const pa::CombineUnit*)(base + o_c);
+    S->punits = (const pa::PrefillUnit*)(base + o_p);
+    S->n_pre = (int32_t)pu.size();
     S->n_tc = (int32_t)tcu.size();
     S->n_simt = (int32_t)simtu.size();
     S->n_comb = (int32_t)cu.size();
@@ -352,6 +390,11 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     p.scale = c.scale;
     p.scale_log2 = (float)((double)c.scale * 1.4426950408889634);
     p.causal = c.causal; p.window = c.window;
+    p.num_queries = P->Nq;
+    p.num_pages = P->num_pages;
+    p.err = P->d_err;
+    p.punits = S->punits;
+    p.num_punits = S->n_pre;
 
     cudaEvent_t* ev = (cudaEvent_t*)c.opts.trace_events;
     cudaError_t e;
@@ -363,6 +406,11 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
         p.num_units = S->n_tc;
         e = pa::launch_decode_mma(p, c.dtype, S->tc_rows_max, st);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode kernel launch failed: %s", cudaGetErrorString(e));
+    }
+    if (S->n_pre > 0) {
+        ++launches;
+        e = pa::launch_prefill_tc(p, c.dtype, P->num_pages, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill kernel launch failed: %s", cudaGetErrorString(e));
     }
     if (S->n_simt > 0) {
         ++launches;
@@ -451,8 +499,8 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
         if (cur != device) return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not %d", cur, device);
         PA_CUDA_TRY(cudaDeviceGetAttribute(&P->num_sms, cudaDevAttrMultiProcessorCount, device));
         const size_t seq_bytes = ((sizeof(pa::SeqInfo) * num_seqs + 255) / 256) * 256;
-        const size_t bt_bytes = sizeof(int32_t) * (size_t)bt_elems;
-        const size_t total = std::max<size_t>(seq_bytes + bt_bytes, 256);
+        const size_t bt_bytes = ((sizeof(int32_t) * (size_t)bt_elems + 255) / 256) * 256;
+        const size_t total = seq_bytes + bt_bytes + 256;  // + the error word
         std::vector<char>& blob = P->meta_host;  // kept alive for the asynchronous copy
         blob.assign(total, 0);
         if (num_seqs) std::memcpy(blob.data(), P->seqs.data(), sizeof(pa::SeqInfo) * num_seqs);
@@ -468,6 +516,7 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
         }
         P->d_seqs = (pa::SeqInfo*)P->d_meta;
         P->d_bt = (int32_t*)((char*)P->d_meta + seq_bytes);
+        P->d_err = (int*)((char*)P->d_meta + seq_bytes + bt_bytes);
     }
     *out_plan = P.release();
     return ok();
@@ -583,6 +632,16 @@ pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_
         st = ensure_workspace(plan, (size_t)S->slots * key.hq * (key.dv + 1) * sizeof(float), (cudaStream_t)stream);
         if (st != PA_OK) return st;
     }
+    return ok();
+}
+
+pa_status pa_plan_device_status(const pa_plan* plan, int32_t* code) {
+    if (!plan || !code) return fail(PA_ERR_INVALID_ARGUMENT, "plan or code is NULL");
+    *code = 0;
+    if (plan->device < 0) return ok();
+    int v = 0;
+    PA_CUDA_TRY(cudaMemcpy(&v, plan->d_err, sizeof v, cudaMemcpyDeviceToHost));
+    *code = v;
     return ok();
 }
 

@@ -100,6 +100,9 @@ template <> __device__ __forceinline__ void mma16816<__half>(float (&d)[4], cons
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
 // Is key t visible to a query at absolute position pos?
 __device__ __forceinline__ bool key_visible(int64_t t, int64_t pos, int causal, int window) {
     return (!causal || t <= pos) && (window == 0 || t + window > pos);

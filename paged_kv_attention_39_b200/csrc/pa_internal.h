@@ -60,12 +60,17 @@ struct AttnParams {
     float scale;       // softmax scale
     float scale_log2;  // scale * log2(e): scores in base-2 units
     int32_t causal, window;
+    int32_t num_queries, num_pages;
+    int* err;          // device error word of the plan (0 = no failure)
 };
 
 // Kernel launchers (one per .cu file). Each returns the launch's cudaError_t.
 cudaError_t launch_simt(const AttnParams& p, pa_dtype dt, cudaStream_t st);
 cudaError_t launch_decode_mma(const AttnParams& p, pa_dtype dt, int rows_max, cudaStream_t st);
 cudaError_t launch_combine(const AttnParams& p, pa_dtype dt, cudaStream_t st);
+cudaError_t launch_prefill_tc(const AttnParams& p, pa_dtype dt, int num_pages, cudaStream_t st);
+// Shapes the tensor-core prefill kernel takes.
+bool prefill_tc_supported(pa_dtype dt, int d, int dv, int group, int page_size);
 
 // Largest row count (queries x group heads per KV head) the tensor-core decode kernel takes.
 constexpr int kDecodeMaxRows = 16;

@@ -1,0 +1,425 @@
+// Chunked-prefill paged attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
+// bf16 / fp16, head_dim 64 or 128, Dv == D.
+//
+// One CTA computes one 128-row tile: 128/G consecutive queries of a sequence times the G
+// query heads that share one KV head (so every K/V tile feeds all G heads), against the keys
+// those queries can see, 128 keys per step, and writes the final output and lse.
+//
+//   warp 4      TMA producer: the Q tile once, then K and V tiles page by page (one box per
+//               page and 64-element half of the head dim, 128-byte swizzle) into a ring of
+//               stages; pages past the sequence's last key are never touched.
+//   warp 5      TMEM owner and MMA issuer (one thread): S = Q K^T into one of two TMEM
+//               buffers, then O += P V with P from shared memory; commits signal completion.
+//               Before P V it zeroes the V rows past the sequence's last key (their bytes are
+//               whatever the page holds there).
+//   warps 0..3  softmax, one thread per row (= TMEM lane): S row from TMEM, scale to base-2
+//               units, causal/window mask at absolute positions on edge tiles, running max and
+//               sum in float32, P = exp2(S - m) as 16-bit into shared memory. The output in TMEM
+//               is rescaled only when the running max grows by more than 2^8, and the epilogue
+//               divides by the sum, rounds once and stores.
+//
+// Every wait on an mbarrier is bounded (Watchdog): a stalled pipeline sets the plan's error
+// word and the CTA leaves through its normal exit, freeing TMEM.
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+
+namespace pa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;  // rows per tile (queries x group heads)
+constexpr int BN = 128;  // keys per step
+constexpr int KST = 2;   // K stages
+constexpr int VST = 2;   // V stages
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
+
+template <int D>
+struct PrefillSmem {
+    static constexpr int KH = D / 64;                 // 128-byte halves of a row
+    static constexpr int HALF_Q = BM * 128;           // bytes of one half of the Q tile
+    static constexpr int HALF_KV = BN * 128;          // bytes of one half of a K or V tile
+    static constexpr int Q = 0;
+    static constexpr int K = Q + KH * HALF_Q;
+    static constexpr int V = K + KST * KH * HALF_KV;
+    static constexpr int P = V + VST * KH * HALF_KV;
+    static constexpr int BAR = P + 2 * BM * 128;      // P: 128 rows x 128 keys, two halves
+    static constexpr int BYTES = BAR + 256;
+    static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
+};
+
+enum BarId { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
+             B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_SFREE = B_SFULL + 2,
+             B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + 1, B_COUNT = B_ODONE + 1 };
+
+}  // namespace
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
+    using L_ = PrefillSmem<D>;
+    constexpr int KH = L_::KH;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr uint32_t IDESC_QK = idesc_f16(BM, BN, kBf16, false, false);
+    constexpr uint32_t IDESC_PV = idesc_f16(BM, D, kBf16, false, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L_::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Watchdog wd{abort_flag, p.err, kWaitLimitNs};
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const PrefillUnit u = p.punits[blockIdx.x];
+    const SeqInfo si = p.seqs[u.seq];
+    const int G = p.group;
+    const int qpt = BM / G;
+    const int live_q = min(qpt, si.n - u.j0);
+    const int live_rows = live_q * G;
+    const int64_t p_first = (int64_t)si.L - si.n + u.j0;
+    const int64_t p_last = p_first + live_q - 1;
+    const int64_t kv_lo = p.window > 0 ? max64(0, p_first - p.window + 1) : 0;
+    const int64_t kv_hi = p.causal ? min64(si.L, p_last + 1) : si.L;
+    const int ps = p.page_size;
+    const int box = ps < BN ? ps : BN;  // keys per TMA box
+    const int64_t kt_start = (kv_lo / box) * box;
+    const int n_tiles = kv_hi > kt_start ? (int)((kv_hi - kt_start + BN - 1) / BN) : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < B_COUNT; ++i) {
+            uint32_t cnt = 1;
+            if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) cnt = 128;
+            mbar_init(&bars[i], cnt);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s0 = tmem, t_s1 = tmem + 128;
+    const uint32_t t_o = tmem + 256;
+    const uint32_t s_base = smem_u32(smem);
+
+    if (warp == 4) {
+        // ===================== TMA producer =====================
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch(&tmq);
+            tma_prefetch(&tmk);
+            tma_prefetch(&tmv);
+            mbar_arrive_expect_tx(&bars[B_QFULL], KH * L_::HALF_Q);
+            for (int h = 0; h < KH; ++h)
+                tma_load_3d(smem + L_::Q + h * L_::HALF_Q, &tmq, &bars[B_QFULL], h * 64, u.kvh * G,
+                            si.q_start + u.j0);
+            const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+            int issued = 0;  // tiles whose K and V loads were issued
+            for (int i = 0; i < n_tiles; ++i) {
+                const int64_t kt0 = kt_start + (int64_t)i * BN;
+                int nb = 0;  // boxes whose first key lies inside the sequence
+                for (int b = 0; b < BN / box; ++b)
+                    if (kt0 + (int64_t)b * box < si.L) nb = b + 1;
+                const uint32_t bytes = (uint32_t)nb * box * 128 * KH;
+                const int ks = i % KST, vs = i % VST;
+                if (i >= KST && !mbar_wait(&bars[B_KEMPTY + ks], ((i / KST) - 1) & 1, wd, 1)) break;
+                mbar_arrive_expect_tx(&bars[B_KFULL + ks], bytes);
+                for (int b = 0; b < nb; ++b) {
+                    const int64_t key = kt0 + (int64_t)b * box;
+                    const int row = (int)((int64_t)bt[key / ps] * ps + key % ps);
+                    for (int h = 0; h < KH; ++h)
+                        tma_load_3d(smem + L_::K + (ks * KH + h) * L_::HALF_KV + b * box * 128, &tmk,
+                                    &bars[B_KFULL + ks], h * 64, u.kvh, row);
+                }
+                if (i >= VST && !mbar_wait(&bars[B_VEMPTY + vs], ((i / VST) - 1) & 1, wd, 2)) break;
+                mbar_arrive_expect_tx(&bars[B_VFULL + vs], bytes);
+                for (int b = 0; b < nb; ++b) {
+                    const int64_t key = kt0 + (int64_t)b * box;
+                    const int row = (int)((int64_t)bt[key / ps] * ps + key % ps);
+                    for (int h = 0; h < KH; ++h)
+                        tma_load_3d(smem + L_::V + (vs * KH + h) * L_::HALF_KV + b * box * 128, &tmv,
+                                    &bars[B_VFULL + vs], h * 64, u.kvh, row);
+                }
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                // Leave no copy in flight into this CTA's shared memory: wait (bounded, ignoring
+                // the abort flag) for the last loads issued into each stage and for Q.
+                const uint64_t t0 = globaltimer_ns();
+                auto drain = [&](uint64_t* bar, uint32_t parity) {
+                    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+                };
+                drain(&bars[B_QFULL], 0);
+                for (int i = max(0, issued - KST); i < issued; ++i) drain(&bars[B_KFULL + i % KST], (i / KST) & 1);
+                for (int i = max(0, issued - VST); i < issued; ++i) drain(&bars[B_VFULL + i % VST], (i / VST) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        // ===================== MMA issuer =====================
+        bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[B_QFULL], 0, wd, 3));
+        for (int i = 0; ok && i <= n_tiles; ++i) {
+            if (i < n_tiles) {
+                const int ks = i % KST, b = i & 1;
+                ok = mbar_wait(&bars[B_KFULL + ks], (i / KST) & 1, wd, 4);
+                if (ok && i >= 2) ok = mbar_wait(&bars[B_SFREE + b], ((i >> 1) - 1) & 1, wd, 5);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t qa = s_base + L_::Q + (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;
+                        const uint32_t ka = s_base + L_::K + (ks * KH + (kk >> 2)) * L_::HALF_KV + (kk & 3) * 32;
+                        mma_f16_ss(b ? t_s1 : t_s0, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), IDESC_QK, kk > 0);
+                    }
+                    mma_commit(&bars[B_SFULL + b]);
+                    mma_commit(&bars[B_KEMPTY + ks]);
+                }
+                __syncwarp();
+            }
+            if (i >= 1) {
+                const int j = i - 1, vs = j % VST;
+                ok = mbar_wait(&bars[B_PFULL], j & 1, wd, 6);
+                if (ok) ok = mbar_wait(&bars[B_VFULL + vs], (j / VST) & 1, wd, 7);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                // V rows past the sequence's end hold arbitrary bytes: make them zero.
+                const int64_t kt0 = kt_start + (int64_t)j * BN;
+                const int nvalid = (int)min64(BN, si.L - kt0);
+                if (nvalid < BN) {
+                    for (int h = 0; h < KH; ++h) {
+                        uint4* base = reinterpret_cast<uint4*>(smem + L_::V + (vs * KH + h) * L_::HALF_KV);
+                        for (int c = nvalid * 8 + lane; c < BN * 8; c += 32) base[c] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                tc_fence_after();
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        const uint32_t pa_ = s_base + L_::P + (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t va = s_base + L_::V + vs * KH * L_::HALF_KV + kk * 16 * 128;
+                        mma_f16_ss(t_o, sdesc_sw128(pa_, 16, 1024), sdesc_sw128(va, L_::HALF_KV, 1024), IDESC_PV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars[B_ODONE]);
+                    mma_commit(&bars[B_VEMPTY + vs]);
+                }
+                __syncwarp();
+            }
+        }
+    } else {
+        // ===================== softmax: thread = row =====================
+        const int r = tid;  // TMEM lane; warp w owns lanes 32w .. 32w+31
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const bool live = r < live_rows;
+        const int64_t pos = p_first + (live ? r / G : 0);
+        // keys every live row sees: [all_lo, all_hi)
+        const int64_t all_lo = p.window > 0 ? p_last - p.window + 1 : INT64_MIN;
+        const int64_t all_hi = min64(p.causal ? p_first + 1 : si.L, si.L);
+        float m_run = neg_inf(), l_run = 0.f;
+        uint8_t* prow = smem + L_::P + r * 128;
+        bool ok = true;
+        for (int i = 0; i < n_tiles; ++i) {
+            const int b = i & 1;
+            const int64_t kt0 = kt_start + (int64_t)i * BN;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (i >> 1) & 1, wd, 8));
+            if (!ok) break;
+            tc_fence_after();
+            float s[BN];
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32((b ? t_s1 : t_s0) + lane_off + c * 32, v);
+                tmem_ld_wait(v);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(v[e]);
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[B_SFREE + b]);
+
+            const bool full = kt0 >= all_lo && kt0 + BN <= all_hi;
+            float m_tile = neg_inf();
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                float x = s[c] * p.scale_log2;
+                if (!full) {
+                    const int64_t t = kt0 + c;
+                    const bool vis = t < si.L && (!live || key_visible(t, pos, p.causal, p.window));
+                    x = vis ? x : neg_inf();
+                }
+                s[c] = x;
+                m_tile = fmaxf(m_tile, x);
+            }
+            const float m_new = fmaxf(m_run, m_tile);
+            if (i > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE], (i - 1) & 1, wd, 9));
+                if (!ok) break;
+            }
+            const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
+            const bool rescale = grow && i > 0 && m_run != neg_inf();
+            if (__any_sync(0xffffffffu, rescale)) {
+                tc_fence_after();
+                const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(t_o + lane_off + c * 32, v);
+                    tmem_ld_wait(v);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                    tmem_st32(t_o + lane_off + c * 32, v);
+                }
+                tmem_st_wait();
+            }
+            if (grow) {
+                l_run *= fast_exp2(m_run - m_new);
+                m_run = m_new;
+            }
+            const float m_use = m_run == neg_inf() ? 0.f : m_run;
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < BN / 8; ++c) {  // 16-byte chunk c holds keys 8c .. 8c+7
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a = fast_exp2(s[c * 8 + 2 * e] - m_use);
+                    const float bb = fast_exp2(s[c * 8 + 2 * e + 1] - m_use);
+                    sum += a + bb;
+                    pk[e] = pack2<T>(a, bb);
+                }
+                const int half = c >> 3, cc = c & 7;
+                *reinterpret_cast<uint4*>(prow + half * (BM * 128) + ((cc ^ (r & 7)) << 4)) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            l_run += sum;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_PFULL]);
+        }
+        // ---- epilogue ----
+        if (ok && n_tiles > 0)
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE], (n_tiles - 1) & 1, wd, 10));
+        tc_fence_after();
+        const bool has = l_run > 0.f;
+        const float inv = has ? 1.0f / l_run : 0.f;
+        const int64_t qrow = (int64_t)(si.q_start + u.j0 + (live ? r / G : 0)) * p.hq + u.kvh * G + (live ? r % G : 0);
+        T* orow = static_cast<T*>(p.out) + qrow * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            if (ok && n_tiles > 0) {
+                tmem_ld32(t_o + lane_off + c * 32, v);
+                tmem_ld_wait(v);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0u;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                pk[e] = pack2<T>(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+            if (live && ok) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+        }
+        if (live && ok) p.lse[qrow] = has ? (m_run + __log2f(l_run)) * kLn2 : neg_inf();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 3-D map over a row-major [d2][d1][d0] tensor of 16-bit elements, box {64, b1, b2}, 128B swizzle.
+bool make_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1,
+              uint32_t b2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t boxd[3] = {64, b1, b2};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3,
+                    const_cast<void*>(base), dims, strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename T, int D>
+cudaError_t launch_t(const AttnParams& p, int num_pages, cudaStream_t st) {
+    using L_ = PrefillSmem<D>;
+    const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+    const int G = p.group, qpt = BM / G;
+    const int ps = p.page_size;
+    const int box = ps < BN ? ps : BN;
+    CUtensorMap tq, tk, tv;  // the Q map spans every packed query row
+    if (!make_map(&tq, bf16, p.q, D, p.hq, (uint64_t)p.num_queries, G, qpt) ||
+        !make_map(&tk, bf16, p.k, D, p.hkv, (uint64_t)num_pages * ps, 1, box) ||
+        !make_map(&tv, bf16, p.v, D, p.hkv, (uint64_t)num_pages * ps, 1, box))
+        return cudaErrorInvalidValue;
+    auto kern = prefill_tc_kernel<T, D>;
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !(configured >> dev & 1ull)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L_::ALLOC);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured |= 1ull << dev;
+    }
+    kern<<<p.num_punits, kThreads, L_::ALLOC, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc_supported(pa_dtype dt, int d, int dv, int group, int page_size) {
+    if (dt == PA_F32 || d != dv || (d != 64 && d != 128)) return false;
+    if (group < 1 || group > BM || BM % group != 0) return false;
+    if (page_size % 16 != 0) return false;
+    if (page_size < BN ? (BN % page_size != 0) : (page_size % BN != 0)) return false;
+    return true;
+}
+
+cudaError_t launch_prefill_tc(const AttnParams& p, pa_dtype dt, int num_pages, cudaStream_t st) {
+    if (p.num_punits == 0) return cudaSuccess;
+    if (dt == PA_BF16) return p.d == 64 ? launch_t<__nv_bfloat16, 64>(p, num_pages, st)
+                                        : launch_t<__nv_bfloat16, 128>(p, num_pages, st);
+    return p.d == 64 ? launch_t<__half, 64>(p, num_pages, st) : launch_t<__half, 128>(p, num_pages, st);
+}
+
+}  // namespace pa
