@@ -293,11 +293,13 @@ def run_ours(args, ws, rank, local):
     return result
 
 
-def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src):
+def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
     """The other configurations, timed the same way (few steps): context for the headline."""
     res = {}
     cfgs = [("bf16_chunked_prefill", W.c3_chunked_prefill), ("bf16_window_mixed", W.c4_window_mixed),
             ("bf16_mla_decode", W.c5_mla_decode)]
+    if only is not None:
+        cfgs = [only]
     for name, fn in cfgs:
         try:
             wl = fn(args.seed)
@@ -319,7 +321,8 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src):
 
                 def step(tr):
                     pa.pa_forward(plan, q, k, v, out, lse, wl.scale, wl.causal, wl.window, trace=tr)
-            ms, kern, comb, _ = time_forward(pa, plan, step, args.extra_steps, 3, True, None, 1)
+            ms, kern, comb, _ = time_forward(pa, plan, step, args.extra_steps, args.warmup if only else 3, True,
+                                             None, 1)
             res[name] = {
                 "ms_per_step": round(ms, 4),
                 "attention_kernels_ms": round(kern, 4),
@@ -337,6 +340,22 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src):
         except Exception as e:  # a failing extra must not hide the headline
             res[name] = {"error": str(e)[:300]}
     return res
+
+
+def run_single(args, ws, rank, local):
+    """One of the other configurations as the only workload (profiling and tuning runs)."""
+    import paged_kv_attention_39_b200 as pa
+    from paged_kv_attention_39_b200 import workloads as W
+    pa.load_library()
+    hbm, tf_burst, _, peak_src = peaks()
+    dev = torch.device("cuda", local)
+    args.extra_steps = args.steps
+    fns = {"bf16_chunked_prefill": W.c3_chunked_prefill, "bf16_window_mixed": W.c4_window_mixed,
+           "bf16_mla_decode": W.c5_mla_decode, "tiny_fp32_decode": W.c1_tiny_fp32_decode}
+    res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
+    r = res[args.workload]
+    return {"metric": METRIC, "workload": args.workload, "value": r.get("tflops"), "unit": "TFLOP/s",
+            "steps": args.steps, "warmup": args.warmup, "detail": r}
 
 
 def cpu_baseline(wl, kv_bytes, budget_s: float = 10.0):
@@ -408,12 +427,18 @@ def main():
     ap.add_argument("--extra-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
+    ap.add_argument("--workload", default="bf16_decode",
+                    choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode",
+                             "tiny_fp32_decode"],
+                    help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     ws, rank, local = dist_setup()
     if args.impl == "reference":
         res = run_reference(args, ws, rank)
+    elif args.workload != "bf16_decode":
+        res = run_single(args, ws, rank, local)
     else:
         res = run_ours(args, ws, rank, local)
     if rank == 0 and res is not None:
