@@ -189,6 +189,38 @@ pa_status pa_mla_forward_ex(pa_plan* plan, const void* q_latent, const void* q_r
                             const pa_forward_options* opts);
 
 /*
+ * pa_forward_static_workspace -- pa_forward's split-KV decode without any memory allocation.
+ * The pages describe no such call: it exists for callers that cannot allocate device memory
+ * while they run attention (a serving loop that must not stall on the allocator mid-step, a
+ * process under a fixed pre-reserved memory budget, a host runtime that forbids cudaMalloc in
+ * plugins). pa_forward may allocate: its split workspace grows on demand and the first call with
+ * a new head configuration uploads a work list into new memory. This call keeps both in one
+ * fixed array of PA_STATIC_WORKSPACE_BYTES in device global memory, defined inside the library;
+ * every GPU that loads the library holds that array until the process exits. The caller still
+ * provides the plan, the inputs and the outputs, exactly as for pa_forward.
+ *
+ * Scope: bf16 or fp16, head_dim == v_head_dim in {64, 128}, and every sequence with at most 16
+ * query rows per KV head (queries x Hq/Hkv): the tensor-core decode kernel's shapes. Other shapes
+ * return PA_ERR_UNSUPPORTED. kv_chunk is pa_forward_options.kv_chunk (0 automatic, -1 never
+ * split, > 0 keys per part). A batch whose work list or float32 split parts do not fit the array
+ * returns PA_ERR_BOUNDS before anything is launched (a larger kv_chunk, or -1, needs fewer parts).
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress, once
+ * per device, with that device current); make that first call before capturing the stream into
+ * a CUDA graph. Every call shares the one array and leaves its contents behind; nothing in it
+ * needs to start at zero (each call writes every part it later reads). Calls whose GPU work
+ * overlaps -- issued on different streams of one process -- race on the array: order them on
+ * one stream. Host threads are serialised inside the call.
+ * All other rules (validation before launch, no host synchronisation, errors) are pa_forward's.
+ */
+#define PA_STATIC_WORKSPACE_BYTES (16u << 20)
+pa_status pa_forward_static_workspace(pa_plan* plan, const void* q, const void* k_cache,
+                                      const void* v_cache, pa_dtype dtype, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t v_head_dim,
+                                      float scale, int causal, int32_t window, int32_t kv_chunk,
+                                      void* out, float* lse, pa_stream stream);
+
+/*
  * pa_plan_prepare -- build and upload the work list of one head configuration ahead of the
  * first forward call (pa_forward does it implicitly). `mla` selects pa_mla_forward's
  * configuration (num_kv_heads is then 1 and v_head_dim == head_dim == latent_dim).

@@ -29,7 +29,8 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
           "PA_ERR_ALIAS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA"]
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
-           "pa_forward_ex", "pa_mla_forward", "pa_mla_forward_ex", "pa_plan_device_status",
+           "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex",
+           "pa_plan_device_status",
            "pa_status_string", "pa_last_error_message", "pa_version"]
 
 _P = ctypes.c_void_p
@@ -87,6 +88,9 @@ def load_library(path: Optional[str] = None):
     lib.pa_mla_forward.argtypes = mla
     lib.pa_mla_forward_ex.restype = ctypes.c_int
     lib.pa_mla_forward_ex.argtypes = mla + [ctypes.POINTER(_Options)]
+    lib.pa_forward_static_workspace.restype = ctypes.c_int
+    lib.pa_forward_static_workspace.argtypes = [_P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _I, ctypes.c_float,
+                                                ctypes.c_int, _I, _I, _P, _P, _P]
     lib.pa_plan_device_status.restype = ctypes.c_int
     lib.pa_plan_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -236,6 +240,20 @@ def pa_forward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _DTYPES[q.dtype], q.shape[1],
         k_cache.shape[2], q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window),
         _ptr(out), _ptr(lse), _stream_ptr(stream, plan.device), _opts(kv_chunk, path, trace)))
+
+
+def pa_forward_static_workspace(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor,
+                                v_cache: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, scale: float,
+                                causal: bool = True, window: int = 0, kv_chunk: int = 0, stream=None) -> None:
+    """Split-KV decode that allocates no memory: scratch in the library's fixed device array
+    (for callers that cannot allocate while attention runs; see include/pa.h)."""
+    for t in (q, k_cache, v_cache, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("pa_forward_static_workspace takes contiguous tensors")
+    _check(load_library().pa_forward_static_workspace(
+        plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _DTYPES[q.dtype], q.shape[1], k_cache.shape[2],
+        q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window), int(kv_chunk), _ptr(out),
+        _ptr(lse), _stream_ptr(stream, plan.device)))
 
 
 def pa_mla_forward(plan: Plan, q_latent: torch.Tensor, q_rope: torch.Tensor,

@@ -437,6 +437,54 @@ pa_forward_options default_opts(const pa_forward_options* o) {
 
 }  // namespace
 
+namespace pa {
+
+pa_status set_error(pa_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+pa_status clear_error() { return ok(); }
+
+pa_status validated_gqa_view(pa_plan* P, const void* q, const void* k, const void* v, pa_dtype dtype, int32_t hq,
+                             int32_t hkv, int32_t d, int32_t dv, float scale, int causal, int32_t window,
+                             void* out, float* lse, PlanView* view) {
+    Call c{};
+    c.mla = false;
+    c.q = q; c.k = k; c.v = v;
+    c.dtype = dtype;
+    c.hq = hq; c.hkv = hkv; c.d = d; c.dv = dv;
+    c.scale = scale; c.causal = causal; c.window = window;
+    c.out = out; c.lse = lse;
+    c.opts = default_opts(nullptr);
+    pa_status vs = validate(P, c);
+    if (vs != PA_OK) return vs;
+    if (P->Nq > 0) {
+        if (P->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to run on");
+        int cur = -1;
+        PA_CUDA_TRY(cudaGetDevice(&cur));
+        if (cur != P->device)
+            return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, P->device);
+    }
+    view->device = P->device;
+    view->num_sms = P->num_sms;
+    view->S = P->S;
+    view->Nq = P->Nq;
+    view->table_width = P->table_width;
+    view->page_size = P->page_size;
+    view->num_pages = P->num_pages;
+    view->host_seqs = P->seqs.data();
+    view->d_seqs = P->d_seqs;
+    view->d_bt = P->d_bt;
+    view->d_err = P->d_err;
+    return PA_OK;
+}
+
+}  // namespace pa
+
 // ---------------------------------------------------------------------------------------
 // C ABI
 // ---------------------------------------------------------------------------------------

@@ -75,4 +75,22 @@ bool prefill_tc_supported(pa_dtype dt, int d, int dv, int group, int page_size);
 // Largest row count (queries x group heads per KV head) the tensor-core decode kernel takes.
 constexpr int kDecodeMaxRows = 16;
 
+// Read-only facts of a plan, for entry points outside the plan's own translation unit.
+struct PlanView {
+    int device, num_sms;
+    int32_t S, Nq, table_width, page_size, num_pages;
+    const SeqInfo* host_seqs;
+    const SeqInfo* d_seqs;
+    const int32_t* d_bt;
+    int* d_err;
+};
+
+// Validates a paged GQA call exactly as pa_forward does and fills `view`.
+pa_status validated_gqa_view(pa_plan* P, const void* q, const void* k, const void* v, pa_dtype dtype, int32_t hq,
+                             int32_t hkv, int32_t d, int32_t dv, float scale, int causal, int32_t window,
+                             void* out, float* lse, PlanView* view);
+// Thread-local error message of the C ABI (pa_last_error_message).
+pa_status set_error(pa_status st, const char* fmt, ...);
+pa_status clear_error();
+
 }  // namespace pa
