@@ -223,7 +223,8 @@ pa_status pa_forward_static_workspace(pa_plan* plan, const void* q, const void* 
 /*
  * pa_plan_prepare -- build and upload the work list of one head configuration ahead of the
  * first forward call (pa_forward does it implicitly). `mla` selects pa_mla_forward's
- * configuration (num_kv_heads is then 1 and v_head_dim == head_dim == latent_dim).
+ * configuration: num_q_heads is then the head count, head_dim the latent width and v_head_dim
+ * the rope width (num_kv_heads is ignored).
  * Uses `stream` for the one upload and the workspace allocation.
  */
 pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_heads,

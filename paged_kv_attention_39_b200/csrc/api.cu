@@ -62,7 +62,7 @@ constexpr int kMaxSplits = 1024;           // parts one sequence's keys may be c
 constexpr int kTargetCtasPerSm = 8;        // automatic split size aims at this many CTAs/SM
 
 struct SchedKey {
-    int mla, dtype, hq, hkv, d, dv, causal, window, path, kv_chunk;
+    int mla, dtype, hq, hkv, d, dv, pr, causal, window, path, kv_chunk;
     bool operator==(const SchedKey& o) const { return std::memcmp(this, &o, sizeof o) == 0; }
 };
 
@@ -74,7 +74,8 @@ struct Schedule {
     const pa::KvUnit* simt_units = nullptr;   // CUDA-core kernel
     const pa::CombineUnit* cunits = nullptr;
     const pa::PrefillUnit* punits = nullptr;  // tensor-core prefill kernel
-    int32_t n_tc = 0, n_simt = 0, n_comb = 0, n_pre = 0;
+    const pa::KvUnit* mla_units = nullptr;    // tensor-core MLA decode kernel (two CTAs per unit)
+    int32_t n_tc = 0, n_simt = 0, n_comb = 0, n_pre = 0, n_mla = 0;
     int32_t tc_rows_max = 0;
     int64_t slots = 0;  // workspace parts
     int32_t kv_chunk = 0;
@@ -133,17 +134,20 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
                            k.d == k.dv && (k.d == 64 || k.d == 128);
     const bool tc_prefill = !k.mla && k.path == PA_PATH_AUTO &&
                             pa::prefill_tc_supported((pa_dtype)k.dtype, k.d, k.dv, G, P->page_size);
+    const bool tc_mla = k.mla && k.path == PA_PATH_AUTO &&
+                        pa::mla_tc_supported((pa_dtype)k.dtype, k.hq, k.d, k.pr, P->page_size);
     std::vector<pa::PrefillUnit> pu;
     std::vector<int64_t> pu_cost;
 
-    struct Block { int32_t seq, j0, j1, lo, hi; bool tc; };
+    struct Block { int32_t seq, j0, j1, lo, hi; int kind; };  // kind: 0 CUDA-core, 1 decode, 2 MLA
     std::vector<Block> blocks;
     int64_t total = 0;  // keys x kv heads, over all blocks
     for (int32_t s = 0; s < P->S; ++s) {
         const pa::SeqInfo& si = P->seqs[s];
         if (si.n == 0) continue;
         const bool tc = tc_decode && (int64_t)si.n * G <= pa::kDecodeMaxRows;
-        if (!tc && tc_prefill) {
+        const bool mla_one = tc_mla && si.n == 1;
+        if (!tc && !mla_one && tc_prefill) {
             // 128-row tiles: 128 / G queries times the G heads of one KV head
             const int32_t qpt = 128 / G;
             for (int32_t j0 = 0; j0 < si.n; j0 += qpt) {
@@ -163,9 +167,9 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
             continue;
         }
         // CUDA-core blocks take few queries so that long prefill chunks spread over CTAs.
-        const int32_t qb = tc ? si.n : std::max<int32_t>(1, 16 / std::min<int32_t>(G, 16));
+        const int32_t qb = (tc || mla_one) ? si.n : std::max<int32_t>(1, 16 / std::min<int32_t>(G, 16));
         for (int32_t j0 = 0; j0 < si.n; j0 += qb) {
-            Block b{s, j0, std::min(si.n, j0 + qb), 0, 0, tc};
+            Block b{s, j0, std::min(si.n, j0 + qb), 0, 0, tc ? 1 : (mla_one ? 2 : 0)};
             visible_union(si.L, si.n, b.j0, b.j1, k.causal, k.window, &b.lo, &b.hi);
             total += (int64_t)(b.hi - b.lo) * (k.mla ? 1 : k.hkv);
             blocks.push_back(b);
@@ -175,13 +179,14 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     if (k.kv_chunk > 0) chunk = k.kv_chunk;
     else if (k.kv_chunk < 0) chunk = INT32_MAX;
     else {
-        const int64_t target = (int64_t)P->num_sms * kTargetCtasPerSm;
+        // The tensor-core MLA kernel runs one CTA per SM, two per unit: aim at one unit per SM.
+        const int64_t target = tc_mla ? (int64_t)P->num_sms : (int64_t)P->num_sms * kTargetCtasPerSm;
         chunk = (total + target - 1) / std::max<int64_t>(1, target);
         chunk = ((chunk + 63) / 64) * 64;
         chunk = std::max<int64_t>(chunk, 256);
     }
 
-    std::vector<pa::KvUnit> tcu, simtu;
+    std::vector<pa::KvUnit> tcu, simtu, mlau;
     std::vector<pa::CombineUnit> cu;
     int64_t slots = 0;
     for (const Block& b : blocks) {
@@ -205,8 +210,8 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
             u.part_base = base;
             u.j0 = b.j0;
             u.j1 = b.j1;
-            (b.tc ? tcu : simtu).push_back(u);
-            if (b.tc) S->tc_rows_max = std::max<int32_t>(S->tc_rows_max, (b.j1 - b.j0) * G);
+            (b.kind == 1 ? tcu : b.kind == 2 ? mlau : simtu).push_back(u);
+            if (b.kind == 1) S->tc_rows_max = std::max<int32_t>(S->tc_rows_max, (b.j1 - b.j0) * G);
         }
     }
     // Longest units first: the block scheduler hands them out in index order.
@@ -215,6 +220,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     };
     std::stable_sort(tcu.begin(), tcu.end(), longer);
     std::stable_sort(simtu.begin(), simtu.end(), longer);
+    std::stable_sort(mlau.begin(), mlau.end(), longer);
     {
         std::vector<size_t> order(pu.size());
         for (size_t i = 0; i < order.size(); ++i) order[i] = i;
@@ -232,12 +238,14 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     const size_t o_simt = align(o_tc + tcu.size() * sizeof(pa::KvUnit));
     const size_t o_c = align(o_simt + simtu.size() * sizeof(pa::KvUnit));
     const size_t o_p = align(o_c + cu.size() * sizeof(pa::CombineUnit));
-    const size_t bytes = align(o_p + pu.size() * sizeof(pa::PrefillUnit));
+    const size_t o_m = align(o_p + pu.size() * sizeof(pa::PrefillUnit));
+    const size_t bytes = align(o_m + mlau.size() * sizeof(pa::KvUnit));
     S->host.assign(std::max<size_t>(bytes, 256), 0);
     if (!tcu.empty()) std::memcpy(S->host.data() + o_tc, tcu.data(), tcu.size() * sizeof(pa::KvUnit));
     if (!simtu.empty()) std::memcpy(S->host.data() + o_simt, simtu.data(), simtu.size() * sizeof(pa::KvUnit));
     if (!cu.empty()) std::memcpy(S->host.data() + o_c, cu.data(), cu.size() * sizeof(pa::CombineUnit));
     if (!pu.empty()) std::memcpy(S->host.data() + o_p, pu.data(), pu.size() * sizeof(pa::PrefillUnit));
+    if (!mlau.empty()) std::memcpy(S->host.data() + o_m, mlau.data(), mlau.size() * sizeof(pa::KvUnit));
     PA_CUDA_TRY(cudaMallocAsync(&S->dev, S->host.size(), st));
     cudaError_t e = cudaMemcpyAsync(S->dev, S->host.data(), S->host.size(), cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) {
@@ -251,6 +259,8 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     S->cunits = (const pa::CombineUnit*)(base + o_c);
     S->punits = (const pa::PrefillUnit*)(base + o_p);
     S->n_pre = (int32_t)pu.size();
+    S->mla_units = (const pa::KvUnit*)(base + o_m);
+    S->n_mla = (int32_t)mlau.size();
     S->n_tc = (int32_t)tcu.size();
     S->n_simt = (int32_t)simtu.size();
     S->n_comb = (int32_t)cu.size();
@@ -361,6 +371,7 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     key.hkv = c.hkv;
     key.d = c.d;
     key.dv = c.dv;
+    key.pr = c.mla ? c.pr : 0;
     key.causal = c.causal;
     key.window = c.window;
     key.path = c.opts.path;
@@ -411,6 +422,13 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
         ++launches;
         e = pa::launch_prefill_tc(p, c.dtype, P->num_pages, st);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill kernel launch failed: %s", cudaGetErrorString(e));
+    }
+    if (S->n_mla > 0) {
+        ++launches;
+        p.units = S->mla_units;
+        p.num_units = S->n_mla;
+        e = pa::launch_mla_tc(p, c.dtype, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "MLA kernel launch failed: %s", cudaGetErrorString(e));
     }
     if (S->n_simt > 0) {
         ++launches;
@@ -666,6 +684,8 @@ pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_
     key.hkv = mla ? 1 : num_kv_heads;
     key.d = head_dim;
     key.dv = mla ? head_dim : v_head_dim;
+    key.pr = mla ? v_head_dim : 0;  // for MLA the fifth size argument is the rope width
+    if (mla) key.dv = head_dim;
     key.causal = causal;
     key.window = window;
     key.path = o.path;

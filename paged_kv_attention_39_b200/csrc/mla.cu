@@ -1,0 +1,415 @@
+// MLA absorbed-latent paged decode on the 5th-generation tensor cores (bf16 / fp16, latent
+// width R = 512, rope width P = 64, up to 128 heads, one query per sequence).
+//
+// Scores s[h, t] = scale * (q_lat[h] . latent[t] + q_rope[h] . rope[t]) take one M = 128 (heads)
+// by N = 32 (keys) by K = R + P = 576 product; the latent rows are also the values, so the same
+// shared-memory tile feeds O += P V. The float32 output of 128 heads x 512 columns would fill
+// all 512 TMEM columns, leaving none for the scores, so each key range is handled by a pair of
+// CTAs: both compute the (identical) scores and softmax, and each accumulates one 256-column
+// half of O (TMEM: two 32-column score buffers + 256 columns of O). The pair's second read of a
+// K/V tile comes mostly from L2.
+//
+//   warp 4      TMA producer: Q (9 boxes of 128 heads x 64 columns, once), then per step the
+//               latent and rope rows of 32 keys page by page into a 2-stage ring
+//   warp 5      TMEM owner, MMA issuer: S = Q K^T (36 k-steps), O_half += P V_half (2 k-steps);
+//               zeroes latent rows past the sequence's last key before P V reads them
+//   warps 0..3  softmax, thread = head: S row from TMEM, mask at the range edges, running max
+//               and sum in float32, P (16-bit, 64-byte swizzled K-major tile) into shared memory
+//
+// Every mbarrier wait is bounded (sm100::mbar_wait).
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+
+namespace pa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int MR = 512;            // latent width
+constexpr int MP = 64;             // rope width
+constexpr int MK = MR + MP;        // score contraction length
+constexpr int MC = MK / 64;        // 128-byte columns of a Q / K row (8 latent + 1 rope)
+constexpr int MBM = 128;           // heads per tile
+constexpr int MBN = 32;            // keys per step
+constexpr int MST = 2;             // K/V stages
+constexpr int MDV = MR / 2;        // output columns per CTA
+constexpr int kMlaThreads = 192;
+constexpr uint32_t kMlaTmemCols = 512;
+constexpr uint64_t kMlaWaitNs = 2000000000ull;
+
+struct MlaSmem {
+    static constexpr int Q_COL = MBM * 128;          // one 64-wide column of Q: 16 KB
+    static constexpr int KV_COL = MBN * 128;         // one 64-wide column of a K/V tile: 4 KB
+    static constexpr int Q = 0;
+    static constexpr int KV = Q + MC * Q_COL;        // 144 KB
+    static constexpr int P = KV + MST * MC * KV_COL; // + 72 KB
+    static constexpr int BAR = P + MBM * 64;         // + 8 KB (128 heads x 32 keys, 16-bit)
+    static constexpr int BYTES = BAR + 256;
+    static constexpr int ALLOC = BYTES + 1024;
+};
+
+enum MBar { M_QFULL = 0, M_FULL = 1, M_EMPTY = M_FULL + MST, M_SFULL = M_EMPTY + MST, M_SFREE = M_SFULL + 2,
+            M_PFULL = M_SFREE + 2, M_ODONE = M_PFULL + 2, M_COUNT = M_ODONE + 2 };
+
+// 64-byte swizzle K-major descriptor (rows of 32 16-bit elements, 8-row atoms of 512 bytes).
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;  // leading byte offset: unused for swizzled K-major
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;  // 64-byte swizzle
+    return d;
+}
+
+}  // namespace
+
+template <typename T>
+__global__ void __launch_bounds__(kMlaThreads, 1)
+    mla_tc_kernel(const __grid_constant__ CUtensorMap tm_ql, const __grid_constant__ CUtensorMap tm_qr,
+                  const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
+                  const AttnParams p) {
+    using L_ = MlaSmem;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr uint32_t IDESC_QK = idesc_f16(MBM, MBN, kBf16, false, false);
+    constexpr uint32_t IDESC_PV = idesc_f16(MBM, MDV, kBf16, false, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L_::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + M_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Watchdog wd{abort_flag, p.err, kMlaWaitNs};
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const KvUnit u = p.units[blockIdx.x >> 1];
+    const int hf = blockIdx.x & 1;  // which half of the 512 output columns
+    const SeqInfo si = p.seqs[u.seq];
+    const int H = p.hq;
+    const int64_t qi = si.q_start;          // one query per sequence on this path
+    const int64_t pos = (int64_t)si.L - 1;  // its absolute position
+    const int ps = p.page_size;
+    const int box = ps < MBN ? ps : MBN;
+    const int64_t kt_start = ((int64_t)u.t0 / box) * box;
+    const int n_tiles = u.t1 > kt_start ? (int)((u.t1 - kt_start + MBN - 1) / MBN) : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < M_COUNT; ++i) {
+            uint32_t cnt = 1;
+            if (i == M_SFREE || i == M_SFREE + 1 || i == M_PFULL || i == M_PFULL + 1) cnt = 128;
+            mbar_init(&bars[i], cnt);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kMlaTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s0 = tmem, t_s1 = tmem + 32, t_o = tmem + 64;
+    const uint32_t s_base = smem_u32(smem);
+
+    if (warp == 4) {
+        // ===================== TMA producer =====================
+        if (lane == 0 && n_tiles > 0) {
+            tma_prefetch(&tm_ql);
+            tma_prefetch(&tm_qr);
+            tma_prefetch(&tm_lat);
+            tma_prefetch(&tm_rope);
+            mbar_arrive_expect_tx(&bars[M_QFULL], MC * L_::Q_COL);
+            for (int c = 0; c < MC - 1; ++c)
+                tma_load_3d(smem + L_::Q + c * L_::Q_COL, &tm_ql, &bars[M_QFULL], c * 64, 0, (int)qi);
+            tma_load_3d(smem + L_::Q + (MC - 1) * L_::Q_COL, &tm_qr, &bars[M_QFULL], 0, 0, (int)qi);
+            const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+            int issued = 0;
+            for (int i = 0; i < n_tiles; ++i) {
+                const int64_t kt0 = kt_start + (int64_t)i * MBN;
+                int nb = 0;
+                for (int b = 0; b < MBN / box; ++b)
+                    if (kt0 + (int64_t)b * box < si.L) nb = b + 1;
+                const int st = i % MST;
+                if (i >= MST && !mbar_wait(&bars[M_EMPTY + st], ((i / MST) - 1) & 1, wd, 21)) break;
+                mbar_arrive_expect_tx(&bars[M_FULL + st], (uint32_t)nb * box * 128 * MC);
+                uint8_t* dst = smem + L_::KV + st * MC * L_::KV_COL;
+                for (int b = 0; b < nb; ++b) {
+                    const int64_t key = kt0 + (int64_t)b * box;
+                    const int row = (int)((int64_t)bt[key / ps] * ps + key % ps);
+                    for (int c = 0; c < MC - 1; ++c)
+                        tma_load_3d(dst + c * L_::KV_COL + b * box * 128, &tm_lat, &bars[M_FULL + st], c * 64, 0, row);
+                    tma_load_3d(dst + (MC - 1) * L_::KV_COL + b * box * 128, &tm_rope, &bars[M_FULL + st], 0, 0, row);
+                }
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                const uint64_t t0 = globaltimer_ns();
+                auto drain = [&](uint64_t* bar, uint32_t parity) {
+                    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kMlaWaitNs) {}
+                };
+                drain(&bars[M_QFULL], 0);
+                for (int i = max(0, issued - MST); i < issued; ++i) drain(&bars[M_FULL + i % MST], (i / MST) & 1);
+            }
+        }
+    } else if (warp == 5) {
+        // ===================== MMA issuer =====================
+        bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[M_QFULL], 0, wd, 23));
+        for (int i = 0; ok && i <= n_tiles; ++i) {
+            if (i < n_tiles) {
+                const int st = i % MST, b = i & 1;
+                ok = mbar_wait(&bars[M_FULL + st], (i / MST) & 1, wd, 24);
+                if (ok && i >= 2) ok = mbar_wait(&bars[M_SFREE + b], ((i >> 1) - 1) & 1, wd, 25);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                // latent rows past the sequence's end hold arbitrary bytes: they are values too
+                const int64_t kt0 = kt_start + (int64_t)i * MBN;
+                const int nvalid = (int)min64(MBN, si.L - kt0);
+                if (nvalid < MBN) {
+                    for (int c = 0; c < MC - 1; ++c) {
+                        uint4* col = reinterpret_cast<uint4*>(smem + L_::KV + (st * MC + c) * L_::KV_COL);
+                        for (int x = nvalid * 8 + lane; x < MBN * 8; x += 32) col[x] = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t kv = s_base + L_::KV + st * MC * L_::KV_COL;
+#pragma unroll 4
+                    for (int kk = 0; kk < MK / 16; ++kk) {
+                        const uint32_t qa = s_base + L_::Q + (kk >> 2) * L_::Q_COL + (kk & 3) * 32;
+                        const uint32_t ka = kv + (kk >> 2) * L_::KV_COL + (kk & 3) * 32;
+                        mma_f16_ss(b ? t_s1 : t_s0, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), IDESC_QK,
+                                   kk > 0);
+                    }
+                    mma_commit(&bars[M_SFULL + b]);
+                }
+                __syncwarp();
+            }
+            if (i >= 1) {
+                const int j = i - 1, st = j % MST;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[M_PFULL + (j & 1)], (j >> 1) & 1, wd, 26));
+                if (!ok) break;
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t vbase = s_base + L_::KV + (st * MC + hf * (MDV / 64)) * L_::KV_COL;
+#pragma unroll
+                    for (int kk = 0; kk < MBN / 16; ++kk) {
+                        const uint32_t pa_ = s_base + L_::P + kk * 32;
+                        const uint32_t va = vbase + kk * 16 * 128;
+                        mma_f16_ss(t_o, sdesc_sw64(pa_, 512), sdesc_sw128(va, L_::KV_COL, 1024), IDESC_PV,
+                                   (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars[M_ODONE + (j & 1)]);
+                    mma_commit(&bars[M_EMPTY + st]);
+                }
+                __syncwarp();
+            }
+        }
+    } else {
+        // ===================== softmax: thread = head =====================
+        const int r = tid;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const bool live = r < H;
+        float m_run = neg_inf(), l_run = 0.f;
+        bool ok = true;
+        for (int i = 0; i < n_tiles; ++i) {
+            const int b = i & 1;
+            const int64_t kt0 = kt_start + (int64_t)i * MBN;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[M_SFULL + b], (i >> 1) & 1, wd, 28));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32((b ? t_s1 : t_s0) + lane_off, v);
+            tmem_ld_wait(v);
+            tc_fence_before();
+            mbar_arrive(&bars[M_SFREE + b]);
+            const bool full = kt0 >= u.t0 && kt0 + MBN <= u.t1;
+            float x[32];
+            float m_tile = neg_inf();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                float y = __uint_as_float(v[e]) * p.scale_log2;
+                if (!full) {
+                    const int64_t t = kt0 + e;
+                    const bool vis = t >= u.t0 && t < u.t1 && key_visible(t, pos, p.causal, p.window);
+                    y = vis ? y : neg_inf();
+                }
+                x[e] = y;
+                m_tile = fmaxf(m_tile, y);
+            }
+            const float m_new = fmaxf(m_run, m_tile);
+            const bool grow = m_new > m_run + 8.0f;
+            const bool rescale = grow && i > 0 && m_run != neg_inf();
+            // the single P buffer was last read by P V of tile i - 1
+            if (i > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[M_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 29));
+                if (!ok) break;
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
+                tc_fence_after();
+                const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll 1
+                for (int c = 0; c < MDV / 32; ++c) {
+                    uint32_t w[32];
+                    tmem_ld32(t_o + lane_off + c * 32, w);
+                    tmem_ld_wait(w);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * alpha);
+                    tmem_st32(t_o + lane_off + c * 32, w);
+                }
+                tmem_st_wait();
+            }
+            if (grow) {
+                l_run *= fast_exp2(m_run - m_new);
+                m_run = m_new;
+            }
+            const float m_use = m_run == neg_inf() ? 0.f : m_run;
+            uint32_t pk[16];
+            float sum = 0.f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float a0 = fast_exp2(x[2 * e] - m_use);
+                const float a1 = fast_exp2(x[2 * e + 1] - m_use);
+                sum += a0 + a1;
+                pk[e] = pack2<T>(a0, a1);
+            }
+            l_run += sum;
+            uint8_t* prow = smem + L_::P + r * 64;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(prow + ((c ^ ((r >> 1) & 3)) << 4)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[M_PFULL + b]);
+        }
+        // ---- epilogue ----
+        if (ok && n_tiles > 0)
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&bars[M_ODONE + ((n_tiles - 1) & 1)], ((n_tiles - 1) >> 1) & 1, wd, 30));
+        tc_fence_after();
+        const bool has = l_run > 0.f;
+        const float inv = has ? 1.0f / l_run : 0.f;
+        const float lse = has ? (m_run + __log2f(l_run)) * kLn2 : neg_inf();
+        const int64_t qrow = qi * H + (live ? r : 0);
+        const bool split = u.nsplit > 1;
+        const int64_t slot = split ? (int64_t)u.part_base + u.split : 0;
+#pragma unroll 1
+        for (int c = 0; c < MDV / 32; ++c) {
+            uint32_t w[32];
+            if (ok && n_tiles > 0) {
+                tmem_ld32(t_o + lane_off + c * 32, w);
+                tmem_ld_wait(w);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) w[e] = 0u;
+            }
+            if (!(live && ok)) continue;
+            const int col0 = hf * MDV + c * 32;
+            if (split) {
+                float4* dst = reinterpret_cast<float4*>(p.ws_o + (slot * H + r) * MR + col0);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    dst[e] = make_float4(__uint_as_float(w[4 * e]) * inv, __uint_as_float(w[4 * e + 1]) * inv,
+                                         __uint_as_float(w[4 * e + 2]) * inv, __uint_as_float(w[4 * e + 3]) * inv);
+            } else {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<T>(__uint_as_float(w[2 * e]) * inv, __uint_as_float(w[2 * e + 1]) * inv);
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<T*>(p.out) + qrow * MR + col0);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
+        }
+        if (live && ok && hf == 0) {
+            if (split) p.ws_lse[slot * H + r] = lse;
+            else p.lse[qrow] = lse;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kMlaTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 mla_encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// Map over a row-major [d2][d1][d0] tensor of 16-bit elements, box {64, b1, b2}, 128B swizzle.
+bool mla_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1,
+             uint32_t b2) {
+    auto fn = mla_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t boxd[3] = {64, b1, b2};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base),
+              dims, strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T>
+cudaError_t mla_launch_t(const AttnParams& p, cudaStream_t st) {
+    const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+    const int ps = p.page_size;
+    const int box = ps < MBN ? ps : MBN;
+    const uint64_t rows = (uint64_t)p.num_pages * ps;
+    CUtensorMap tql, tqr, tlat, trope;
+    // Q maps: [Nq][H][R] and [Nq][H][P], one query x 128 heads x 64 columns per box
+    if (!mla_map(&tql, bf16, p.q, MR, p.hq, (uint64_t)p.num_queries, MBM, 1) ||
+        !mla_map(&tqr, bf16, p.qr, MP, p.hq, (uint64_t)p.num_queries, MBM, 1) ||
+        !mla_map(&tlat, bf16, p.k, MR, 1, rows, 1, box) || !mla_map(&trope, bf16, p.kr, MP, 1, rows, 1, box))
+        return cudaErrorInvalidValue;
+    auto kern = mla_tc_kernel<T>;
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !(configured >> dev & 1ull)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, MlaSmem::ALLOC);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured |= 1ull << dev;
+    }
+    kern<<<2 * p.num_units, kMlaThreads, MlaSmem::ALLOC, st>>>(tql, tqr, tlat, trope, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool mla_tc_supported(pa_dtype dt, int heads, int latent_dim, int rope_dim, int page_size) {
+    if (dt == PA_F32 || latent_dim != MR || rope_dim != MP || heads < 1 || heads > MBM) return false;
+    if (page_size % 16 != 0) return false;
+    if (page_size < MBN ? (MBN % page_size != 0) : (page_size % MBN != 0)) return false;
+    return true;
+}
+
+cudaError_t launch_mla_tc(const AttnParams& p, pa_dtype dt, cudaStream_t st) {
+    if (p.num_units == 0) return cudaSuccess;
+    if (dt == PA_BF16) return mla_launch_t<__nv_bfloat16>(p, st);
+    return mla_launch_t<__half>(p, st);
+}
+
+}  // namespace pa

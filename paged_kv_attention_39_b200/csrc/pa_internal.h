@@ -71,6 +71,9 @@ cudaError_t launch_combine(const AttnParams& p, pa_dtype dt, cudaStream_t st);
 cudaError_t launch_prefill_tc(const AttnParams& p, pa_dtype dt, int num_pages, cudaStream_t st);
 // Shapes the tensor-core prefill kernel takes.
 bool prefill_tc_supported(pa_dtype dt, int d, int dv, int group, int page_size);
+cudaError_t launch_mla_tc(const AttnParams& p, pa_dtype dt, cudaStream_t st);
+// Shapes the tensor-core MLA decode kernel takes (one query per sequence).
+bool mla_tc_supported(pa_dtype dt, int heads, int latent_dim, int rope_dim, int page_size);
 
 // Largest row count (queries x group heads per KV head) the tensor-core decode kernel takes.
 constexpr int kDecodeMaxRows = 16;

@@ -47,16 +47,118 @@ struct PrefillSmem {
     static constexpr int K = Q + KH * HALF_Q;
     static constexpr int V = K + KST * KH * HALF_KV;
     static constexpr int P = V + VST * KH * HALF_KV;
-    static constexpr int BAR = P + 2 * BM * 128;      // P: 128 rows x 128 keys, two halves
+    static constexpr int BAR = P + 2 * 2 * BM * 128;  // P: two buffers of 128 rows x 128 keys
     static constexpr int BYTES = BAR + 256;
     static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
 };
 
+// Barriers used once per tile in alternation come in pairs indexed by tile parity, so that no
+// waiter can ever find its barrier two phases ahead of the phase it waits for.
 enum BarId { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
              B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_SFREE = B_SFULL + 2,
-             B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + 1, B_COUNT = B_ODONE + 1 };
+             B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + 2, B_COUNT = B_ODONE + 2 };
 
 }  // namespace
+
+// ---- softmax helpers: one thread owns one row of a 128-key score tile in TMEM -------------------
+// Column c of the tile is masked when c + off_lo < 0 or c + off_hi >= 0, where off_lo = kt0 - row_lo
+// and off_hi = kt0 - row_hi (the row's visible keys are [row_lo, row_hi)).
+
+__device__ __forceinline__ float tile_max_full(uint32_t taddr) {
+    float m0 = neg_inf(), m1 = neg_inf(), m2 = neg_inf(), m3 = neg_inf();
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait(v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+            m0 = fmaxf(m0, __uint_as_float(v[e]));
+            m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+            m2 = fmaxf(m2, __uint_as_float(v[e + 2]));
+            m3 = fmaxf(m3, __uint_as_float(v[e + 3]));
+        }
+    }
+    return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+__device__ __forceinline__ float tile_max_masked(uint32_t taddr, int off_lo, int off_hi) {
+    float m0 = neg_inf(), m1 = neg_inf();
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait(v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const int k0 = c * 32 + e;
+            const float x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? __uint_as_float(v[e]) : neg_inf();
+            const float x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? __uint_as_float(v[e + 1]) : neg_inf();
+            m0 = fmaxf(m0, x0);
+            m1 = fmaxf(m1, x1);
+        }
+    }
+    return fmaxf(m0, m1);
+}
+
+// Stores 16-byte chunk `chunk` (keys 8*chunk .. +7) of row r of a K-major, 128B-swizzled P tile.
+__device__ __forceinline__ void store_p_chunk(uint8_t* prow, int r, int chunk, uint32_t a, uint32_t b, uint32_t c,
+                                              uint32_t d) {
+    const int half = chunk >> 3, cc = chunk & 7;
+    *reinterpret_cast<uint4*>(prow + half * (BM * 128) + ((cc ^ (r & 7)) << 4)) = make_uint4(a, b, c, d);
+}
+
+template <typename T>
+__device__ __forceinline__ float tile_exp_full(uint32_t taddr, float scale, float m, uint8_t* prow, int r) {
+    float s0 = 0.f, s1 = 0.f;
+    const float nm = -m;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait(v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float a0 = fast_exp2(fmaf(__uint_as_float(v[2 * e]), scale, nm));
+            const float a1 = fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), scale, nm));
+            s0 += a0;
+            s1 += a1;
+            pk[e] = pack2<T>(a0, a1);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) store_p_chunk(prow, r, c * 4 + q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+    return s0 + s1;
+}
+
+template <typename T>
+__device__ __forceinline__ float tile_exp_masked(uint32_t taddr, float scale, float m, uint8_t* prow, int r,
+                                                 int off_lo, int off_hi) {
+    float s0 = 0.f, s1 = 0.f;
+    const float nm = -m;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait(v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int k0 = c * 32 + 2 * e;
+            const bool v0 = k0 + off_lo >= 0 && k0 + off_hi < 0;
+            const bool v1 = k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0;
+            const float a0 = v0 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), scale, nm)) : 0.f;
+            const float a1 = v1 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), scale, nm)) : 0.f;
+            s0 += a0;
+            s1 += a1;
+            pk[e] = pack2<T>(a0, a1);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) store_p_chunk(prow, r, c * 4 + q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+    return s0 + s1;
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -94,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) cnt = 128;
+            if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_PFULL + 1) cnt = 128;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -189,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (i >= 1) {
                 const int j = i - 1, vs = j % VST;
-                ok = mbar_wait(&bars[B_PFULL], j & 1, wd, 6);
+                ok = mbar_wait(&bars[B_PFULL + (j & 1)], (j >> 1) & 1, wd, 6);
                 if (ok) ok = mbar_wait(&bars[B_VFULL + vs], (j / VST) & 1, wd, 7);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
@@ -208,12 +310,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint32_t pa_ = s_base + L_::P + (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+                        const uint32_t pa_ = s_base + L_::P + (j & 1) * (2 * BM * 128) + (kk >> 2) * (BM * 128) +
+                                             (kk & 3) * 32;
                         const uint32_t va = s_base + L_::V + vs * KH * L_::HALF_KV + kk * 16 * 128;
                         mma_f16_ss(t_o, sdesc_sw128(pa_, 16, 1024), sdesc_sw128(va, L_::HALF_KV, 1024), IDESC_PV,
                                    (j > 0 || kk > 0) ? 1u : 0u);
                     }
-                    mma_commit(&bars[B_ODONE]);
+                    mma_commit(&bars[B_ODONE + (j & 1)]);
                     mma_commit(&bars[B_VEMPTY + vs]);
                 }
                 __syncwarp();
@@ -225,54 +328,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const bool live = r < live_rows;
         const int64_t pos = p_first + (live ? r / G : 0);
+        // keys this row sees: [row_lo, row_hi) (padding rows: every key of the sequence)
+        const int64_t row_lo = (live && p.window > 0) ? max64(0, pos - p.window + 1) : 0;
+        const int64_t row_hi = (live && p.causal) ? min64(si.L, pos + 1) : si.L;
         // keys every live row sees: [all_lo, all_hi)
         const int64_t all_lo = p.window > 0 ? p_last - p.window + 1 : INT64_MIN;
         const int64_t all_hi = min64(p.causal ? p_first + 1 : si.L, si.L);
         float m_run = neg_inf(), l_run = 0.f;
-        uint8_t* prow = smem + L_::P + r * 128;
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const int b = i & 1;
             const int64_t kt0 = kt_start + (int64_t)i * BN;
+            const uint32_t t_sb = (b ? t_s1 : t_s0) + lane_off;
+            const bool full = kt0 >= all_lo && kt0 + BN <= all_hi;
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (i >> 1) & 1, wd, 8));
             if (!ok) break;
             tc_fence_after();
-            float s[BN];
-#pragma unroll
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32((b ? t_s1 : t_s0) + lane_off + c * 32, v);
-                tmem_ld_wait(v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(v[e]);
-            }
-            tc_fence_before();
-            mbar_arrive(&bars[B_SFREE + b]);
-
-            const bool full = kt0 >= all_lo && kt0 + BN <= all_hi;
-            float m_tile = neg_inf();
-#pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                float x = s[c] * p.scale_log2;
-                if (!full) {
-                    const int64_t t = kt0 + c;
-                    const bool vis = t < si.L && (!live || key_visible(t, pos, p.causal, p.window));
-                    x = vis ? x : neg_inf();
-                }
-                s[c] = x;
-                m_tile = fmaxf(m_tile, x);
-            }
+            // pass 1: tile max of the raw scores (S read from TMEM 32 columns at a time); the
+            // scale is positive, so it is applied to the max once. Edge tiles mask keys outside
+            // the row's visible range [row_lo, row_hi) first.
+            float m_raw;
+            if (full) m_raw = tile_max_full(t_sb);
+            else m_raw = tile_max_masked(t_sb, (int)(kt0 - row_lo), (int)(kt0 - row_hi));
+            const float m_tile = m_raw * p.scale_log2;
             const float m_new = fmaxf(m_run, m_tile);
-            if (i > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE], (i - 1) & 1, wd, 9));
-                if (!ok) break;
-            }
             const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
             const bool rescale = grow && i > 0 && m_run != neg_inf();
             if (__any_sync(0xffffffffu, rescale)) {
+                // the output must hold every earlier tile before it is rescaled
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 9));
+                if (!ok) break;
                 tc_fence_after();
                 const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t v[32];
                     tmem_ld32(t_o + lane_off + c * 32, v);
@@ -288,29 +376,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m_run = m_new;
             }
             const float m_use = m_run == neg_inf() ? 0.f : m_run;
-            float sum = 0.f;
-#pragma unroll
-            for (int c = 0; c < BN / 8; ++c) {  // 16-byte chunk c holds keys 8c .. 8c+7
-                uint32_t pk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a = fast_exp2(s[c * 8 + 2 * e] - m_use);
-                    const float bb = fast_exp2(s[c * 8 + 2 * e + 1] - m_use);
-                    sum += a + bb;
-                    pk[e] = pack2<T>(a, bb);
-                }
-                const int half = c >> 3, cc = c & 7;
-                *reinterpret_cast<uint4*>(prow + half * (BM * 128) + ((cc ^ (r & 7)) << 4)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            // P buffer b was last read by P V of tile i - 2
+            if (i >= 2) {
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((i - 2) >> 1) & 1, wd, 11));
+                if (!ok) break;
             }
+            // pass 2: probabilities p = 2^(s * scale - m), 16-bit, into the swizzled K-major P tile
+            uint8_t* prow = smem + L_::P + b * (2 * BM * 128) + r * 128;
+            const float sum = full ? tile_exp_full<T>(t_sb, p.scale_log2, m_use, prow, r)
+                                   : tile_exp_masked<T>(t_sb, p.scale_log2, m_use, prow, r, (int)(kt0 - row_lo),
+                                                        (int)(kt0 - row_hi));
+            tc_fence_before();
+            mbar_arrive(&bars[B_SFREE + b]);  // S buffer b may be overwritten
             l_run += sum;
             fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[B_PFULL]);
+            mbar_arrive(&bars[B_PFULL + b]);
         }
         // ---- epilogue ----
         if (ok && n_tiles > 0)
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE], (n_tiles - 1) & 1, wd, 10));
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(&bars[B_ODONE + ((n_tiles - 1) & 1)], ((n_tiles - 1) >> 1) & 1, wd, 10));
         tc_fence_after();
         const bool has = l_run > 0.f;
         const float inv = has ? 1.0f / l_run : 0.f;

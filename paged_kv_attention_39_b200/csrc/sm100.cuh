@@ -37,6 +37,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait with a suspend-time hint: the thread may sleep up to `hint_ns` unless the phase
+// completes first.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
@@ -54,13 +65,15 @@ struct Watchdog {
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Watchdog& w, int code) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        if (*w.abort_flag) return false;
-        if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > w.limit_ns) {
-            *w.abort_flag = 1;
-            if (w.err) atomicCAS(w.err, 0, code);
-            return false;
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if ((it & 7) == 0) {  // the clock and the abort flag are checked now and then only
+            if (*w.abort_flag) return false;
+            if (globaltimer_ns() - t0 > w.limit_ns) {
+                *w.abort_flag = 1;
+                if (w.err) atomicCAS(w.err, 0, code);
+                return false;
+            }
         }
     }
 }
