@@ -118,36 +118,50 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
     if (warp == 4) {
         // ===================== TMA producer =====================
-        if (lane == 0 && n_tiles > 0) {
-            tma_prefetch(&tm_ql);
-            tma_prefetch(&tm_qr);
-            tma_prefetch(&tm_lat);
-            tma_prefetch(&tm_rope);
-            mbar_arrive_expect_tx(&bars[M_QFULL], MC * L_::Q_COL);
-            for (int c = 0; c < MC - 1; ++c)
-                tma_load_3d(smem + L_::Q + c * L_::Q_COL, &tm_ql, &bars[M_QFULL], c * 64, 0, (int)qi);
-            tma_load_3d(smem + L_::Q + (MC - 1) * L_::Q_COL, &tm_qr, &bars[M_QFULL], 0, 0, (int)qi);
+        // Whole warp in the loop, lane 0 issues; page ids of the next 32 boxes come from one
+        // lane-parallel block-table read.
+        if (n_tiles > 0) {
+            if (lane == 0) {
+                tma_prefetch(&tm_ql);
+                tma_prefetch(&tm_qr);
+                tma_prefetch(&tm_lat);
+                tma_prefetch(&tm_rope);
+                mbar_arrive_expect_tx(&bars[M_QFULL], MC * L_::Q_COL);
+                for (int c = 0; c < MC - 1; ++c)
+                    tma_load_3d(smem + L_::Q + c * L_::Q_COL, &tm_ql, &bars[M_QFULL], c * 64, 0, (int)qi);
+                tma_load_3d(smem + L_::Q + (MC - 1) * L_::Q_COL, &tm_qr, &bars[M_QFULL], 0, 0, (int)qi);
+            }
             const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+            const int bpt = MBN / box;
+            int base_g = -(1 << 30), my_row = 0;
             int issued = 0;
             for (int i = 0; i < n_tiles; ++i) {
                 const int64_t kt0 = kt_start + (int64_t)i * MBN;
                 int nb = 0;
-                for (int b = 0; b < MBN / box; ++b)
+                for (int b = 0; b < bpt; ++b)
                     if (kt0 + (int64_t)b * box < si.L) nb = b + 1;
+                const int g0 = i * bpt;
+                if (g0 + nb > base_g + 32) {
+                    base_g = g0;
+                    const int64_t key = kt_start + (int64_t)(base_g + lane) * box;
+                    my_row = key < si.L ? (int)((int64_t)bt[key / ps] * ps + key % ps) : 0;
+                }
                 const int st = i % MST;
-                if (i >= MST && !mbar_wait(&bars[M_EMPTY + st], ((i / MST) - 1) & 1, wd, 21)) break;
-                mbar_arrive_expect_tx(&bars[M_FULL + st], (uint32_t)nb * box * 128 * MC);
+                if (i >= MST && !__all_sync(0xffffffffu, mbar_wait(&bars[M_EMPTY + st], ((i / MST) - 1) & 1, wd, 21)))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(&bars[M_FULL + st], (uint32_t)nb * box * 128 * MC);
                 uint8_t* dst = smem + L_::KV + st * MC * L_::KV_COL;
                 for (int b = 0; b < nb; ++b) {
-                    const int64_t key = kt0 + (int64_t)b * box;
-                    const int row = (int)((int64_t)bt[key / ps] * ps + key % ps);
-                    for (int c = 0; c < MC - 1; ++c)
-                        tma_load_3d(dst + c * L_::KV_COL + b * box * 128, &tm_lat, &bars[M_FULL + st], c * 64, 0, row);
-                    tma_load_3d(dst + (MC - 1) * L_::KV_COL + b * box * 128, &tm_rope, &bars[M_FULL + st], 0, 0, row);
+                    const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
+                    if (lane == 0) {
+                        for (int c = 0; c < MC - 1; ++c)
+                            tma_load_3d(dst + c * L_::KV_COL + b * box * 128, &tm_lat, &bars[M_FULL + st], c * 64, 0, row);
+                        tma_load_3d(dst + (MC - 1) * L_::KV_COL + b * box * 128, &tm_rope, &bars[M_FULL + st], 0, 0, row);
+                    }
                 }
                 issued = i + 1;
             }
-            if (*abort_flag) {
+            if (lane == 0 && *abort_flag) {
                 const uint64_t t0 = globaltimer_ns();
                 auto drain = [&](uint64_t* bar, uint32_t parity) {
                     while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kMlaWaitNs) {}
@@ -158,6 +172,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
     } else if (warp == 5) {
         // ===================== MMA issuer =====================
+        const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
+        const uint64_t dKV = sdesc_sw128(s_base + L_::KV, 16, 1024);
+        const uint64_t dV = sdesc_sw128(s_base + L_::KV, L_::KV_COL, 1024);
+        const uint64_t dP = sdesc_sw64(s_base + L_::P, 512);
         bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[M_QFULL], 0, wd, 23));
         for (int i = 0; ok && i <= n_tiles; ++i) {
             if (i < n_tiles) {
@@ -179,14 +197,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t kv = s_base + L_::KV + st * MC * L_::KV_COL;
-#pragma unroll 4
-                    for (int kk = 0; kk < MK / 16; ++kk) {
-                        const uint32_t qa = s_base + L_::Q + (kk >> 2) * L_::Q_COL + (kk & 3) * 32;
-                        const uint32_t ka = kv + (kk >> 2) * L_::KV_COL + (kk & 3) * 32;
-                        mma_f16_ss(b ? t_s1 : t_s0, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), IDESC_QK,
-                                   kk > 0);
-                    }
+                    const uint32_t d_s = b ? t_s1 : t_s0;
+                    const uint64_t dKst = desc_add(dKV, st * MC * L_::KV_COL);
+#pragma unroll
+                    for (int kk = 0; kk < MK / 16; ++kk)
+                        mma_f16_ss(d_s, desc_add(dQ, (kk >> 2) * L_::Q_COL + (kk & 3) * 32),
+                                   desc_add(dKst, (kk >> 2) * L_::KV_COL + (kk & 3) * 32), IDESC_QK, kk > 0);
                     mma_commit(&bars[M_SFULL + b]);
                 }
                 __syncwarp();
@@ -197,14 +213,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t vbase = s_base + L_::KV + (st * MC + hf * (MDV / 64)) * L_::KV_COL;
+                    const uint64_t dVs = desc_add(dV, (st * MC + hf * (MDV / 64)) * L_::KV_COL);
+                    const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < MBN / 16; ++kk) {
-                        const uint32_t pa_ = s_base + L_::P + kk * 32;
-                        const uint32_t va = vbase + kk * 16 * 128;
-                        mma_f16_ss(t_o, sdesc_sw64(pa_, 512), sdesc_sw128(va, L_::KV_COL, 1024), IDESC_PV,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < MBN / 16; ++kk)
+                        mma_f16_ss(t_o, desc_add(dP, kk * 32), desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
                     mma_commit(&bars[M_ODONE + (j & 1)]);
                     mma_commit(&bars[M_EMPTY + st]);
                 }
@@ -216,6 +229,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         const int r = tid;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const bool live = r < H;
+        const int64_t vis_lo = p.window > 0 ? max64(u.t0, pos - p.window + 1) : u.t0;
+        const int64_t vis_hi = p.causal ? min64(u.t1, pos + 1) : u.t1;
         float m_run = neg_inf(), l_run = 0.f;
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
@@ -229,20 +244,29 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             tmem_ld_wait(v);
             tc_fence_before();
             mbar_arrive(&bars[M_SFREE + b]);
-            const bool full = kt0 >= u.t0 && kt0 + MBN <= u.t1;
-            float x[32];
-            float m_tile = neg_inf();
+            // keys of this unit the query sees: [vis_lo, vis_hi), the same for every head
+            const bool full = kt0 >= vis_lo && kt0 + MBN <= vis_hi;
+            const int off_lo = (int)(kt0 - vis_lo), off_hi = (int)(kt0 - vis_hi);
+            float m0 = neg_inf(), m1 = neg_inf();
+            if (full) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                float y = __uint_as_float(v[e]) * p.scale_log2;
-                if (!full) {
-                    const int64_t t = kt0 + e;
-                    const bool vis = t >= u.t0 && t < u.t1 && key_visible(t, pos, p.causal, p.window);
-                    y = vis ? y : neg_inf();
+                for (int e = 0; e < 32; e += 2) {
+                    m0 = fmaxf(m0, __uint_as_float(v[e]));
+                    m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
                 }
-                x[e] = y;
-                m_tile = fmaxf(m_tile, y);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const bool vis = e + off_lo >= 0 && e + off_hi < 0;
+                    v[e] = vis ? v[e] : __float_as_uint(neg_inf());
+                }
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    m0 = fmaxf(m0, __uint_as_float(v[e]));
+                    m1 = fmaxf(m1, __uint_as_float(v[e + 1]));
+                }
             }
+            const float m_tile = fmaxf(m0, m1) * p.scale_log2;  // scale > 0 commutes with the max
             const float m_new = fmaxf(m_run, m_tile);
             const bool grow = m_new > m_run + 8.0f;
             const bool rescale = grow && i > 0 && m_run != neg_inf();
@@ -269,17 +293,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 l_run *= fast_exp2(m_run - m_new);
                 m_run = m_new;
             }
-            const float m_use = m_run == neg_inf() ? 0.f : m_run;
+            const float nm = -(m_run == neg_inf() ? 0.f : m_run);
             uint32_t pk[16];
-            float sum = 0.f;
+            float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const float a0 = fast_exp2(x[2 * e] - m_use);
-                const float a1 = fast_exp2(x[2 * e + 1] - m_use);
-                sum += a0 + a1;
+            for (int e = 0; e < 16; ++e) {  // masked scores are -inf: exp2 gives 0
+                const float a0 = fast_exp2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, nm));
+                const float a1 = fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, nm));
+                s0 += a0;
+                s1 += a1;
                 pk[e] = pack2<T>(a0, a1);
             }
-            l_run += sum;
+            l_run += s0 + s1;
             uint8_t* prow = smem + L_::P + r * 64;
 #pragma unroll
             for (int c = 0; c < 4; ++c)

@@ -160,6 +160,43 @@ __device__ __forceinline__ float tile_exp_masked(uint32_t taddr, float scale, fl
     return s0 + s1;
 }
 
+// One pass over the tile with the row's running max m (known finite): probabilities relative to m
+// go straight to the P tile while the tile max of the raw scores is tracked; the caller keeps
+// them when the max grew by at most 2^8 (so p <= 256), and otherwise redoes the tile.
+template <typename T, bool MASKED>
+__device__ __forceinline__ float tile_fused(uint32_t taddr, float scale, float m, uint8_t* prow, int r, int off_lo,
+                                            int off_hi, float& m_raw) {
+    float s0 = 0.f, s1 = 0.f, m0 = neg_inf(), m1 = neg_inf();
+    const float nm = -m;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait(v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+            if (MASKED) {
+                const int k0 = c * 32 + 2 * e;
+                x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? x0 : neg_inf();
+                x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? x1 : neg_inf();
+            }
+            m0 = fmaxf(m0, x0);
+            m1 = fmaxf(m1, x1);
+            const float a0 = fast_exp2(fmaf(x0, scale, nm));
+            const float a1 = fast_exp2(fmaf(x1, scale, nm));
+            s0 += a0;
+            s1 += a1;
+            pk[e] = pack2<T>(a0, a1);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) store_p_chunk(prow, r, c * 4 + q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+    m_raw = fmaxf(m0, m1);
+    return s0 + s1;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -217,44 +254,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 4) {
         // ===================== TMA producer =====================
-        if (lane == 0 && n_tiles > 0) {
-            tma_prefetch(&tmq);
-            tma_prefetch(&tmk);
-            tma_prefetch(&tmv);
-            mbar_arrive_expect_tx(&bars[B_QFULL], KH * L_::HALF_Q);
-            for (int h = 0; h < KH; ++h)
-                tma_load_3d(smem + L_::Q + h * L_::HALF_Q, &tmq, &bars[B_QFULL], h * 64, u.kvh * G,
-                            si.q_start + u.j0);
+        // The whole warp runs the loop; lane 0 issues. Page ids of the next 32 boxes are read
+        // from the block table by the 32 lanes at once and handed to lane 0 by shuffles, so a
+        // table read never sits between two loads.
+        if (n_tiles > 0) {
+            if (lane == 0) {
+                tma_prefetch(&tmq);
+                tma_prefetch(&tmk);
+                tma_prefetch(&tmv);
+                mbar_arrive_expect_tx(&bars[B_QFULL], KH * L_::HALF_Q);
+                for (int h = 0; h < KH; ++h)
+                    tma_load_3d(smem + L_::Q + h * L_::HALF_Q, &tmq, &bars[B_QFULL], h * 64, u.kvh * G,
+                                si.q_start + u.j0);
+            }
             const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
-            int issued = 0;  // tiles whose K and V loads were issued
+            const int bpt = BN / box;  // boxes per tile (<= 8)
+            int base_g = -(1 << 30);   // first box whose page id the lanes hold
+            int my_row = 0;            // lane l: first cache row of box base_g + l
+            int issued = 0;            // tiles whose K and V loads were issued
             for (int i = 0; i < n_tiles; ++i) {
                 const int64_t kt0 = kt_start + (int64_t)i * BN;
                 int nb = 0;  // boxes whose first key lies inside the sequence
-                for (int b = 0; b < BN / box; ++b)
+                for (int b = 0; b < bpt; ++b)
                     if (kt0 + (int64_t)b * box < si.L) nb = b + 1;
+                const int g0 = i * bpt;
+                if (g0 + nb > base_g + 32) {
+                    base_g = g0;
+                    const int64_t key = kt_start + (int64_t)(base_g + lane) * box;
+                    my_row = key < si.L ? (int)((int64_t)bt[key / ps] * ps + key % ps) : 0;
+                }
                 const uint32_t bytes = (uint32_t)nb * box * 128 * KH;
                 const int ks = i % KST, vs = i % VST;
-                if (i >= KST && !mbar_wait(&bars[B_KEMPTY + ks], ((i / KST) - 1) & 1, wd, 1)) break;
-                mbar_arrive_expect_tx(&bars[B_KFULL + ks], bytes);
+                if (i >= KST && !__all_sync(0xffffffffu, mbar_wait(&bars[B_KEMPTY + ks], ((i / KST) - 1) & 1, wd, 1)))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(&bars[B_KFULL + ks], bytes);
                 for (int b = 0; b < nb; ++b) {
-                    const int64_t key = kt0 + (int64_t)b * box;
-                    const int row = (int)((int64_t)bt[key / ps] * ps + key % ps);
-                    for (int h = 0; h < KH; ++h)
-                        tma_load_3d(smem + L_::K + (ks * KH + h) * L_::HALF_KV + b * box * 128, &tmk,
-                                    &bars[B_KFULL + ks], h * 64, u.kvh, row);
+                    const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
+                    if (lane == 0)
+                        for (int h = 0; h < KH; ++h)
+                            tma_load_3d(smem + L_::K + (ks * KH + h) * L_::HALF_KV + b * box * 128, &tmk,
+                                        &bars[B_KFULL + ks], h * 64, u.kvh, row);
                 }
-                if (i >= VST && !mbar_wait(&bars[B_VEMPTY + vs], ((i / VST) - 1) & 1, wd, 2)) break;
-                mbar_arrive_expect_tx(&bars[B_VFULL + vs], bytes);
+                if (i >= VST && !__all_sync(0xffffffffu, mbar_wait(&bars[B_VEMPTY + vs], ((i / VST) - 1) & 1, wd, 2)))
+                    break;
+                if (lane == 0) mbar_arrive_expect_tx(&bars[B_VFULL + vs], bytes);
                 for (int b = 0; b < nb; ++b) {
-                    const int64_t key = kt0 + (int64_t)b * box;
-                    const int row = (int)((int64_t)bt[key / ps] * ps + key % ps);
-                    for (int h = 0; h < KH; ++h)
-                        tma_load_3d(smem + L_::V + (vs * KH + h) * L_::HALF_KV + b * box * 128, &tmv,
-                                    &bars[B_VFULL + vs], h * 64, u.kvh, row);
+                    const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
+                    if (lane == 0)
+                        for (int h = 0; h < KH; ++h)
+                            tma_load_3d(smem + L_::V + (vs * KH + h) * L_::HALF_KV + b * box * 128, &tmv,
+                                        &bars[B_VFULL + vs], h * 64, u.kvh, row);
                 }
                 issued = i + 1;
             }
-            if (*abort_flag) {
+            if (lane == 0 && *abort_flag) {
                 // Leave no copy in flight into this CTA's shared memory: wait (bounded, ignoring
                 // the abort flag) for the last loads issued into each stage and for Q.
                 const uint64_t t0 = globaltimer_ns();
@@ -268,6 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 5) {
         // ===================== MMA issuer =====================
+        // Descriptors are built once; a k-step or stage offset is an add to the address field.
+        const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
+        const uint64_t dK = sdesc_sw128(s_base + L_::K, 16, 1024);
+        const uint64_t dP = sdesc_sw128(s_base + L_::P, 16, 1024);
+        const uint64_t dV = sdesc_sw128(s_base + L_::V, L_::HALF_KV, 1024);
         bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[B_QFULL], 0, wd, 3));
         for (int i = 0; ok && i <= n_tiles; ++i) {
             if (i < n_tiles) {
@@ -278,11 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
+                    const uint32_t d_s = b ? t_s1 : t_s0;
+                    const uint64_t dKs = desc_add(dK, ks * KH * L_::HALF_KV);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t qa = s_base + L_::Q + (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;
-                        const uint32_t ka = s_base + L_::K + (ks * KH + (kk >> 2)) * L_::HALF_KV + (kk & 3) * 32;
-                        mma_f16_ss(b ? t_s1 : t_s0, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), IDESC_QK, kk > 0);
+                        const uint32_t off = (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;  // HALF_Q == HALF_KV
+                        mma_f16_ss(d_s, desc_add(dQ, off), desc_add(dKs, off), IDESC_QK, kk > 0);
                     }
                     mma_commit(&bars[B_SFULL + b]);
                     mma_commit(&bars[B_KEMPTY + ks]);
@@ -308,14 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
+                    const uint64_t dPj = desc_add(dP, (j & 1) * (2 * BM * 128));
+                    const uint64_t dVs = desc_add(dV, vs * KH * L_::HALF_KV);
+                    const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk) {
-                        const uint32_t pa_ = s_base + L_::P + (j & 1) * (2 * BM * 128) + (kk >> 2) * (BM * 128) +
-                                             (kk & 3) * 32;
-                        const uint32_t va = s_base + L_::V + vs * KH * L_::HALF_KV + kk * 16 * 128;
-                        mma_f16_ss(t_o, sdesc_sw128(pa_, 16, 1024), sdesc_sw128(va, L_::HALF_KV, 1024), IDESC_PV,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < BN / 16; ++kk)
+                        mma_f16_ss(t_o, desc_add(dPj, (kk >> 2) * (BM * 128) + (kk & 3) * 32),
+                                   desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
                     mma_commit(&bars[B_ODONE + (j & 1)]);
                     mma_commit(&bars[B_VEMPTY + vs]);
                 }
@@ -344,48 +402,57 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (i >> 1) & 1, wd, 8));
             if (!ok) break;
             tc_fence_after();
-            // pass 1: tile max of the raw scores (S read from TMEM 32 columns at a time); the
-            // scale is positive, so it is applied to the max once. Edge tiles mask keys outside
-            // the row's visible range [row_lo, row_hi) first.
-            float m_raw;
-            if (full) m_raw = tile_max_full(t_sb);
-            else m_raw = tile_max_masked(t_sb, (int)(kt0 - row_lo), (int)(kt0 - row_hi));
-            const float m_tile = m_raw * p.scale_log2;
-            const float m_new = fmaxf(m_run, m_tile);
-            const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
-            const bool rescale = grow && i > 0 && m_run != neg_inf();
-            if (__any_sync(0xffffffffu, rescale)) {
-                // the output must hold every earlier tile before it is rescaled
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 9));
-                if (!ok) break;
-                tc_fence_after();
-                const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(t_o + lane_off + c * 32, v);
-                    tmem_ld_wait(v);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                    tmem_st32(t_o + lane_off + c * 32, v);
-                }
-                tmem_st_wait();
-            }
-            if (grow) {
-                l_run *= fast_exp2(m_run - m_new);
-                m_run = m_new;
-            }
-            const float m_use = m_run == neg_inf() ? 0.f : m_run;
             // P buffer b was last read by P V of tile i - 2
             if (i >= 2) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((i - 2) >> 1) & 1, wd, 11));
                 if (!ok) break;
             }
-            // pass 2: probabilities p = 2^(s * scale - m), 16-bit, into the swizzled K-major P tile
             uint8_t* prow = smem + L_::P + b * (2 * BM * 128) + r * 128;
-            const float sum = full ? tile_exp_full<T>(t_sb, p.scale_log2, m_use, prow, r)
-                                   : tile_exp_masked<T>(t_sb, p.scale_log2, m_use, prow, r, (int)(kt0 - row_lo),
-                                                        (int)(kt0 - row_hi));
+            const int off_lo = (int)(kt0 - row_lo), off_hi = (int)(kt0 - row_hi);
+            // Fast path: one pass with the running max when every row of the warp has one.
+            bool redo = true;
+            float sum = 0.f;
+            if (__all_sync(0xffffffffu, m_run != neg_inf())) {
+                float m_raw;
+                sum = full ? tile_fused<T, false>(t_sb, p.scale_log2, m_run, prow, r, 0, 0, m_raw)
+                           : tile_fused<T, true>(t_sb, p.scale_log2, m_run, prow, r, off_lo, off_hi, m_raw);
+                redo = __any_sync(0xffffffffu, m_raw * p.scale_log2 > m_run + 8.0f);
+            }
+            if (redo) {
+                // pass 1: tile max of the raw scores (S read from TMEM 32 columns at a time); the
+                // scale is positive, so it is applied to the max once. Edge tiles mask keys
+                // outside the row's visible range [row_lo, row_hi) first.
+                const float m_raw = full ? tile_max_full(t_sb) : tile_max_masked(t_sb, off_lo, off_hi);
+                const float m_tile = m_raw * p.scale_log2;
+                const float m_new = fmaxf(m_run, m_tile);
+                const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
+                const bool rescale = grow && i > 0 && m_run != neg_inf();
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // the output must hold every earlier tile before it is rescaled
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 9));
+                    if (!ok) break;
+                    tc_fence_after();
+                    const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t v[32];
+                        tmem_ld32(t_o + lane_off + c * 32, v);
+                        tmem_ld_wait(v);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                        tmem_st32(t_o + lane_off + c * 32, v);
+                    }
+                    tmem_st_wait();
+                }
+                if (grow) {
+                    l_run *= fast_exp2(m_run - m_new);
+                    m_run = m_new;
+                }
+                const float m_use = m_run == neg_inf() ? 0.f : m_run;
+                // pass 2: probabilities p = 2^(s * scale - m), 16-bit, into the swizzled K-major P tile
+                sum = full ? tile_exp_full<T>(t_sb, p.scale_log2, m_use, prow, r)
+                           : tile_exp_masked<T>(t_sb, p.scale_log2, m_use, prow, r, off_lo, off_hi);
+            }
             tc_fence_before();
             mbar_arrive(&bars[B_SFREE + b]);  // S buffer b may be overwritten
             l_run += sum;

@@ -170,6 +170,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     return d;
 }
 
+// Descriptor of the same layout `bytes` further on (the start-address field holds address / 16;
+// shared-memory addresses stay below 2^18, so the add never carries out of the field).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 // Instruction descriptor of kind::f16: float32 accumulator, A and B both bf16 (or both f16),
 // A/B K-major (0) or MN-major (1), shape M x N.
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool a_mn, bool b_mn) {
