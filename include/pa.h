@@ -189,6 +189,30 @@ pa_status pa_mla_forward_ex(pa_plan* plan, const void* q_latent, const void* q_r
                             const pa_forward_options* opts);
 
 /*
+ * pa_append -- write each query row's new key and value into its cache slot (ruDNN
+ * `DevicePlan::append`; the step that precedes attention). Query j of sequence s sits at
+ * absolute position p = L_s - n_s + j, so its rows go to page block_tables[s][p / page_size],
+ * slot p % page_size:
+ *   k_cache[page, slot, h, :] = new_k[q, h, :]   and   v_cache[page, slot, h, :] = new_v[q, h, :]
+ *
+ *   new_k   [N_q, num_kv_heads, head_dim]   dtype (read)
+ *   new_v   [N_q, num_kv_heads, v_head_dim] dtype (read)
+ *   k_cache [num_pages, page_size, num_kv_heads, head_dim]   (written in place)
+ *   v_cache [num_pages, page_size, num_kv_heads, v_head_dim] (written in place)
+ * MLA: pass the new latent rows as new_k with the latent cache, and the new rope rows as new_v
+ * with the rope cache (num_kv_heads = 1).
+ *
+ * Rows must be multiples of 16 bytes (PA_ERR_UNSUPPORTED otherwise). The caches must not
+ * overlap each other or the new rows (PA_ERR_ALIAS), and no two query rows of the plan may map
+ * to one slot (PA_ERR_ALIAS; checked once per plan on the host). The caller owns the caches:
+ * this call does not copy shared pages (ruDNN's copy-on-write decision belongs to the caller's
+ * page allocator here). Stream-ordered, no host synchronisation.
+ */
+pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k_cache, void* v_cache,
+                    pa_dtype dtype, int32_t num_kv_heads, int32_t head_dim, int32_t v_head_dim,
+                    pa_stream stream);
+
+/*
  * pa_forward_static_workspace -- pa_forward's split-KV decode without any memory allocation.
  * The pages describe no such call: it exists for callers that cannot allocate device memory
  * while they run attention (a serving loop that must not stall on the allocator mid-step, a

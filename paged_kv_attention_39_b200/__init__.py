@@ -29,7 +29,7 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
           "PA_ERR_ALIAS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA"]
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
-           "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex",
+           "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex", "pa_append",
            "pa_plan_device_status",
            "pa_status_string", "pa_last_error_message", "pa_version"]
 
@@ -91,6 +91,8 @@ def load_library(path: Optional[str] = None):
     lib.pa_forward_static_workspace.restype = ctypes.c_int
     lib.pa_forward_static_workspace.argtypes = [_P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _I, ctypes.c_float,
                                                 ctypes.c_int, _I, _I, _P, _P, _P]
+    lib.pa_append.restype = ctypes.c_int
+    lib.pa_append.argtypes = [_P, _P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _P]
     lib.pa_plan_device_status.restype = ctypes.c_int
     lib.pa_plan_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -240,6 +242,17 @@ def pa_forward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _DTYPES[q.dtype], q.shape[1],
         k_cache.shape[2], q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window),
         _ptr(out), _ptr(lse), _stream_ptr(stream, plan.device), _opts(kv_chunk, path, trace)))
+
+
+def pa_append(plan: Plan, new_k: torch.Tensor, new_v: torch.Tensor, k_cache: torch.Tensor,
+              v_cache: torch.Tensor, stream=None) -> None:
+    """Write new_k [Nq, Hkv, D] / new_v [Nq, Hkv, Dv] into the plan's cache slots (in place)."""
+    for t in (new_k, new_v, k_cache, v_cache):
+        if not t.is_contiguous():
+            raise ValueError("pa_append takes contiguous tensors")
+    _check(load_library().pa_append(plan.handle, _ptr(new_k), _ptr(new_v), _ptr(k_cache), _ptr(v_cache),
+                                    _DTYPES[new_k.dtype], k_cache.shape[2], k_cache.shape[3], v_cache.shape[3],
+                                    _stream_ptr(stream, plan.device)))
 
 
 def pa_forward_static_workspace(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor,

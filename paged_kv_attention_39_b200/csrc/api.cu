@@ -94,6 +94,8 @@ struct pa_plan {
     pa::SeqInfo* d_seqs = nullptr;
     int32_t* d_bt = nullptr;
     int* d_err = nullptr;  // kernels' error word (bounded waits that ran out)
+    int32_t* d_q2seq = nullptr;  // sequence of each packed query row
+    int writes_checked = 0;      // 0 unknown, 1 every query row owns a distinct cache slot, -1 not
     std::vector<std::unique_ptr<Schedule>> scheds;  // most recent last
     float* ws = nullptr;
     size_t ws_bytes = 0;
@@ -566,11 +568,17 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
         PA_CUDA_TRY(cudaDeviceGetAttribute(&P->num_sms, cudaDevAttrMultiProcessorCount, device));
         const size_t seq_bytes = ((sizeof(pa::SeqInfo) * num_seqs + 255) / 256) * 256;
         const size_t bt_bytes = ((sizeof(int32_t) * (size_t)bt_elems + 255) / 256) * 256;
-        const size_t total = seq_bytes + bt_bytes + 256;  // + the error word
+        const size_t q2s_bytes = ((sizeof(int32_t) * (size_t)nq + 255) / 256) * 256;
+        const size_t total = seq_bytes + bt_bytes + 256 + q2s_bytes;  // + the error word + query->sequence
         std::vector<char>& blob = P->meta_host;  // kept alive for the asynchronous copy
         blob.assign(total, 0);
         if (num_seqs) std::memcpy(blob.data(), P->seqs.data(), sizeof(pa::SeqInfo) * num_seqs);
-        if (bt_elems) std::memcpy(blob.data() + seq_bytes, P->bt.data(), bt_bytes);
+        if (bt_elems) std::memcpy(blob.data() + seq_bytes, P->bt.data(), sizeof(int32_t) * (size_t)bt_elems);
+        {
+            int32_t* q2s = reinterpret_cast<int32_t*>(blob.data() + seq_bytes + bt_bytes + 256);
+            for (int32_t s = 0; s < num_seqs; ++s)
+                for (int32_t q = query_offsets[s]; q < query_offsets[s + 1]; ++q) q2s[q] = s;
+        }
         PA_CUDA_TRY(cudaMallocAsync(&P->d_meta, total, (cudaStream_t)upload_stream));
         cudaError_t e = cudaMemcpyAsync(P->d_meta, blob.data(), total, cudaMemcpyHostToDevice,
                                         (cudaStream_t)upload_stream);
@@ -583,6 +591,7 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
         P->d_seqs = (pa::SeqInfo*)P->d_meta;
         P->d_bt = (int32_t*)((char*)P->d_meta + seq_bytes);
         P->d_err = (int*)((char*)P->d_meta + seq_bytes + bt_bytes);
+        P->d_q2seq = (int32_t*)((char*)P->d_meta + seq_bytes + bt_bytes + 256);
     }
     *out_plan = P.release();
     return ok();
@@ -700,6 +709,61 @@ pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_
         st = ensure_workspace(plan, (size_t)S->slots * key.hq * (key.dv + 1) * sizeof(float), (cudaStream_t)stream);
         if (st != PA_OK) return st;
     }
+    return ok();
+}
+
+pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k_cache, void* v_cache,
+                    pa_dtype dtype, int32_t num_kv_heads, int32_t head_dim, int32_t v_head_dim, pa_stream stream) {
+    if (!plan) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return fail(PA_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+    if (num_kv_heads <= 0 || head_dim <= 0 || v_head_dim <= 0)
+        return fail(PA_ERR_SHAPE, "kv heads and head dims must be positive");
+    if (head_dim > 1024 || v_head_dim > 1024) return fail(PA_ERR_UNSUPPORTED, "head dims above 1024 are not supported");
+    const int64_t es = (int64_t)dtype_size(dtype);
+    const int64_t kb = head_dim * es, vb = v_head_dim * es;
+    if (kb % 16 || vb % 16) return fail(PA_ERR_UNSUPPORTED, "rows must be multiples of 16 bytes (head_dim * element size)");
+    int64_t n_new_k, n_new_v, n_k, n_v;
+    if (!product({plan->Nq, num_kv_heads, kb}, &n_new_k) || !product({plan->Nq, num_kv_heads, vb}, &n_new_v) ||
+        !product({plan->num_pages, plan->page_size, num_kv_heads, kb}, &n_k) ||
+        !product({plan->num_pages, plan->page_size, num_kv_heads, vb}, &n_v))
+        return fail(PA_ERR_BOUNDS, "tensor size overflows 64-bit byte counts");
+    if (plan->Nq == 0) return ok();
+    if (!new_k || !new_v || !k_cache || !v_cache) return fail(PA_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    for (const void* ptr : {new_k, new_v, (const void*)k_cache, (const void*)v_cache})
+        if ((uintptr_t)ptr % 16 != 0) return fail(PA_ERR_INVALID_ARGUMENT, "device pointers must be 16-byte aligned");
+    auto R = [](const void* p, int64_t n) { return Range{(uintptr_t)p, (uintptr_t)p + (uintptr_t)n}; };
+    const Range rk = R(k_cache, n_k), rv = R(v_cache, n_v), rnk = R(new_k, n_new_k), rnv = R(new_v, n_new_v);
+    if (overlap(rk, rv)) return fail(PA_ERR_ALIAS, "k_cache and v_cache overlap");
+    if (overlap(rk, rnk) || overlap(rk, rnv) || overlap(rv, rnk) || overlap(rv, rnv))
+        return fail(PA_ERR_ALIAS, "new rows overlap a cache");
+    // Every query row must own a distinct cache slot, or two rows would race for one slot
+    // (e.g. sequences sharing a prefix page). Checked once per plan.
+    if (plan->writes_checked == 0) {
+        std::vector<int64_t> slots;
+        slots.reserve((size_t)plan->Nq);
+        for (int32_t s = 0; s < plan->S; ++s) {
+            const pa::SeqInfo& si = plan->seqs[s];
+            for (int32_t j = 0; j < si.n; ++j) {
+                const int64_t pos = (int64_t)si.L - si.n + j;
+                slots.push_back((int64_t)plan->bt[(int64_t)s * plan->table_width + pos / plan->page_size] * plan->page_size +
+                                pos % plan->page_size);
+            }
+        }
+        std::sort(slots.begin(), slots.end());
+        plan->writes_checked = std::adjacent_find(slots.begin(), slots.end()) == slots.end() ? 1 : -1;
+    }
+    if (plan->writes_checked < 0) return fail(PA_ERR_ALIAS, "two query rows of the plan map to the same cache slot");
+    if (plan->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to run on");
+    int cur = -1;
+    PA_CUDA_TRY(cudaGetDevice(&cur));
+    if (cur != plan->device)
+        return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
+    cudaError_t e = pa::launch_append(new_k, new_v, k_cache, v_cache, plan->d_seqs, plan->d_q2seq, plan->d_bt,
+                                      plan->table_width, plan->page_size, num_kv_heads, (int32_t)kb, (int32_t)vb,
+                                      (int64_t)plan->Nq * num_kv_heads, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "append kernel launch failed: %s", cudaGetErrorString(e));
+    plan->last_stream = (cudaStream_t)stream;
+    plan->last_launches = 1;
     return ok();
 }
 

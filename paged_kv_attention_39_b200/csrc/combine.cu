@@ -2,13 +2,45 @@
 // Part i of a row holds its normalised output o_i and logsumexp lse_i over its keys; the
 // merged lse is logsumexp_i(lse_i) and the merged output is sum_i exp(lse_i - lse) * o_i.
 // Parts without keys carry lse_i = -inf and weight 0; a row whose parts are all empty gets
-// out = 0 and lse = -inf. One warp per (query, head); lanes run over the value dimension.
+// out = 0 and lse = -inf.
+//
+// One warp per (query, head). The weights go to shared memory first; then each lane owns four
+// consecutive output columns (float4) and walks the parts four at a time, so that every lane
+// keeps several independent loads in flight -- the merge is a short, latency-bound HBM read.
 #include "device_common.cuh"
 
 namespace pa {
 
 constexpr int kCombineWarps = 4;
 constexpr int kCombineMaxSplits = 1024;
+
+template <typename T>
+__device__ __forceinline__ void store4(T* dst, float4 v);
+template <>
+__device__ __forceinline__ void store4<float>(float* dst, float4 v) {
+    *reinterpret_cast<float4*>(dst) = v;
+}
+template <>
+__device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* dst, float4 v) {
+    uint2 u;
+    u.x = pack2<__nv_bfloat16>(v.x, v.y);
+    u.y = pack2<__nv_bfloat16>(v.z, v.w);
+    *reinterpret_cast<uint2*>(dst) = u;
+}
+template <>
+__device__ __forceinline__ void store4<__half>(__half* dst, float4 v) {
+    uint2 u;
+    u.x = pack2<__half>(v.x, v.y);
+    u.y = pack2<__half>(v.z, v.w);
+    *reinterpret_cast<uint2*>(dst) = u;
+}
+
+__device__ __forceinline__ void fma4(float4& a, float w, const float4 b) {
+    a.x = fmaf(w, b.x, a.x);
+    a.y = fmaf(w, b.y, a.y);
+    a.z = fmaf(w, b.z, a.z);
+    a.w = fmaf(w, b.w, a.w);
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnParams p) {
@@ -38,10 +70,31 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
     __syncwarp();
     const float* op = p.ws_o + ((int64_t)cu.part_base * p.hq + h) * p.dv;
     const int64_t step = (int64_t)p.hq * p.dv;
-    for (int c = lane; c < p.dv; c += 32) {
-        float acc = 0.f;
-        for (int i = 0; i < n; ++i) acc += wts[warp][i] * op[i * step + c];
-        o[c] = from_f32<T>(acc);
+    if ((p.dv & 3) == 0) {
+        for (int c = lane * 4; c < p.dv; c += 128) {
+            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
+            int i = 0;
+            for (; i + 4 <= n; i += 4) {
+                const float4 b0 = *reinterpret_cast<const float4*>(op + (i + 0) * step + c);
+                const float4 b1 = *reinterpret_cast<const float4*>(op + (i + 1) * step + c);
+                const float4 b2 = *reinterpret_cast<const float4*>(op + (i + 2) * step + c);
+                const float4 b3 = *reinterpret_cast<const float4*>(op + (i + 3) * step + c);
+                fma4(a0, wts[warp][i + 0], b0);
+                fma4(a1, wts[warp][i + 1], b1);
+                fma4(a2, wts[warp][i + 2], b2);
+                fma4(a3, wts[warp][i + 3], b3);
+            }
+            for (; i < n; ++i) fma4(a0, wts[warp][i], *reinterpret_cast<const float4*>(op + i * step + c));
+            const float4 r = make_float4(a0.x + a1.x + a2.x + a3.x, a0.y + a1.y + a2.y + a3.y,
+                                         a0.z + a1.z + a2.z + a3.z, a0.w + a1.w + a2.w + a3.w);
+            store4<T>(o + c, r);
+        }
+    } else {
+        for (int c = lane; c < p.dv; c += 32) {
+            float acc = 0.f;
+            for (int i = 0; i < n; ++i) acc += wts[warp][i] * op[i * step + c];
+            o[c] = from_f32<T>(acc);
+        }
     }
     if (lane == 0) p.lse[row] = lse;
 }

@@ -9,14 +9,19 @@
 //               page and 64-element half of the head dim, 128-byte swizzle) into a ring of
 //               stages; pages past the sequence's last key are never touched.
 //   warp 5      TMEM owner and MMA issuer (one thread): S = Q K^T into one of two TMEM
-//               buffers, then O += P V with P from shared memory; commits signal completion.
-//               Before P V it zeroes the V rows past the sequence's last key (their bytes are
-//               whatever the page holds there).
+//               buffers, then O += P V with P read from TMEM; commits signal completion. Before
+//               P V it zeroes the V rows past the sequence's last key (their bytes are whatever
+//               the page holds there).
 //   warps 0..3  softmax, one thread per row (= TMEM lane): S row from TMEM, scale to base-2
 //               units, causal/window mask at absolute positions on edge tiles, running max and
-//               sum in float32, P = exp2(S - m) as 16-bit into shared memory. The output in TMEM
-//               is rescaled only when the running max grows by more than 2^8, and the epilogue
-//               divides by the sum, rounds once and stores.
+//               sum in float32, P = exp2(S - m) packed to 16-bit into one of two TMEM P buffers.
+//               Usually one pass with the running max; the output in TMEM is rescaled only when
+//               the max grows by more than 2^8. The epilogue divides by the sum, rounds once
+//               and stores.
+//
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+D) P0, P1 (64 columns each) after O.
+// The tensor core runs one thread's MMAs in issue order, so QK of tile i+2 (issued after P V of
+// tile i) never overwrites a score buffer that is still being read.
 //
 // Every wait on an mbarrier is bounded (Watchdog): a stalled pipeline sets the plan's error
 // word and the CTA leaves through its normal exit, freeing TMEM.
@@ -32,8 +37,8 @@ namespace {
 
 constexpr int BM = 128;  // rows per tile (queries x group heads)
 constexpr int BN = 128;  // keys per step
-constexpr int KST = 2;   // K stages
-constexpr int VST = 2;   // V stages
+constexpr int KST = 3;   // K stages
+constexpr int VST = 3;   // V stages
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
@@ -46,8 +51,7 @@ struct PrefillSmem {
     static constexpr int Q = 0;
     static constexpr int K = Q + KH * HALF_Q;
     static constexpr int V = K + KST * KH * HALF_KV;
-    static constexpr int P = V + VST * KH * HALF_KV;
-    static constexpr int BAR = P + 2 * 2 * BM * 128;  // P: two buffers of 128 rows x 128 keys
+    static constexpr int BAR = V + VST * KH * HALF_KV;
     static constexpr int BYTES = BAR + 256;
     static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
 };
@@ -55,8 +59,8 @@ struct PrefillSmem {
 // Barriers used once per tile in alternation come in pairs indexed by tile parity, so that no
 // waiter can ever find its barrier two phases ahead of the phase it waits for.
 enum BarId { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
-             B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_SFREE = B_SFULL + 2,
-             B_PFULL = B_SFREE + 2, B_ODONE = B_PFULL + 2, B_COUNT = B_ODONE + 2 };
+             B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2,
+             B_COUNT = B_ODONE + 2 };
 
 }  // namespace
 
@@ -101,100 +105,73 @@ __device__ __forceinline__ float tile_max_masked(uint32_t taddr, int off_lo, int
     return fmaxf(m0, m1);
 }
 
-// Stores 16-byte chunk `chunk` (keys 8*chunk .. +7) of row r of a K-major, 128B-swizzled P tile.
-__device__ __forceinline__ void store_p_chunk(uint8_t* prow, int r, int chunk, uint32_t a, uint32_t b, uint32_t c,
-                                              uint32_t d) {
-    const int half = chunk >> 3, cc = chunk & 7;
-    *reinterpret_cast<uint4*>(prow + half * (BM * 128) + ((cc ^ (r & 7)) << 4)) = make_uint4(a, b, c, d);
-}
-
-template <typename T>
-__device__ __forceinline__ float tile_exp_full(uint32_t taddr, float scale, float m, uint8_t* prow, int r) {
-    float s0 = 0.f, s1 = 0.f;
-    const float nm = -m;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + c * 32, v);
-        tmem_ld_wait(v);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const float a0 = fast_exp2(fmaf(__uint_as_float(v[2 * e]), scale, nm));
-            const float a1 = fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), scale, nm));
-            s0 += a0;
-            s1 += a1;
-            pk[e] = pack2<T>(a0, a1);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) store_p_chunk(prow, r, c * 4 + q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-    }
-    return s0 + s1;
-}
-
-template <typename T>
-__device__ __forceinline__ float tile_exp_masked(uint32_t taddr, float scale, float m, uint8_t* prow, int r,
-                                                 int off_lo, int off_hi) {
-    float s0 = 0.f, s1 = 0.f;
-    const float nm = -m;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + c * 32, v);
-        tmem_ld_wait(v);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int k0 = c * 32 + 2 * e;
-            const bool v0 = k0 + off_lo >= 0 && k0 + off_hi < 0;
-            const bool v1 = k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0;
-            const float a0 = v0 ? fast_exp2(fmaf(__uint_as_float(v[2 * e]), scale, nm)) : 0.f;
-            const float a1 = v1 ? fast_exp2(fmaf(__uint_as_float(v[2 * e + 1]), scale, nm)) : 0.f;
-            s0 += a0;
-            s1 += a1;
-            pk[e] = pack2<T>(a0, a1);
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) store_p_chunk(prow, r, c * 4 + q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-    }
-    return s0 + s1;
-}
-
-// One pass over the tile with the row's running max m (known finite): probabilities relative to m
-// go straight to the P tile while the tile max of the raw scores is tracked; the caller keeps
-// them when the max grew by at most 2^8 (so p <= 256), and otherwise redoes the tile.
+// Probabilities of columns 32c .. 32c+31 of a row, packed two per 32-bit word, go to TMEM
+// columns 16c .. 16c+15 of the row's P buffer (the A operand layout of the P V MMA).
 template <typename T, bool MASKED>
-__device__ __forceinline__ float tile_fused(uint32_t taddr, float scale, float m, uint8_t* prow, int r, int off_lo,
-                                            int off_hi, float& m_raw) {
-    float s0 = 0.f, s1 = 0.f, m0 = neg_inf(), m1 = neg_inf();
-    const float nm = -m;
+__device__ __forceinline__ float exp_chunk(const uint32_t (&v)[32], int c, float scale, float nm, uint32_t p_taddr,
+                                           int off_lo, int off_hi) {
+    uint32_t pk[16];
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+        if (MASKED) {
+            const int k0 = c * 32 + 2 * e;
+            x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? x0 : neg_inf();
+            x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? x1 : neg_inf();
+        }
+        const float a0 = fast_exp2(fmaf(x0, scale, nm));
+        const float a1 = fast_exp2(fmaf(x1, scale, nm));
+        s0 += a0;
+        s1 += a1;
+        pk[e] = pack2<T>(a0, a1);
+    }
+    tmem_st16(p_taddr + c * 16, pk);
+    return s0 + s1;
+}
+
+// Second pass of the two-pass path: probabilities against the (new) row max m.
+template <typename T, bool MASKED>
+__device__ __forceinline__ float tile_exp(uint32_t taddr, float scale, float m, uint32_t p_taddr, int off_lo,
+                                          int off_hi) {
+    float sum = 0.f;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
-        uint32_t pk[16];
+        sum += exp_chunk<T, MASKED>(v, c, scale, -m, p_taddr, off_lo, off_hi);
+    }
+    return sum;
+}
+
+// One pass with the row's running max m (known finite): probabilities relative to m go to the
+// P buffer while the tile max of the raw scores is tracked; the caller keeps them when the max
+// grew by at most 2^8 (so p <= 256), and otherwise redoes the tile.
+template <typename T, bool MASKED>
+__device__ __forceinline__ float tile_fused(uint32_t taddr, float scale, float m, uint32_t p_taddr, int off_lo,
+                                            int off_hi, float& m_raw) {
+    float sum = 0.f, m0 = neg_inf(), m1 = neg_inf();
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait(v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            float x0 = __uint_as_float(v[2 * e]), x1 = __uint_as_float(v[2 * e + 1]);
+        for (int e = 0; e < 32; e += 2) {
+            float x0 = __uint_as_float(v[e]), x1 = __uint_as_float(v[e + 1]);
             if (MASKED) {
-                const int k0 = c * 32 + 2 * e;
+                const int k0 = c * 32 + e;
                 x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? x0 : neg_inf();
                 x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? x1 : neg_inf();
             }
             m0 = fmaxf(m0, x0);
             m1 = fmaxf(m1, x1);
-            const float a0 = fast_exp2(fmaf(x0, scale, nm));
-            const float a1 = fast_exp2(fmaf(x1, scale, nm));
-            s0 += a0;
-            s1 += a1;
-            pk[e] = pack2<T>(a0, a1);
         }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) store_p_chunk(prow, r, c * 4 + q, pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        sum += exp_chunk<T, MASKED>(v, c, scale, -m, p_taddr, off_lo, off_hi);
     }
     m_raw = fmaxf(m0, m1);
-    return s0 + s1;
+    return sum;
 }
 
 template <typename T, int D>
@@ -233,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL || i == B_PFULL + 1) cnt = 128;
+            if (i == B_PFULL || i == B_PFULL + 1) cnt = 128;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -250,6 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t t_s0 = tmem, t_s1 = tmem + 128;
     const uint32_t t_o = tmem + 256;
+    const uint32_t t_p0 = t_o + D, t_p1 = t_o + D + 64;
     const uint32_t s_base = smem_u32(smem);
 
     if (warp == 4) {
@@ -324,15 +302,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Descriptors are built once; a k-step or stage offset is an add to the address field.
         const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
         const uint64_t dK = sdesc_sw128(s_base + L_::K, 16, 1024);
-        const uint64_t dP = sdesc_sw128(s_base + L_::P, 16, 1024);
         const uint64_t dV = sdesc_sw128(s_base + L_::V, L_::HALF_KV, 1024);
         bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[B_QFULL], 0, wd, 3));
         for (int i = 0; ok && i <= n_tiles; ++i) {
             if (i < n_tiles) {
                 const int ks = i % KST, b = i & 1;
-                ok = mbar_wait(&bars[B_KFULL + ks], (i / KST) & 1, wd, 4);
-                if (ok && i >= 2) ok = mbar_wait(&bars[B_SFREE + b], ((i >> 1) - 1) & 1, wd, 5);
-                ok = __all_sync(0xffffffffu, ok);
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_KFULL + ks], (i / KST) & 1, wd, 4));
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
@@ -367,13 +342,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint64_t dPj = desc_add(dP, (j & 1) * (2 * BM * 128));
+                    const uint32_t t_pj = (j & 1) ? t_p1 : t_p0;
                     const uint64_t dVs = desc_add(dV, vs * KH * L_::HALF_KV);
                     const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        mma_f16_ss(t_o, desc_add(dPj, (kk >> 2) * (BM * 128) + (kk & 3) * 32),
-                                   desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
+                    for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
+                        mma_f16_ts(t_o, t_pj + kk * 8, desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
                     mma_commit(&bars[B_ODONE + (j & 1)]);
                     mma_commit(&bars[B_VEMPTY + vs]);
                 }
@@ -407,15 +381,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((i - 2) >> 1) & 1, wd, 11));
                 if (!ok) break;
             }
-            uint8_t* prow = smem + L_::P + b * (2 * BM * 128) + r * 128;
+            const uint32_t t_pb = (b ? t_p1 : t_p0) + lane_off;
             const int off_lo = (int)(kt0 - row_lo), off_hi = (int)(kt0 - row_hi);
             // Fast path: one pass with the running max when every row of the warp has one.
             bool redo = true;
             float sum = 0.f;
             if (__all_sync(0xffffffffu, m_run != neg_inf())) {
                 float m_raw;
-                sum = full ? tile_fused<T, false>(t_sb, p.scale_log2, m_run, prow, r, 0, 0, m_raw)
-                           : tile_fused<T, true>(t_sb, p.scale_log2, m_run, prow, r, off_lo, off_hi, m_raw);
+                sum = full ? tile_fused<T, false>(t_sb, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
+                           : tile_fused<T, true>(t_sb, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
                 redo = __any_sync(0xffffffffu, m_raw * p.scale_log2 > m_run + 8.0f);
             }
             if (redo) {
@@ -442,21 +416,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
                         tmem_st32(t_o + lane_off + c * 32, v);
                     }
-                    tmem_st_wait();
                 }
                 if (grow) {
                     l_run *= fast_exp2(m_run - m_new);
                     m_run = m_new;
                 }
                 const float m_use = m_run == neg_inf() ? 0.f : m_run;
-                // pass 2: probabilities p = 2^(s * scale - m), 16-bit, into the swizzled K-major P tile
-                sum = full ? tile_exp_full<T>(t_sb, p.scale_log2, m_use, prow, r)
-                           : tile_exp_masked<T>(t_sb, p.scale_log2, m_use, prow, r, off_lo, off_hi);
+                // pass 2: probabilities p = 2^(s * scale - m) into the P buffer
+                sum = full ? tile_exp<T, false>(t_sb, p.scale_log2, m_use, t_pb, 0, 0)
+                           : tile_exp<T, true>(t_sb, p.scale_log2, m_use, t_pb, off_lo, off_hi);
             }
-            tc_fence_before();
-            mbar_arrive(&bars[B_SFREE + b]);  // S buffer b may be overwritten
+            tmem_st_wait();
             l_run += sum;
-            fence_proxy_async_smem();
+            tc_fence_before();
             mbar_arrive(&bars[B_PFULL + b]);
         }
         // ---- epilogue ----

@@ -167,3 +167,20 @@ def test_binding_functions_compile_their_calls():
     plan = pa.pa_plan_create([5], [0, 1], torch.zeros(1, 1, dtype=torch.int32), 16, 1, device=-1)
     with pytest.raises(pa.PaError):
         pa.pa_plan_prepare(plan, torch.bfloat16, 4, 2, 64, 64)
+
+
+def test_append_validation(lib):
+    wl, plan = host_plan()
+    q, k, v, o, l = fake_ptrs(wl)
+    def app(nk=q, nv=q + 4096 * 64, kc=k, vc=v, hkv=2, d=64, dv=64, dtype=1, pl=plan):
+        return pa.STATUS[lib.pa_append(pl.handle, nk, nv, kc, vc, dtype, hkv, d, dv, None)]
+    assert app() == "PA_ERR_INVALID_ARGUMENT"          # host-only plan, after all checks
+    assert app(kc=k, vc=k) == "PA_ERR_ALIAS"            # caches overlap
+    assert app(nk=k) == "PA_ERR_ALIAS"                  # new rows inside a cache
+    assert app(d=4) == "PA_ERR_UNSUPPORTED"             # 8-byte rows
+    assert app(hkv=0) == "PA_ERR_SHAPE"
+    assert app(dtype=9) == "PA_ERR_DTYPE"
+    # two sequences that append into the same page slot
+    bt = torch.tensor([[0, 1], [0, 1]], dtype=torch.int32)
+    shared = pa.pa_plan_create([20, 20], [0, 1, 2], bt, 16, 4, device=-1)
+    assert app(pl=shared) == "PA_ERR_ALIAS"
