@@ -213,6 +213,30 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
                     pa_stream stream);
 
 /*
+ * pa_backward -- gradients of paged GQA attention (boostr `standard_attention_bwd`; ruDNN
+ * `attention_backward`: weights recomputed from Q and K, not saved). For the upstream gradient
+ * d_out of out = softmax(scale Q K^T + mask) V:
+ *     dV_t += P_t dO,  dP_t = dO . V_t,  D = dO . out,  dS_t = P_t (dP_t - D),
+ *     dQ = scale sum_t dS_t K_t,  dK_t += scale dS_t Q
+ * with P recomputed from the forward's lse. Query head h reads KV head h / G, so the G heads of a
+ * group (and every query, and every sequence sharing a page) add into the same cache slot.
+ *
+ *   q, k_cache, v_cache  the forward's inputs (dtype, same layouts as pa_forward)
+ *   out, lse             the forward's outputs
+ *   d_out                [N_q, Hq, Dv] dtype
+ *   d_q                  [N_q, Hq, D] float32, written
+ *   d_k_cache            [pages, page_size, Hkv, D] float32, ADDED INTO (zero it first)
+ *   d_v_cache            [pages, page_size, Hkv, Dv] float32, ADDED INTO (zero it first)
+ * Float32 atomics make the summation order of dK/dV vary between runs. Validation and errors as
+ * pa_forward (gradient outputs must not overlap each other or any input).
+ */
+pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                      const void* out, const float* lse, const void* d_out, pa_dtype dtype,
+                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                      int32_t v_head_dim, float scale, int causal, int32_t window, float* d_q,
+                      float* d_k_cache, float* d_v_cache, pa_stream stream);
+
+/*
  * pa_forward_static_workspace -- pa_forward's split-KV decode without any memory allocation.
  * The pages describe no such call: it exists for callers that cannot allocate device memory
  * while they run attention (a serving loop that must not stall on the allocator mid-step, a

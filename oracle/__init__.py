@@ -45,6 +45,10 @@ class Oracle:
         lib.pao_mla_attention.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I,
                                           _I, _I, _I, ctypes.c_double, ctypes.c_int, _I, _P, _P,
                                           _P, _P, _P, ctypes.c_int]
+        lib.pao_paged_attention_backward.restype = ctypes.c_int
+        lib.pao_paged_attention_backward.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I, _I, _I,
+                                                     _I, _I, ctypes.c_double, ctypes.c_int, _I, _P, _P, _P,
+                                                     ctypes.c_int]
         lib.pao_lse_combine.restype = None
         lib.pao_lse_combine.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _I, _P, _P]
         self.lib = lib
@@ -99,6 +103,31 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle rejected the schedule (code {rc})")
         return out, lse
+
+    # -- backward of paged GQA attention -----------------------------------------------------
+    def attention_backward(self, q, k_cache, v_cache, d_out, seq_lens, query_offsets, block_tables, page_size,
+                           scale, causal=True, window=0, nthreads=None):
+        """(dq [Nq, Hq, D], dk [P, ps, Hkv, D], dv [P, ps, Hkv, Dv]) float64 for upstream d_out."""
+        dt = q.dtype
+        assert k_cache.dtype == dt and v_cache.dtype == dt and d_out.dtype == dt and dt in _DT
+        q, k_cache, v_cache, d_out = self._c(q), self._c(k_cache), self._c(v_cache), self._c(d_out)
+        nq, hq, d = q.shape
+        num_pages, ps, hkv, _ = k_cache.shape
+        dv = v_cache.shape[3]
+        sl = self._c(seq_lens, torch.int32)
+        qo = self._c(query_offsets, torch.int32)
+        bt = self._c(block_tables, torch.int32)
+        dq = torch.zeros((nq, hq, d), dtype=torch.float64)
+        dk = torch.zeros((num_pages, ps, hkv, d), dtype=torch.float64)
+        dvv = torch.zeros((num_pages, ps, hkv, dv), dtype=torch.float64)
+        rc = self.lib.pao_paged_attention_backward(
+            q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), d_out.data_ptr(), _DT[dt], sl.data_ptr(),
+            qo.data_ptr(), sl.numel(), bt.data_ptr(), bt.shape[1], page_size, num_pages, hq, hkv, d, dv,
+            float(scale), int(bool(causal)), int(window), dq.data_ptr(), dk.data_ptr(), dvv.data_ptr(),
+            self._threads(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle rejected the schedule (code {rc})")
+        return dq, dk, dvv
 
     # -- MLA absorbed-latent attention ------------------------------------------------------
     def mla(self, q_latent, q_rope, latent_cache, rope_cache, seq_lens, query_offsets,

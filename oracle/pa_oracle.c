@@ -357,3 +357,164 @@ void pao_lse_combine(const double* o_parts, const double* lse_parts, int64_t npa
         }
     }
 }
+
+/*
+ * Backward of paged GQA attention (boostr `standard_attention_bwd`, recomputing the weights from
+ * Q and K): with P = softmax(scale * Q K^T + mask) per row, O = P V, and the upstream gradient
+ * dO,
+ *     dV_t += P_t dO,   dP_t = dO . V_t,   D = dO . O,   dS_t = P_t (dP_t - D),
+ *     dQ = scale * sum_t dS_t K_t,   dK_t += scale * dS_t Q.
+ * Query head h reads KV head h / G, so dK and dV sum over the G heads of a group (boostr
+ * `sum_gqa_grads`), and over every query and sequence whose visible keys include the slot
+ * (a page shared by several sequences receives all their contributions).
+ * dq [Nq, Hq, D] is written; dk [P, ps, Hkv, D] and dv [P, ps, Hkv, Dv] are zeroed and then
+ * accumulated. Same masking readings as the forward. Returns 0, or -1/-2/-3 as the forward.
+ */
+typedef struct {
+    pao_job J;
+    const void* dout;
+    double* dq;
+    double* dk;
+    double* dv;
+    pthread_mutex_t acc_lock;
+} pao_bwd_job;
+
+static void pao_bwd_item(pao_bwd_job* B, int32_t s, int32_t kvh, double* kbuf, double* vbuf, double* xbuf,
+                         double* qbuf, double* dkl, double* dvl, double* obuf, double* gbuf) {
+    pao_job* J = &B->J;
+    const int64_t L = J->seq_lens[s];
+    const int64_t q0 = J->query_offsets[s];
+    const int64_t n = J->query_offsets[s + 1] - q0;
+    const int32_t ps = J->page_size;
+    const int32_t G = J->hq / J->hkv;
+    const int32_t kd = J->d, vd = J->dv;
+    if (n == 0) return;
+    for (int64_t t = 0; t < L; ++t) {
+        int64_t page = J->block_tables[(int64_t)s * J->table_width + t / ps];
+        int64_t row = (page * ps + t % ps) * J->hkv + kvh;
+        for (int32_t c = 0; c < kd; ++c) kbuf[t * kd + c] = pao_load(J->k, J->dtype, row * kd + c);
+        for (int32_t c = 0; c < vd; ++c) vbuf[t * vd + c] = pao_load(J->v, J->dtype, row * vd + c);
+        for (int32_t c = 0; c < kd; ++c) dkl[t * kd + c] = 0.0;
+        for (int32_t c = 0; c < vd; ++c) dvl[t * vd + c] = 0.0;
+    }
+    for (int32_t g = 0; g < G; ++g) {
+        const int32_t h = kvh * G + g;
+        for (int64_t j = 0; j < n; ++j) {
+            const int64_t r = (q0 + j) * J->hq + h;
+            const int64_t p = L - n + j;
+            for (int32_t c = 0; c < kd; ++c) qbuf[c] = pao_load(J->q, J->dtype, r * kd + c);
+            for (int32_t c = 0; c < vd; ++c) gbuf[c] = pao_load(B->dout, J->dtype, r * vd + c);
+            double m = -INFINITY;
+            for (int64_t t = 0; t < L; ++t) {
+                if (!pao_visible(J, s, t, p)) { xbuf[t] = -INFINITY; continue; }
+                double acc = 0.0;
+                for (int32_t c = 0; c < kd; ++c) acc += qbuf[c] * kbuf[t * kd + c];
+                xbuf[t] = J->scale * acc;
+                if (xbuf[t] > m) m = xbuf[t];
+            }
+            double* dq = B->dq + r * kd;
+            for (int32_t c = 0; c < kd; ++c) dq[c] = 0.0;
+            if (m == -INFINITY) continue;
+            double sum = 0.0;
+            for (int64_t t = 0; t < L; ++t)
+                if (xbuf[t] != -INFINITY) sum += exp(xbuf[t] - m);
+            const double lse = m + log(sum);
+            for (int32_t c = 0; c < vd; ++c) obuf[c] = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                if (xbuf[t] == -INFINITY) continue;
+                xbuf[t] = exp(xbuf[t] - lse); /* now P_t */
+                for (int32_t c = 0; c < vd; ++c) obuf[c] += xbuf[t] * vbuf[t * vd + c];
+            }
+            double Dr = 0.0;
+#ifndef PAO_MUTANT_BWD_NO_D
+            for (int32_t c = 0; c < vd; ++c) Dr += gbuf[c] * obuf[c];
+#endif
+            for (int64_t t = 0; t < L; ++t) {
+                if (xbuf[t] == -INFINITY) continue;
+                const double P = xbuf[t];
+                double dp = 0.0;
+                for (int32_t c = 0; c < vd; ++c) dp += gbuf[c] * vbuf[t * vd + c];
+                const double ds = P * (dp - Dr);
+                for (int32_t c = 0; c < kd; ++c) dq[c] += J->scale * ds * kbuf[t * kd + c];
+                for (int32_t c = 0; c < kd; ++c) dkl[t * kd + c] += J->scale * ds * qbuf[c];
+                for (int32_t c = 0; c < vd; ++c) dvl[t * vd + c] += P * gbuf[c];
+            }
+        }
+    }
+    pthread_mutex_lock(&B->acc_lock);
+    for (int64_t t = 0; t < L; ++t) {
+        int64_t page = J->block_tables[(int64_t)s * J->table_width + t / ps];
+        int64_t row = (page * ps + t % ps) * J->hkv + kvh;
+        for (int32_t c = 0; c < kd; ++c) B->dk[row * kd + c] += dkl[t * kd + c];
+        for (int32_t c = 0; c < vd; ++c) B->dv[row * vd + c] += dvl[t * vd + c];
+    }
+    pthread_mutex_unlock(&B->acc_lock);
+}
+
+static void* pao_bwd_worker(void* arg) {
+    pao_bwd_job* B = (pao_bwd_job*)arg;
+    pao_job* J = &B->J;
+    int64_t maxL = 1;
+    for (int32_t s = 0; s < J->num_seqs; ++s)
+        if (J->seq_lens[s] > maxL) maxL = J->seq_lens[s];
+    double* kbuf = (double*)malloc(sizeof(double) * maxL * J->d);
+    double* vbuf = (double*)malloc(sizeof(double) * maxL * J->dv);
+    double* dkl = (double*)malloc(sizeof(double) * maxL * J->d);
+    double* dvl = (double*)malloc(sizeof(double) * maxL * J->dv);
+    double* xbuf = (double*)malloc(sizeof(double) * maxL);
+    double* qbuf = (double*)malloc(sizeof(double) * J->d);
+    double* obuf = (double*)malloc(sizeof(double) * J->dv);
+    double* gbuf = (double*)malloc(sizeof(double) * J->dv);
+    if (!kbuf || !vbuf || !dkl || !dvl || !xbuf || !qbuf || !obuf || !gbuf) {
+        pthread_mutex_lock(&J->lock);
+        J->error = 1;
+        pthread_mutex_unlock(&J->lock);
+    } else {
+        for (;;) {
+            pthread_mutex_lock(&J->lock);
+            int64_t it = J->next_item++;
+            pthread_mutex_unlock(&J->lock);
+            if (it >= (int64_t)J->num_seqs * J->hkv) break;
+            pao_bwd_item(B, (int32_t)(it / J->hkv), (int32_t)(it % J->hkv), kbuf, vbuf, xbuf, qbuf, dkl, dvl, obuf,
+                         gbuf);
+        }
+    }
+    free(kbuf); free(vbuf); free(dkl); free(dvl); free(xbuf); free(qbuf); free(obuf); free(gbuf);
+    return NULL;
+}
+
+int pao_paged_attention_backward(const void* q, const void* k_cache, const void* v_cache, const void* d_out,
+                                 int dtype, const int32_t* seq_lens, const int32_t* query_offsets, int32_t num_seqs,
+                                 const int32_t* block_tables, int32_t table_width, int32_t page_size,
+                                 int32_t num_pages, int32_t hq, int32_t hkv, int32_t d, int32_t dv, double scale,
+                                 int causal, int32_t window, double* dq, double* dk, double* dvout, int nthreads) {
+    if (hq <= 0 || hkv <= 0 || hq % hkv || d <= 0 || dv <= 0 || window < 0) return -1;
+    pao_bwd_job B;
+    memset(&B, 0, sizeof B);
+    pao_job* J = &B.J;
+    J->q = q; J->k = k_cache; J->v = v_cache; J->dtype = dtype; J->mla = 0;
+    J->seq_lens = seq_lens; J->query_offsets = query_offsets; J->num_seqs = num_seqs;
+    J->block_tables = block_tables; J->table_width = table_width; J->page_size = page_size;
+    J->num_pages = num_pages; J->hq = hq; J->hkv = hkv; J->d = d; J->dv = dv;
+    J->scale = scale; J->causal = causal; J->window = window;
+    int rc = pao_check_schedule(J);
+    if (rc) return rc;
+    B.dout = d_out; B.dq = dq; B.dk = dk; B.dv = dvout;
+    memset(dk, 0, sizeof(double) * (size_t)num_pages * page_size * hkv * d);
+    memset(dvout, 0, sizeof(double) * (size_t)num_pages * page_size * hkv * dv);
+    pthread_mutex_init(&J->lock, NULL);
+    pthread_mutex_init(&B.acc_lock, NULL);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, pao_bwd_worker, &B) == 0) ++started;
+        else break;
+    }
+    if (started == 0) pao_bwd_worker(&B);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    pthread_mutex_destroy(&J->lock);
+    pthread_mutex_destroy(&B.acc_lock);
+    return J->error ? -3 : 0;
+}

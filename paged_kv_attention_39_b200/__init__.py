@@ -29,7 +29,7 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
           "PA_ERR_ALIAS", "PA_ERR_UNSUPPORTED", "PA_ERR_CUDA"]
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
-           "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex", "pa_append",
+           "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex", "pa_append", "pa_backward",
            "pa_plan_device_status",
            "pa_status_string", "pa_last_error_message", "pa_version"]
 
@@ -93,6 +93,9 @@ def load_library(path: Optional[str] = None):
                                                 ctypes.c_int, _I, _I, _P, _P, _P]
     lib.pa_append.restype = ctypes.c_int
     lib.pa_append.argtypes = [_P, _P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _P]
+    lib.pa_backward.restype = ctypes.c_int
+    lib.pa_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _I, ctypes.c_float, ctypes.c_int,
+                                _I, _P, _P, _P, _P]
     lib.pa_plan_device_status.restype = ctypes.c_int
     lib.pa_plan_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
     lib.pa_status_string.restype = ctypes.c_char_p
@@ -253,6 +256,19 @@ def pa_append(plan: Plan, new_k: torch.Tensor, new_v: torch.Tensor, k_cache: tor
     _check(load_library().pa_append(plan.handle, _ptr(new_k), _ptr(new_v), _ptr(k_cache), _ptr(v_cache),
                                     _DTYPES[new_k.dtype], k_cache.shape[2], k_cache.shape[3], v_cache.shape[3],
                                     _stream_ptr(stream, plan.device)))
+
+
+def pa_backward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, out: torch.Tensor,
+                lse: torch.Tensor, d_out: torch.Tensor, d_q: torch.Tensor, d_k_cache: torch.Tensor,
+                d_v_cache: torch.Tensor, scale: float, causal: bool = True, window: int = 0, stream=None) -> None:
+    """Gradients of pa_forward: d_q written, d_k_cache / d_v_cache (float32) accumulated."""
+    for t in (q, k_cache, v_cache, out, lse, d_out, d_q, d_k_cache, d_v_cache):
+        if not t.is_contiguous():
+            raise ValueError("pa_backward takes contiguous tensors")
+    _check(load_library().pa_backward(
+        plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), _ptr(d_out), _DTYPES[q.dtype],
+        q.shape[1], k_cache.shape[2], q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window),
+        _ptr(d_q), _ptr(d_k_cache), _ptr(d_v_cache), _stream_ptr(stream, plan.device)))
 
 
 def pa_forward_static_workspace(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor,

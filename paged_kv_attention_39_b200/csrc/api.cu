@@ -767,6 +767,59 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
     return ok();
 }
 
+pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache, const void* out,
+                      const float* lse, const void* d_out, pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads,
+                      int32_t head_dim, int32_t v_head_dim, float scale, int causal, int32_t window, float* d_q,
+                      float* d_k_cache, float* d_v_cache, pa_stream stream) {
+    if (!plan) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    {
+        if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return fail(PA_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+        if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads)
+            return fail(PA_ERR_SHAPE, "query heads (%d) must be a positive multiple of kv heads (%d)", num_q_heads, num_kv_heads);
+        if (head_dim <= 0 || v_head_dim <= 0) return fail(PA_ERR_SHAPE, "head dims must be positive");
+        if (head_dim > 1024 || v_head_dim > 1024) return fail(PA_ERR_UNSUPPORTED, "head dims above 1024 are not supported");
+        if (!std::isfinite(scale) || !(scale > 0.0f)) return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and > 0");
+        if (causal != 0 && causal != 1) return fail(PA_ERR_INVALID_ARGUMENT, "causal must be 0 or 1");
+        if (window < 0) return fail(PA_ERR_INVALID_ARGUMENT, "window must be >= 0");
+    }
+    const int64_t es = (int64_t)dtype_size(dtype);
+    const int64_t nq = plan->Nq, pages = plan->num_pages, ps = plan->page_size;
+    int64_t n_q, n_k, n_v, n_o, n_l, n_dq, n_dk, n_dv;
+    if (!product({nq, num_q_heads, head_dim, es}, &n_q) || !product({pages, ps, num_kv_heads, head_dim, es}, &n_k) ||
+        !product({pages, ps, num_kv_heads, v_head_dim, es}, &n_v) || !product({nq, num_q_heads, v_head_dim, es}, &n_o) ||
+        !product({nq, num_q_heads, 4}, &n_l) || !product({nq, num_q_heads, head_dim, 4}, &n_dq) ||
+        !product({pages, ps, num_kv_heads, head_dim, 4}, &n_dk) || !product({pages, ps, num_kv_heads, v_head_dim, 4}, &n_dv))
+        return fail(PA_ERR_BOUNDS, "tensor size overflows 64-bit byte counts");
+    if (nq == 0) return ok();
+    if (!q || !k_cache || !v_cache || !out || !lse || !d_out || !d_q || !d_k_cache || !d_v_cache)
+        return fail(PA_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    for (const void* ptr : {q, k_cache, v_cache, out, (const void*)lse, d_out, (const void*)d_q, (const void*)d_k_cache,
+                            (const void*)d_v_cache})
+        if ((uintptr_t)ptr % 16 != 0) return fail(PA_ERR_INVALID_ARGUMENT, "device pointers must be 16-byte aligned");
+    auto R = [](const void* p, int64_t n) { return Range{(uintptr_t)p, (uintptr_t)p + (uintptr_t)n}; };
+    const Range outs[3] = {R(d_q, n_dq), R(d_k_cache, n_dk), R(d_v_cache, n_dv)};
+    const Range ins[6] = {R(q, n_q), R(k_cache, n_k), R(v_cache, n_v), R(out, n_o), R(lse, n_l), R(d_out, n_o)};
+    for (int a = 0; a < 3; ++a) {
+        for (int b = a + 1; b < 3; ++b)
+            if (overlap(outs[a], outs[b])) return fail(PA_ERR_ALIAS, "gradient outputs overlap");
+        for (const Range& r : ins)
+            if (overlap(outs[a], r)) return fail(PA_ERR_ALIAS, "a gradient output overlaps an input");
+    }
+    if (plan->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to run on");
+    int cur = -1;
+    PA_CUDA_TRY(cudaGetDevice(&cur));
+    if (cur != plan->device)
+        return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
+    cudaError_t e = pa::launch_backward(q, k_cache, v_cache, out, lse, d_out, d_q, d_k_cache, d_v_cache,
+                                        plan->d_seqs, plan->d_q2seq, plan->d_bt, plan->table_width, plan->page_size,
+                                        num_q_heads, num_kv_heads, head_dim, v_head_dim, scale, causal, window,
+                                        nq * num_q_heads, dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "backward kernel launch failed: %s", cudaGetErrorString(e));
+    plan->last_stream = (cudaStream_t)stream;
+    plan->last_launches = 1;
+    return ok();
+}
+
 pa_status pa_plan_device_status(const pa_plan* plan, int32_t* code) {
     if (!plan || !code) return fail(PA_ERR_INVALID_ARGUMENT, "plan or code is NULL");
     *code = 0;

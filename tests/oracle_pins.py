@@ -325,10 +325,82 @@ def pin_half_precision_widening(orc):
         assert torch.equal(o[0, 0], vals[page, 0, 0].double())
 
 
+def _backward_cases():
+    return [
+        W.make_gqa("b1", 31, [9, 20], [3, 20], 4, 2, 8, 8, 4, torch.float32, causal=True),
+        W.make_gqa("b2", 32, [25, 6], [4, 2], 6, 3, 8, 4, 8, torch.float32, causal=True, window=5),
+        W.make_gqa("b3", 33, [12], [5], 2, 2, 8, 8, 4, torch.float32, causal=False, window=4),
+    ]
+
+
+def pin_backward_vs_autograd(orc):
+    """dq, dk, dv against torch autograd of fp64 SDPA on the dense gather (GQA by repeat_interleave,
+    whose backward sums the group), scattered back to the cache slots through the block table."""
+    for wl in _backward_cases():
+        s_ = wl.sched
+        g = torch.Generator().manual_seed(9)
+        dout = torch.randn(wl.q.shape[0], wl.num_q_heads, wl.v_head_dim, generator=g).to(wl.q.dtype)
+        dq, dk, dv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s_.seq_lens, s_.query_offsets,
+                                            s_.block_tables, s_.page_size, wl.scale, wl.causal, wl.window)
+        G = wl.num_q_heads // wl.num_kv_heads
+        ref_dk = torch.zeros_like(dk)
+        ref_dv = torch.zeros_like(dv)
+        for s in range(s_.num_seqs):
+            L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+            t = torch.arange(L)
+            pages = s_.block_tables[s, t // s_.page_size].long()
+            K = wl.k_cache[pages, t % s_.page_size].double().requires_grad_(True)
+            V = wl.v_cache[pages, t % s_.page_size].double().requires_grad_(True)
+            Q = wl.q[q0:q0 + n].double().requires_grad_(True)
+            pos = torch.arange(L - n, L).view(n, 1)
+            keep = torch.ones(n, L, dtype=torch.bool)
+            if wl.causal:
+                keep &= t.view(1, L) <= pos
+            if wl.window > 0:
+                keep &= t.view(1, L) + wl.window > pos
+            o = F.scaled_dot_product_attention(Q.transpose(0, 1), K.repeat_interleave(G, 1).transpose(0, 1),
+                                               V.repeat_interleave(G, 1).transpose(0, 1), attn_mask=keep,
+                                               scale=wl.scale)
+            (o * dout[q0:q0 + n].double().transpose(0, 1)).sum().backward()
+            assert torch.allclose(dq[q0:q0 + n], Q.grad, rtol=1e-10, atol=1e-12), (wl.name, s)
+            ref_dk.index_put_((pages, t % s_.page_size), K.grad, accumulate=True)
+            ref_dv.index_put_((pages, t % s_.page_size), V.grad, accumulate=True)
+        assert torch.allclose(dk, ref_dk, rtol=1e-10, atol=1e-12), wl.name
+        assert torch.allclose(dv, ref_dv, rtol=1e-10, atol=1e-12), wl.name
+
+
+def pin_backward_finite_differences(orc):
+    """Central differences of L = sum(out * dO) (forward oracle) at a few entries of q, k, v."""
+    wl = W.make_gqa("fd", 34, [10, 7], [4, 2], 4, 2, 8, 8, 4, torch.float32, causal=True, window=6)
+    s_ = wl.sched
+    g = torch.Generator().manual_seed(10)
+    dout = torch.randn(wl.q.shape[0], 4, 8, generator=g).to(torch.float32)
+    dq, dk, dv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s_.seq_lens, s_.query_offsets,
+                                        s_.block_tables, 4, wl.scale, True, 6)
+
+    def loss(q, k, v):
+        out, _ = orc.attention(q, k, v, s_.seq_lens, s_.query_offsets, s_.block_tables, 4, wl.scale, True, 6)
+        return float((out * dout.double()).sum())
+
+    probes = [("q", (1, 2, 3)), ("q", (5, 0, 7)), ("k", (int(s_.block_tables[0, 1]), 2, 1, 4)),
+              ("v", (int(s_.block_tables[1, 0]), 3, 0, 6)), ("v", (int(s_.block_tables[0, 2]), 1, 1, 0))]
+    for name, idx in probes:
+        base = {"q": wl.q, "k": wl.k_cache, "v": wl.v_cache}[name]
+        plus, minus = base.clone(), base.clone()
+        plus[idx] += 1e-2
+        minus[idx] -= 1e-2
+        h2 = float(plus[idx]) - float(minus[idx])
+        args_p = {"q": wl.q, "k": wl.k_cache, "v": wl.v_cache}; args_p[name] = plus
+        args_m = {"q": wl.q, "k": wl.k_cache, "v": wl.v_cache}; args_m[name] = minus
+        fd = (loss(args_p["q"], args_p["k"], args_p["v"]) - loss(args_m["q"], args_m["k"], args_m["v"])) / h2
+        an = float({"q": dq, "k": dk, "v": dv}[name][idx])
+        assert abs(fd - an) <= 1e-4 * max(1.0, abs(an)), (name, idx, fd, an)
+
+
 ALL_PINS = [
     pin_sdpa_bruteforce, pin_alice_fixture_dense, pin_single_key, pin_constant_v_per_kv_head,
     pin_q_zero_counts_and_mean, pin_position_probe, pin_large_score_selects_target,
     pin_page_permutation_invariance, pin_split_equals_unsplit, pin_chunked_equals_oneshot,
     pin_window_cases, pin_gqa_equals_mha_repeated, pin_mla_equals_gqa_concat,
-    pin_half_precision_widening,
+    pin_half_precision_widening, pin_backward_vs_autograd, pin_backward_finite_differences,
 ]

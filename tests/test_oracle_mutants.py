@@ -22,6 +22,7 @@ MUTANTS = [
     "PAO_MUTANT_LSE_NO_MAX",      # lse loses the max shift
     "PAO_MUTANT_UNNORMALISED",    # output not divided by the softmax sum
     "PAO_MUTANT_SCALE_DROPPED",   # scores not scaled
+    "PAO_MUTANT_BWD_NO_D",        # backward without the rowsum(dO * O) term
 ]
 
 
