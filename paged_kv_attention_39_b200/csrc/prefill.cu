@@ -5,14 +5,15 @@
 // query heads that share one KV head (so every K/V tile feeds all G heads), against the keys
 // those queries can see, 128 keys per step, and writes the final output and lse.
 //
-//   warp 4      TMA producer: the Q tile once, then K and V tiles page by page (one box per
+//   warp 8      TMA producer: the Q tile once, then K and V tiles page by page (one box per
 //               page and 64-element half of the head dim, 128-byte swizzle) into a ring of
 //               stages; pages past the sequence's last key are never touched.
-//   warp 5      TMEM owner and MMA issuer (one thread): S = Q K^T into one of two TMEM
+//   warp 9      TMEM owner and MMA issuer (one thread): S = Q K^T into one of two TMEM
 //               buffers, then O += P V with P read from TMEM; commits signal completion. Before
 //               P V it zeroes the V rows past the sequence's last key (their bytes are whatever
 //               the page holds there).
-//   warps 0..3  softmax, one thread per row (= TMEM lane): S row from TMEM, scale to base-2
+//   warps 0..7  softmax, two warps per row (each owning one half of the tile's columns; a warp's
+//               lanes are the TMEM lanes of its quadrant): S from TMEM, scale to base-2
 //               units, causal/window mask at absolute positions on edge tiles, running max and
 //               sum in float32, P = exp2(S - m) packed to 16-bit into one of two TMEM P buffers.
 //               Usually one pass with the running max; the output in TMEM is rescaled only when
@@ -39,7 +40,9 @@ constexpr int BM = 128;  // rows per tile (queries x group heads)
 constexpr int BN = 128;  // keys per step
 constexpr int KST = 3;   // K stages
 constexpr int VST = 3;   // V stages
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quadrant, each owning half of the columns
+constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
@@ -52,7 +55,8 @@ struct PrefillSmem {
     static constexpr int K = Q + KH * HALF_Q;
     static constexpr int V = K + KST * KH * HALF_KV;
     static constexpr int BAR = V + VST * KH * HALF_KV;
-    static constexpr int BYTES = BAR + 256;
+    static constexpr int XCH = BAR + 256;  // 128 rows x 2 column halves of float: row statistics
+    static constexpr int BYTES = XCH + 2 * BM * 4;
     static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
 };
 
@@ -68,10 +72,11 @@ enum BarId { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEM
 // Column c of the tile is masked when c + off_lo < 0 or c + off_hi >= 0, where off_lo = kt0 - row_lo
 // and off_hi = kt0 - row_hi (the row's visible keys are [row_lo, row_hi)).
 
-__device__ __forceinline__ float tile_max_full(uint32_t taddr) {
+// Each helper covers the 32-column chunks [c0, c0 + 2): one half of the tile's columns.
+__device__ __forceinline__ float tile_max_full(uint32_t taddr, int c0) {
     float m0 = neg_inf(), m1 = neg_inf(), m2 = neg_inf(), m3 = neg_inf();
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c0; c < c0 + 2; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -86,10 +91,10 @@ __device__ __forceinline__ float tile_max_full(uint32_t taddr) {
     return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-__device__ __forceinline__ float tile_max_masked(uint32_t taddr, int off_lo, int off_hi) {
+__device__ __forceinline__ float tile_max_masked(uint32_t taddr, int c0, int off_lo, int off_hi) {
     float m0 = neg_inf(), m1 = neg_inf();
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c0; c < c0 + 2; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -132,11 +137,11 @@ __device__ __forceinline__ float exp_chunk(const uint32_t (&v)[32], int c, float
 
 // Second pass of the two-pass path: probabilities against the (new) row max m.
 template <typename T, bool MASKED>
-__device__ __forceinline__ float tile_exp(uint32_t taddr, float scale, float m, uint32_t p_taddr, int off_lo,
-                                          int off_hi) {
+__device__ __forceinline__ float tile_exp(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
+                                          int off_lo, int off_hi) {
     float sum = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c0; c < c0 + 2; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -149,11 +154,11 @@ __device__ __forceinline__ float tile_exp(uint32_t taddr, float scale, float m, 
 // P buffer while the tile max of the raw scores is tracked; the caller keeps them when the max
 // grew by at most 2^8 (so p <= 256), and otherwise redoes the tile.
 template <typename T, bool MASKED>
-__device__ __forceinline__ float tile_fused(uint32_t taddr, float scale, float m, uint32_t p_taddr, int off_lo,
-                                            int off_hi, float& m_raw) {
+__device__ __forceinline__ float tile_fused(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
+                                            int off_lo, int off_hi, float& m_raw) {
     float sum = 0.f, m0 = neg_inf(), m1 = neg_inf();
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c0; c < c0 + 2; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -210,14 +215,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i == B_PFULL || i == B_PFULL + 1) cnt = 128;
+            if (i == B_PFULL || i == B_PFULL + 1) cnt = kSoftmaxWarps * 32;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -230,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_p0 = t_o + D, t_p1 = t_o + D + 64;
     const uint32_t s_base = smem_u32(smem);
 
-    if (warp == 4) {
+    if (warp == kTmaWarp) {
         // ===================== TMA producer =====================
         // The whole warp runs the loop; lane 0 issues. Page ids of the next 32 boxes are read
         // from the block table by the 32 lanes at once and handed to lane 0 by shuffles, so a
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = max(0, issued - VST); i < issued; ++i) drain(&bars[B_VFULL + i % VST], (i / VST) & 1);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ===================== MMA issuer =====================
         // Descriptors are built once; a k-step or stage offset is an add to the address field.
         const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
@@ -355,9 +360,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else {
-        // ===================== softmax: thread = row =====================
-        const int r = tid;  // TMEM lane; warp w owns lanes 32w .. 32w+31
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // ===================== softmax: thread = row, two warps per row =====================
+        // Warp w owns TMEM lanes 32(w % 4) .. +31 (its rows) and columns half (w / 4) of every
+        // tile; the two warps of a row keep identical running maxima, exchange their partial
+        // maxima through shared memory when needed and add their partial sums at the end.
+        const int quad = warp & 3, half = warp >> 2;
+        const int r = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        const int c0 = half * 2;  // first 32-column chunk of this warp's half
+        float* xch = reinterpret_cast<float*>(smem + L_::XCH);
+        auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;\n" ::"r"(1 + quad) : "memory"); };
+        // max (or sum) of this row's two halves
+        auto exchange = [&](float mine, bool is_max) {
+            xch[half * BM + r] = mine;
+            pair_sync();
+            const float other = xch[(1 - half) * BM + r];
+            pair_sync();  // the slot may be written again only after the partner has read it
+            return is_max ? fmaxf(mine, other) : mine + other;
+        };
         const bool live = r < live_rows;
         const int64_t pos = p_first + (live ? r / G : 0);
         // keys this row sees: [row_lo, row_hi) (padding rows: every key of the sequence)
@@ -366,49 +386,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         // keys every live row sees: [all_lo, all_hi)
         const int64_t all_lo = p.window > 0 ? p_last - p.window + 1 : INT64_MIN;
         const int64_t all_hi = min64(p.causal ? p_first + 1 : si.L, si.L);
-        float m_run = neg_inf(), l_run = 0.f;
+        float m_run = neg_inf(), l_part = 0.f;
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
             const int b = i & 1;
             const int64_t kt0 = kt_start + (int64_t)i * BN;
             const uint32_t t_sb = (b ? t_s1 : t_s0) + lane_off;
             const bool full = kt0 >= all_lo && kt0 + BN <= all_hi;
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (i >> 1) & 1, wd, 8));
-            if (!ok) break;
+            // After an abort the loop still runs to its end (every wait then returns at once), so
+            // that both warps of a row reach the same row-statistics exchanges.
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (i >> 1) & 1, wd, 8)) && ok;
             tc_fence_after();
             // P buffer b was last read by P V of tile i - 2
             if (i >= 2) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((i - 2) >> 1) & 1, wd, 11));
-                if (!ok) break;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((i - 2) >> 1) & 1, wd, 11)) && ok;
             }
             const uint32_t t_pb = (b ? t_p1 : t_p0) + lane_off;
             const int off_lo = (int)(kt0 - row_lo), off_hi = (int)(kt0 - row_hi);
-            // Fast path: one pass with the running max when every row of the warp has one.
+            // Fast path: one pass with the running max when every row of the warp has one (both
+            // warps of a row decide alike: their running maxima are equal).
             bool redo = true;
             float sum = 0.f;
             if (__all_sync(0xffffffffu, m_run != neg_inf())) {
                 float m_raw;
-                sum = full ? tile_fused<T, false>(t_sb, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
-                           : tile_fused<T, true>(t_sb, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
+                sum = full ? tile_fused<T, false>(t_sb, c0, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
+                           : tile_fused<T, true>(t_sb, c0, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
+                m_raw = exchange(m_raw, true);
                 redo = __any_sync(0xffffffffu, m_raw * p.scale_log2 > m_run + 8.0f);
             }
             if (redo) {
-                // pass 1: tile max of the raw scores (S read from TMEM 32 columns at a time); the
-                // scale is positive, so it is applied to the max once. Edge tiles mask keys
-                // outside the row's visible range [row_lo, row_hi) first.
-                const float m_raw = full ? tile_max_full(t_sb) : tile_max_masked(t_sb, off_lo, off_hi);
+                // pass 1: tile max of the raw scores; the scale is positive, so it is applied to
+                // the max once. Edge tiles mask keys outside [row_lo, row_hi) first.
+                float m_raw = full ? tile_max_full(t_sb, c0) : tile_max_masked(t_sb, c0, off_lo, off_hi);
+                m_raw = exchange(m_raw, true);
                 const float m_tile = m_raw * p.scale_log2;
                 const float m_new = fmaxf(m_run, m_tile);
                 const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
                 const bool rescale = grow && i > 0 && m_run != neg_inf();
                 if (__any_sync(0xffffffffu, rescale)) {
                     // the output must hold every earlier tile before it is rescaled
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 9));
-                    if (!ok) break;
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 9)) && ok;
                     tc_fence_after();
                     const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {  // this warp's half of O
                         uint32_t v[32];
                         tmem_ld32(t_o + lane_off + c * 32, v);
                         tmem_ld_wait(v);
@@ -418,30 +439,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 if (grow) {
-                    l_run *= fast_exp2(m_run - m_new);
+                    l_part *= fast_exp2(m_run - m_new);
                     m_run = m_new;
                 }
                 const float m_use = m_run == neg_inf() ? 0.f : m_run;
                 // pass 2: probabilities p = 2^(s * scale - m) into the P buffer
-                sum = full ? tile_exp<T, false>(t_sb, p.scale_log2, m_use, t_pb, 0, 0)
-                           : tile_exp<T, true>(t_sb, p.scale_log2, m_use, t_pb, off_lo, off_hi);
+                sum = full ? tile_exp<T, false>(t_sb, c0, p.scale_log2, m_use, t_pb, 0, 0)
+                           : tile_exp<T, true>(t_sb, c0, p.scale_log2, m_use, t_pb, off_lo, off_hi);
             }
             tmem_st_wait();
-            l_run += sum;
+            l_part += sum;
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + b]);
         }
-        // ---- epilogue ----
+        // ---- epilogue: each warp of the pair stores its half of the output columns ----
         if (ok && n_tiles > 0)
             ok = __all_sync(0xffffffffu,
                             mbar_wait(&bars[B_ODONE + ((n_tiles - 1) & 1)], ((n_tiles - 1) >> 1) & 1, wd, 10));
+        ok = __all_sync(0xffffffffu, ok);
+        const float l_run = exchange(l_part, false);
         tc_fence_after();
         const bool has = l_run > 0.f;
         const float inv = has ? 1.0f / l_run : 0.f;
         const int64_t qrow = (int64_t)(si.q_start + u.j0 + (live ? r / G : 0)) * p.hq + u.kvh * G + (live ? r % G : 0);
         T* orow = static_cast<T*>(p.out) + qrow * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+#pragma unroll 1
+        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
             uint32_t v[32];
             if (ok && n_tiles > 0) {
                 tmem_ld32(t_o + lane_off + c * 32, v);
@@ -460,12 +483,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
             }
         }
-        if (live && ok) p.lse[qrow] = has ? (m_run + __log2f(l_run)) * kLn2 : neg_inf();
+        if (live && ok && half == 0) p.lse[qrow] = has ? (m_run + __log2f(l_run)) * kLn2 : neg_inf();
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
