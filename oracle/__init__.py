@@ -11,8 +11,10 @@ Pins (tests/test_oracle_pins.py): brute force against torch's fp64 SDPA/logsumex
 dense cases, closed forms (single key, constant V, Q = 0 -> exp(lse) counts the visible keys,
 W = 1 -> own value row, position probe), invariances (page permutation, split == unsplit,
 chunked == one-shot prefill, window >= context == no window, GQA == MHA on a repeated cache,
-MLA == single-head GQA on a concatenated key), and compile-time mutants of this file that the
-pins must reject.
+MLA == single-head GQA on a concatenated key), sparse top-K pins (every block selected ==
+dense attention, a planted block wins a top-1 selection and then equals attention restricted to
+that block, integer-valued scores fix ties exactly, a brute-force restatement on tiny cases), and
+compile-time mutants of the C file that the pins must reject.
 """
 from __future__ import annotations
 
@@ -49,6 +51,15 @@ class Oracle:
         lib.pao_paged_attention_backward.argtypes = [_P, _P, _P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                                      _I, _I, ctypes.c_double, ctypes.c_int, _I, _P, _P, _P,
                                                      ctypes.c_int]
+        lib.pao_sparse_block_scores.restype = ctypes.c_int
+        lib.pao_sparse_block_scores.argtypes = [_P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                                ctypes.c_double, ctypes.c_int, _I, _I, _I, _P, ctypes.c_int]
+        lib.pao_sparse_topk.restype = ctypes.c_int
+        lib.pao_sparse_topk.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
+        lib.pao_sparse_attention.restype = ctypes.c_int
+        lib.pao_sparse_attention.argtypes = [_P, _P, _P, ctypes.c_int, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                             _I, ctypes.c_double, ctypes.c_int, _I, _I, _P, _I, _P, _P, _P,
+                                             ctypes.c_int]
         lib.pao_lse_combine.restype = None
         lib.pao_lse_combine.argtypes = [_P, _P, ctypes.c_int64, ctypes.c_int64, _I, _P, _P]
         self.lib = lib
@@ -158,6 +169,90 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle rejected the schedule (code {rc})")
         return out, lse
+
+    # -- sparse top-K block attention ---------------------------------------------------------
+    @staticmethod
+    def num_blocks(seq_lens, block_size: int) -> torch.Tensor:
+        """Sparse blocks per sequence: ceil(L / block_size) (the last block may be partial)."""
+        sl = torch.as_tensor(seq_lens, dtype=torch.int64)
+        return (sl + block_size - 1) // block_size
+
+    def sparse_block_scores(self, q, k_cache, seq_lens, query_offsets, block_tables, page_size, scale,
+                            block_size, causal=True, window=0, max_blocks=None, nthreads=None):
+        """Proxy block scores [Nq, Hkv, max_blocks] float64 (-inf past a sequence's blocks)."""
+        dt = q.dtype
+        assert k_cache.dtype == dt and dt in _DT
+        q, k_cache = self._c(q), self._c(k_cache)
+        nq, hq, d = q.shape
+        num_pages, ps, hkv, _ = k_cache.shape
+        sl = self._c(seq_lens, torch.int32)
+        qo = self._c(query_offsets, torch.int32)
+        bt = self._c(block_tables, torch.int32)
+        if max_blocks is None:
+            max_blocks = int(self.num_blocks(sl, block_size).max().item()) if sl.numel() else 0
+        scores = torch.full((nq, hkv, max_blocks), float("nan"), dtype=torch.float64)
+        rc = self.lib.pao_sparse_block_scores(
+            q.data_ptr(), k_cache.data_ptr(), _DT[dt], sl.data_ptr(), qo.data_ptr(), sl.numel(), bt.data_ptr(),
+            bt.shape[1], page_size, num_pages, hq, hkv, d, float(scale), int(bool(causal)), int(window),
+            int(block_size), int(max_blocks), scores.data_ptr(), self._threads(nthreads))
+        if rc != 0:
+            raise ValueError(f"oracle rejected the arguments (code {rc})")
+        return scores
+
+    def sparse_topk(self, scores, seq_lens, query_offsets, block_size, topk, width=None):
+        """Selected blocks [Nq, Hkv, width] int32, ascending, -1 past the row's count."""
+        scores = self._c(scores, torch.float64)
+        nq, hkv, max_blocks = scores.shape
+        sl = self._c(seq_lens, torch.int32)
+        qo = self._c(query_offsets, torch.int32)
+        if width is None:
+            width = topk if topk > 0 else max_blocks
+        sel = torch.full((nq, hkv, width), -7, dtype=torch.int32)
+        rc = self.lib.pao_sparse_topk(scores.data_ptr(), sl.data_ptr(), qo.data_ptr(), sl.numel(), hkv, max_blocks,
+                                      int(block_size), int(topk), int(width), sel.data_ptr())
+        if rc != 0:
+            raise ValueError(f"oracle rejected the arguments (code {rc})")
+        return sel
+
+    def sparse_attention(self, q, k_cache, v_cache, seq_lens, query_offsets, block_tables, page_size, scale,
+                         block_size, selection, causal=True, window=0, rows=None, nthreads=None):
+        """Attention over the selected blocks: out [Nq, Hq, Dv], lse [Nq, Hq] float64."""
+        dt = q.dtype
+        assert k_cache.dtype == dt and v_cache.dtype == dt and dt in _DT
+        q, k_cache, v_cache = self._c(q), self._c(k_cache), self._c(v_cache)
+        nq, hq, d = q.shape
+        num_pages, ps, hkv, _ = k_cache.shape
+        dv = v_cache.shape[3]
+        sl = self._c(seq_lens, torch.int32)
+        qo = self._c(query_offsets, torch.int32)
+        bt = self._c(block_tables, torch.int32)
+        sel = self._c(selection, torch.int32)
+        assert sel.shape[0] == nq and sel.shape[1] == hkv
+        want = self._want(nq * hq, rows)
+        out = torch.full((nq, hq, dv), float("nan"), dtype=torch.float64)
+        lse = torch.full((nq, hq), float("nan"), dtype=torch.float64)
+        rc = self.lib.pao_sparse_attention(
+            q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), _DT[dt], sl.data_ptr(), qo.data_ptr(), sl.numel(),
+            bt.data_ptr(), bt.shape[1], page_size, num_pages, hq, hkv, d, dv, float(scale), int(bool(causal)),
+            int(window), int(block_size), sel.data_ptr(), sel.shape[2],
+            want.data_ptr() if want is not None else None, out.data_ptr(), lse.data_ptr(), self._threads(nthreads))
+        if rc == -4:
+            raise ValueError("selection entry out of range or repeated")
+        if rc != 0:
+            raise ValueError(f"oracle rejected the arguments (code {rc})")
+        return out, lse
+
+    def sparse(self, wl, block_size, topk, rows=None, nthreads=None):
+        """Proxy scores, selection and attention for a GQA workload: (scores, sel, out, lse)."""
+        s = wl.sched
+        scores = self.sparse_block_scores(wl.q, wl.k_cache, s.seq_lens, s.query_offsets, s.block_tables,
+                                          s.page_size, wl.scale, block_size, wl.causal, wl.window,
+                                          nthreads=nthreads)
+        sel = self.sparse_topk(scores, s.seq_lens, s.query_offsets, block_size, topk)
+        out, lse = self.sparse_attention(wl.q, wl.k_cache, wl.v_cache, s.seq_lens, s.query_offsets, s.block_tables,
+                                         s.page_size, wl.scale, block_size, sel, wl.causal, wl.window, rows,
+                                         nthreads)
+        return scores, sel, out, lse
 
     # -- merge of partial results -------------------------------------------------------------
     def lse_combine(self, o_parts: torch.Tensor, lse_parts: torch.Tensor):

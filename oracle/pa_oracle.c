@@ -25,6 +25,12 @@
  *  - lse is the natural-log logsumexp of the scaled, masked scores.
  * MLA (ruDNN `DevicePlan::mla`): score = scale * (q_lat . latent_t + q_rope . rope_t); the
  * latent is both key and value, so out has the latent width R.
+ * Sparse top-K (alice-llm `llama3_sparse_attention`): proxy block scores from the first query
+ * head of each group, top-K blocks per (query, kv head), attention over the selected blocks.
+ * Readings: a sequence has ceil(L / block_size) blocks (the last may be partial), so that
+ * "every block selected" is dense attention; the proxy score of a block is the largest scaled
+ * score over the keys of the block the query can see (-inf if none); equal scores rank the
+ * lower block index first.
  *
  * Inputs are the exact stored values (fp32, bf16 or fp16 bit patterns) widened to double.
  */
@@ -90,6 +96,13 @@ typedef struct {
     const uint8_t* want;      /* optional [Nq*Hq]: compute only rows with want != 0 */
     double* out;              /* [Nq, Hq, Dv] */
     double* lse;              /* [Nq, Hq] */
+    /* sparse top-K block selection */
+    int mode;                 /* 0: attention, 1: proxy block scores */
+    int32_t block_size;       /* keys per sparse block */
+    const int32_t* sel;       /* optional [Nq, Hkv, sel_width]: selected blocks, -1 = unused */
+    int32_t sel_width;
+    double* scores;           /* mode 1: [Nq, Hkv, max_blocks] */
+    int32_t max_blocks;
     /* work distribution over (sequence, kv head) */
     int64_t next_item;
     pthread_mutex_t lock;
@@ -114,7 +127,7 @@ static int pao_visible(const pao_job* J, int32_t s, int64_t t, int64_t p) {
 }
 
 static void pao_run_item(pao_job* J, int32_t s, int32_t kvh, double* kbuf, double* vbuf,
-                         double* krbuf, double* xbuf, double* qbuf) {
+                         double* krbuf, double* xbuf, double* qbuf, uint8_t* smask) {
     const int64_t L = J->seq_lens[s];
     const int64_t q0 = J->query_offsets[s];
     const int64_t n = J->query_offsets[s + 1] - q0;
@@ -170,9 +183,19 @@ static void pao_run_item(pao_job* J, int32_t s, int32_t kvh, double* kbuf, doubl
 #endif
             for (int32_t c = 0; c < kd; ++c) qbuf[c] = pao_load(J->q, J->dtype, r * kd + c);
             for (int32_t c = 0; c < J->pr; ++c) qbuf[kd + c] = pao_load(J->qr, J->dtype, r * J->pr + c);
+            if (J->sel) { /* sparse: only the keys of the blocks selected for (query, kv head) */
+                const int64_t nb = (L + J->block_size - 1) / J->block_size;
+                const int32_t* row_sel = J->sel + (qi * J->hkv + kvh) * (int64_t)J->sel_width;
+                for (int64_t b = 0; b < nb; ++b) smask[b] = 0;
+                for (int32_t e = 0; e < J->sel_width; ++e)
+                    if (row_sel[e] >= 0) smask[row_sel[e]] = 1;
+            }
             double m = -INFINITY;
             for (int64_t t = 0; t < L; ++t) {
-                if (!pao_visible(J, s, t, p)) { xbuf[t] = -INFINITY; continue; }
+                if (!pao_visible(J, s, t, p) || (J->sel && !smask[t / J->block_size])) {
+                    xbuf[t] = -INFINITY;
+                    continue;
+                }
                 double acc = 0.0;
                 for (int32_t c = 0; c < kd; ++c) acc += qbuf[c] * kbuf[t * kd + c];
 #ifndef PAO_MUTANT_DROP_ROPE
@@ -211,6 +234,63 @@ static void pao_run_item(pao_job* J, int32_t s, int32_t kvh, double* kbuf, doubl
     }
 }
 
+/* Number of sparse blocks of a sequence with L keys: the last block may be partial. */
+static int64_t pao_num_blocks(int64_t L, int32_t block_size) {
+#ifdef PAO_MUTANT_SPARSE_FLOOR
+    return L / block_size; /* wrong: drops a partial last block */
+#else
+    return (L + block_size - 1) / block_size;
+#endif
+}
+
+/*
+ * Proxy block scores of one (sequence, kv head): for every query of the sequence, the proxy
+ * query is the first query head of the KV head's group (alice-llm `llama3_sparse_attention`,
+ * "cheap proxy"), and the score of block b is the largest scaled score q_proxy . k_t over the
+ * keys t of the block the query can see; a block without a visible key scores -inf.
+ */
+static void pao_scores_item(pao_job* J, int32_t s, int32_t kvh, double* kbuf, double* qbuf) {
+    const int64_t L = J->seq_lens[s];
+    const int64_t q0 = J->query_offsets[s];
+    const int64_t n = J->query_offsets[s + 1] - q0;
+    const int32_t ps = J->page_size, kd = J->d, bs = J->block_size;
+    const int32_t G = J->hq / J->hkv;
+    if (n == 0) return;
+    for (int64_t t = 0; t < L; ++t) {
+        int64_t page = J->block_tables[(int64_t)s * J->table_width + t / ps];
+        int64_t row = (page * ps + t % ps) * J->hkv + kvh;
+        for (int32_t c = 0; c < kd; ++c) kbuf[t * kd + c] = pao_load(J->k, J->dtype, row * kd + c);
+    }
+    const int64_t nb = pao_num_blocks(L, bs);
+#ifdef PAO_MUTANT_SPARSE_PROXY_LAST
+    const int32_t h = kvh * G + G - 1; /* wrong proxy head */
+#else
+    const int32_t h = kvh * G;
+#endif
+    for (int64_t j = 0; j < n; ++j) {
+        const int64_t qi = q0 + j;
+        const int64_t p = L - n + j;
+        for (int32_t c = 0; c < kd; ++c) qbuf[c] = pao_load(J->q, J->dtype, (qi * J->hq + h) * kd + c);
+        double* out = J->scores + (qi * J->hkv + kvh) * (int64_t)J->max_blocks;
+        for (int64_t b = 0; b < J->max_blocks; ++b) {
+            double best = -INFINITY;
+            if (b < nb) {
+                const int64_t t1 = (b + 1) * bs < L ? (b + 1) * bs : L;
+                for (int64_t t = b * bs; t < t1; ++t) {
+#ifndef PAO_MUTANT_SPARSE_UNMASKED
+                    if (!pao_visible(J, s, t, p)) continue;
+#endif
+                    double acc = 0.0;
+                    for (int32_t c = 0; c < kd; ++c) acc += qbuf[c] * kbuf[t * kd + c];
+                    acc *= J->scale;
+                    if (acc > best) best = acc;
+                }
+            }
+            out[b] = best;
+        }
+    }
+}
+
 static void* pao_worker(void* arg) {
     pao_job* J = (pao_job*)arg;
     int64_t maxL = 0;
@@ -222,7 +302,8 @@ static void* pao_worker(void* arg) {
     double* krbuf = J->mla ? (double*)malloc(sizeof(double) * rows * (size_t)(J->pr > 0 ? J->pr : 1)) : NULL;
     double* xbuf = (double*)malloc(sizeof(double) * rows);
     double* qbuf = (double*)malloc(sizeof(double) * (size_t)(J->d + J->pr));
-    if (!kbuf || (!J->mla && !vbuf) || (J->mla && !krbuf) || !xbuf || !qbuf) {
+    uint8_t* smask = J->sel ? (uint8_t*)malloc((size_t)(rows / (J->block_size > 0 ? J->block_size : 1) + 2)) : NULL;
+    if (!kbuf || (!J->mla && !vbuf) || (J->mla && !krbuf) || !xbuf || !qbuf || (J->sel && !smask)) {
         pthread_mutex_lock(&J->lock);
         J->error = 1;
         pthread_mutex_unlock(&J->lock);
@@ -233,9 +314,14 @@ static void* pao_worker(void* arg) {
             int64_t it = J->next_item++;
             pthread_mutex_unlock(&J->lock);
             if (it >= (int64_t)J->num_seqs * kheads) break;
-            pao_run_item(J, (int32_t)(it / kheads), (int32_t)(it % kheads), kbuf, vbuf, krbuf, xbuf, qbuf);
+            if (J->mode == 1)
+                pao_scores_item(J, (int32_t)(it / kheads), (int32_t)(it % kheads), kbuf, qbuf);
+            else
+                pao_run_item(J, (int32_t)(it / kheads), (int32_t)(it % kheads), kbuf, vbuf, krbuf, xbuf, qbuf,
+                             smask);
         }
     }
+    free(smask);
     free(kbuf);
     free(vbuf);
     free(krbuf);
@@ -356,6 +442,123 @@ void pao_lse_combine(const double* o_parts, const double* lse_parts, int64_t npa
             for (int32_t c = 0; c < dv; ++c) o[c] += w * o_parts[(i * rows + r) * dv + c];
         }
     }
+}
+
+/*
+ * Sparse top-K block attention (alice-llm `llama3_sparse_attention`: proxy block scores,
+ * top-K block selection, attention over the selected blocks, merge of the partials). The keys
+ * of sequence s are cut into ceil(L_s / block_size) blocks of block_size consecutive positions
+ * (the last one may be partial); queries attend only to the keys of the blocks selected for
+ * their (query, kv head), with the usual causal/window mask on top. All G query heads of a
+ * group share their KV head's selection.
+ */
+
+/* Proxy block scores, [Nq, Hkv, max_blocks] (blocks past a sequence's count: -inf). */
+int pao_sparse_block_scores(const void* q, const void* k_cache, int dtype, const int32_t* seq_lens,
+                            const int32_t* query_offsets, int32_t num_seqs, const int32_t* block_tables,
+                            int32_t table_width, int32_t page_size, int32_t num_pages, int32_t hq,
+                            int32_t hkv, int32_t d, double scale, int causal, int32_t window,
+                            int32_t block_size, int32_t max_blocks, double* scores, int nthreads) {
+    if (hq <= 0 || hkv <= 0 || hq % hkv || d <= 0 || window < 0 || block_size <= 0 || max_blocks < 0)
+        return -1;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        if (pao_num_blocks(seq_lens[s], block_size) > max_blocks) return -1;
+    pao_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k_cache; J.v = NULL; J.dtype = dtype; J.mla = 0; J.mode = 1;
+    J.seq_lens = seq_lens; J.query_offsets = query_offsets; J.num_seqs = num_seqs;
+    J.block_tables = block_tables; J.table_width = table_width; J.page_size = page_size;
+    J.num_pages = num_pages; J.hq = hq; J.hkv = hkv; J.d = d; J.dv = d; J.pr = 0;
+    J.scale = scale; J.causal = causal; J.window = window;
+    J.block_size = block_size; J.scores = scores; J.max_blocks = max_blocks;
+    return pao_run(&J, nthreads);
+}
+
+/*
+ * Top-K selection per (query, kv head) row from the proxy scores. A sequence with nb blocks
+ * keeps k = nb blocks when topk is 0 or at least nb (the dense case), else k = topk: the k
+ * highest scores, equal scores going to the lower block index. The selected indices are
+ * written in ascending order into [Nq, Hkv, width], the rest of the row set to -1.
+ * Returns -1 when width < k for some sequence.
+ */
+int pao_sparse_topk(const double* scores, const int32_t* seq_lens, const int32_t* query_offsets,
+                    int32_t num_seqs, int32_t hkv, int32_t max_blocks, int32_t block_size, int32_t topk,
+                    int32_t width, int32_t* sel) {
+    if (hkv <= 0 || block_size <= 0 || topk < 0 || width < 0) return -1;
+    uint8_t* picked = (uint8_t*)malloc((size_t)max_blocks + 1);
+    if (!picked) return -3;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        const int64_t nb = pao_num_blocks(seq_lens[s], block_size);
+        if (nb > max_blocks) { free(picked); return -1; }
+        const int64_t k = (topk == 0 || topk >= nb) ? nb : topk;
+        if (k > width) { free(picked); return -1; }
+        for (int64_t qi = query_offsets[s]; qi < query_offsets[s + 1]; ++qi) {
+            for (int32_t h = 0; h < hkv; ++h) {
+                const double* sc = scores + (qi * hkv + h) * (int64_t)max_blocks;
+                int32_t* out = sel + (qi * hkv + h) * (int64_t)width;
+                for (int64_t b = 0; b < nb; ++b) picked[b] = 0;
+                for (int64_t r = 0; r < k; ++r) { /* take the best block not taken yet */
+                    int64_t best = -1;
+                    for (int64_t b = 0; b < nb; ++b) {
+                        if (picked[b]) continue;
+#if defined(PAO_MUTANT_SPARSE_TIES_HIGH)
+                        if (best < 0 || sc[b] >= sc[best]) best = b;
+#elif defined(PAO_MUTANT_SPARSE_MIN)
+                        if (best < 0 || sc[b] < sc[best]) best = b;
+#else
+                        if (best < 0 || sc[b] > sc[best]) best = b;
+#endif
+                    }
+                    if (best < 0) break;
+                    picked[best] = 1;
+                }
+                int32_t e = 0;
+                for (int64_t b = 0; b < nb; ++b)
+                    if (picked[b]) out[e++] = (int32_t)b;
+                for (; e < width; ++e) out[e] = -1;
+            }
+        }
+    }
+    free(picked);
+    return 0;
+}
+
+/*
+ * Attention restricted to selected blocks. selection [Nq, Hkv, width]: block indices, -1 for
+ * an unused entry. Returns -4 if an entry lies outside [0, nb) of its sequence or repeats a
+ * block of its row; otherwise as pao_paged_attention.
+ */
+int pao_sparse_attention(const void* q, const void* k_cache, const void* v_cache, int dtype,
+                         const int32_t* seq_lens, const int32_t* query_offsets, int32_t num_seqs,
+                         const int32_t* block_tables, int32_t table_width, int32_t page_size,
+                         int32_t num_pages, int32_t hq, int32_t hkv, int32_t d, int32_t dv, double scale,
+                         int causal, int32_t window, int32_t block_size, const int32_t* selection,
+                         int32_t width, const uint8_t* want_rows, double* out, double* lse, int nthreads) {
+    if (hq <= 0 || hkv <= 0 || hq % hkv || d <= 0 || dv <= 0 || window < 0 || block_size <= 0 || width < 0)
+        return -1;
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        const int64_t nb = pao_num_blocks(seq_lens[s], block_size);
+        for (int64_t qi = query_offsets[s]; qi < query_offsets[s + 1]; ++qi)
+            for (int32_t h = 0; h < hkv; ++h) {
+                const int32_t* row = selection + (qi * hkv + h) * (int64_t)width;
+                for (int32_t e = 0; e < width; ++e) {
+                    if (row[e] == -1) continue;
+                    if (row[e] < 0 || row[e] >= nb) return -4;
+                    for (int32_t f = 0; f < e; ++f)
+                        if (row[f] == row[e]) return -4;
+                }
+            }
+    }
+    pao_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.k = k_cache; J.v = v_cache; J.dtype = dtype; J.mla = 0;
+    J.seq_lens = seq_lens; J.query_offsets = query_offsets; J.num_seqs = num_seqs;
+    J.block_tables = block_tables; J.table_width = table_width; J.page_size = page_size;
+    J.num_pages = num_pages; J.hq = hq; J.hkv = hkv; J.d = d; J.dv = dv; J.pr = 0;
+    J.scale = scale; J.causal = causal; J.window = window;
+    J.want = want_rows; J.out = out; J.lse = lse;
+    J.block_size = block_size; J.sel = selection; J.sel_width = width;
+    return pao_run(&J, nthreads);
 }
 
 /*

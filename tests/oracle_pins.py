@@ -13,7 +13,11 @@ when the oracle disagrees with the fact it checks. Sources of truth:
     merging the parts (ruDNN "merge FP32 statistics"; alice-llm `lse_combine`), splitting a
     prefill chunk in two, a window wider than the context, GQA on a repeated cache, MLA as
     single-head attention on the concatenated key;
-  * exact widening of bf16/fp16 inputs (same values given as fp32 give identical results).
+  * exact widening of bf16/fp16 inputs (same values given as fp32 give identical results);
+  * sparse top-K (alice-llm `llama3_sparse_attention`): a torch restatement on tiny cases, every
+    block selected == dense attention, a planted block wins top-1 and then equals attention
+    restricted to its keys, Q = 0 makes all visible blocks tie (lowest indices win, uniform
+    weights), and the page's own bridge tests on `fixture_gqa`.
 """
 from __future__ import annotations
 
@@ -397,10 +401,178 @@ def pin_backward_finite_differences(orc):
         assert abs(fd - an) <= 1e-4 * max(1.0, abs(an)), (name, idx, fd, an)
 
 
+# ---- sparse top-K block selection (alice-llm `llama3_sparse_attention`) -------------------------
+
+def _sparse_cases():
+    """(workload, block_size) pairs: decode and prefill chunks, windows, ragged last blocks."""
+    return [
+        (W.make_gqa("s1", 21, [37, 100, 64], [1, 1, 1], 4, 2, 8, 8, 4, torch.float32, causal=True), 8),
+        (W.make_gqa("s2", 22, [45, 30], [9, 30], 6, 3, 16, 8, 8, torch.float32, causal=True, window=13), 8),
+        (W.make_gqa("s3", 23, [50, 19], [5, 19], 4, 1, 8, 12, 4, torch.bfloat16, causal=False), 12),
+        (W.make_gqa("s4", 24, [70], [16], 8, 2, 8, 8, 16, torch.float32, causal=True), 16),
+    ]
+
+
+def _brute_sparse(wl, bs, topk):
+    """Proxy scores, selection and attention restated with torch on the dense gather."""
+    s_ = wl.sched
+    G = wl.num_q_heads // wl.num_kv_heads
+    nq = s_.num_queries
+    nb_max = max(1, max((int(L) + bs - 1) // bs for L in s_.seq_lens))
+    scores = torch.full((nq, wl.num_kv_heads, nb_max), float("-inf"), dtype=torch.float64)
+    width = topk if topk > 0 else nb_max
+    sel = torch.full((nq, wl.num_kv_heads, width), -1, dtype=torch.int32)
+    out = torch.zeros(nq, wl.num_q_heads, wl.v_head_dim, dtype=torch.float64)
+    lse = torch.full((nq, wl.num_q_heads), float("-inf"), dtype=torch.float64)
+    for s in range(s_.num_seqs):
+        L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+        if n == 0:
+            continue
+        nb = (L + bs - 1) // bs
+        k = nb if (topk == 0 or topk >= nb) else topk
+        K = _dense_kv(wl.k_cache, s_.block_tables, s, L, s_.page_size)
+        V = _dense_kv(wl.v_cache, s_.block_tables, s, L, s_.page_size)
+        for j in range(n):
+            p = L - n + j
+            t = torch.arange(L)
+            vis = torch.ones(L, dtype=torch.bool)
+            if wl.causal:
+                vis &= t <= p
+            if wl.window > 0:
+                vis &= t + wl.window > p
+            for kvh in range(wl.num_kv_heads):
+                qp = wl.q[q0 + j, kvh * G].double()
+                sc = (K[:, kvh] @ qp) * wl.scale
+                blk = []
+                for b in range(nb):
+                    m = sc[b * bs:(b + 1) * bs][vis[b * bs:(b + 1) * bs]]
+                    blk.append(float(m.max()) if m.numel() else float("-inf"))
+                scores[q0 + j, kvh, :nb] = torch.tensor(blk, dtype=torch.float64)
+                chosen = sorted(sorted(range(nb), key=lambda b: (-blk[b], b))[:k])
+                sel[q0 + j, kvh, :k] = torch.tensor(chosen, dtype=torch.int32)
+                keep = vis & torch.isin(t // bs, torch.tensor(chosen, dtype=torch.int64))
+                for g in range(G):
+                    h = kvh * G + g
+                    x = (K[:, kvh] @ wl.q[q0 + j, h].double()) * wl.scale
+                    if keep.any():
+                        w = torch.softmax(x[keep], dim=0)
+                        out[q0 + j, h] = w @ V[keep, kvh]
+                        lse[q0 + j, h] = torch.logsumexp(x[keep], dim=0)
+    return scores, sel, out, lse
+
+
+def pin_sparse_bruteforce(orc):
+    """Scores, the exact selection and the output against a torch restatement, for top-k below,
+    at and above the block count."""
+    for wl, bs in _sparse_cases():
+        for topk in (1, 2, 3, 0):
+            rs, rsel, rout, rlse = _brute_sparse(wl, bs, topk)
+            sc, sel, out, lse = orc.sparse(wl, bs, topk)
+            assert sc.shape == rs.shape and torch.allclose(sc, rs, rtol=1e-12, atol=1e-12, equal_nan=False), wl.name
+            assert torch.equal(sel, rsel), (wl.name, topk)
+            assert torch.allclose(out, rout, rtol=1e-11, atol=1e-12), (wl.name, topk, (out - rout).abs().max())
+            assert torch.allclose(lse, rlse, rtol=1e-12, atol=1e-12), (wl.name, topk)
+
+
+def pin_sparse_dense_fallback(orc):
+    """Every block selected (top-k 0, equal to or above the block count) is dense attention: the
+    selection is 0 .. nb-1 and out/lse equal the dense oracle's."""
+    for wl, bs in _sparse_cases():
+        dout, dlse = orc.run(wl)
+        s_ = wl.sched
+        nbs = orc.num_blocks(s_.seq_lens, bs)
+        for topk in (0, int(nbs.max()), int(nbs.max()) + 5):
+            sc, sel, out, lse = orc.sparse(wl, bs, topk)
+            for s in range(s_.num_seqs):
+                nb = int(nbs[s])
+                rows = sel[int(s_.query_offsets[s]):int(s_.query_offsets[s + 1])]
+                assert torch.equal(rows[..., :nb], torch.arange(nb, dtype=torch.int32).expand_as(rows[..., :nb]))
+                assert bool((rows[..., nb:] == -1).all())
+            assert torch.allclose(out, dout, rtol=1e-13, atol=1e-14), (wl.name, topk)
+            assert torch.allclose(lse, dlse, rtol=1e-13, atol=1e-14), (wl.name, topk)
+
+
+def pin_sparse_planted_block(orc):
+    """Decode: one key of block b*_s is a large multiple of the proxy query of every KV head, so a
+    top-1 selection is b*_s for all heads, and the output equals dense attention restricted to
+    the keys of b*_s (key_begin/key_end)."""
+    bs = 8
+    wl = W.make_gqa("plant", 31, [37, 100, 64, 8], [1, 1, 1, 1], 4, 2, 8, 8, 4, torch.float32, causal=True)
+    s_ = wl.sched
+    G = 2
+    gen = torch.Generator().manual_seed(5)
+    kb, ke = [], []
+    for s in range(s_.num_seqs):
+        L = int(s_.seq_lens[s])
+        nb = (L + bs - 1) // bs
+        b = int(torch.randint(0, nb, (1,), generator=gen))
+        t = min(L - 1, b * bs + int(torch.randint(0, bs, (1,), generator=gen)))
+        page = int(s_.block_tables[s, t // s_.page_size])
+        for kvh in range(wl.num_kv_heads):
+            wl.k_cache[page, t % s_.page_size, kvh] = 40.0 * wl.q[int(s_.query_offsets[s]), kvh * G]
+        kb.append(b * bs)
+        ke.append(min(L, (b + 1) * bs))
+    sc, sel, out, lse = orc.sparse(wl, bs, 1)
+    for s in range(s_.num_seqs):
+        assert bool((sel[s, :, 0] == kb[s] // bs).all()), (s, sel[s])
+    kb_t = torch.tensor(kb, dtype=torch.int32)
+    ke_t = torch.tensor(ke, dtype=torch.int32)
+    rout, rlse = orc.attention(wl.q, wl.k_cache, wl.v_cache, s_.seq_lens, s_.query_offsets, s_.block_tables,
+                               s_.page_size, wl.scale, True, 0, key_begin=kb_t, key_end=ke_t)
+    assert torch.equal(out, rout) and torch.equal(lse, rlse)
+
+
+def pin_sparse_ties_lower_index(orc):
+    """Q = 0: every visible block scores exactly 0 and blocks without a visible key -inf, so the
+    selection is the lowest-indexed k visible blocks; the output is the mean of V over their
+    visible keys and exp(lse) their count."""
+    bs = 4
+    wl = W.make_gqa("ties", 41, [30, 23, 40], [1, 6, 1], 4, 2, 8, 8, 4, torch.float32, causal=True, window=11)
+    wl.q.zero_()
+    s_ = wl.sched
+    topk = 2
+    sc, sel, out, lse = orc.sparse(wl, bs, topk)
+    for s in range(s_.num_seqs):
+        L = int(s_.seq_lens[s]); q0 = int(s_.query_offsets[s]); n = int(s_.query_offsets[s + 1]) - q0
+        V = _dense_kv(wl.v_cache, s_.block_tables, s, L, s_.page_size)
+        for j in range(n):
+            p = L - n + j
+            lo = max(0, p - wl.window + 1)
+            first = lo // bs
+            want = [first, first + 1] if first + 1 <= p // bs else [first]
+            for kvh in range(wl.num_kv_heads):
+                got = [b for b in sel[q0 + j, kvh].tolist() if b >= 0]
+                assert got == want, (s, j, got, want)
+                keys = [t for t in range(lo, p + 1) if t // bs in want]
+                ref = V[keys, kvh].mean(dim=0)
+                for g in range(2):
+                    h = kvh * 2 + g
+                    assert torch.allclose(out[q0 + j, h], ref, rtol=1e-13, atol=1e-14)
+                    assert abs(math.exp(float(lse[q0 + j, h])) - len(keys)) < 1e-9 * len(keys)
+
+
+def pin_sparse_alice_fixture(orc):
+    """alice-llm bridge tests on `fixture_gqa` (blocks and pages of 4 keys, non-causal): top-k 0
+    and top-k 3 (= the block count) match dense attention; top-2 of 3 gives finite values."""
+    q, k, v, sl, qo, bt, ps, scale = alice_fixture()
+    dout, _ = orc.attention(q, k, v, sl, qo, bt, ps, scale, causal=False, window=0)
+    for topk in (0, 3, 2):
+        sc = orc.sparse_block_scores(q, k, sl, qo, bt, ps, scale, 4, causal=False)
+        sel = orc.sparse_topk(sc, sl, qo, 4, topk)
+        out, _ = orc.sparse_attention(q, k, v, sl, qo, bt, ps, scale, 4, sel, causal=False)
+        if topk == 2:
+            assert bool(torch.isfinite(out).all()) and bool((sel >= 0).sum(-1).eq(2).all())
+        else:
+            rel = ((out - dout).abs() / dout.abs().clamp_min(1e-6)).max()
+            assert rel < 1e-12, (topk, rel)
+
+
 ALL_PINS = [
     pin_sdpa_bruteforce, pin_alice_fixture_dense, pin_single_key, pin_constant_v_per_kv_head,
     pin_q_zero_counts_and_mean, pin_position_probe, pin_large_score_selects_target,
     pin_page_permutation_invariance, pin_split_equals_unsplit, pin_chunked_equals_oneshot,
     pin_window_cases, pin_gqa_equals_mha_repeated, pin_mla_equals_gqa_concat,
     pin_half_precision_widening, pin_backward_vs_autograd, pin_backward_finite_differences,
+    pin_sparse_bruteforce, pin_sparse_dense_fallback, pin_sparse_planted_block, pin_sparse_ties_lower_index,
+    pin_sparse_alice_fixture,
 ]

@@ -23,6 +23,11 @@ MUTANTS = [
     "PAO_MUTANT_UNNORMALISED",    # output not divided by the softmax sum
     "PAO_MUTANT_SCALE_DROPPED",   # scores not scaled
     "PAO_MUTANT_BWD_NO_D",        # backward without the rowsum(dO * O) term
+    "PAO_MUTANT_SPARSE_FLOOR",    # partial last block dropped (floor block count)
+    "PAO_MUTANT_SPARSE_PROXY_LAST",  # proxy from the last query head of the group
+    "PAO_MUTANT_SPARSE_TIES_HIGH",   # equal scores rank the higher block index first
+    "PAO_MUTANT_SPARSE_MIN",      # lowest-scoring blocks selected
+    "PAO_MUTANT_SPARSE_UNMASKED", # proxy ignores the causal/window mask
 ]
 
 
