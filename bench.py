@@ -297,10 +297,13 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
     """The other configurations, timed the same way (few steps): context for the headline."""
     res = {}
     cfgs = [("bf16_chunked_prefill", W.c3_chunked_prefill), ("bf16_window_mixed", W.c4_window_mixed),
-            ("bf16_mla_decode", W.c5_mla_decode)]
+            ("bf16_mla_decode", W.c5_mla_decode), ("bf16_sparse_topk_decode", W.sparse_bf16_decode)]
     if only is not None:
         cfgs = [only]
     for name, fn in cfgs:
+        if name == "bf16_sparse_topk_decode":
+            res[name] = run_sparse(args, pa, W, dev, hbm, peak_src, only is not None)
+            continue
         try:
             wl = fn(args.seed)
             flops = W.algorithmic_flops(wl)
@@ -342,6 +345,33 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
     return res
 
 
+def run_sparse(args, pa, W, dev, hbm, peak_src, alone):
+    """Sparse top-K decode: one step = proxy scores + top-K selection + attention over the
+    selected blocks + merge (pa_sparse_select then pa_sparse_forward)."""
+    try:
+        wl, bs, topk = W.sparse_bf16_decode(args.seed)
+        plan = pa.plan_for(wl, device=dev.index)
+        q, k, v = wl.q.to(dev), wl.k_cache.to(dev), wl.v_cache.to(dev)
+        out = torch.empty(q.shape[0], q.shape[1], wl.v_head_dim, dtype=q.dtype, device=dev)
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+        sel = torch.empty(q.shape[0], wl.num_kv_heads, topk, dtype=torch.int32, device=dev)
+
+        def step(tr):
+            pa.pa_sparse_select(plan, q, k, sel, wl.scale, bs, topk, wl.causal, wl.window)
+            pa.pa_sparse_forward(plan, q, k, v, sel, out, lse, wl.scale, bs, wl.causal, wl.window)
+        ms, _, _, _ = time_forward(pa, plan, step, args.extra_steps, args.warmup if alone else 3, False, None, 1)
+        launches = pa.pa_plan_get_info(plan)["last_launches"] + 2
+        nbytes = W.sparse_bytes(wl, bs, sel)
+        plan.close()
+        return {"ms_per_step": round(ms, 4), "block_size": bs, "topk": topk,
+                "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                "frac_hbm_of_%s" % peak_src: round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4),
+                "algorithmic_mb": round(nbytes / 1e6, 1),
+                "dense_kv_mb": round(W.algorithmic_kv_bytes(wl) / 1e6, 1), "launches": launches}
+    except Exception as e:  # a failing extra must not hide the headline
+        return {"error": str(e)[:300]}
+
+
 def run_single(args, ws, rank, local):
     """One of the other configurations as the only workload (profiling and tuning runs)."""
     import paged_kv_attention_39_b200 as pa
@@ -351,9 +381,13 @@ def run_single(args, ws, rank, local):
     dev = torch.device("cuda", local)
     args.extra_steps = args.steps
     fns = {"bf16_chunked_prefill": W.c3_chunked_prefill, "bf16_window_mixed": W.c4_window_mixed,
-           "bf16_mla_decode": W.c5_mla_decode, "tiny_fp32_decode": W.c1_tiny_fp32_decode}
+           "bf16_mla_decode": W.c5_mla_decode, "tiny_fp32_decode": W.c1_tiny_fp32_decode,
+           "bf16_sparse_topk_decode": W.sparse_bf16_decode}
     res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
     r = res[args.workload]
+    if args.workload == "bf16_sparse_topk_decode":
+        return {"metric": METRIC, "workload": args.workload, "value": r.get("gbs"), "unit": "GB/s",
+                "steps": args.steps, "warmup": args.warmup, "detail": r}
     return {"metric": METRIC, "workload": args.workload, "value": r.get("tflops"), "unit": "TFLOP/s",
             "steps": args.steps, "warmup": args.warmup, "detail": r}
 
@@ -428,7 +462,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--workload", default="bf16_decode",
-                    choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode",
+                    choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode", "bf16_sparse_topk_decode",
                              "tiny_fp32_decode"],
                     help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()

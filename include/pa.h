@@ -281,6 +281,74 @@ pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_
                           const pa_forward_options* opts);
 
 /*
+ * Sparse top-K block attention (alice-llm 2.0.0, sparse_attention/llama3_bridge.rs,
+ * `llama3_sparse_attention`): a cheap proxy pass scores fixed-size blocks of keys, each
+ * (query, KV head) keeps its top-K blocks, and attention runs over the keys of those blocks only;
+ * the per-block partials are merged with the split-KV logsumexp merge (alice-llm `lse_combine`).
+ *
+ * Blocks. The keys of sequence s are cut into nb_s = ceil(L_s / block_size) blocks of
+ * block_size consecutive positions (the last one may be partial; reading of the page's
+ * num_pages / (block_size / page_size), which drops a partial last block and would break its
+ * "top-K 0 equals dense attention" guarantee). block_size must be a positive multiple of the
+ * plan's page_size (the page's BlockPageMismatch rule) and nb_s <= PA_SPARSE_MAX_BLOCKS.
+ */
+#define PA_SPARSE_MAX_BLOCKS 16384
+
+/*
+ * pa_sparse_select -- proxy block scores and top-K block selection, on `stream`.
+ *
+ * Proxy: for query i of sequence s and KV head h the proxy query is the first query head of
+ * the group, q[i, h * G, :] (the page's "cheap proxy = the first Q lane of each KV head"). The
+ * score of block b is the largest scaled score scale * q_proxy . k[t, h, :] over the keys t of
+ * b that query i can see (causal/window at absolute positions as in pa_forward); a block
+ * without a visible key scores -inf. Scores are float32 dot products of the stored values.
+ * Selection: k_i = nb_s when topk == 0 or topk >= nb_s (every block: the dense case), else
+ * topk; the k_i blocks with the highest scores, equal scores ranking the lower block index
+ * first, are written in ascending block order to selection[i, h, 0 .. k_i), and the rest of
+ * the row is set to -1.
+ *
+ *   q, k_cache    as pa_forward (v is not read)
+ *   topk          >= 0
+ *   selection     [N_q, num_kv_heads, width] int32 device, written; width >= max_s k_s
+ *   block_scores  NULL, or [N_q, num_kv_heads, scores_width] float32 device, written with the
+ *                 proxy scores (-inf past a sequence's blocks); scores_width >= max_s nb_s
+ *
+ * Errors: as pa_forward, plus PA_ERR_SHAPE (block_size not a positive multiple of page_size,
+ * width or scores_width too small), PA_ERR_UNSUPPORTED (more than PA_SPARSE_MAX_BLOCKS blocks
+ * in a sequence), PA_ERR_ALIAS (selection or block_scores overlapping q, k_cache or each other).
+ */
+pa_status pa_sparse_select(pa_plan* plan, const void* q, const void* k_cache, pa_dtype dtype,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                           int causal, int32_t window, int32_t block_size, int32_t topk,
+                           int32_t* selection, int32_t width, float* block_scores,
+                           int32_t scores_width, pa_stream stream);
+
+/*
+ * pa_sparse_forward -- attention over selected key blocks (alice-llm `kvouter_attention` /
+ * `kvouter_forward` + `lse_combine`), on `stream`.
+ *
+ * Query row (i, h) attends to the keys t of the blocks listed in selection[i, h / G, :] that
+ * it can see (causal/window as in pa_forward); out and lse are those of softmax over exactly
+ * those keys (a row left with no key gets out = 0, lse = -inf). A selection row holds block
+ * indices of its sequence, in any order, and -1 for unused entries; every G query heads of a
+ * KV head share its row. The selection is read on the device only: an entry outside
+ * [-1, nb_s) or a block listed twice in one row sets the plan's device error word
+ * (pa_plan_device_status reports 64) and is skipped; that call's results are then undefined.
+ *
+ *   q, k_cache, v_cache, dtype, heads, dims, scale, causal, window, out, lse   as pa_forward
+ *   block_size   as pa_sparse_select
+ *   selection    [N_q, num_kv_heads, width] int32 device (e.g. pa_sparse_select's), width >= 0
+ *
+ * Errors: as pa_forward, plus PA_ERR_SHAPE for block_size, PA_ERR_UNSUPPORTED for more than
+ * PA_SPARSE_MAX_BLOCKS blocks in a sequence, PA_ERR_ALIAS if out or lse overlaps selection.
+ */
+pa_status pa_sparse_forward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                            pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t v_head_dim, float scale, int causal,
+                            int32_t window, int32_t block_size, const int32_t* selection,
+                            int32_t width, void* out, float* lse, pa_stream stream);
+
+/*
  * pa_plan_device_status -- diagnostic read of the plan's device error word (synchronous copy:
  * not for the hot path). 0 means no kernel reported a failure; a non-zero code means a kernel
  * gave up a bounded wait in its pipeline (the results of that call are undefined).

@@ -30,8 +30,9 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
            "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex", "pa_append", "pa_backward",
-           "pa_plan_device_status",
+           "pa_plan_device_status", "pa_sparse_select", "pa_sparse_forward",
            "pa_status_string", "pa_last_error_message", "pa_version"]
+PA_SPARSE_MAX_BLOCKS = 16384
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -98,6 +99,12 @@ def load_library(path: Optional[str] = None):
                                 _I, _P, _P, _P, _P]
     lib.pa_plan_device_status.restype = ctypes.c_int
     lib.pa_plan_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
+    lib.pa_sparse_select.restype = ctypes.c_int
+    lib.pa_sparse_select.argtypes = [_P, _P, _P, ctypes.c_int, _I, _I, _I, ctypes.c_float, ctypes.c_int, _I, _I, _I,
+                                     _P, _I, _P, _I, _P]
+    lib.pa_sparse_forward.restype = ctypes.c_int
+    lib.pa_sparse_forward.argtypes = [_P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _I, ctypes.c_float, ctypes.c_int, _I,
+                                      _I, _P, _I, _P, _P, _P]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_status_string.argtypes = [ctypes.c_int]
     lib.pa_last_error_message.restype = ctypes.c_char_p
@@ -245,6 +252,41 @@ def pa_forward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _DTYPES[q.dtype], q.shape[1],
         k_cache.shape[2], q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window),
         _ptr(out), _ptr(lse), _stream_ptr(stream, plan.device), _opts(kv_chunk, path, trace)))
+
+
+def pa_sparse_select(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, selection: torch.Tensor, scale: float,
+                     block_size: int, topk: int, causal: bool = True, window: int = 0,
+                     block_scores: Optional[torch.Tensor] = None, num_q_heads: Optional[int] = None,
+                     stream=None) -> None:
+    """Proxy block scores and top-K selection: selection [Nq, Hkv, width] int32 (in place), and
+    block_scores [Nq, Hkv, scores_width] float32 when given."""
+    for t in (q, k_cache, selection) + ((block_scores,) if block_scores is not None else ()):
+        if not t.is_contiguous():
+            raise ValueError("pa_sparse_select takes contiguous tensors")
+    if selection.dtype != torch.int32:
+        raise ValueError("selection must be int32")
+    if block_scores is not None and block_scores.dtype != torch.float32:
+        raise ValueError("block_scores must be float32")
+    _check(load_library().pa_sparse_select(
+        plan.handle, _ptr(q), _ptr(k_cache), _DTYPES[q.dtype], num_q_heads or q.shape[1], k_cache.shape[2],
+        q.shape[2], float(scale), int(bool(causal)), int(window), int(block_size), int(topk), _ptr(selection),
+        selection.shape[2], _ptr(block_scores), block_scores.shape[2] if block_scores is not None else 0,
+        _stream_ptr(stream, plan.device)))
+
+
+def pa_sparse_forward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      selection: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, scale: float, block_size: int,
+                      causal: bool = True, window: int = 0, stream=None) -> None:
+    """Attention over the blocks in selection [Nq, Hkv, width] int32 -> out, lse (in place)."""
+    for t in (q, k_cache, v_cache, selection, out, lse):
+        if not t.is_contiguous():
+            raise ValueError("pa_sparse_forward takes contiguous tensors")
+    if lse.dtype != torch.float32 or selection.dtype != torch.int32:
+        raise ValueError("lse must be float32 and selection int32")
+    _check(load_library().pa_sparse_forward(
+        plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _DTYPES[q.dtype], q.shape[1], k_cache.shape[2],
+        q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window), int(block_size),
+        _ptr(selection), selection.shape[2], _ptr(out), _ptr(lse), _stream_ptr(stream, plan.device)))
 
 
 def pa_append(plan: Plan, new_k: torch.Tensor, new_v: torch.Tensor, k_cache: torch.Tensor,

@@ -63,6 +63,7 @@ constexpr int kTargetCtasPerSm = 8;        // automatic split size aims at this 
 
 struct SchedKey {
     int mla, dtype, hq, hkv, d, dv, pr, causal, window, path, kv_chunk;
+    int sparse_bs, sparse_w;  // sparse top-K: block size and selection width (0 = dense)
     bool operator==(const SchedKey& o) const { return std::memcmp(this, &o, sizeof o) == 0; }
 };
 
@@ -99,6 +100,10 @@ struct pa_plan {
     std::vector<std::unique_ptr<Schedule>> scheds;  // most recent last
     float* ws = nullptr;
     size_t ws_bytes = 0;
+    int32_t* sel_ws = nullptr;  // checked, compacted sparse selection
+    size_t sel_ws_bytes = 0;
+    float* score_ws = nullptr;  // proxy block scores when the caller keeps none
+    size_t score_ws_bytes = 0;
     cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
     int32_t last_launches = 0;
     int64_t uploaded_bytes = 0;
@@ -144,7 +149,20 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     struct Block { int32_t seq, j0, j1, lo, hi; int kind; };  // kind: 0 CUDA-core, 1 decode, 2 MLA
     std::vector<Block> blocks;
     int64_t total = 0;  // keys x kv heads, over all blocks
-    for (int32_t s = 0; s < P->S; ++s) {
+    // Sparse top-K: every query is its own row set; its keys are the concatenation of up to
+    // sparse_w selected blocks (positions through the selection, see AttnParams::sel).
+    const bool tc_sparse = tc_decode && G <= pa::kDecodeMaxRows && k.sparse_bs % 16 == 0;
+    for (int32_t s = 0; k.sparse_bs > 0 && s < P->S; ++s) {
+        const pa::SeqInfo& si = P->seqs[s];
+        const int64_t nb = ((int64_t)si.L + k.sparse_bs - 1) / k.sparse_bs;
+        const int64_t w = std::min<int64_t>(k.sparse_w, nb);
+        for (int32_t j = 0; j < si.n; ++j) {
+            Block b{s, j, j + 1, 0, (int32_t)(w * k.sparse_bs), tc_sparse ? 1 : 0};
+            total += (int64_t)b.hi * k.hkv;
+            blocks.push_back(b);
+        }
+    }
+    for (int32_t s = 0; k.sparse_bs == 0 && s < P->S; ++s) {
         const pa::SeqInfo& si = P->seqs[s];
         if (si.n == 0) continue;
         const bool tc = tc_decode && (int64_t)si.n * G <= pa::kDecodeMaxRows;
@@ -178,7 +196,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
         }
     }
     int64_t chunk;
-    if (k.kv_chunk > 0) chunk = k.kv_chunk;
+    if (k.kv_chunk > 0) chunk = k.sparse_bs > 0 ? ((int64_t)k.kv_chunk + 15) / 16 * 16 : k.kv_chunk;
     else if (k.kv_chunk < 0) chunk = INT32_MAX;
     else {
         // The tensor-core MLA kernel runs one CTA per SM, two per unit: aim at one unit per SM.
@@ -195,7 +213,11 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
         const int64_t len = b.hi - b.lo;
         int64_t c = chunk;
         int32_t nsplit = len <= 0 ? 1 : ceil_div(len, c);
-        if (nsplit > kMaxSplits) { c = (len + kMaxSplits - 1) / kMaxSplits; nsplit = ceil_div(len, c); }
+        if (nsplit > kMaxSplits) {
+            c = (len + kMaxSplits - 1) / kMaxSplits;
+            if (k.sparse_bs > 0) c = (c + 15) / 16 * 16;  // tiles of 16 keys stay inside one block
+            nsplit = ceil_div(len, c);
+        }
         const int32_t base = nsplit > 1 ? (int32_t)slots : -1;
         if (nsplit > 1) {
             for (int32_t j = b.j0; j < b.j1; ++j)
@@ -294,6 +316,21 @@ pa_status ensure_workspace(pa_plan* P, size_t bytes, cudaStream_t st) {
     return PA_OK;
 }
 
+template <typename P_>
+pa_status grow_buffer(P_** buf, size_t* have, size_t bytes, cudaStream_t st) {
+    if (bytes <= *have) return PA_OK;
+    if (*buf) {
+        PA_CUDA_TRY(cudaFreeAsync(*buf, st));
+        *buf = nullptr;
+        *have = 0;
+    }
+    void* p = nullptr;
+    PA_CUDA_TRY(cudaMallocAsync(&p, bytes, st));
+    *buf = (P_*)p;
+    *have = bytes;
+    return PA_OK;
+}
+
 // ---------------------------------------------------------------------------------------
 // Shared validation of a forward call
 // ---------------------------------------------------------------------------------------
@@ -309,7 +346,25 @@ struct Call {
     void* out;
     float* lse;
     pa_forward_options opts;
+    int32_t block_size;         // sparse top-K (0 = dense)
+    const int32_t* selection;   // [Nq, Hkv, width]
+    int32_t width;
 };
+
+int32_t max_blocks(const pa_plan* P, int32_t bs) {
+    int64_t m = 0;
+    for (const pa::SeqInfo& si : P->seqs) m = std::max<int64_t>(m, ((int64_t)si.L + bs - 1) / bs);
+    return (int32_t)std::min<int64_t>(m, INT32_MAX);
+}
+
+// Block size rule and block count limit of the sparse entry points.
+pa_status check_sparse_blocks(const pa_plan* P, int32_t bs) {
+    if (bs <= 0 || bs % P->page_size != 0)
+        return fail(PA_ERR_SHAPE, "block_size (%d) must be a positive multiple of page_size (%d)", bs, P->page_size);
+    if (max_blocks(P, bs) > PA_SPARSE_MAX_BLOCKS)
+        return fail(PA_ERR_UNSUPPORTED, "a sequence has more than %d blocks of %d keys", PA_SPARSE_MAX_BLOCKS, bs);
+    return PA_OK;
+}
 
 pa_status validate(pa_plan* P, const Call& c) {
     if (!P) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
@@ -330,6 +385,11 @@ pa_status validate(pa_plan* P, const Call& c) {
     if (c.opts.path != PA_PATH_AUTO && c.opts.path != PA_PATH_SIMT)
         return fail(PA_ERR_INVALID_ARGUMENT, "unknown path %d", c.opts.path);
     if (c.opts.kv_chunk < -1) return fail(PA_ERR_INVALID_ARGUMENT, "kv_chunk must be -1, 0 or > 0");
+    if (c.block_size != 0) {
+        pa_status bs = check_sparse_blocks(P, c.block_size);
+        if (bs != PA_OK) return bs;
+        if (c.width < 0) return fail(PA_ERR_SHAPE, "selection width must be >= 0");
+    }
 
     const int64_t es = (int64_t)dtype_size(c.dtype);
     int64_t nq = P->Nq, pages = P->num_pages, ps = P->page_size;
@@ -351,6 +411,14 @@ pa_status validate(pa_plan* P, const Call& c) {
     if (overlap(ro, rl)) return fail(PA_ERR_ALIAS, "out and lse overlap");
     for (const Range& r : ins)
         if (overlap(ro, r) || overlap(rl, r)) return fail(PA_ERR_ALIAS, "out or lse overlaps an input");
+    if (c.block_size > 0) {
+        int64_t n_sel = 0;
+        if (!product({nq, c.hkv, c.width, 4}, &n_sel)) return fail(PA_ERR_BOUNDS, "selection size overflows");
+        if (n_sel > 0 && !c.selection) return fail(PA_ERR_INVALID_ARGUMENT, "selection is NULL");
+        if ((uintptr_t)c.selection % 4 != 0) return fail(PA_ERR_INVALID_ARGUMENT, "selection must be 4-byte aligned");
+        const Range rs = R(c.selection, n_sel);
+        if (overlap(ro, rs) || overlap(rl, rs)) return fail(PA_ERR_ALIAS, "out or lse overlaps the selection");
+    }
     return PA_OK;
 }
 
@@ -378,9 +446,19 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     key.window = c.window;
     key.path = c.opts.path;
     key.kv_chunk = c.opts.kv_chunk;
+    int32_t wout = 0;  // width of the compacted selection
+    if (c.block_size > 0) {
+        wout = std::min<int32_t>(c.width, max_blocks(P, c.block_size));
+        key.sparse_bs = c.block_size;
+        key.sparse_w = wout;
+    }
     Schedule* S = nullptr;
     pa_status bs = build_schedule(P, key, st, &S);
     if (bs != PA_OK) return bs;
+    if (c.block_size > 0 && wout > 0) {
+        pa_status gs = grow_buffer(&P->sel_ws, &P->sel_ws_bytes, (size_t)P->Nq * c.hkv * wout * sizeof(int32_t), st);
+        if (gs != PA_OK) return gs;
+    }
     if (S->slots > 0) {
         const size_t need = (size_t)S->slots * c.hq * (c.dv + 1) * sizeof(float);
         pa_status ws = ensure_workspace(P, need, st);
@@ -412,6 +490,17 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     cudaEvent_t* ev = (cudaEvent_t*)c.opts.trace_events;
     cudaError_t e;
     int launches = 0;
+    if (c.block_size > 0) {
+        p.sel = P->sel_ws;
+        p.sel_width = wout;
+        p.block_size = c.block_size;
+        if (wout > 0) {
+            ++launches;
+            e = pa::launch_sparse_prep(c.selection, c.width, P->sel_ws, wout, P->d_seqs, P->d_q2seq, c.hkv,
+                                       c.block_size, max_blocks(P, c.block_size), P->Nq, P->d_err, st);
+            if (e != cudaSuccess) return fail(PA_ERR_CUDA, "selection check launch failed: %s", cudaGetErrorString(e));
+        }
+    }
     if (ev) PA_CUDA_TRY(cudaEventRecord(ev[0], st));
     if (S->n_tc > 0) {
         ++launches;
@@ -605,6 +694,8 @@ pa_status pa_plan_destroy(pa_plan* plan) {
         // once the stream reaches this point.
         cudaStream_t st = plan->last_stream;
         if (plan->ws) cudaFreeAsync(plan->ws, st);
+        if (plan->sel_ws) cudaFreeAsync(plan->sel_ws, st);
+        if (plan->score_ws) cudaFreeAsync(plan->score_ws, st);
         for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
         if (plan->d_meta) cudaFreeAsync(plan->d_meta, st);
         cudaError_t e = cudaLaunchHostFunc(st, [](void* ud) { delete static_cast<pa_plan*>(ud); }, plan);
@@ -678,6 +769,100 @@ pa_status pa_mla_forward(pa_plan* plan, const void* q_latent, const void* q_rope
                          int causal, int32_t window, void* out, float* lse, pa_stream stream) {
     return pa_mla_forward_ex(plan, q_latent, q_rope, latent_cache, rope_cache, dtype, num_heads,
                              latent_dim, rope_dim, scale, causal, window, out, lse, stream, nullptr);
+}
+
+pa_status pa_sparse_forward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                            pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t v_head_dim, float scale, int causal, int32_t window, int32_t block_size,
+                            const int32_t* selection, int32_t width, void* out, float* lse, pa_stream stream) {
+    if (!plan) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    if (block_size <= 0) return fail(PA_ERR_SHAPE, "block_size must be > 0");
+    Call c{};
+    c.mla = false;
+    c.q = q; c.k = k_cache; c.v = v_cache;
+    c.dtype = dtype;
+    c.hq = num_q_heads; c.hkv = num_kv_heads; c.d = head_dim; c.dv = v_head_dim;
+    c.scale = scale; c.causal = causal; c.window = window;
+    c.out = out; c.lse = lse;
+    c.opts = default_opts(nullptr);
+    c.block_size = block_size;
+    c.selection = selection;
+    c.width = width;
+    return run_forward(plan, c, (cudaStream_t)stream);
+}
+
+pa_status pa_sparse_select(pa_plan* plan, const void* q, const void* k_cache, pa_dtype dtype,
+                           int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                           int causal, int32_t window, int32_t block_size, int32_t topk,
+                           int32_t* selection, int32_t width, float* block_scores, int32_t scores_width,
+                           pa_stream stream) {
+    pa_plan* P = plan;
+    if (!P) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return fail(PA_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+    if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0)
+        return fail(PA_ERR_SHAPE, "query heads (%d) must be a positive multiple of kv heads (%d)", num_q_heads,
+                    num_kv_heads);
+    if (head_dim <= 0) return fail(PA_ERR_SHAPE, "head_dim must be positive");
+    if (head_dim > 1024) return fail(PA_ERR_UNSUPPORTED, "head dims above 1024 are not supported");
+    if (!std::isfinite(scale) || !(scale > 0.0f)) return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and > 0");
+    if (causal != 0 && causal != 1) return fail(PA_ERR_INVALID_ARGUMENT, "causal must be 0 or 1");
+    if (window < 0) return fail(PA_ERR_INVALID_ARGUMENT, "window must be >= 0");
+    if (topk < 0) return fail(PA_ERR_INVALID_ARGUMENT, "topk must be >= 0");
+    pa_status bst = check_sparse_blocks(P, block_size);
+    if (bst != PA_OK) return bst;
+    const int32_t nb_max = max_blocks(P, block_size);
+    int64_t k_max = 0;
+    for (const pa::SeqInfo& si : P->seqs) {
+        if (si.n == 0) continue;
+        const int64_t nb = ((int64_t)si.L + block_size - 1) / block_size;
+        k_max = std::max<int64_t>(k_max, (topk == 0 || topk >= nb) ? nb : topk);
+    }
+    if (width < k_max) return fail(PA_ERR_SHAPE, "selection width %d is below the %lld blocks kept", width, (long long)k_max);
+    if (block_scores && scores_width < nb_max)
+        return fail(PA_ERR_SHAPE, "scores_width %d is below the %d blocks of the longest sequence", scores_width, nb_max);
+    const int64_t es = (int64_t)dtype_size(dtype);
+    int64_t n_q, n_k, n_sel, n_sc = 0;
+    if (!product({P->Nq, num_q_heads, head_dim, es}, &n_q) ||
+        !product({P->num_pages, P->page_size, num_kv_heads, head_dim, es}, &n_k) ||
+        !product({P->Nq, num_kv_heads, width, 4}, &n_sel) ||
+        (block_scores && !product({P->Nq, num_kv_heads, scores_width, 4}, &n_sc)))
+        return fail(PA_ERR_BOUNDS, "tensor size overflows 64-bit byte counts");
+    if (P->Nq == 0) return ok();
+    if (!q || (n_k > 0 && !k_cache) || (n_sel > 0 && !selection))
+        return fail(PA_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    if ((uintptr_t)q % 16 || (uintptr_t)k_cache % 16 || (uintptr_t)selection % 4 || (uintptr_t)block_scores % 4)
+        return fail(PA_ERR_INVALID_ARGUMENT, "q and k_cache must be 16-byte aligned, selection and scores 4-byte");
+    auto R = [](const void* p, int64_t n) { return Range{(uintptr_t)p, (uintptr_t)p + (uintptr_t)n}; };
+    const Range rq = R(q, n_q), rk = R(k_cache, n_k), rs = R(selection, n_sel), rc = R(block_scores, n_sc);
+    if (overlap(rs, rq) || overlap(rs, rk) || overlap(rc, rq) || overlap(rc, rk) || overlap(rs, rc))
+        return fail(PA_ERR_ALIAS, "selection or block_scores overlaps an input or each other");
+    if (P->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to run on");
+    int cur = -1;
+    PA_CUDA_TRY(cudaGetDevice(&cur));
+    if (cur != P->device) return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, P->device);
+
+    std::lock_guard<std::mutex> lock(P->mu);
+    cudaStream_t st = (cudaStream_t)stream;
+    P->last_stream = st;
+    float* scores = block_scores;
+    int32_t sw = scores_width;
+    if (!scores) {
+        sw = nb_max;
+        pa_status gs = grow_buffer(&P->score_ws, &P->score_ws_bytes, std::max<size_t>(4, (size_t)P->Nq * num_kv_heads * sw * 4), st);
+        if (gs != PA_OK) return gs;
+        scores = P->score_ws;
+    }
+    cudaError_t e = pa::launch_sparse_scores(q, k_cache, scores, sw, P->d_seqs, P->d_q2seq, P->d_bt, P->table_width,
+                                             P->page_size, num_q_heads, num_kv_heads, head_dim, block_size, scale,
+                                             causal, window, P->Nq, dtype, st);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "proxy score launch failed: %s", cudaGetErrorString(e));
+    if (width > 0) {
+        e = pa::launch_sparse_topk(scores, sw, selection, width, P->d_seqs, P->d_q2seq, num_kv_heads, block_size, topk,
+                                   nb_max, P->Nq, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "top-k launch failed: %s", cudaGetErrorString(e));
+    }
+    P->last_launches = width > 0 ? 2 : 1;
+    return ok();
 }
 
 pa_status pa_plan_prepare(pa_plan* plan, int mla, pa_dtype dtype, int32_t num_q_heads,

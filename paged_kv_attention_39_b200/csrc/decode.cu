@@ -42,7 +42,7 @@ __device__ __forceinline__ int swz(int row, int chunk) { return chunk ^ (row & 7
 
 }  // namespace
 
-template <typename T, int D, int NT, int MT, int STAGES>
+template <typename T, int D, int NT, int MT, int STAGES, bool SPARSE>
 __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParams p) {
     using C = DecodeCfg<D, MT, STAGES>;
     constexpr int TT = C::TT, CH = C::CH, KK = D / 16;
@@ -56,6 +56,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParam
     const int R = (u.j1 - u.j0) * G;  // live rows, <= 8 * NT
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gq = lane >> 2, tq = lane & 3;  // fragment row group / thread-in-group
+    // Sparse: one query per unit; its keys are reached through the selection row of (query, kvh)
+    // and a tile of TT keys never straddles two blocks (TT divides block_size and t0).
+    const int32_t* selrow = nullptr;
+    if constexpr (SPARSE) selrow = p.sel + ((int64_t)(si.q_start + u.j0) * p.hkv + kvh) * p.sel_width;
+    const int bs = p.block_size;
 
     // ---- query fragments (B operand of S^T = K Q^T): column n = row gq of the n-tile ------
     uint32_t qf[NT][KK][2];
@@ -113,8 +118,17 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParam
         const int tok0 = u.t0 + (warp + it * kWarps) * TT;
         int64_t off = -1;
         if (lane < TT) {
-            const int t = tok0 + lane;
-            if (t < u.t1) off = ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D;
+            if constexpr (SPARSE) {
+                const int vk = tok0 + lane;
+                if (vk < u.t1) {
+                    const int32_t blk = selrow[vk / bs];
+                    const int64_t t = (int64_t)blk * bs + vk % bs;
+                    if (blk >= 0 && t < si.L) off = ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D;
+                }
+            } else {
+                const int t = tok0 + lane;
+                if (t < u.t1) off = ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D;
+            }
         }
         T* dk = wbuf + stage * 2 * C::TILE;
         T* dv = dk + C::TILE;
@@ -165,7 +179,17 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParam
             }
         }
         // ---- scale, mask, running max ----------------------------------------------------
-        const bool full = tok0 + TT <= u.t1 && tok0 >= all_lo && tok0 + TT - 1 < all_hi;
+        bool full;
+        int64_t tbase = tok0;  // position of the tile's first key
+        bool tvalid = true;
+        if constexpr (SPARSE) {
+            const int32_t blk = selrow[tok0 / bs];
+            tvalid = blk >= 0;
+            tbase = (int64_t)blk * bs + tok0 % bs;
+            full = tvalid && tok0 + TT <= u.t1 && tbase + TT <= si.L && tbase >= all_lo && tbase + TT - 1 < all_hi;
+        } else {
+            full = tok0 + TT <= u.t1 && tok0 >= all_lo && tok0 + TT - 1 < all_hi;
+        }
         float tmax[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) tmax[nt][0] = tmax[nt][1] = neg_inf();
@@ -177,9 +201,10 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParam
                 for (int e = 0; e < 4; ++e) {
                     float x = s[mt][nt][e] * p.scale_log2;
                     if (!full) {
-                        const int t = tok0 + mt * 16 + gq + 8 * (e >> 1);
+                        const int o = mt * 16 + gq + 8 * (e >> 1);
+                        const int64_t t = tbase + o;
                         const int c = e & 1;
-                        const bool vis = t < u.t1 &&
+                        const bool vis = tvalid && tok0 + o < u.t1 && (!SPARSE || t < si.L) &&
                                          (!livec[nt][c] || key_visible(t, posc[nt][c], p.causal, p.window));
                         if (!vis) x = neg_inf();
                     }
@@ -310,11 +335,11 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParam
 
 namespace {
 
-template <typename T, int D, int NT>
+template <typename T, int D, int NT, bool SPARSE>
 cudaError_t launch_cfg(const AttnParams& p, cudaStream_t st) {
     constexpr int MT = 1, STAGES = 3;
     using C = DecodeCfg<D, MT, STAGES>;
-    auto kern = decode_mma_kernel<T, D, NT, MT, STAGES>;
+    auto kern = decode_mma_kernel<T, D, NT, MT, STAGES, SPARSE>;
     static unsigned long long configured = 0;  // one bit per device ordinal
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -328,19 +353,23 @@ cudaError_t launch_cfg(const AttnParams& p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <typename T>
+template <typename T, bool SPARSE>
 cudaError_t launch_t(const AttnParams& p, int rows_max, cudaStream_t st) {
     const bool two = rows_max > 8;
-    if (p.d == 64) return two ? launch_cfg<T, 64, 2>(p, st) : launch_cfg<T, 64, 1>(p, st);
-    return two ? launch_cfg<T, 128, 2>(p, st) : launch_cfg<T, 128, 1>(p, st);
+    if (p.d == 64) return two ? launch_cfg<T, 64, 2, SPARSE>(p, st) : launch_cfg<T, 64, 1, SPARSE>(p, st);
+    return two ? launch_cfg<T, 128, 2, SPARSE>(p, st) : launch_cfg<T, 128, 1, SPARSE>(p, st);
 }
 
 }  // namespace
 
 cudaError_t launch_decode_mma(const AttnParams& p, pa_dtype dt, int rows_max, cudaStream_t st) {
     if (p.num_units == 0) return cudaSuccess;
-    if (dt == PA_BF16) return launch_t<__nv_bfloat16>(p, rows_max, st);
-    return launch_t<__half>(p, rows_max, st);
+    if (p.sel) {
+        if (dt == PA_BF16) return launch_t<__nv_bfloat16, true>(p, rows_max, st);
+        return launch_t<__half, true>(p, rows_max, st);
+    }
+    if (dt == PA_BF16) return launch_t<__nv_bfloat16, false>(p, rows_max, st);
+    return launch_t<__half, false>(p, rows_max, st);
 }
 
 }  // namespace pa

@@ -62,6 +62,11 @@ struct AttnParams {
     int32_t causal, window;
     int32_t num_queries, num_pages;
     int* err;          // device error word of the plan (0 = no failure)
+    // Sparse top-K attention: when sel is set, a unit's keys [t0, t1) are positions in the
+    // concatenation of the row's selected blocks: key v is position sel[row][v / block_size] *
+    // block_size + v % block_size of the sequence (entries of -1 hold no keys).
+    const int32_t* sel;  // [Nq, Hkv, sel_width] checked, compacted selection
+    int32_t sel_width, block_size;
 };
 
 // Kernel launchers (one per .cu file). Each returns the launch's cudaError_t.
@@ -80,6 +85,18 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
 cudaError_t launch_append(const void* new_k, const void* new_v, void* k_cache, void* v_cache, const SeqInfo* seqs,
                           const int32_t* q2seq, const int32_t* block_tables, int32_t table_width, int32_t page_size,
                           int32_t hkv, int32_t k_row_bytes, int32_t v_row_bytes, int64_t rows, cudaStream_t st);
+// Sparse top-K block selection (sparse.cu).
+cudaError_t launch_sparse_scores(const void* q, const void* k, float* scores, int32_t sw, const SeqInfo* seqs,
+                                 const int32_t* q2seq, const int32_t* block_tables, int32_t table_width,
+                                 int32_t page_size, int32_t hq, int32_t hkv, int32_t d, int32_t block_size,
+                                 float scale, int causal, int32_t window, int64_t num_queries, pa_dtype dt,
+                                 cudaStream_t st);
+cudaError_t launch_sparse_topk(const float* scores, int32_t sw, int32_t* sel, int32_t width, const SeqInfo* seqs,
+                               const int32_t* q2seq, int32_t hkv, int32_t block_size, int32_t topk,
+                               int32_t nb_max, int64_t num_queries, cudaStream_t st);
+cudaError_t launch_sparse_prep(const int32_t* in, int32_t width, int32_t* out, int32_t wout, const SeqInfo* seqs,
+                               const int32_t* q2seq, int32_t hkv, int32_t block_size, int32_t nb_max,
+                               int64_t num_queries, int* err, cudaStream_t st);
 // Shapes the tensor-core MLA decode kernel takes (one query per sequence).
 bool mla_tc_supported(pa_dtype dt, int heads, int latent_dim, int rope_dim, int page_size);
 

@@ -5,7 +5,8 @@
 // accumulators, then either the final output/lse or one float32 split part.
 //
 // This is the exact-precision path (no 16-bit rounding of probabilities), used for fp32 and
-// for shapes the tensor-core kernels do not take.
+// for shapes the tensor-core kernels do not take. With a sparse selection the unit's keys are
+// positions in the concatenation of the row's selected blocks (see AttnParams::sel).
 #include "device_common.cuh"
 
 namespace pa {
@@ -40,7 +41,17 @@ __global__ void __launch_bounds__(128) simt_kernel(const AttnParams p) {
             acc[i] = 0.f;
         }
         float m = neg_inf(), l = 0.f;
-        for (int t = u.t0; t < u.t1; ++t) {
+        const int32_t* selrow = p.sel ? p.sel + ((int64_t)(si.q_start + j) * p.hkv + kvh) * p.sel_width : nullptr;
+        for (int vk = u.t0; vk < u.t1; ++vk) {
+            int64_t t = vk;
+            if (selrow) {  // sparse: key vk of the concatenated selected blocks
+                const int32_t blk = selrow[vk / p.block_size];
+                t = (int64_t)blk * p.block_size + vk % p.block_size;
+                if (blk < 0 || t >= si.L) {  // nothing left in this block entry
+                    vk += p.block_size - 1 - vk % p.block_size;
+                    continue;
+                }
+            }
             if (!key_visible(t, pos, p.causal, p.window)) continue;
             const int64_t slot = (int64_t)bt[t / ps] * ps + t % ps;
             const int64_t krow = (slot * p.hkv + kvh) * p.d;

@@ -265,6 +265,40 @@ def c5_mla_decode(seed: int = 0, batch: int = 32, lmin: int = 1024, lmax: int = 
                     pin=pin)
 
 
+def sparse_bf16_decode(seed: int = 0, block_size: int = 64, topk: int = 16, pin: bool = False):
+    """The bf16 decode batch (64 sequences, context U[512, 8192], Hq=32, Hkv=8, D=128, page 16)
+    with sparse top-K attention over blocks of `block_size` keys: (workload, block_size, topk).
+    Blocks of 64 and a handful of them per query follow the page's bridge (blocks of 64 keys)."""
+    return c2_bf16_decode(seed, pin=pin), block_size, topk
+
+
+def sparse_bytes(wl, block_size: int, selection) -> int:
+    """Algorithmic HBM bytes of one sparse step: the proxy pass reads the K row of every key a
+    query sees once per (query, KV head); attention reads the K and V rows of the keys it sees in
+    the selected blocks (selection [Nq, Hkv, width], -1 = unused)."""
+    sched = wl.sched
+    esz = wl.k_cache.element_size()
+    krow, kvrow = wl.head_dim * esz, (wl.head_dim + wl.v_head_dim) * esz
+    sel = selection.cpu()
+    total = 0
+    W = wl.window
+    for s in range(sched.num_seqs):
+        L = int(sched.seq_lens[s])
+        q0, q1 = int(sched.query_offsets[s]), int(sched.query_offsets[s + 1])
+        for qi in range(q0, q1):
+            p = L - (q1 - q0) + (qi - q0)
+            hi = p + 1 if wl.causal else L
+            lo = max(0, p - W + 1) if W > 0 else 0
+            total += max(0, hi - lo) * krow * wl.num_kv_heads
+            for h in range(wl.num_kv_heads):
+                for b in sel[qi, h].tolist():
+                    if b < 0:
+                        continue
+                    a, e = max(lo, b * block_size), min(hi, (b + 1) * block_size)
+                    total += max(0, e - a) * kvrow
+    return total
+
+
 FULL_CONFIGS = {
     "tiny_fp32_decode": c1_tiny_fp32_decode,
     "bf16_decode": c2_bf16_decode,

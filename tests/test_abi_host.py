@@ -184,3 +184,51 @@ def test_append_validation(lib):
     bt = torch.tensor([[0, 1], [0, 1]], dtype=torch.int32)
     shared = pa.pa_plan_create([20, 20], [0, 1, 2], bt, 16, 4, device=-1)
     assert app(pl=shared) == "PA_ERR_ALIAS"
+
+
+def test_sparse_validation(lib):
+    """pa_sparse_select / pa_sparse_forward check every argument before the host-only refusal.
+    Plan: L = 37 and 100 keys in pages of 16, so blocks of 16 keys give 3 and 7 blocks."""
+    wl, plan = host_plan()
+    q, k, v, o, l = fake_ptrs(wl)
+    sel = l + (1 << 30)
+    scores = sel + (1 << 30)
+    def select(bs=16, topk=4, width=4, sc=None, scw=0, s=sel, hq=4, hkv=2, d=64, scale=0.125, causal=1, window=0):
+        st = lib.pa_sparse_select(plan.handle, q, k, 1, hq, hkv, d, ctypes.c_float(scale), causal, window, bs, topk, s,
+                                  width, sc, scw, None)
+        return pa.STATUS[st]
+    assert select() == "PA_ERR_INVALID_ARGUMENT"          # all valid -> host-only plan refusal
+    assert "host-only" in pa.pa_last_error_message()
+    assert select(bs=24) == "PA_ERR_SHAPE"                # not a multiple of the page size
+    assert select(bs=0) == "PA_ERR_SHAPE"
+    assert select(width=3) == "PA_ERR_SHAPE"              # the longer sequence keeps 4 blocks
+    assert select(topk=0, width=6) == "PA_ERR_SHAPE"      # every block: 7 for the longer one
+    assert select(topk=0, width=7) == "PA_ERR_INVALID_ARGUMENT"
+    assert select(topk=9, width=7) == "PA_ERR_INVALID_ARGUMENT"  # topk above the block count: all 7
+    assert select(sc=scores, scw=6) == "PA_ERR_SHAPE"     # scores need 7 columns
+    assert select(sc=scores, scw=7) == "PA_ERR_INVALID_ARGUMENT"
+    assert select(topk=-1) == "PA_ERR_INVALID_ARGUMENT"
+    assert select(s=q) == "PA_ERR_ALIAS"                  # selection over q
+    assert select(sc=k, scw=7) == "PA_ERR_ALIAS"          # scores inside K
+    assert select(s=None) == "PA_ERR_INVALID_ARGUMENT"
+    assert select(hq=5) == "PA_ERR_SHAPE"
+    assert select(d=2048) == "PA_ERR_UNSUPPORTED"
+    assert select(scale=0.0) == "PA_ERR_INVALID_ARGUMENT"
+    def fwd(bs=16, width=4, s=sel, out=o, lse=l):
+        st = lib.pa_sparse_forward(plan.handle, q, k, v, 1, 4, 2, 64, 64, ctypes.c_float(0.125), 1, 0, bs, s, width,
+                                   out, lse, None)
+        return pa.STATUS[st]
+    assert fwd() == "PA_ERR_INVALID_ARGUMENT" and "host-only" in pa.pa_last_error_message()
+    assert fwd(bs=24) == "PA_ERR_SHAPE"
+    assert fwd(bs=0) == "PA_ERR_SHAPE"
+    assert fwd(width=-1) == "PA_ERR_SHAPE"
+    assert fwd(s=None) == "PA_ERR_INVALID_ARGUMENT"
+    assert fwd(out=sel) == "PA_ERR_ALIAS"                  # out over the selection
+    assert fwd(s=sel + 2) == "PA_ERR_INVALID_ARGUMENT"     # misaligned selection
+    # more blocks than PA_SPARSE_MAX_BLOCKS in one sequence
+    L = (pa.PA_SPARSE_MAX_BLOCKS + 1) * 16
+    big = pa.pa_plan_create([L], [0, 1], torch.arange(L // 16, dtype=torch.int32).view(1, -1), 16, L // 16, device=-1)
+    st = lib.pa_sparse_select(big.handle, q, k, 1, 4, 2, 64, ctypes.c_float(0.1), 1, 0, 16, 4, sel, 4, None, 0, None)
+    assert pa.STATUS[st] == "PA_ERR_UNSUPPORTED"
+    assert pa.STATUS[lib.pa_sparse_select(big.handle, q, k, 1, 4, 2, 64, ctypes.c_float(0.1), 1, 0, 32, 4, sel, 4,
+                                          None, 0, None)] == "PA_ERR_INVALID_ARGUMENT"  # blocks of 32: fits
