@@ -8,10 +8,10 @@
 //   warp 8      TMA producer: the Q tile once, then K and V tiles page by page (one box per
 //               page and 64-element half of the head dim, 128-byte swizzle) into a ring of
 //               stages; pages past the sequence's last key are never touched.
-//   warp 9      TMEM owner and MMA issuer (one thread): S = Q K^T into one of two TMEM
-//               buffers, then O += P V with P read from TMEM; commits signal completion. Before
-//               P V it zeroes the V rows past the sequence's last key (their bytes are whatever
-//               the page holds there).
+//   warp 9      TMEM owner and issuer (one thread) of S = Q K^T into one of two TMEM buffers.
+//   warp 10     issuer (one thread) of O += P V with P read from TMEM; before it, the warp
+//               zeroes the V rows past the sequence's last key (their bytes are whatever the page
+//               holds there). Commits signal completion.
 //   warps 0..7  softmax, two warps per row (each owning one half of the tile's columns; a warp's
 //               lanes are the TMEM lanes of its quadrant): S from TMEM, scale to base-2
 //               units, causal/window mask at absolute positions on edge tiles, running max and
@@ -21,8 +21,9 @@
 //               and stores.
 //
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+D) P0, P1 (64 columns each) after O.
-// The tensor core runs one thread's MMAs in issue order, so QK of tile i+2 (issued after P V of
-// tile i) never overwrites a score buffer that is still being read.
+// QK of tile i+2 goes into score buffer i & 1 only after the softmax has marked P of tile i
+// ready (it has then read all of S of tile i). The QK and the P V chains come from two issuing
+// warps so that the tensor core overlaps them.
 //
 // Every wait on an mbarrier is bounded (Watchdog): a stalled pipeline sets the plan's error
 // word and the CTA leaves through its normal exit, freeing TMEM.
@@ -41,8 +42,8 @@ constexpr int BN = 128;  // keys per step
 constexpr int KST = 3;   // K stages
 constexpr int VST = 3;   // V stages
 constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quadrant, each owning half of the columns
-constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1;
-constexpr int kThreads = (kSoftmaxWarps + 2) * 32;
+constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1, kPvWarp = kSoftmaxWarps + 2;
+constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
@@ -156,27 +157,29 @@ __device__ __forceinline__ float tile_exp(uint32_t taddr, int c0, float scale, f
 template <typename T, bool MASKED>
 __device__ __forceinline__ float tile_fused(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
                                             int off_lo, int off_hi, float& m_raw) {
-    float sum = 0.f, m0 = neg_inf(), m1 = neg_inf();
-#pragma unroll 1
-    for (int c = c0; c < c0 + 2; ++c) {
-        uint32_t v[32];
-        tmem_ld32(taddr + c * 32, v);
-        tmem_ld_wait(v);
+    uint32_t v0[32], v1[32];
+    tmem_ld32(taddr + c0 * 32, v0);  // both chunks in flight before the one wait
+    tmem_ld32(taddr + (c0 + 1) * 32, v1);
+    tmem_ld_wait(v0);
+    tmem_regs_ready(v1);
+    float m0 = neg_inf(), m1 = neg_inf();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            float x0 = __uint_as_float(v[e]), x1 = __uint_as_float(v[e + 1]);
-            if (MASKED) {
-                const int k0 = c * 32 + e;
-                x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? x0 : neg_inf();
-                x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? x1 : neg_inf();
-            }
-            m0 = fmaxf(m0, x0);
-            m1 = fmaxf(m1, x1);
+    for (int e = 0; e < 32; e += 2) {
+        float x0 = __uint_as_float(v0[e]), x1 = __uint_as_float(v0[e + 1]);
+        float y0 = __uint_as_float(v1[e]), y1 = __uint_as_float(v1[e + 1]);
+        if (MASKED) {
+            const int k0 = c0 * 32 + e, k1 = k0 + 32;
+            x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? x0 : neg_inf();
+            x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? x1 : neg_inf();
+            y0 = (k1 + off_lo >= 0 && k1 + off_hi < 0) ? y0 : neg_inf();
+            y1 = (k1 + 1 + off_lo >= 0 && k1 + 1 + off_hi < 0) ? y1 : neg_inf();
         }
-        sum += exp_chunk<T, MASKED>(v, c, scale, -m, p_taddr, off_lo, off_hi);
+        m0 = fmaxf(m0, fmaxf(x0, y0));
+        m1 = fmaxf(m1, fmaxf(x1, y1));
     }
     m_raw = fmaxf(m0, m1);
-    return sum;
+    return exp_chunk<T, MASKED>(v0, c0, scale, -m, p_taddr, off_lo, off_hi) +
+           exp_chunk<T, MASKED>(v1, c0 + 1, scale, -m, p_taddr, off_lo, off_hi);
 }
 
 template <typename T, int D>
@@ -302,17 +305,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = max(0, issued - VST); i < issued; ++i) drain(&bars[B_VFULL + i % VST], (i / VST) & 1);
             }
         }
-    } else if (warp == kMmaWarp) {
-        // ===================== MMA issuer =====================
-        // Descriptors are built once; a k-step or stage offset is an add to the address field.
+    } else if (warp == kMmaWarp || warp == kPvWarp) {
+        // ===================== MMA issuers =====================
+        // Two warps issue: one the S = Q K^T chains, one the O += P V chains. The tensor core
+        // runs the MMAs of one issuing warp one after the other, each k-step paying a latency
+        // well above its throughput (about twice as much for the TMEM-operand form of P V);
+        // chains from two warps overlap. Descriptors are built once; a k-step or stage offset
+        // is an add to the address field.
         const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
         const uint64_t dK = sdesc_sw128(s_base + L_::K, 16, 1024);
         const uint64_t dV = sdesc_sw128(s_base + L_::V, L_::HALF_KV, 1024);
-        bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[B_QFULL], 0, wd, 3));
-        for (int i = 0; ok && i <= n_tiles; ++i) {
-            if (i < n_tiles) {
+        if (warp == kMmaWarp) {
+            // S of tile i goes into score buffer i & 1. Both buffers start free; after that,
+            // buffer j & 1 is free again once the softmax has marked P of tile j ready (it has
+            // then read all of S of tile j).
+            bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[B_QFULL], 0, wd, 3));
+            for (int i = 0; ok && i < n_tiles; ++i) {
                 const int ks = i % KST, b = i & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_KFULL + ks], (i / KST) & 1, wd, 4));
+                if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + b], ((i - 2) >> 1) & 1, wd, 6));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_KFULL + ks], (i / KST) & 1, wd, 4));
                 if (!ok) break;
                 tc_fence_after();
                 if (lane == 0) {
@@ -328,11 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 __syncwarp();
             }
-            if (i >= 1) {
-                const int j = i - 1, vs = j % VST;
-                ok = mbar_wait(&bars[B_PFULL + (j & 1)], (j >> 1) & 1, wd, 6);
-                if (ok) ok = mbar_wait(&bars[B_VFULL + vs], (j / VST) & 1, wd, 7);
-                ok = __all_sync(0xffffffffu, ok);
+        } else {
+            // O += P V of tile j once P of tile j and V tile j are in place.
+            for (int j = 0; j < n_tiles; ++j) {
+                const int vs = j % VST;
+                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + (j & 1)], (j >> 1) & 1, wd, 6));
+                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_VFULL + vs], (j / VST) & 1, wd, 7));
                 if (!ok) break;
                 // V rows past the sequence's end hold arbitrary bytes: make them zero.
                 const int64_t kt0 = kt_start + (int64_t)j * BN;
