@@ -6,13 +6,15 @@
 // shared-memory tile feeds O += P V. The float32 output of 128 heads x 512 columns would fill
 // all 512 TMEM columns, leaving none for the scores, so each key range is handled by a pair of
 // CTAs: both compute the (identical) scores and softmax, and each accumulates one 256-column
-// half of O (TMEM: two 32-column score buffers + 256 columns of O). The pair's second read of a
-// K/V tile comes mostly from L2.
+// half of O (TMEM: two score buffers of four 32-column partials + 256 columns of O). The pair's
+// second read of a K/V tile comes mostly from L2.
 //
 //   warp 4      TMA producer: Q (9 boxes of 128 heads x 64 columns, once), then per step the
 //               latent and rope rows of 32 keys page by page into a 2-stage ring
-//   warp 5      TMEM owner, MMA issuer: S = Q K^T (36 k-steps), O_half += P V_half (2 k-steps);
-//               zeroes latent rows past the sequence's last key before P V reads them
+//   warps 5..8  S = Q K^T, nine of the 36 k-steps each into a partial score buffer (warp 5 also
+//               owns TMEM)
+//   warp 9      O_half += P V_half (2 k-steps); zeroes latent rows past the sequence's last key
+//               before P V reads them
 //   warps 0..3  softmax, thread = head: S row from TMEM, mask at the range edges, running max
 //               and sum in float32, P (16-bit, 64-byte swizzled K-major tile) into shared memory
 //
@@ -35,7 +37,10 @@ constexpr int MBM = 128;           // heads per tile
 constexpr int MBN = 32;            // keys per step
 constexpr int MST = 2;             // K/V stages
 constexpr int MDV = MR / 2;        // output columns per CTA
-constexpr int kMlaThreads = 192;
+constexpr int kQkWarps = 4;                   // issuers of S = Q K^T, each a quarter of the k-steps
+constexpr int kQkSteps = MK / 16 / kQkWarps;  // 9 k-steps per issuer
+constexpr int kQkWarp0 = 5, kPvWarp = kQkWarp0 + kQkWarps;
+constexpr int kMlaThreads = (kPvWarp + 1) * 32;
 constexpr uint32_t kMlaTmemCols = 512;
 constexpr uint64_t kMlaWaitNs = 2000000000ull;
 
@@ -99,13 +104,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         for (int i = 0; i < M_COUNT; ++i) {
             uint32_t cnt = 1;
             if (i == M_SFREE || i == M_SFREE + 1 || i == M_PFULL || i == M_PFULL + 1) cnt = 128;
+            if (i == M_SFULL || i == M_SFULL + 1) cnt = kQkWarps;
+            if (i >= M_EMPTY && i < M_EMPTY + MST) cnt = kQkWarps + 1;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
     }
-    if (warp == 5) {
+    if (warp == kQkWarp0) {
         tmem_alloc(tmem_slot, kMlaTmemCols);
         tmem_relinquish();
     }
@@ -113,7 +120,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s0 = tmem, t_s1 = tmem + 32, t_o = tmem + 64;
+    // score buffer b, partial g (one per QK issuer): columns 128 b + 32 g; O: columns 256 .. 511
+    const uint32_t t_o = tmem + 256;
     const uint32_t s_base = smem_u32(smem);
 
     if (warp == 4) {
@@ -170,59 +178,69 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 for (int i = max(0, issued - MST); i < issued; ++i) drain(&bars[M_FULL + i % MST], (i / MST) & 1);
             }
         }
-    } else if (warp == 5) {
-        // ===================== MMA issuer =====================
+    } else if (warp >= kQkWarp0 && warp < kPvWarp) {
+        // ===================== S = Q K^T issuers =====================
+        // Each of the kQkWarps warps issues one quarter of the 36 k-steps into its own partial
+        // score buffer: a single chain of N = 32 MMAs pays the per-step latency 36 times, four
+        // chains from four warps overlap on the tensor core. The softmax adds the partials.
+        const int g = warp - kQkWarp0;
         const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
         const uint64_t dKV = sdesc_sw128(s_base + L_::KV, 16, 1024);
+        bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[M_QFULL], 0, wd, 23));
+        for (int i = 0; ok && i < n_tiles; ++i) {
+            const int st = i % MST, b = i & 1;
+            ok = mbar_wait(&bars[M_FULL + st], (i / MST) & 1, wd, 24);
+            if (ok && i >= 2) ok = mbar_wait(&bars[M_SFREE + b], ((i >> 1) - 1) & 1, wd, 25);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t d_s = tmem + b * 128 + g * 32;
+                const uint64_t dKst = desc_add(dKV, st * MC * L_::KV_COL);
+#pragma unroll
+                for (int s2 = 0; s2 < kQkSteps; ++s2) {
+                    const int kk = g * kQkSteps + s2;
+                    mma_f16_ss(d_s, desc_add(dQ, (kk >> 2) * L_::Q_COL + (kk & 3) * 32),
+                               desc_add(dKst, (kk >> 2) * L_::KV_COL + (kk & 3) * 32), IDESC_QK, s2 > 0);
+                }
+                mma_commit(&bars[M_SFULL + b]);
+                mma_commit(&bars[M_EMPTY + st]);
+            }
+            __syncwarp();
+        }
+    } else if (warp == kPvWarp) {
+        // ===================== O_half += P V_half issuer =====================
         const uint64_t dV = sdesc_sw128(s_base + L_::KV, L_::KV_COL, 1024);
         const uint64_t dP = sdesc_sw64(s_base + L_::P, 512);
-        bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[M_QFULL], 0, wd, 23));
-        for (int i = 0; ok && i <= n_tiles; ++i) {
-            if (i < n_tiles) {
-                const int st = i % MST, b = i & 1;
-                ok = mbar_wait(&bars[M_FULL + st], (i / MST) & 1, wd, 24);
-                if (ok && i >= 2) ok = mbar_wait(&bars[M_SFREE + b], ((i >> 1) - 1) & 1, wd, 25);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                // latent rows past the sequence's end hold arbitrary bytes: they are values too
-                const int64_t kt0 = kt_start + (int64_t)i * MBN;
-                const int nvalid = (int)min64(MBN, si.L - kt0);
-                if (nvalid < MBN) {
-                    for (int c = 0; c < MC - 1; ++c) {
-                        uint4* col = reinterpret_cast<uint4*>(smem + L_::KV + (st * MC + c) * L_::KV_COL);
-                        for (int x = nvalid * 8 + lane; x < MBN * 8; x += 32) col[x] = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
+        for (int j = 0; j < n_tiles; ++j) {
+            const int st = j % MST;
+            bool ok = mbar_wait(&bars[M_FULL + st], (j / MST) & 1, wd, 24);
+            if (ok) ok = mbar_wait(&bars[M_PFULL + (j & 1)], (j >> 1) & 1, wd, 26);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            // latent rows past the sequence's end hold arbitrary bytes and are values too; the
+            // scores of tile j (which read them as keys, masked) are complete by now
+            const int64_t kt0 = kt_start + (int64_t)j * MBN;
+            const int nvalid = (int)min64(MBN, si.L - kt0);
+            if (nvalid < MBN) {
+                for (int c = 0; c < MC - 1; ++c) {
+                    uint4* col = reinterpret_cast<uint4*>(smem + L_::KV + (st * MC + c) * L_::KV_COL);
+                    for (int x = nvalid * 8 + lane; x < MBN * 8; x += 32) col[x] = make_uint4(0, 0, 0, 0);
                 }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t d_s = b ? t_s1 : t_s0;
-                    const uint64_t dKst = desc_add(dKV, st * MC * L_::KV_COL);
-#pragma unroll
-                    for (int kk = 0; kk < MK / 16; ++kk)
-                        mma_f16_ss(d_s, desc_add(dQ, (kk >> 2) * L_::Q_COL + (kk & 3) * 32),
-                                   desc_add(dKst, (kk >> 2) * L_::KV_COL + (kk & 3) * 32), IDESC_QK, kk > 0);
-                    mma_commit(&bars[M_SFULL + b]);
-                }
+                fence_proxy_async_smem();
                 __syncwarp();
             }
-            if (i >= 1) {
-                const int j = i - 1, st = j % MST;
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[M_PFULL + (j & 1)], (j >> 1) & 1, wd, 26));
-                if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint64_t dVs = desc_add(dV, (st * MC + hf * (MDV / 64)) * L_::KV_COL);
-                    const uint32_t acc0 = j > 0 ? 1u : 0u;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint64_t dVs = desc_add(dV, (st * MC + hf * (MDV / 64)) * L_::KV_COL);
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < MBN / 16; ++kk)
-                        mma_f16_ss(t_o, desc_add(dP, kk * 32), desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
-                    mma_commit(&bars[M_ODONE + (j & 1)]);
-                    mma_commit(&bars[M_EMPTY + st]);
-                }
-                __syncwarp();
+                for (int kk = 0; kk < MBN / 16; ++kk)
+                    mma_f16_ss(t_o, desc_add(dP, kk * 32), desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
+                mma_commit(&bars[M_ODONE + (j & 1)]);
+                mma_commit(&bars[M_EMPTY + st]);
             }
+            __syncwarp();
         }
     } else {
         // ===================== softmax: thread = head =====================
@@ -239,9 +257,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[M_SFULL + b], (i >> 1) & 1, wd, 28));
             if (!ok) break;
             tc_fence_after();
-            uint32_t v[32];
-            tmem_ld32((b ? t_s1 : t_s0) + lane_off, v);
+            uint32_t v[32], w[32];
+            const uint32_t t_sb = tmem + b * 128 + lane_off;
+            tmem_ld32(t_sb, v);
+            tmem_ld32(t_sb + 32, w);
             tmem_ld_wait(v);
+            tmem_regs_ready(w);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+#pragma unroll 1
+            for (int g = 2; g < kQkWarps; ++g) {
+                tmem_ld32(t_sb + g * 32, w);
+                tmem_ld_wait(w);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) + __uint_as_float(w[e]));
+            }
             tc_fence_before();
             mbar_arrive(&bars[M_SFREE + b]);
             // keys of this unit the query sees: [vis_lo, vis_hi), the same for every head
@@ -361,7 +391,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kQkWarp0) {
         tc_fence_after();
         tmem_dealloc(tmem, kMlaTmemCols);
     }
