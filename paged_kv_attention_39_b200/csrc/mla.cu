@@ -9,8 +9,10 @@
 // half of O (TMEM: two score buffers of four 32-column partials + 256 columns of O). The pair's
 // second read of a K/V tile comes mostly from L2.
 //
-//   warp 4      TMA producer: Q (9 boxes of 128 heads x 64 columns, once), then per step the
-//               latent and rope rows of 32 keys page by page into a 2-stage ring
+//   warp 4      TMA producer: Q (two boxes: 128 heads x all 8 latent column blocks, and the rope
+//               part), then per step the latent rows of 32 keys (one box with all 8 column
+//               blocks when a page holds the whole step) and the rope rows into a 2-stage ring,
+//               with an L2 prefetch a few steps ahead
 //   warps 5..8  S = Q K^T, nine of the 36 k-steps each into a partial score buffer (warp 5 also
 //               owns TMEM)
 //   warp 9      O_half += P V_half (2 k-steps); zeroes latent rows past the sequence's last key
@@ -41,6 +43,7 @@ constexpr int kQkWarps = 4;                   // issuers of S = Q K^T, each a qu
 constexpr int kQkSteps = MK / 16 / kQkWarps;  // 9 k-steps per issuer
 constexpr int kQkWarp0 = 5, kPvWarp = kQkWarp0 + kQkWarps;
 constexpr int kMlaThreads = (kPvWarp + 1) * 32;
+constexpr int kPrefetchTiles = 4;             // L2 prefetch distance of the TMA producer (tiles)
 constexpr uint32_t kMlaTmemCols = 512;
 constexpr uint64_t kMlaWaitNs = 2000000000ull;
 
@@ -74,8 +77,8 @@ __device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t sbo_byte
 template <typename T>
 __global__ void __launch_bounds__(kMlaThreads, 1)
     mla_tc_kernel(const __grid_constant__ CUtensorMap tm_ql, const __grid_constant__ CUtensorMap tm_qr,
-                  const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_rope,
-                  const AttnParams p) {
+                  const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_latw,
+                  const __grid_constant__ CUtensorMap tm_rope, const AttnParams p) {
     using L_ = MlaSmem;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t IDESC_QK = idesc_f16(MBM, MBN, kBf16, false, false);
@@ -133,10 +136,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 tma_prefetch(&tm_ql);
                 tma_prefetch(&tm_qr);
                 tma_prefetch(&tm_lat);
+                tma_prefetch(&tm_latw);
                 tma_prefetch(&tm_rope);
                 mbar_arrive_expect_tx(&bars[M_QFULL], MC * L_::Q_COL);
-                for (int c = 0; c < MC - 1; ++c)
-                    tma_load_3d(smem + L_::Q + c * L_::Q_COL, &tm_ql, &bars[M_QFULL], c * 64, 0, (int)qi);
+                // all 8 latent columns of the 128 heads in one box: [column][head][64 elements]
+                tma_load_4d(smem + L_::Q, &tm_ql, &bars[M_QFULL], 0, 0, 0, (int)qi);
                 tma_load_3d(smem + L_::Q + (MC - 1) * L_::Q_COL, &tm_qr, &bars[M_QFULL], 0, 0, (int)qi);
             }
             const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
@@ -149,10 +153,27 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 for (int b = 0; b < bpt; ++b)
                     if (kt0 + (int64_t)b * box < si.L) nb = b + 1;
                 const int g0 = i * bpt;
-                if (g0 + nb > base_g + 32) {
+                if (g0 + (kPrefetchTiles + 1) * bpt > base_g + 32) {  // ids of this tile and the prefetched one
                     base_g = g0;
                     const int64_t key = kt_start + (int64_t)(base_g + lane) * box;
                     my_row = key < si.L ? (int)((int64_t)bt[key / ps] * ps + key % ps) : 0;
+                }
+                // Warm L2 with the tile kPrefetchTiles ahead: with only two stages, a load issued
+                // when a stage frees up would otherwise pay the full HBM latency.
+                if (i + kPrefetchTiles < n_tiles) {
+                    const int gp = g0 + kPrefetchTiles * bpt;
+                    const int64_t ktp = kt0 + (int64_t)kPrefetchTiles * MBN;
+                    for (int b = 0; b < bpt; ++b) {
+                        const int prow = __shfl_sync(0xffffffffu, my_row, gp + b - base_g);
+                        if (lane == 0 && ktp + (int64_t)b * box < si.L) {
+                            if (bpt == 1) {
+                                tma_prefetch_l2_3d(&tm_latw, 0, prow, 0);
+                            } else {
+                                for (int c = 0; c < MC - 1; ++c) tma_prefetch_l2_3d(&tm_lat, c * 64, 0, prow);
+                            }
+                            tma_prefetch_l2_3d(&tm_rope, 0, 0, prow);
+                        }
+                    }
                 }
                 const int st = i % MST;
                 if (i >= MST && !__all_sync(0xffffffffu, mbar_wait(&bars[M_EMPTY + st], ((i / MST) - 1) & 1, wd, 21)))
@@ -162,8 +183,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 for (int b = 0; b < nb; ++b) {
                     const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
                     if (lane == 0) {
-                        for (int c = 0; c < MC - 1; ++c)
-                            tma_load_3d(dst + c * L_::KV_COL + b * box * 128, &tm_lat, &bars[M_FULL + st], c * 64, 0, row);
+                        if (bpt == 1) {  // one page box holds the whole tile: 8 latent columns in one load
+                            tma_load_3d(dst, &tm_latw, &bars[M_FULL + st], 0, row, 0);
+                        } else {
+                            for (int c = 0; c < MC - 1; ++c)
+                                tma_load_3d(dst + c * L_::KV_COL + b * box * 128, &tm_lat, &bars[M_FULL + st], c * 64,
+                                            0, row);
+                        }
                         tma_load_3d(dst + (MC - 1) * L_::KV_COL + b * box * 128, &tm_rope, &bars[M_FULL + st], 0, 0, row);
                     }
                 }
@@ -412,6 +438,19 @@ PFN_cuTensorMapEncodeTiled_v12000 mla_encode_fn() {
     return fn;
 }
 
+// Tiled map of 16-bit elements with 128B swizzle: `rank` dims (innermost first), byte strides of
+// dims 1.., and the box.
+bool mla_encode(CUtensorMap* m, bool bf16, const void* base, int rank, const cuuint64_t* dims,
+                const cuuint64_t* strides, const cuuint32_t* boxd) {
+    auto fn = mla_encode_fn();
+    if (!fn) return false;
+    cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank,
+              const_cast<void*>(base), dims, strides, boxd, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Map over a row-major [d2][d1][d0] tensor of 16-bit elements, box {64, b1, b2}, 128B swizzle.
 bool mla_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1,
              uint32_t b2) {
@@ -432,11 +471,21 @@ cudaError_t mla_launch_t(const AttnParams& p, cudaStream_t st) {
     const int ps = p.page_size;
     const int box = ps < MBN ? ps : MBN;
     const uint64_t rows = (uint64_t)p.num_pages * ps;
-    CUtensorMap tql, tqr, tlat, trope;
-    // Q maps: [Nq][H][R] and [Nq][H][P], one query x 128 heads x 64 columns per box
-    if (!mla_map(&tql, bf16, p.q, MR, p.hq, (uint64_t)p.num_queries, MBM, 1) ||
+    CUtensorMap tql, tqr, tlat, tlatw, trope;
+    // Absorbed Q [Nq][H][R] seen as {64 elements, head, 64-column block, query}: one box brings the
+    // 8 column blocks of 128 heads, laid out [block][head][64 elements] as the MMA reads them.
+    const cuuint64_t qdims[4] = {64, (cuuint64_t)p.hq, MR / 64, (cuuint64_t)p.num_queries};
+    const cuuint64_t qstr[3] = {MR * 2, 128, (cuuint64_t)p.hq * MR * 2};
+    const cuuint32_t qbox[4] = {64, MBM, MR / 64, 1};
+    // Latent cache rows [rows][R] seen as {64 elements, row, 64-column block}: one box brings a page
+    // box of keys with all 8 column blocks, laid out [block][key][64 elements].
+    const cuuint64_t ldims[3] = {64, rows, MR / 64};
+    const cuuint64_t lstr[2] = {MR * 2, 128};
+    const cuuint32_t lbox[3] = {64, (cuuint32_t)box, MR / 64};
+    if (!mla_encode(&tql, bf16, p.q, 4, qdims, qstr, qbox) ||
         !mla_map(&tqr, bf16, p.qr, MP, p.hq, (uint64_t)p.num_queries, MBM, 1) ||
-        !mla_map(&tlat, bf16, p.k, MR, 1, rows, 1, box) || !mla_map(&trope, bf16, p.kr, MP, 1, rows, 1, box))
+        !mla_map(&tlat, bf16, p.k, MR, 1, rows, 1, box) || !mla_encode(&tlatw, bf16, p.k, 3, ldims, lstr, lbox) ||
+        !mla_map(&trope, bf16, p.kr, MP, 1, rows, 1, box))
         return cudaErrorInvalidValue;
     auto kern = mla_tc_kernel<T>;
     static unsigned long long configured = 0;
@@ -448,7 +497,7 @@ cudaError_t mla_launch_t(const AttnParams& p, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<2 * p.num_units, kMlaThreads, MlaSmem::ALLOC, st>>>(tql, tqr, tlat, trope, p);
+    kern<<<2 * p.num_units, kMlaThreads, MlaSmem::ALLOC, st>>>(tql, tqr, tlat, tlatw, trope, p);
     return cudaGetLastError();
 }
 
