@@ -297,6 +297,7 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
     """The other configurations, timed the same way (few steps): context for the headline."""
     res = {}
     cfgs = [("bf16_chunked_prefill", W.c3_chunked_prefill), ("bf16_window_mixed", W.c4_window_mixed),
+            ("bf16_window_mixed_decode_part", W.c4_decode_part), ("bf16_window_mixed_prefill_part", W.c4_prefill_part),
             ("bf16_mla_decode", W.c5_mla_decode), ("bf16_sparse_topk_decode", W.sparse_bf16_decode)]
     if only is not None:
         cfgs = [only]
@@ -382,7 +383,8 @@ def run_single(args, ws, rank, local):
     args.extra_steps = args.steps
     fns = {"bf16_chunked_prefill": W.c3_chunked_prefill, "bf16_window_mixed": W.c4_window_mixed,
            "bf16_mla_decode": W.c5_mla_decode, "tiny_fp32_decode": W.c1_tiny_fp32_decode,
-           "bf16_sparse_topk_decode": W.sparse_bf16_decode}
+           "bf16_sparse_topk_decode": W.sparse_bf16_decode, "bf16_window_mixed_decode_part": W.c4_decode_part,
+           "bf16_window_mixed_prefill_part": W.c4_prefill_part}
     res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
     r = res[args.workload]
     if args.workload == "bf16_sparse_topk_decode":
@@ -463,6 +465,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffer) leg")
     ap.add_argument("--workload", default="bf16_decode",
                     choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode", "bf16_sparse_topk_decode",
+                             "bf16_window_mixed_decode_part", "bf16_window_mixed_prefill_part",
                              "tiny_fp32_decode"],
                     help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()

@@ -255,6 +255,22 @@ def c4_window_mixed(seed: int = 0, n_decode: int = 16, ctx: int = 32768, n_prefi
                     window=window, pin=pin)
 
 
+def c4_decode_part(seed: int = 0, n_decode: int = 16, ctx: int = 32768, window: int = 4096,
+                   pin: bool = False) -> GqaWorkload:
+    """The decode sub-batch of the window + mixed batch alone: n_decode sequences of context ctx,
+    one query each, Hq=64, Hkv=8, D=128, page 64, window, causal, bf16."""
+    return make_gqa(f"bf16_window{window}_decode_{n_decode}x{ctx}", seed, [ctx] * n_decode, [1] * n_decode, 64, 8,
+                    128, 128, 64, torch.bfloat16, causal=True, window=window, pin=pin)
+
+
+def c4_prefill_part(seed: int = 0, n_prefill: int = 4, hist: int = 8192, chunk: int = 1024, window: int = 4096,
+                    pin: bool = False) -> GqaWorkload:
+    """The prefill sub-batch of the window + mixed batch alone: n_prefill chunks of `chunk` queries
+    after `hist` keys of history, Hq=64, Hkv=8, D=128, page 64, window, causal, bf16."""
+    return make_gqa(f"bf16_window{window}_prefill_{n_prefill}x{hist}+{chunk}", seed, [hist + chunk] * n_prefill,
+                    [chunk] * n_prefill, 64, 8, 128, 128, 64, torch.bfloat16, causal=True, window=window, pin=pin)
+
+
 def c5_mla_decode(seed: int = 0, batch: int = 32, lmin: int = 1024, lmax: int = 16384,
                   pin: bool = False) -> MlaWorkload:
     """MLA absorbed-latent decode: batch, context U[lmin, lmax], H=128, R=512, rope 64,
