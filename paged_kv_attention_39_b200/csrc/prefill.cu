@@ -5,9 +5,10 @@
 // query heads that share one KV head (so every K/V tile feeds all G heads), against the keys
 // those queries can see, 128 keys per step, and writes the final output and lse.
 //
-//   warp 8      TMA producer: the Q tile once, then K and V tiles page by page (one box per
-//               page and 64-element half of the head dim, 128-byte swizzle) into a ring of
-//               stages; pages past the sequence's last key are never touched.
+//   warps 8, 11 TMA producers: warp 8 the Q tile once and the K tiles, warp 11 the V tiles, page
+//               by page (one box per page and 64-element half of the head dim, 128-byte
+//               swizzle) into rings of stages; pages past the sequence's last key are never
+//               touched.
 //   warp 9      TMEM owner and issuer (one thread) of S = Q K^T into one of two TMEM buffers.
 //   warp 10     issuer (one thread) of O += P V with P read from TMEM; before it, the warp
 //               zeroes the V rows past the sequence's last key (their bytes are whatever the page
@@ -43,7 +44,8 @@ constexpr int KST = 3;   // K stages
 constexpr int VST = 3;   // V stages
 constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quadrant, each owning half of the columns
 constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1, kPvWarp = kSoftmaxWarps + 2;
-constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
+constexpr int kTmaVWarp = kSoftmaxWarps + 3;  // the V producer (kTmaWarp loads Q and K)
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
@@ -238,26 +240,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_p0 = t_o + D, t_p1 = t_o + D + 64;
     const uint32_t s_base = smem_u32(smem);
 
-    if (warp == kTmaWarp) {
-        // ===================== TMA producer =====================
-        // The whole warp runs the loop; lane 0 issues. Page ids of the next 32 boxes are read
-        // from the block table by the 32 lanes at once and handed to lane 0 by shuffles, so a
-        // table read never sits between two loads.
+    if (warp == kTmaWarp || warp == kTmaVWarp) {
+        // ===================== TMA producers =====================
+        // One warp loads Q and the K tiles, another the V tiles, so that neither waits for the
+        // other's stages. The whole warp runs the loop; lane 0 issues. Page ids of the next 32
+        // boxes are read from the block table by the 32 lanes at once and handed to lane 0 by
+        // shuffles, so a table read never sits between two loads.
+        const bool is_v = warp == kTmaVWarp;
+        const int NST = is_v ? VST : KST;
+        const CUtensorMap* tm = is_v ? &tmv : &tmk;
+        uint64_t* full = &bars[is_v ? B_VFULL : B_KFULL];
+        uint64_t* empty = &bars[is_v ? B_VEMPTY : B_KEMPTY];
+        uint8_t* ring = smem + (is_v ? L_::V : L_::K);
         if (n_tiles > 0) {
             if (lane == 0) {
-                tma_prefetch(&tmq);
-                tma_prefetch(&tmk);
-                tma_prefetch(&tmv);
-                mbar_arrive_expect_tx(&bars[B_QFULL], KH * L_::HALF_Q);
-                for (int h = 0; h < KH; ++h)
-                    tma_load_3d(smem + L_::Q + h * L_::HALF_Q, &tmq, &bars[B_QFULL], h * 64, u.kvh * G,
-                                si.q_start + u.j0);
+                tma_prefetch(tm);
+                if (!is_v) {
+                    tma_prefetch(&tmq);
+                    mbar_arrive_expect_tx(&bars[B_QFULL], KH * L_::HALF_Q);
+                    for (int h = 0; h < KH; ++h)
+                        tma_load_3d(smem + L_::Q + h * L_::HALF_Q, &tmq, &bars[B_QFULL], h * 64, u.kvh * G,
+                                    si.q_start + u.j0);
+                }
             }
             const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
             const int bpt = BN / box;  // boxes per tile (<= 8)
             int base_g = -(1 << 30);   // first box whose page id the lanes hold
             int my_row = 0;            // lane l: first cache row of box base_g + l
-            int issued = 0;            // tiles whose K and V loads were issued
+            int issued = 0;            // tiles whose loads were issued
             for (int i = 0; i < n_tiles; ++i) {
                 const int64_t kt0 = kt_start + (int64_t)i * BN;
                 int nb = 0;  // boxes whose first key lies inside the sequence
@@ -269,40 +279,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int64_t key = kt_start + (int64_t)(base_g + lane) * box;
                     my_row = key < si.L ? (int)((int64_t)bt[key / ps] * ps + key % ps) : 0;
                 }
-                const uint32_t bytes = (uint32_t)nb * box * 128 * KH;
-                const int ks = i % KST, vs = i % VST;
-                if (i >= KST && !__all_sync(0xffffffffu, mbar_wait(&bars[B_KEMPTY + ks], ((i / KST) - 1) & 1, wd, 1)))
+                const int st = i % NST;
+                if (i >= NST && !__all_sync(0xffffffffu, mbar_wait(empty + st, ((i / NST) - 1) & 1, wd, is_v ? 2 : 1)))
                     break;
-                if (lane == 0) mbar_arrive_expect_tx(&bars[B_KFULL + ks], bytes);
+                if (lane == 0) mbar_arrive_expect_tx(full + st, (uint32_t)nb * box * 128 * KH);
                 for (int b = 0; b < nb; ++b) {
                     const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
                     if (lane == 0)
                         for (int h = 0; h < KH; ++h)
-                            tma_load_3d(smem + L_::K + (ks * KH + h) * L_::HALF_KV + b * box * 128, &tmk,
-                                        &bars[B_KFULL + ks], h * 64, u.kvh, row);
-                }
-                if (i >= VST && !__all_sync(0xffffffffu, mbar_wait(&bars[B_VEMPTY + vs], ((i / VST) - 1) & 1, wd, 2)))
-                    break;
-                if (lane == 0) mbar_arrive_expect_tx(&bars[B_VFULL + vs], bytes);
-                for (int b = 0; b < nb; ++b) {
-                    const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
-                    if (lane == 0)
-                        for (int h = 0; h < KH; ++h)
-                            tma_load_3d(smem + L_::V + (vs * KH + h) * L_::HALF_KV + b * box * 128, &tmv,
-                                        &bars[B_VFULL + vs], h * 64, u.kvh, row);
+                            tma_load_3d(ring + (st * KH + h) * L_::HALF_KV + b * box * 128, tm, full + st, h * 64,
+                                        u.kvh, row);
                 }
                 issued = i + 1;
             }
             if (lane == 0 && *abort_flag) {
                 // Leave no copy in flight into this CTA's shared memory: wait (bounded, ignoring
-                // the abort flag) for the last loads issued into each stage and for Q.
+                // the abort flag) for the last loads issued into each stage (and for Q).
                 const uint64_t t0 = globaltimer_ns();
                 auto drain = [&](uint64_t* bar, uint32_t parity) {
                     while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {}
                 };
-                drain(&bars[B_QFULL], 0);
-                for (int i = max(0, issued - KST); i < issued; ++i) drain(&bars[B_KFULL + i % KST], (i / KST) & 1);
-                for (int i = max(0, issued - VST); i < issued; ++i) drain(&bars[B_VFULL + i % VST], (i / VST) & 1);
+                if (!is_v) drain(&bars[B_QFULL], 0);
+                for (int i = max(0, issued - NST); i < issued; ++i) drain(full + i % NST, (i / NST) & 1);
             }
         }
     } else if (warp == kMmaWarp || warp == kPvWarp) {
