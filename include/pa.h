@@ -348,6 +348,16 @@ pa_status pa_sparse_forward(pa_plan* plan, const void* q, const void* k_cache, c
                             int32_t window, int32_t block_size, const int32_t* selection,
                             int32_t width, void* out, float* lse, pa_stream stream);
 
+/* pa_sparse_forward with options (pa_forward_options: key-part length of the split, counted in
+ * keys of the concatenated selected blocks and rounded up to a multiple of 16; path; trace events:
+ * the first after the selection check, then around the attention kernels and the merge). */
+pa_status pa_sparse_forward_ex(pa_plan* plan, const void* q, const void* k_cache,
+                               const void* v_cache, pa_dtype dtype, int32_t num_q_heads,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t v_head_dim,
+                               float scale, int causal, int32_t window, int32_t block_size,
+                               const int32_t* selection, int32_t width, void* out, float* lse,
+                               pa_stream stream, const pa_forward_options* opts);
+
 /*
  * pa_plan_device_status -- diagnostic read of the plan's device error word (synchronous copy:
  * not for the hot path). 0 means no kernel reported a failure; a non-zero code means a kernel

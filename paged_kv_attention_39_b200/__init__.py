@@ -30,7 +30,7 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
            "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex", "pa_append", "pa_backward",
-           "pa_plan_device_status", "pa_sparse_select", "pa_sparse_forward",
+           "pa_plan_device_status", "pa_sparse_select", "pa_sparse_forward", "pa_sparse_forward_ex",
            "pa_status_string", "pa_last_error_message", "pa_version"]
 PA_SPARSE_MAX_BLOCKS = 16384
 
@@ -105,6 +105,8 @@ def load_library(path: Optional[str] = None):
     lib.pa_sparse_forward.restype = ctypes.c_int
     lib.pa_sparse_forward.argtypes = [_P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _I, ctypes.c_float, ctypes.c_int, _I,
                                       _I, _P, _I, _P, _P, _P]
+    lib.pa_sparse_forward_ex.restype = ctypes.c_int
+    lib.pa_sparse_forward_ex.argtypes = lib.pa_sparse_forward.argtypes + [ctypes.POINTER(_Options)]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_status_string.argtypes = [ctypes.c_int]
     lib.pa_last_error_message.restype = ctypes.c_char_p
@@ -276,17 +278,19 @@ def pa_sparse_select(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, selecti
 
 def pa_sparse_forward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                       selection: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, scale: float, block_size: int,
-                      causal: bool = True, window: int = 0, stream=None) -> None:
+                      causal: bool = True, window: int = 0, stream=None, kv_chunk: int = 0,
+                      path: int = PA_PATH_AUTO, trace=None) -> None:
     """Attention over the blocks in selection [Nq, Hkv, width] int32 -> out, lse (in place)."""
     for t in (q, k_cache, v_cache, selection, out, lse):
         if not t.is_contiguous():
             raise ValueError("pa_sparse_forward takes contiguous tensors")
     if lse.dtype != torch.float32 or selection.dtype != torch.int32:
         raise ValueError("lse must be float32 and selection int32")
-    _check(load_library().pa_sparse_forward(
+    _check(load_library().pa_sparse_forward_ex(
         plan.handle, _ptr(q), _ptr(k_cache), _ptr(v_cache), _DTYPES[q.dtype], q.shape[1], k_cache.shape[2],
         q.shape[2], v_cache.shape[3], float(scale), int(bool(causal)), int(window), int(block_size),
-        _ptr(selection), selection.shape[2], _ptr(out), _ptr(lse), _stream_ptr(stream, plan.device)))
+        _ptr(selection), selection.shape[2], _ptr(out), _ptr(lse), _stream_ptr(stream, plan.device),
+        _opts(kv_chunk, path, trace)))
 
 
 def pa_append(plan: Plan, new_k: torch.Tensor, new_v: torch.Tensor, k_cache: torch.Tensor,

@@ -203,7 +203,9 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
         const int64_t target = tc_mla ? (int64_t)P->num_sms : (int64_t)P->num_sms * kTargetCtasPerSm;
         chunk = (total + target - 1) / std::max<int64_t>(1, target);
         chunk = ((chunk + 63) / 64) * 64;
-        chunk = std::max<int64_t>(chunk, 256);
+        // Sparse rows are short runs of selected blocks: whole rows up to 1024 keys per unit (no
+        // merge) beat finer splits; dense decode rows are split down to 256 keys.
+        chunk = std::max<int64_t>(chunk, k.sparse_bs > 0 ? 1024 : 256);
     }
 
     std::vector<pa::KvUnit> tcu, simtu, mlau;
@@ -775,6 +777,15 @@ pa_status pa_sparse_forward(pa_plan* plan, const void* q, const void* k_cache, c
                             pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                             int32_t v_head_dim, float scale, int causal, int32_t window, int32_t block_size,
                             const int32_t* selection, int32_t width, void* out, float* lse, pa_stream stream) {
+    return pa_sparse_forward_ex(plan, q, k_cache, v_cache, dtype, num_q_heads, num_kv_heads, head_dim, v_head_dim,
+                                scale, causal, window, block_size, selection, width, out, lse, stream, nullptr);
+}
+
+pa_status pa_sparse_forward_ex(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
+                               pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t v_head_dim, float scale, int causal, int32_t window, int32_t block_size,
+                               const int32_t* selection, int32_t width, void* out, float* lse, pa_stream stream,
+                               const pa_forward_options* opts) {
     if (!plan) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
     if (block_size <= 0) return fail(PA_ERR_SHAPE, "block_size must be > 0");
     Call c{};
@@ -784,7 +795,7 @@ pa_status pa_sparse_forward(pa_plan* plan, const void* q, const void* k_cache, c
     c.hq = num_q_heads; c.hkv = num_kv_heads; c.d = head_dim; c.dv = v_head_dim;
     c.scale = scale; c.causal = causal; c.window = window;
     c.out = out; c.lse = lse;
-    c.opts = default_opts(nullptr);
+    c.opts = default_opts(opts);
     c.block_size = block_size;
     c.selection = selection;
     c.width = width;

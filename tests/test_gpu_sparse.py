@@ -43,7 +43,7 @@ def gpu_select(wl, bs, topk, plan=None, width=None, with_scores=True):
     return (sc.cpu() if sc is not None else None), sel.cpu()
 
 
-def gpu_sparse_forward(wl, bs, sel, plan=None):
+def gpu_sparse_forward(wl, bs, sel, plan=None, kv_chunk=0, path=pa.PA_PATH_AUTO):
     own = plan is None
     if own:
         plan = pa.plan_for(wl)
@@ -51,7 +51,7 @@ def gpu_sparse_forward(wl, bs, sel, plan=None):
     out = torch.full((q.shape[0], wl.num_q_heads, wl.v_head_dim), float("nan"), dtype=q.dtype, device="cuda")
     lse = torch.full((q.shape[0], wl.num_q_heads), float("nan"), dtype=torch.float32, device="cuda")
     pa.pa_sparse_forward(plan, q, k, v, sel.to(torch.int32).cuda().contiguous(), out, lse, wl.scale, bs, wl.causal,
-                         wl.window)
+                         wl.window, kv_chunk=kv_chunk, path=path)
     torch.cuda.synchronize()
     status = pa.pa_plan_device_status(plan)
     if own:
@@ -245,3 +245,19 @@ def test_full_size_sparse_decode_sampled(orc):
                                             s.block_tables, s.page_size, wl.scale, bs, ref_sel, wl.causal, wl.window,
                                             rows=rows)
     check(wl, out, lse, ref_out, ref_lse, rows=rows, tag="full-size sparse")
+
+
+@pytest.mark.parametrize("kv_chunk,path", [(-1, pa.PA_PATH_AUTO), (16, pa.PA_PATH_AUTO), (40, pa.PA_PATH_AUTO),
+                                           (0, pa.PA_PATH_SIMT), (24, pa.PA_PATH_SIMT)])
+def test_forward_split_and_path(orc, kv_chunk, path):
+    """Any split of the selected keys into parts (rounded to 16 keys), and the CUDA-core path."""
+    name, wl, bs, topk = sparse_cases()[0]
+    s = wl.sched
+    ref_sc = orc.sparse_block_scores(wl.q, wl.k_cache, s.seq_lens, s.query_offsets, s.block_tables, s.page_size,
+                                     wl.scale, bs, wl.causal, wl.window)
+    ref_sel = orc.sparse_topk(ref_sc, s.seq_lens, s.query_offsets, bs, topk)
+    out, lse, status = gpu_sparse_forward(wl, bs, ref_sel, kv_chunk=kv_chunk, path=path)
+    assert status == 0
+    ref_out, ref_lse = orc.sparse_attention(wl.q, wl.k_cache, wl.v_cache, s.seq_lens, s.query_offsets,
+                                            s.block_tables, s.page_size, wl.scale, bs, ref_sel, wl.causal, wl.window)
+    check(wl, out, lse, ref_out, ref_lse, tag=f"chunk {kv_chunk} path {path}")
