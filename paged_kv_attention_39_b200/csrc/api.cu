@@ -138,7 +138,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     S->key = k;
     const int32_t G = k.hq / k.hkv;
     const bool tc_decode = !k.mla && k.path == PA_PATH_AUTO && k.dtype != PA_F32 &&
-                           k.d == k.dv && (k.d == 64 || k.d == 128);
+                           k.d == k.dv && (k.d == 64 || k.d == 128 || k.d == 256);
     const bool tc_prefill = !k.mla && k.path == PA_PATH_AUTO &&
                             pa::prefill_tc_supported((pa_dtype)k.dtype, k.d, k.dv, G, P->page_size);
     const bool tc_mla = k.mla && k.path == PA_PATH_AUTO &&

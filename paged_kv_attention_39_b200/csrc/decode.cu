@@ -1,4 +1,4 @@
-// Split-KV paged decode on the tensor cores (bf16 / fp16, head_dim 64 or 128, Dv == D).
+// Split-KV paged decode on the tensor cores (bf16 / fp16, head_dim 64, 128 or 256, Dv == D).
 //
 // A CTA owns one KvUnit for one KV head: up to 16 rows (the queries of a sequence times the
 // G query heads that share the KV head) against keys [t0, t1). The K/V bytes of a key are
@@ -357,6 +357,7 @@ template <typename T, bool SPARSE>
 cudaError_t launch_t(const AttnParams& p, int rows_max, cudaStream_t st) {
     const bool two = rows_max > 8;
     if (p.d == 64) return two ? launch_cfg<T, 64, 2, SPARSE>(p, st) : launch_cfg<T, 64, 1, SPARSE>(p, st);
+    if (p.d == 256) return two ? launch_cfg<T, 256, 2, SPARSE>(p, st) : launch_cfg<T, 256, 1, SPARSE>(p, st);
     return two ? launch_cfg<T, 128, 2, SPARSE>(p, st) : launch_cfg<T, 128, 1, SPARSE>(p, st);
 }
 

@@ -33,7 +33,7 @@ def small_decode(seed, dtype=torch.bfloat16, hq=32, hkv=8, d=128, batch=8, lmin=
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("kv_chunk", [0, -1, 48, 100])
 def test_small_decode_tensor_core(orc, dtype, d, kv_chunk):
     wl = small_decode(1, dtype=dtype, d=d)
@@ -51,6 +51,16 @@ def test_decode_groups_and_multi_query(orc, hq, hkv, qn):
     for kv_chunk in (0, 32):
         out, lse = run_gqa(wl, kv_chunk=kv_chunk)
         check(wl, out, lse, *ref, tag=f"G{hq // hkv} n{qn} chunk {kv_chunk}")
+
+
+@pytest.mark.parametrize("hq,hkv,qn", [(16, 1, 1), (8, 2, 4), (4, 4, 1)])
+def test_decode_head_dim_256(orc, hq, hkv, qn):
+    """head_dim 256 on the tensor-core decode kernel, up to 16 rows per KV head (two n-tiles)."""
+    wl = small_decode(3, hq=hq, hkv=hkv, d=256, qn=qn, lmin=qn, lmax=400)
+    ref = orc.run(wl)
+    for kv_chunk in (0, 64):
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+        check(wl, out, lse, *ref, tag=f"d256 G{hq // hkv} n{qn} chunk {kv_chunk}")
 
 
 @pytest.mark.parametrize("window", [1, 7, 100, 5000])
