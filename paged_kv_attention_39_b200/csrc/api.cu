@@ -59,6 +59,57 @@ struct Range {
 bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
 
 constexpr int kMaxSplits = 1024;           // parts one sequence's keys may be cut into
+
+// ---------------------------------------------------------------------------------------
+// Host-to-device uploads through pinned staging
+// ---------------------------------------------------------------------------------------
+// A copy from pageable memory makes the driver stage it itself (synchronously, and it may wait
+// for the stream); copies through page-locked slots are true asynchronous DMA. The slots are
+// allocated once per process and shared by every plan; a slot is reused once the event recorded
+// after its last copy has completed. Uploads larger than a slot go straight from pageable memory.
+constexpr int kStageSlots = 16;
+constexpr size_t kStageSlotBytes = 256 << 10;
+
+struct Staging {
+    std::mutex mu;
+    char* slot[kStageSlots] = {};
+    cudaEvent_t done[kStageSlots] = {};
+    bool used[kStageSlots] = {};
+    int next = 0;
+};
+constexpr int kStageDevices = 64;
+Staging* staging(int dev) {  // one set of slots per device (events belong to a device)
+    static std::mutex mu;
+    static Staging* per_dev[kStageDevices] = {};  // never destroyed: outlive any plan released at exit
+    if (dev < 0 || dev >= kStageDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!per_dev[dev]) per_dev[dev] = new Staging();
+    return per_dev[dev];
+}
+
+cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+    int dev = -1;
+    Staging* gp = bytes <= kStageSlotBytes && cudaGetDevice(&dev) == cudaSuccess ? staging(dev) : nullptr;
+    if (!gp) return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st);
+    Staging& g = *gp;
+    std::lock_guard<std::mutex> lock(g.mu);
+    const int i = g.next;
+    g.next = (g.next + 1) % kStageSlots;
+    cudaError_t e;
+    if (!g.slot[i]) {
+        if ((e = cudaMallocHost(reinterpret_cast<void**>(&g.slot[i]), kStageSlotBytes)) != cudaSuccess) {
+            g.slot[i] = nullptr;
+            return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st);
+        }
+        if ((e = cudaEventCreateWithFlags(&g.done[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+    } else if (g.used[i] && (e = cudaEventSynchronize(g.done[i])) != cudaSuccess) {
+        return e;  // the slot's previous copy has to finish before it is overwritten
+    }
+    std::memcpy(g.slot[i], src, bytes);
+    if ((e = cudaMemcpyAsync(dst, g.slot[i], bytes, cudaMemcpyHostToDevice, st)) != cudaSuccess) return e;
+    g.used[i] = true;
+    return cudaEventRecord(g.done[i], st);
+}
 constexpr int kTargetCtasPerSm = 8;        // automatic split size aims at this many CTAs/SM
 
 struct SchedKey {
@@ -273,7 +324,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     if (!pu.empty()) std::memcpy(S->host.data() + o_p, pu.data(), pu.size() * sizeof(pa::PrefillUnit));
     if (!mlau.empty()) std::memcpy(S->host.data() + o_m, mlau.data(), mlau.size() * sizeof(pa::KvUnit));
     PA_CUDA_TRY(cudaMallocAsync(&S->dev, S->host.size(), st));
-    cudaError_t e = cudaMemcpyAsync(S->dev, S->host.data(), S->host.size(), cudaMemcpyHostToDevice, st);
+    cudaError_t e = upload(S->dev, S->host.data(), S->host.size(), st);
     if (e != cudaSuccess) {
         cudaFreeAsync(S->dev, st);
         return fail(PA_ERR_CUDA, "schedule upload failed: %s", cudaGetErrorString(e));
@@ -671,8 +722,7 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
                 for (int32_t q = query_offsets[s]; q < query_offsets[s + 1]; ++q) q2s[q] = s;
         }
         PA_CUDA_TRY(cudaMallocAsync(&P->d_meta, total, (cudaStream_t)upload_stream));
-        cudaError_t e = cudaMemcpyAsync(P->d_meta, blob.data(), total, cudaMemcpyHostToDevice,
-                                        (cudaStream_t)upload_stream);
+        cudaError_t e = upload(P->d_meta, blob.data(), total, (cudaStream_t)upload_stream);
         P->last_stream = (cudaStream_t)upload_stream;
         P->uploaded_bytes = (int64_t)total;
         if (e != cudaSuccess) {
