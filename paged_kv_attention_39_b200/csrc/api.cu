@@ -87,6 +87,39 @@ Staging* staging(int dev) {  // one set of slots per device (events belong to a 
     return per_dev[dev];
 }
 
+// Device memory of plans (metadata, work lists, workspaces) comes from a pool of the library's
+// own per device that keeps freed memory cached (release threshold at its maximum): a plan per
+// decode step then allocates without going back to the driver, and the process's default pool
+// is left as the caller configured it.
+cudaError_t lib_malloc(void** ptr, size_t bytes, cudaStream_t st) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[kStageDevices] = {};
+    static bool tried[kStageDevices] = {};
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    cudaMemPool_t pool = nullptr;
+    if (dev >= 0 && dev < kStageDevices) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!tried[dev]) {
+            tried[dev] = true;
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t pl = nullptr;
+            if (cudaMemPoolCreate(&pl, &props) == cudaSuccess) {
+                uint64_t keep = UINT64_MAX;
+                cudaMemPoolSetAttribute(pl, cudaMemPoolAttrReleaseThreshold, &keep);
+                pools[dev] = pl;
+            }
+        }
+        pool = pools[dev];
+    }
+    if (!pool) return cudaMallocAsync(ptr, bytes, st);
+    return cudaMallocFromPoolAsync(ptr, bytes, pool, st);
+}
+
 cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     int dev = -1;
     Staging* gp = bytes <= kStageSlotBytes && cudaGetDevice(&dev) == cudaSuccess ? staging(dev) : nullptr;
@@ -323,7 +356,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     if (!cu.empty()) std::memcpy(S->host.data() + o_c, cu.data(), cu.size() * sizeof(pa::CombineUnit));
     if (!pu.empty()) std::memcpy(S->host.data() + o_p, pu.data(), pu.size() * sizeof(pa::PrefillUnit));
     if (!mlau.empty()) std::memcpy(S->host.data() + o_m, mlau.data(), mlau.size() * sizeof(pa::KvUnit));
-    PA_CUDA_TRY(cudaMallocAsync(&S->dev, S->host.size(), st));
+    PA_CUDA_TRY(lib_malloc(&S->dev, S->host.size(), st));
     cudaError_t e = upload(S->dev, S->host.data(), S->host.size(), st);
     if (e != cudaSuccess) {
         cudaFreeAsync(S->dev, st);
@@ -363,7 +396,7 @@ pa_status ensure_workspace(pa_plan* P, size_t bytes, cudaStream_t st) {
         P->ws_bytes = 0;
     }
     void* p = nullptr;
-    PA_CUDA_TRY(cudaMallocAsync(&p, bytes, st));
+    PA_CUDA_TRY(lib_malloc(&p, bytes, st));
     P->ws = (float*)p;
     P->ws_bytes = bytes;
     return PA_OK;
@@ -378,7 +411,7 @@ pa_status grow_buffer(P_** buf, size_t* have, size_t bytes, cudaStream_t st) {
         *have = 0;
     }
     void* p = nullptr;
-    PA_CUDA_TRY(cudaMallocAsync(&p, bytes, st));
+    PA_CUDA_TRY(lib_malloc(&p, bytes, st));
     *buf = (P_*)p;
     *have = bytes;
     return PA_OK;
@@ -721,7 +754,7 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
             for (int32_t s = 0; s < num_seqs; ++s)
                 for (int32_t q = query_offsets[s]; q < query_offsets[s + 1]; ++q) q2s[q] = s;
         }
-        PA_CUDA_TRY(cudaMallocAsync(&P->d_meta, total, (cudaStream_t)upload_stream));
+        PA_CUDA_TRY(lib_malloc(&P->d_meta, total, (cudaStream_t)upload_stream));
         cudaError_t e = upload(P->d_meta, blob.data(), total, (cudaStream_t)upload_stream);
         P->last_stream = (cudaStream_t)upload_stream;
         P->uploaded_bytes = (int64_t)total;
