@@ -1,9 +1,13 @@
 // Chunked-prefill paged attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
 // bf16 / fp16, head_dim 64 or 128, Dv == D.
 //
-// One CTA computes one 128-row tile: 128/G consecutive queries of a sequence times the G
-// query heads that share one KV head (so every K/V tile feeds all G heads), against the keys
-// those queries can see, 128 keys per step, and writes the final output and lse.
+// A unit is one 128-row tile: 128/G consecutive queries of a sequence times the G query heads
+// that share one KV head (so every K/V tile feeds all G heads), against the keys those queries
+// can see, 128 keys per step; it ends with the final output and lse. The kernel is persistent:
+// one CTA per SM walks the units in strides of the grid, and its pipelines run on from one unit
+// into the next (the Q of the next unit loads as soon as the last score product of the current
+// one has completed; K/V loads and score products of the next unit overlap the current unit's
+// last softmax and output store).
 //
 //   warps 8, 11 TMA producers: warp 8 the Q tile once and the K tiles, warp 11 the V tiles, page
 //               by page (one box per page and 64-element half of the head dim, 128-byte
@@ -67,7 +71,7 @@ struct PrefillSmem {
 // waiter can ever find its barrier two phases ahead of the phase it waits for.
 enum BarId { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
              B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2,
-             B_COUNT = B_ODONE + 2 };
+             B_QEMPTY = B_ODONE + 2, B_COUNT = B_QEMPTY + 1 };
 
 }  // namespace
 
@@ -202,20 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const Watchdog wd{abort_flag, p.err, kWaitLimitNs};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const PrefillUnit u = p.punits[blockIdx.x];
-    const SeqInfo si = p.seqs[u.seq];
     const int G = p.group;
     const int qpt = BM / G;
-    const int live_q = min(qpt, si.n - u.j0);
-    const int live_rows = live_q * G;
-    const int64_t p_first = (int64_t)si.L - si.n + u.j0;
-    const int64_t p_last = p_first + live_q - 1;
-    const int64_t kv_lo = p.window > 0 ? max64(0, p_first - p.window + 1) : 0;
-    const int64_t kv_hi = p.causal ? min64(si.L, p_last + 1) : si.L;
     const int ps = p.page_size;
     const int box = ps < BN ? ps : BN;  // keys per TMA box
-    const int64_t kt_start = (kv_lo / box) * box;
-    const int n_tiles = kv_hi > kt_start ? (int)((kv_hi - kt_start + BN - 1) / BN) : 0;
 
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
@@ -240,6 +234,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_p0 = t_o + D, t_p1 = t_o + D + 64;
     const uint32_t s_base = smem_u32(smem);
 
+    // Units come longest first from the host. In round rr the CTA takes unit rr * grid + b, with b
+    // = blockIdx.x on even rounds and grid - 1 - blockIdx.x on odd ones (a snake over the sorted
+    // list keeps the work per CTA even). Every role walks the same sequence and counts the key
+    // tiles it has passed (gt) and the units with at least one tile (kq); stage indices and
+    // barrier phases follow those running counts across units.
+    const int rounds = (p.num_punits + (int)gridDim.x - 1) / (int)gridDim.x;
+    auto unit_of = [&](int rr) {
+        return rr * (int)gridDim.x + ((rr & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x);
+    };
+    auto view_of = [&](int ui, PrefillUnit& u, SeqInfo& si, int& live_q, int64_t& p_first, int64_t& kt_start,
+                       int& n_tiles) {
+        u = p.punits[ui];
+        si = p.seqs[u.seq];
+        live_q = min(qpt, si.n - u.j0);
+        p_first = (int64_t)si.L - si.n + u.j0;
+        const int64_t p_last = p_first + live_q - 1;
+        const int64_t kv_lo = p.window > 0 ? max64(0, p_first - p.window + 1) : 0;
+        const int64_t kv_hi = p.causal ? min64(si.L, p_last + 1) : si.L;
+        kt_start = (kv_lo / box) * box;
+        n_tiles = kv_hi > kt_start ? (int)((kv_hi - kt_start + BN - 1) / BN) : 0;
+    };
+
     if (warp == kTmaWarp || warp == kTmaVWarp) {
         // ===================== TMA producers =====================
         // One warp loads Q and the K tiles, another the V tiles, so that neither waits for the
@@ -252,23 +268,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint64_t* full = &bars[is_v ? B_VFULL : B_KFULL];
         uint64_t* empty = &bars[is_v ? B_VEMPTY : B_KEMPTY];
         uint8_t* ring = smem + (is_v ? L_::V : L_::K);
-        if (n_tiles > 0) {
-            if (lane == 0) {
-                tma_prefetch(tm);
-                if (!is_v) {
-                    tma_prefetch(&tmq);
+        if (lane == 0) {
+            tma_prefetch(tm);
+            if (!is_v) tma_prefetch(&tmq);
+        }
+        const int bpt = BN / box;  // boxes per tile (<= 8)
+        int gt = 0, kq = 0;        // tiles and Q tiles issued
+        bool ok = true;
+        for (int rr = 0; ok && rr < rounds; ++rr) {
+            const int ui = unit_of(rr);
+            if (ui >= p.num_punits) continue;
+            PrefillUnit u;
+            SeqInfo si;
+            int live_q, n_tiles;
+            int64_t p_first, kt_start;
+            view_of(ui, u, si, live_q, p_first, kt_start, n_tiles);
+            if (n_tiles == 0) continue;
+            if (!is_v) {
+                // the Q buffer is free once every S = Q K^T of the previous unit has completed
+                if (kq > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[B_QEMPTY], (kq - 1) & 1, wd, 12))) break;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(&bars[B_QFULL], KH * L_::HALF_Q);
                     for (int h = 0; h < KH; ++h)
                         tma_load_3d(smem + L_::Q + h * L_::HALF_Q, &tmq, &bars[B_QFULL], h * 64, u.kvh * G,
                                     si.q_start + u.j0);
                 }
             }
+            ++kq;
             const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
-            const int bpt = BN / box;  // boxes per tile (<= 8)
-            int base_g = -(1 << 30);   // first box whose page id the lanes hold
-            int my_row = 0;            // lane l: first cache row of box base_g + l
-            int issued = 0;            // tiles whose loads were issued
-            for (int i = 0; i < n_tiles; ++i) {
+            int base_g = -(1 << 30);  // first box whose page id the lanes hold
+            int my_row = 0;           // lane l: first cache row of box base_g + l
+            for (int i = 0; i < n_tiles; ++i, ++gt) {
                 const int64_t kt0 = kt_start + (int64_t)i * BN;
                 int nb = 0;  // boxes whose first key lies inside the sequence
                 for (int b = 0; b < bpt; ++b)
@@ -279,9 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int64_t key = kt_start + (int64_t)(base_g + lane) * box;
                     my_row = key < si.L ? (int)((int64_t)bt[key / ps] * ps + key % ps) : 0;
                 }
-                const int st = i % NST;
-                if (i >= NST && !__all_sync(0xffffffffu, mbar_wait(empty + st, ((i / NST) - 1) & 1, wd, is_v ? 2 : 1)))
+                const int st = gt % NST;
+                if (gt >= NST && !__all_sync(0xffffffffu, mbar_wait(empty + st, ((gt / NST) - 1) & 1, wd, is_v ? 2 : 1))) {
+                    ok = false;
                     break;
+                }
                 if (lane == 0) mbar_arrive_expect_tx(full + st, (uint32_t)nb * box * 128 * KH);
                 for (int b = 0; b < nb; ++b) {
                     const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
@@ -290,18 +322,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_3d(ring + (st * KH + h) * L_::HALF_KV + b * box * 128, tm, full + st, h * 64,
                                         u.kvh, row);
                 }
-                issued = i + 1;
             }
-            if (lane == 0 && *abort_flag) {
-                // Leave no copy in flight into this CTA's shared memory: wait (bounded, ignoring
-                // the abort flag) for the last loads issued into each stage (and for Q).
-                const uint64_t t0 = globaltimer_ns();
-                auto drain = [&](uint64_t* bar, uint32_t parity) {
-                    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {}
-                };
-                if (!is_v) drain(&bars[B_QFULL], 0);
-                for (int i = max(0, issued - NST); i < issued; ++i) drain(full + i % NST, (i / NST) & 1);
-            }
+        }
+        if (lane == 0 && *abort_flag) {
+            // Leave no copy in flight into this CTA's shared memory: wait (bounded, ignoring the
+            // abort flag) for the last loads issued into each stage (and for the last Q).
+            const uint64_t t0 = globaltimer_ns();
+            auto drain = [&](uint64_t* bar, uint32_t parity) {
+                while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {}
+            };
+            if (!is_v && kq > 0) drain(&bars[B_QFULL], (kq - 1) & 1);
+            for (int i = max(0, gt - NST); i < gt; ++i) drain(full + i % NST, (i / NST) & 1);
         }
     } else if (warp == kMmaWarp || warp == kPvWarp) {
         // ===================== MMA issuers =====================
@@ -313,61 +344,76 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
         const uint64_t dK = sdesc_sw128(s_base + L_::K, 16, 1024);
         const uint64_t dV = sdesc_sw128(s_base + L_::V, L_::HALF_KV, 1024);
-        if (warp == kMmaWarp) {
-            // S of tile i goes into score buffer i & 1. Both buffers start free; after that,
-            // buffer j & 1 is free again once the softmax has marked P of tile j ready (it has
-            // then read all of S of tile j).
-            bool ok = __all_sync(0xffffffffu, n_tiles == 0 || mbar_wait(&bars[B_QFULL], 0, wd, 3));
-            for (int i = 0; ok && i < n_tiles; ++i) {
-                const int ks = i % KST, b = i & 1;
-                if (i >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + b], ((i - 2) >> 1) & 1, wd, 6));
-                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_KFULL + ks], (i / KST) & 1, wd, 4));
-                if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t d_s = b ? t_s1 : t_s0;
-                    const uint64_t dKs = desc_add(dK, ks * KH * L_::HALF_KV);
+        int gt = 0, kq = 0;
+        bool ok = true;
+        for (int rr = 0; ok && rr < rounds; ++rr) {
+            const int ui = unit_of(rr);
+            if (ui >= p.num_punits) continue;
+            PrefillUnit u;
+            SeqInfo si;
+            int live_q, n_tiles;
+            int64_t p_first, kt_start;
+            view_of(ui, u, si, live_q, p_first, kt_start, n_tiles);
+            if (n_tiles == 0) continue;
+            if (warp == kMmaWarp) {
+                // S of tile gt goes into score buffer gt & 1, free again once the softmax has
+                // marked P of tile gt - 2 ready (it has then read all of S of that tile).
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_QFULL], kq & 1, wd, 3));
+                for (int i = 0; ok && i < n_tiles; ++i, ++gt) {
+                    const int ks = gt % KST, b = gt & 1;
+                    if (gt >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + b], ((gt - 2) >> 1) & 1, wd, 6));
+                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_KFULL + ks], (gt / KST) & 1, wd, 4));
+                    if (!ok) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t d_s = b ? t_s1 : t_s0;
+                        const uint64_t dKs = desc_add(dK, ks * KH * L_::HALF_KV);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;  // HALF_Q == HALF_KV
-                        mma_f16_ss(d_s, desc_add(dQ, off), desc_add(dKs, off), IDESC_QK, kk > 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t off = (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;  // HALF_Q == HALF_KV
+                            mma_f16_ss(d_s, desc_add(dQ, off), desc_add(dKs, off), IDESC_QK, kk > 0);
+                        }
+                        mma_commit(&bars[B_SFULL + b]);
+                        mma_commit(&bars[B_KEMPTY + ks]);
+                        if (i == n_tiles - 1) mma_commit(&bars[B_QEMPTY]);
                     }
-                    mma_commit(&bars[B_SFULL + b]);
-                    mma_commit(&bars[B_KEMPTY + ks]);
-                }
-                __syncwarp();
-            }
-        } else {
-            // O += P V of tile j once P of tile j and V tile j are in place.
-            for (int j = 0; j < n_tiles; ++j) {
-                const int vs = j % VST;
-                bool ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + (j & 1)], (j >> 1) & 1, wd, 6));
-                if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_VFULL + vs], (j / VST) & 1, wd, 7));
-                if (!ok) break;
-                // V rows past the sequence's end hold arbitrary bytes: make them zero.
-                const int64_t kt0 = kt_start + (int64_t)j * BN;
-                const int nvalid = (int)min64(BN, si.L - kt0);
-                if (nvalid < BN) {
-                    for (int h = 0; h < KH; ++h) {
-                        uint4* base = reinterpret_cast<uint4*>(smem + L_::V + (vs * KH + h) * L_::HALF_KV);
-                        for (int c = nvalid * 8 + lane; c < BN * 8; c += 32) base[c] = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
                     __syncwarp();
                 }
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t t_pj = (j & 1) ? t_p1 : t_p0;
-                    const uint64_t dVs = desc_add(dV, vs * KH * L_::HALF_KV);
-                    const uint32_t acc0 = j > 0 ? 1u : 0u;
+            } else {
+                // O += P V of tile gt once P of that tile and its V tile are in place; the first
+                // tile of a unit starts O afresh (the softmax has read the previous unit's O
+                // before it marks that P ready).
+                for (int j = 0; ok && j < n_tiles; ++j, ++gt) {
+                    const int vs = gt % VST;
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_PFULL + (gt & 1)], (gt >> 1) & 1, wd, 6));
+                    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_VFULL + vs], (gt / VST) & 1, wd, 7));
+                    if (!ok) break;
+                    // V rows past the sequence's end hold arbitrary bytes: make them zero.
+                    const int64_t kt0 = kt_start + (int64_t)j * BN;
+                    const int nvalid = (int)min64(BN, si.L - kt0);
+                    if (nvalid < BN) {
+                        for (int h = 0; h < KH; ++h) {
+                            uint4* base = reinterpret_cast<uint4*>(smem + L_::V + (vs * KH + h) * L_::HALF_KV);
+                            for (int c = nvalid * 8 + lane; c < BN * 8; c += 32) base[c] = make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t t_pj = (gt & 1) ? t_p1 : t_p0;
+                        const uint64_t dVs = desc_add(dV, vs * KH * L_::HALF_KV);
+                        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
-                        mma_f16_ts(t_o, t_pj + kk * 8, desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
-                    mma_commit(&bars[B_ODONE + (j & 1)]);
-                    mma_commit(&bars[B_VEMPTY + vs]);
+                        for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 8 TMEM columns of P
+                            mma_f16_ts(t_o, t_pj + kk * 8, desc_add(dVs, kk * 16 * 128), IDESC_PV, kk > 0 ? 1u : acc0);
+                        mma_commit(&bars[B_ODONE + (gt & 1)]);
+                        mma_commit(&bars[B_VEMPTY + vs]);
+                    }
+                    __syncwarp();
                 }
-                __syncwarp();
             }
+            ++kq;
         }
     } else {
         // ===================== softmax: thread = row, two warps per row =====================
@@ -388,112 +434,126 @@ __global__ void __launch_bounds__(kThreads, 1)
             pair_sync();  // the slot may be written again only after the partner has read it
             return is_max ? fmaxf(mine, other) : mine + other;
         };
-        const bool live = r < live_rows;
-        const int64_t pos = p_first + (live ? r / G : 0);
-        // keys this row sees: [row_lo, row_hi) (padding rows: every key of the sequence)
-        const int64_t row_lo = (live && p.window > 0) ? max64(0, pos - p.window + 1) : 0;
-        const int64_t row_hi = (live && p.causal) ? min64(si.L, pos + 1) : si.L;
-        // keys every live row sees: [all_lo, all_hi)
-        const int64_t all_lo = p.window > 0 ? p_last - p.window + 1 : INT64_MIN;
-        const int64_t all_hi = min64(p.causal ? p_first + 1 : si.L, si.L);
-        float m_run = neg_inf(), l_part = 0.f;
+        int gt = 0;
         bool ok = true;
-        for (int i = 0; i < n_tiles; ++i) {
-            const int b = i & 1;
-            const int64_t kt0 = kt_start + (int64_t)i * BN;
-            const uint32_t t_sb = (b ? t_s1 : t_s0) + lane_off;
-            const bool full = kt0 >= all_lo && kt0 + BN <= all_hi;
-            // After an abort the loop still runs to its end (every wait then returns at once), so
-            // that both warps of a row reach the same row-statistics exchanges.
-            ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (i >> 1) & 1, wd, 8)) && ok;
-            tc_fence_after();
-            // P buffer b was last read by P V of tile i - 2
-            if (i >= 2) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((i - 2) >> 1) & 1, wd, 11)) && ok;
-            }
-            const uint32_t t_pb = (b ? t_p1 : t_p0) + lane_off;
-            const int off_lo = (int)(kt0 - row_lo), off_hi = (int)(kt0 - row_hi);
-            // Fast path: one pass with the running max when every row of the warp has one (both
-            // warps of a row decide alike: their running maxima are equal).
-            bool redo = true;
-            float sum = 0.f;
-            if (__all_sync(0xffffffffu, m_run != neg_inf())) {
-                float m_raw;
-                sum = full ? tile_fused<T, false>(t_sb, c0, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
-                           : tile_fused<T, true>(t_sb, c0, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
-                m_raw = exchange(m_raw, true);
-                redo = __any_sync(0xffffffffu, m_raw * p.scale_log2 > m_run + 8.0f);
-            }
-            if (redo) {
-                // pass 1: tile max of the raw scores; the scale is positive, so it is applied to
-                // the max once. Edge tiles mask keys outside [row_lo, row_hi) first.
-                float m_raw = full ? tile_max_full(t_sb, c0) : tile_max_masked(t_sb, c0, off_lo, off_hi);
-                m_raw = exchange(m_raw, true);
-                const float m_tile = m_raw * p.scale_log2;
-                const float m_new = fmaxf(m_run, m_tile);
-                const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
-                const bool rescale = grow && i > 0 && m_run != neg_inf();
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // the output must hold every earlier tile before it is rescaled
-                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((i - 1) & 1)], ((i - 1) >> 1) & 1, wd, 9)) && ok;
-                    tc_fence_after();
-                    const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
+        // After an abort the loops still run to their ends (every wait then returns at once), so
+        // that both warps of a row reach the same row-statistics exchanges.
+        for (int rr = 0; rr < rounds; ++rr) {
+            const int ui = unit_of(rr);
+            if (ui >= p.num_punits) continue;
+            PrefillUnit u;
+            SeqInfo si;
+            int live_q, n_tiles;
+            int64_t p_first, kt_start;
+            view_of(ui, u, si, live_q, p_first, kt_start, n_tiles);
+            const int live_rows = live_q * G;
+            const int64_t p_last = p_first + live_q - 1;
+            const bool live = r < live_rows;
+            const int64_t pos = p_first + (live ? r / G : 0);
+            // keys this row sees: [row_lo, row_hi) (padding rows: every key of the sequence)
+            const int64_t row_lo = (live && p.window > 0) ? max64(0, pos - p.window + 1) : 0;
+            const int64_t row_hi = (live && p.causal) ? min64(si.L, pos + 1) : si.L;
+            // keys every live row sees: [all_lo, all_hi)
+            const int64_t all_lo = p.window > 0 ? p_last - p.window + 1 : INT64_MIN;
+            const int64_t all_hi = min64(p.causal ? p_first + 1 : si.L, si.L);
+            float m_run = neg_inf(), l_part = 0.f;
+            for (int i = 0; i < n_tiles; ++i, ++gt) {
+                const int b = gt & 1;
+                const int64_t kt0 = kt_start + (int64_t)i * BN;
+                const uint32_t t_sb = (b ? t_s1 : t_s0) + lane_off;
+                const bool full = kt0 >= all_lo && kt0 + BN <= all_hi;
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_SFULL + b], (gt >> 1) & 1, wd, 8)) && ok;
+                tc_fence_after();
+                // P buffer b was last read by P V of tile gt - 2
+                if (gt >= 2) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + b], ((gt - 2) >> 1) & 1, wd, 11)) && ok;
+                }
+                const uint32_t t_pb = (b ? t_p1 : t_p0) + lane_off;
+                const int off_lo = (int)(kt0 - row_lo), off_hi = (int)(kt0 - row_hi);
+                // Fast path: one pass with the running max when every row of the warp has one (both
+                // warps of a row decide alike: their running maxima are equal).
+                bool redo = true;
+                float sum = 0.f;
+                if (__all_sync(0xffffffffu, m_run != neg_inf())) {
+                    float m_raw;
+                    sum = full ? tile_fused<T, false>(t_sb, c0, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
+                               : tile_fused<T, true>(t_sb, c0, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
+                    m_raw = exchange(m_raw, true);
+                    redo = __any_sync(0xffffffffu, m_raw * p.scale_log2 > m_run + 8.0f);
+                }
+                if (redo) {
+                    // pass 1: tile max of the raw scores; the scale is positive, so it is applied to
+                    // the max once. Edge tiles mask keys outside [row_lo, row_hi) first.
+                    float m_raw = full ? tile_max_full(t_sb, c0) : tile_max_masked(t_sb, c0, off_lo, off_hi);
+                    m_raw = exchange(m_raw, true);
+                    const float m_tile = m_raw * p.scale_log2;
+                    const float m_new = fmaxf(m_run, m_tile);
+                    const bool grow = m_new > m_run + 8.0f;  // also true when m_run is -inf and m_new finite
+                    const bool rescale = grow && i > 0 && m_run != neg_inf();
+                    if (__any_sync(0xffffffffu, rescale)) {
+                        // the output must hold every earlier tile of the unit before it is rescaled
+                        ok = __all_sync(0xffffffffu, mbar_wait(&bars[B_ODONE + ((gt - 1) & 1)], ((gt - 1) >> 1) & 1, wd, 9)) && ok;
+                        tc_fence_after();
+                        const float alpha = rescale ? fast_exp2(m_run - m_new) : 1.0f;
 #pragma unroll 1
-                    for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {  // this warp's half of O
-                        uint32_t v[32];
-                        tmem_ld32(t_o + lane_off + c * 32, v);
-                        tmem_ld_wait(v);
+                        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {  // this warp's half of O
+                            uint32_t v[32];
+                            tmem_ld32(t_o + lane_off + c * 32, v);
+                            tmem_ld_wait(v);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                        tmem_st32(t_o + lane_off + c * 32, v);
+                            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                            tmem_st32(t_o + lane_off + c * 32, v);
+                        }
                     }
+                    if (grow) {
+                        l_part *= fast_exp2(m_run - m_new);
+                        m_run = m_new;
+                    }
+                    const float m_use = m_run == neg_inf() ? 0.f : m_run;
+                    // pass 2: probabilities p = 2^(s * scale - m) into the P buffer
+                    sum = full ? tile_exp<T, false>(t_sb, c0, p.scale_log2, m_use, t_pb, 0, 0)
+                               : tile_exp<T, true>(t_sb, c0, p.scale_log2, m_use, t_pb, off_lo, off_hi);
                 }
-                if (grow) {
-                    l_part *= fast_exp2(m_run - m_new);
-                    m_run = m_new;
-                }
-                const float m_use = m_run == neg_inf() ? 0.f : m_run;
-                // pass 2: probabilities p = 2^(s * scale - m) into the P buffer
-                sum = full ? tile_exp<T, false>(t_sb, c0, p.scale_log2, m_use, t_pb, 0, 0)
-                           : tile_exp<T, true>(t_sb, c0, p.scale_log2, m_use, t_pb, off_lo, off_hi);
+                tmem_st_wait();
+                l_part += sum;
+                tc_fence_before();
+                mbar_arrive(&bars[B_PFULL + b]);
             }
-            tmem_st_wait();
-            l_part += sum;
-            tc_fence_before();
-            mbar_arrive(&bars[B_PFULL + b]);
-        }
-        // ---- epilogue: each warp of the pair stores its half of the output columns ----
-        if (ok && n_tiles > 0)
-            ok = __all_sync(0xffffffffu,
-                            mbar_wait(&bars[B_ODONE + ((n_tiles - 1) & 1)], ((n_tiles - 1) >> 1) & 1, wd, 10));
-        ok = __all_sync(0xffffffffu, ok);
-        const float l_run = exchange(l_part, false);
-        tc_fence_after();
-        const bool has = l_run > 0.f;
-        const float inv = has ? 1.0f / l_run : 0.f;
-        const int64_t qrow = (int64_t)(si.q_start + u.j0 + (live ? r / G : 0)) * p.hq + u.kvh * G + (live ? r % G : 0);
-        T* orow = static_cast<T*>(p.out) + qrow * D;
+            // ---- epilogue: each warp of the pair stores its half of the output columns ----
+            if (ok && n_tiles > 0)
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(&bars[B_ODONE + ((gt - 1) & 1)], ((gt - 1) >> 1) & 1, wd, 10));
+            ok = __all_sync(0xffffffffu, ok);
+            const float l_run = exchange(l_part, false);
+            tc_fence_after();
+            const bool has = l_run > 0.f;
+            const float inv = has ? 1.0f / l_run : 0.f;
+            const int64_t qrow = (int64_t)(si.q_start + u.j0 + (live ? r / G : 0)) * p.hq + u.kvh * G + (live ? r % G : 0);
+            T* orow = static_cast<T*>(p.out) + qrow * D;
 #pragma unroll 1
-        for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
-            uint32_t v[32];
-            if (ok && n_tiles > 0) {
-                tmem_ld32(t_o + lane_off + c * 32, v);
-                tmem_ld_wait(v);
-            } else {
+            for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
+                uint32_t v[32];
+                if (ok && n_tiles > 0) {
+                    tmem_ld32(t_o + lane_off + c * 32, v);
+                    tmem_ld_wait(v);
+                } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = 0u;
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack2<T>(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+                if (live && ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
             }
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-                pk[e] = pack2<T>(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
-            if (live && ok) {
-                uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-            }
+            if (live && ok && half == 0) p.lse[qrow] = has ? (m_run + __log2f(l_run)) * kLn2 : neg_inf();
+            // the next unit's first P V overwrites O: this warp's reads of it are complete
+            tc_fence_before();
         }
-        if (live && ok && half == 0) p.lse[qrow] = has ? (m_run + __log2f(l_run)) * kLn2 : neg_inf();
     }
 
     tc_fence_before();
@@ -558,7 +618,16 @@ cudaError_t launch_t(const AttnParams& p, int num_pages, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<p.num_punits, kThreads, L_::ALLOC, st>>>(tq, tk, tv, p);
+    // persistent: one CTA per SM (shared memory allows no more), each walking units in strides
+    static int sms[64] = {0};
+    int nsm = dev < 64 ? sms[dev] : 0;
+    if (nsm == 0) {
+        e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) sms[dev] = nsm;
+    }
+    const int grid = p.num_punits < nsm ? p.num_punits : nsm;
+    kern<<<grid, kThreads, L_::ALLOC, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 

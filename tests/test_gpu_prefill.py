@@ -67,6 +67,23 @@ def test_prefill_masks(orc, window, causal):
     check(wl, out, lse, *ref, tag=f"window {window} causal {causal}")
 
 
+@pytest.mark.parametrize("d,dtype,window,causal,ps", [(64, torch.bfloat16, 0, True, 64), (128, torch.float16, 100, True, 16),
+                                                    (128, torch.bfloat16, 0, False, 128)])
+def test_prefill_many_units_per_cta(orc, d, dtype, window, causal, ps):
+    """Several hundred 128-row tiles, so that each CTA of the persistent kernel runs one unit after
+    another (stage indices and barrier phases carried across units, Q reloaded per unit), with
+    ragged last tiles and histories from empty to 600 keys."""
+    wl = prefill_wl(8, hq=16, hkv=4, d=d, ps=ps, dtype=dtype, hist=(0, 600), chunk=70, batch=48,
+                    window=window, causal=causal)
+    ref = orc.run(wl)
+    plan = pa.plan_for(wl)
+    out, lse = run_gqa(wl, plan=plan)
+    assert pa.pa_plan_get_info(plan)["last_launches"] == 1
+    assert pa.pa_plan_device_status(plan) == 0
+    plan.close()
+    check(wl, out, lse, *ref, tag=f"many units d{d} {dtype} w{window} c{causal} ps{ps}")
+
+
 def test_prefill_without_history_and_single_query_tiles(orc):
     wl = W.make_gqa("p0", 6, [1, 33, 128, 129, 300], [1, 33, 128, 129, 300], 32, 8, 128, 128, 64,
                     torch.bfloat16, causal=True)
