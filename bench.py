@@ -298,12 +298,22 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
     res = {}
     cfgs = [("bf16_chunked_prefill", W.c3_chunked_prefill), ("bf16_window_mixed", W.c4_window_mixed),
             ("bf16_window_mixed_decode_part", W.c4_decode_part), ("bf16_window_mixed_prefill_part", W.c4_prefill_part),
-            ("bf16_mla_decode", W.c5_mla_decode), ("bf16_sparse_topk_decode", W.sparse_bf16_decode)]
+            ("bf16_mla_decode", W.c5_mla_decode), ("bf16_sparse_topk_decode", W.sparse_bf16_decode),
+            ("fp16_decode", lambda sd: W.c2_decode_variant(sd, torch.float16, 128)),
+            ("bf16_decode_d64", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 64)),
+            ("bf16_decode_d256", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256)),
+            ("bf16_append_chunk", W.append_chunk), ("bf16_backward_chunk", W.backward_chunk)]
     if only is not None:
         cfgs = [only]
     for name, fn in cfgs:
         if name == "bf16_sparse_topk_decode":
             res[name] = run_sparse(args, pa, W, dev, hbm, peak_src, only is not None)
+            continue
+        if name == "bf16_append_chunk":
+            res[name] = run_append(args, pa, W, dev, hbm, peak_src)
+            continue
+        if name == "bf16_backward_chunk":
+            res[name] = run_backward(args, pa, W, dev, tf_burst, peak_src)
             continue
         try:
             wl = fn(args.seed)
@@ -373,6 +383,75 @@ def run_sparse(args, pa, W, dev, hbm, peak_src, alone):
         return {"error": str(e)[:300]}
 
 
+def event_median(fn, before, steps, warmup):
+    """Median device time of fn() over `steps` calls, each timed alone with CUDA events; before()
+    runs untimed ahead of every call (an L2 flush, zeroing an accumulator)."""
+    for _ in range(warmup):
+        before()
+        fn()
+    ts = []
+    for _ in range(steps):
+        before()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def run_append(args, pa, W, dev, hbm, peak_src):
+    """Paged append of the chunked-prefill batch's 4096 new K/V rows (33.6 MB read and written).
+    The data is smaller than L2, so a 256 MB write flushes L2 before every timed call."""
+    try:
+        wl, nk, nv = W.append_chunk(args.seed)
+        plan = pa.plan_for(wl, device=dev.index)
+        k, v = wl.k_cache.to(dev), wl.v_cache.to(dev)
+        nk, nv = nk.to(dev), nv.to(dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        ms = event_median(lambda: pa.pa_append(plan, nk, nv, k, v), flush.zero_, max(args.extra_steps, 10), 3)
+        nbytes = W.append_bytes(wl)
+        plan.close()
+        return {"ms_per_step": round(ms, 4), "rows": wl.sched.num_queries * wl.num_kv_heads,
+                "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                "frac_hbm_of_%s" % peak_src: round(nbytes / (ms * 1e-3) / 1e9 / hbm, 4),
+                "algorithmic_mb": round(nbytes / 1e6, 1), "launches": 1, "l2": "flushed before each call"}
+    except Exception as e:  # a failing extra must not hide the headline
+        return {"error": str(e)[:300]}
+
+
+def run_backward(args, pa, W, dev, tf_burst, peak_src):
+    """Recompute-based backward of a chunked-prefill batch (4 sequences, history U[0, 2048] plus
+    256 queries): d_q written, d_k / d_v caches (float32) zeroed before and accumulated by each
+    timed call. CUDA-core float32 arithmetic with atomics for dK/dV."""
+    try:
+        wl, d_out = W.backward_chunk(args.seed)
+        plan = pa.plan_for(wl, device=dev.index)
+        q, k, v = wl.q.to(dev), wl.k_cache.to(dev), wl.v_cache.to(dev)
+        d_out = d_out.to(dev)
+        out = torch.empty(q.shape[0], q.shape[1], wl.v_head_dim, dtype=q.dtype, device=dev)
+        lse = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+        pa.pa_forward(plan, q, k, v, out, lse, wl.scale, wl.causal, wl.window)
+        d_q = torch.empty(q.shape, dtype=torch.float32, device=dev)
+        d_k = torch.empty(k.shape, dtype=torch.float32, device=dev)
+        d_v = torch.empty(v.shape, dtype=torch.float32, device=dev)
+
+        def zero():
+            d_k.zero_()
+            d_v.zero_()
+        ms = event_median(lambda: pa.pa_backward(plan, q, k, v, out, lse, d_out, d_q, d_k, d_v, wl.scale,
+                                                 wl.causal, wl.window), zero, max(args.extra_steps, 3), 2)
+        flops = W.backward_flops(wl)
+        plan.close()
+        return {"ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                "frac_tensor_of_%s" % peak_src: round(flops / (ms * 1e-3) / 1e12 / tf_burst, 4),
+                "algorithmic_gflop": round(flops / 1e9, 2), "launches": 1,
+                "note": "float32 CUDA-core kernel with atomics (correctness path), not tensor cores"}
+    except Exception as e:  # a failing extra must not hide the headline
+        return {"error": str(e)[:300]}
+
+
 def run_single(args, ws, rank, local):
     """One of the other configurations as the only workload (profiling and tuning runs)."""
     import paged_kv_attention_39_b200 as pa
@@ -384,11 +463,18 @@ def run_single(args, ws, rank, local):
     fns = {"bf16_chunked_prefill": W.c3_chunked_prefill, "bf16_window_mixed": W.c4_window_mixed,
            "bf16_mla_decode": W.c5_mla_decode, "tiny_fp32_decode": W.c1_tiny_fp32_decode,
            "bf16_sparse_topk_decode": W.sparse_bf16_decode, "bf16_window_mixed_decode_part": W.c4_decode_part,
-           "bf16_window_mixed_prefill_part": W.c4_prefill_part}
+           "bf16_window_mixed_prefill_part": W.c4_prefill_part,
+           "fp16_decode": lambda sd: W.c2_decode_variant(sd, torch.float16, 128),
+           "bf16_decode_d64": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 64),
+           "bf16_decode_d256": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256),
+           "bf16_append_chunk": W.append_chunk, "bf16_backward_chunk": W.backward_chunk}
     res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
     r = res[args.workload]
-    if args.workload == "bf16_sparse_topk_decode":
+    if args.workload in ("bf16_sparse_topk_decode", "bf16_append_chunk"):
         return {"metric": METRIC, "workload": args.workload, "value": r.get("gbs"), "unit": "GB/s",
+                "steps": args.steps, "warmup": args.warmup, "detail": r}
+    if args.workload in ("fp16_decode", "bf16_decode_d64", "bf16_decode_d256"):
+        return {"metric": METRIC, "workload": args.workload, "value": r.get("kv_gbs"), "unit": "GB/s",
                 "steps": args.steps, "warmup": args.warmup, "detail": r}
     return {"metric": METRIC, "workload": args.workload, "value": r.get("tflops"), "unit": "TFLOP/s",
             "steps": args.steps, "warmup": args.warmup, "detail": r}
@@ -466,7 +552,8 @@ def main():
     ap.add_argument("--workload", default="bf16_decode",
                     choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode", "bf16_sparse_topk_decode",
                              "bf16_window_mixed_decode_part", "bf16_window_mixed_prefill_part",
-                             "tiny_fp32_decode"],
+                             "tiny_fp32_decode", "fp16_decode", "bf16_decode_d64", "bf16_decode_d256",
+                             "bf16_append_chunk", "bf16_backward_chunk"],
                     help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()
     if args.warmup < 3:

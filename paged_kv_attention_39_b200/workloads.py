@@ -281,6 +281,46 @@ def c5_mla_decode(seed: int = 0, batch: int = 32, lmin: int = 1024, lmax: int = 
                     pin=pin)
 
 
+def c2_decode_variant(seed: int = 0, dtype: torch.dtype = torch.float16, d: int = 128, batch: int = 64,
+                      pin: bool = False) -> GqaWorkload:
+    """The bf16 decode batch's shape (64 sequences, context U[512, 8192], Hq=32, Hkv=8, page 16)
+    in another element type or head size (D = Dv = d)."""
+    lens = _uniform_ints(seed, 0xC2, batch, 512, 8192)
+    tag = {torch.float16: "fp16", torch.bfloat16: "bf16", torch.float32: "fp32"}[dtype]
+    return make_gqa(f"{tag}_decode_d{d}_b{batch}", seed, lens, [1] * batch, 32, 8, d, d, 16, dtype,
+                    causal=True, window=0, pin=pin)
+
+
+def append_chunk(seed: int = 0):
+    """Paged append of the chunked-prefill batch's new rows (8 sequences x 512 queries, Hkv=8,
+    D=Dv=128, pages of 64, bf16): (workload, new_k [Nq, Hkv, D], new_v [Nq, Hkv, Dv])."""
+    wl = c3_chunked_prefill(seed)
+    nq = wl.sched.num_queries
+    new_k = randn((nq, wl.num_kv_heads, wl.head_dim), seed, 21, wl.k_cache.dtype)
+    new_v = randn((nq, wl.num_kv_heads, wl.v_head_dim), seed, 22, wl.v_cache.dtype)
+    return wl, new_k, new_v
+
+
+def append_bytes(wl) -> int:
+    """Algorithmic HBM bytes of one append: every new K/V row read once and written once."""
+    esz = wl.k_cache.element_size()
+    return 2 * wl.sched.num_queries * wl.num_kv_heads * (wl.head_dim + wl.v_head_dim) * esz
+
+
+def backward_chunk(seed: int = 0, batch: int = 4, hmax: int = 2048, chunk: int = 256):
+    """Backward of a chunked-prefill batch (history U[0, hmax] plus `chunk` queries, Hq=32,
+    Hkv=8, D=128, pages of 64, bf16, causal): (workload, d_out [Nq, Hq, Dv])."""
+    wl = c3_chunked_prefill(seed, batch=batch, hmax=hmax, chunk=chunk)
+    d_out = randn((wl.sched.num_queries, wl.num_q_heads, wl.v_head_dim), seed, 23, wl.q.dtype)
+    return wl, d_out
+
+
+def backward_flops(wl) -> int:
+    """2 flops per multiply-add of the recompute-based backward over visible pairs, every query
+    head: the scores q.k (D), dP = dO.v (Dv), dV += P dO (Dv), dQ += dS k (D), dK += dS q (D)."""
+    return visible_pairs(wl) * wl.num_q_heads * 2 * (3 * wl.head_dim + 2 * wl.v_head_dim)
+
+
 def sparse_bf16_decode(seed: int = 0, block_size: int = 64, topk: int = 16, pin: bool = False):
     """The bf16 decode batch (64 sequences, context U[512, 8192], Hq=32, Hkv=8, D=128, page 16)
     with sparse top-K attention over blocks of `block_size` keys: (workload, block_size, topk).
