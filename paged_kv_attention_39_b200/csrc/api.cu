@@ -188,6 +188,13 @@ struct pa_plan {
     size_t sel_ws_bytes = 0;
     float* score_ws = nullptr;  // proxy block scores when the caller keeps none
     size_t score_ws_bytes = 0;
+    // tensor-core backward: work lists for one group size (key tiles, then row blocks) and Drow
+    void* bwd_dev = nullptr;
+    int32_t bwd_group = 0, bwd_causal = -1, bwd_window = -1, bwd_nkey = 0, bwd_nrow = 0;
+    size_t bwd_row_off = 0;
+    std::vector<std::vector<char>> bwd_host;  // host blobs of the uploads (kept with the plan)
+    float* bwd_drow = nullptr;
+    size_t bwd_drow_bytes = 0;
     cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
     int32_t last_launches = 0;
     int64_t uploaded_bytes = 0;
@@ -781,6 +788,8 @@ pa_status pa_plan_destroy(pa_plan* plan) {
         if (plan->ws) cudaFreeAsync(plan->ws, st);
         if (plan->sel_ws) cudaFreeAsync(plan->sel_ws, st);
         if (plan->score_ws) cudaFreeAsync(plan->score_ws, st);
+        if (plan->bwd_dev) cudaFreeAsync(plan->bwd_dev, st);
+        if (plan->bwd_drow) cudaFreeAsync(plan->bwd_drow, st);
         for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
         if (plan->d_meta) cudaFreeAsync(plan->d_meta, st);
         cudaError_t e = cudaLaunchHostFunc(st, [](void* ud) { delete static_cast<pa_plan*>(ud); }, plan);
@@ -1089,6 +1098,75 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
     PA_CUDA_TRY(cudaGetDevice(&cur));
     if (cur != plan->device)
         return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
+    const int32_t G = num_q_heads / num_kv_heads;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (pa::backward_mma_supported(dtype, head_dim, v_head_dim, G)) {
+        std::lock_guard<std::mutex> lock(plan->mu);
+        if (plan->bwd_group != G || plan->bwd_causal != causal || plan->bwd_window != window) {
+            // Work lists, longest first: 64-key tiles of every sequence (cost: the rows that see
+            // them) for dK/dV, and blocks of at most 16 rows (cost: the keys they see) for dQ.
+            const int KT = pa::backward_key_tile(), qpb = std::max(1, pa::backward_row_block() / G);
+            std::vector<std::pair<int64_t, pa::BwdKeyUnit>> ku;
+            std::vector<std::pair<int64_t, pa::BwdRowUnit>> ru;
+            for (int32_t si = 0; si < plan->S; ++si) {
+                const pa::SeqInfo& q_ = plan->seqs[si];
+                if (q_.n == 0) continue;
+                const int64_t base = (int64_t)q_.L - q_.n;
+                for (int64_t k0 = 0; k0 < q_.L; k0 += KT) {
+                    const int64_t kmax = std::min<int64_t>(k0 + KT, q_.L);
+                    const int64_t jlo = causal ? std::max<int64_t>(0, k0 - base) : 0;
+                    const int64_t jhi = window > 0 ? std::min<int64_t>(q_.n, kmax - 1 + window - base) : q_.n;
+                    if (jhi <= jlo) continue;
+                    ku.push_back({jhi - jlo, pa::BwdKeyUnit{si, (int32_t)k0}});
+                }
+                for (int32_t j0 = 0; j0 < q_.n; j0 += qpb) {
+                    const int32_t j1 = std::min(q_.n, j0 + qpb);
+                    int32_t lo = 0, hi = 0;
+                    visible_union(q_.L, q_.n, j0, j1, causal != 0, window, &lo, &hi);
+                    ru.push_back({(int64_t)hi - lo, pa::BwdRowUnit{si, j0, j1, 0}});
+                }
+            }
+            auto longer = [](const auto& a, const auto& b) { return a.first > b.first; };
+            std::stable_sort(ku.begin(), ku.end(), longer);
+            std::stable_sort(ru.begin(), ru.end(), longer);
+            const size_t row_off = (ku.size() * sizeof(pa::BwdKeyUnit) + 255) & ~size_t(255);
+            std::vector<char> blob(std::max<size_t>(16, row_off + ru.size() * sizeof(pa::BwdRowUnit)));
+            for (size_t i = 0; i < ku.size(); ++i) std::memcpy(blob.data() + i * sizeof(pa::BwdKeyUnit), &ku[i].second, sizeof(pa::BwdKeyUnit));
+            for (size_t i = 0; i < ru.size(); ++i)
+                std::memcpy(blob.data() + row_off + i * sizeof(pa::BwdRowUnit), &ru[i].second, sizeof(pa::BwdRowUnit));
+            if (plan->bwd_dev) {
+                PA_CUDA_TRY(cudaFreeAsync(plan->bwd_dev, st));
+                plan->bwd_dev = nullptr;
+            }
+            PA_CUDA_TRY(lib_malloc(&plan->bwd_dev, blob.size(), st));
+            PA_CUDA_TRY(upload(plan->bwd_dev, blob.data(), blob.size(), st));
+            plan->bwd_host.push_back(std::move(blob));
+            plan->bwd_group = G;
+            plan->bwd_causal = causal;
+            plan->bwd_window = window;
+            plan->bwd_nkey = (int32_t)ku.size();
+            plan->bwd_nrow = (int32_t)ru.size();
+            plan->bwd_row_off = row_off;
+            plan->uploaded_bytes += (int64_t)plan->bwd_host.back().size();
+        }
+        pa_status gs = grow_buffer(&plan->bwd_drow, &plan->bwd_drow_bytes, (size_t)nq * num_q_heads * sizeof(float), st);
+        if (gs != PA_OK) return gs;
+        pa::BwdParams2 bp{};
+        bp.q = q; bp.k = k_cache; bp.v = v_cache; bp.out = out; bp.lse = lse; bp.dout = d_out;
+        bp.drow = plan->bwd_drow; bp.dq = d_q; bp.dk = d_k_cache; bp.dv = d_v_cache;
+        bp.seqs = plan->d_seqs; bp.block_tables = plan->d_bt;
+        bp.key_units = (const pa::BwdKeyUnit*)plan->bwd_dev;
+        bp.row_units = (const pa::BwdRowUnit*)((const char*)plan->bwd_dev + plan->bwd_row_off);
+        bp.table_width = plan->table_width; bp.page_size = plan->page_size;
+        bp.hq = num_q_heads; bp.hkv = num_kv_heads; bp.group = G; bp.d = head_dim;
+        bp.scale = scale; bp.scale_log2 = scale * 1.4426950408889634f;
+        bp.causal = causal; bp.window = window;
+        cudaError_t e = pa::launch_backward_mma(bp, dtype, plan->bwd_nkey, plan->bwd_nrow, nq * num_q_heads, st);
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "backward kernel launch failed: %s", cudaGetErrorString(e));
+        plan->last_stream = st;
+        plan->last_launches = 1 + (plan->bwd_nkey > 0 ? 1 : 0) + (plan->bwd_nrow > 0 ? 1 : 0);
+        return ok();
+    }
     cudaError_t e = pa::launch_backward(q, k_cache, v_cache, out, lse, d_out, d_q, d_k_cache, d_v_cache,
                                         plan->d_seqs, plan->d_q2seq, plan->d_bt, plan->table_width, plan->page_size,
                                         num_q_heads, num_kv_heads, head_dim, v_head_dim, scale, causal, window,

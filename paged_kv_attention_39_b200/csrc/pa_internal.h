@@ -38,6 +38,35 @@ struct PrefillUnit {
     int32_t kvh, pad0, pad1, pad2;
 };
 
+// Backward on the tensor cores: a 64-key tile of sequence `seq` starting at key k0 (dK/dV
+// kernel), and queries j0 .. j1-1 of a sequence, at most 16 rows per KV head (dQ kernel).
+struct BwdKeyUnit {
+    int32_t seq, k0;
+};
+struct BwdRowUnit {
+    int32_t seq, j0, j1, pad;
+};
+
+struct BwdParams2 {
+    const void* q;       // [Nq, Hq, D]
+    const void* k;       // [P, ps, Hkv, D]
+    const void* v;       // [P, ps, Hkv, D]
+    const void* out;     // [Nq, Hq, D] forward output
+    const float* lse;    // [Nq, Hq] forward logsumexp (natural log)
+    const void* dout;    // [Nq, Hq, D]
+    float* drow;         // [Nq, Hq] dO . O, written by the first kernel
+    float* dq;           // [Nq, Hq, D] written
+    float* dk;           // [P, ps, Hkv, D] added into
+    float* dv;           // [P, ps, Hkv, D] added into
+    const SeqInfo* seqs;
+    const int32_t* block_tables;
+    const BwdKeyUnit* key_units;
+    const BwdRowUnit* row_units;
+    int32_t table_width, page_size, hq, hkv, group, d;
+    float scale, scale_log2;
+    int32_t causal, window;
+};
+
 // Everything a kernel needs; passed by value.
 struct AttnParams {
     const void* q;    // [Nq, Hq, D]   (MLA: absorbed q [Nq, H, R])
@@ -85,6 +114,13 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
 cudaError_t launch_append(const void* new_k, const void* new_v, void* k_cache, void* v_cache, const SeqInfo* seqs,
                           const int32_t* q2seq, const int32_t* block_tables, int32_t table_width, int32_t page_size,
                           int32_t hkv, int32_t k_row_bytes, int32_t v_row_bytes, int64_t rows, cudaStream_t st);
+// Tensor-core backward (backward_mma.cu): shapes it takes, its tile sizes and the launch of its
+// three kernels (Drow, dK/dV, dQ).
+bool backward_mma_supported(pa_dtype dt, int d, int dv, int group);
+int backward_key_tile();
+int backward_row_block();
+cudaError_t launch_backward_mma(const BwdParams2& p, pa_dtype dt, int num_key_units, int num_row_units, int64_t rows,
+                                cudaStream_t st);
 // Sparse top-K block selection (sparse.cu).
 cudaError_t launch_sparse_scores(const void* q, const void* k, float* scores, int32_t sw, const SeqInfo* seqs,
                                  const int32_t* q2seq, const int32_t* block_tables, int32_t table_width,

@@ -1,4 +1,5 @@
-"""GPU backward (recompute-based, float32 atomics for dK/dV) against the fp64 oracle's backward."""
+"""GPU backward against the fp64 oracle's backward: the tensor-core path (bf16 / fp16, D in {64, 128},
+at most 16 heads per group; deterministic dK/dV) and the float32 CUDA-core kernel (other shapes)."""
 import pytest
 import torch
 
@@ -26,6 +27,17 @@ def run_backward(wl, g):
     return dout, dq.cpu(), dk.cpu(), dv.cpu()
 
 
+# Tolerances. float32: the CUDA-core kernel computes in float32 throughout (1e-4 of the largest
+# gradient element). bf16 / fp16: the tensor-core path rounds P and dS to the 16-bit input type
+# before the dV, dK and dQ products (as the forward rounds P before P V). With unit roundoff u
+# (2^-8 bf16, 2^-11 fp16) an element summed over N keys is off by about u * sqrt(N) * |term|,
+# which does not shrink where the terms cancel, so the bound is set against the largest element:
+# an fp64 emulation of exactly that rounding on the 1000-key shape below gives 0.34 % of the
+# largest |dQ|; the bounds leave about three times that.
+TOL_MAX = {torch.bfloat16: 1e-2, torch.float16: 2.5e-3}
+TOL_REL = {torch.bfloat16: 2e-2, torch.float16: 1e-2}
+
+
 def close(got, ref, dtype, tag):
     got, ref = got.double(), ref.double()
     owned = torch.isfinite(ref)
@@ -34,7 +46,7 @@ def close(got, ref, dtype, tag):
         tol = 1e-4 * scale
         assert float((got - ref)[owned].abs().max()) <= tol, (tag, float((got - ref)[owned].abs().max()), tol)
     else:
-        bad = (got - ref).abs() > 2e-3 * scale + 2e-2 * ref.abs()
+        bad = (got - ref).abs() > TOL_MAX[dtype] * scale + TOL_REL[dtype] * ref.abs()
         assert not bool(bad[owned].any()), (tag, float((got - ref)[owned].abs().max()), scale)
 
 
@@ -65,3 +77,64 @@ def test_backward_shared_prefix_page_accumulates(orc):
     close(dq, rq, torch.float32, "dq")
     close(dk, rk, torch.float32, "dk")
     close(dv, rv, torch.float32, "dv")
+
+
+@pytest.mark.parametrize("hq,hkv,d,ps,causal,window,dtype", [
+    (32, 8, 128, 64, True, 0, torch.bfloat16),
+    (16, 16, 128, 16, True, 0, torch.float16),   # one head per group
+    (16, 1, 64, 32, True, 100, torch.bfloat16),  # sixteen heads per group, window
+    (8, 2, 128, 16, False, 0, torch.bfloat16),
+    (8, 4, 64, 128, True, 0, torch.float16),
+])
+def test_backward_tensor_core_shapes(orc, hq, hkv, d, ps, causal, window, dtype):
+    """The tensor-core backward (key-major dK/dV, query-major dQ): chunked prefills with history,
+    a prefill from empty history, many 64-key tiles and 16-row blocks, ragged ends."""
+    wl = W.make_gqa("bwd_tc", 5, [300, 513, 64, 1000], [100, 200, 64, 17], hq, hkv, d, d, ps, dtype,
+                    causal=causal, window=window)
+    g = torch.Generator().manual_seed(11)
+    dout, dq, dk, dv = run_backward(wl, g)
+    s = wl.sched
+    rq, rk, rv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s.seq_lens, s.query_offsets,
+                                        s.block_tables, s.page_size, wl.scale, causal, window)
+    tag = f"hq{hq} hkv{hkv} d{d} ps{ps} c{causal} w{window}"
+    close(dq, rq, dtype, "dq " + tag)
+    close(dk, rk, dtype, "dk " + tag)
+    close(dv, rv, dtype, "dv " + tag)
+
+
+def test_backward_tensor_core_shared_pages_and_launches(orc):
+    """bf16 on the tensor-core path with two sequences sharing their first pages: each CTA adds its
+    finished key rows once, so the shared slots receive both sequences' gradients. The path runs
+    three kernels (Drow, dK/dV, dQ)."""
+    wl = W.make_gqa("share_tc", 6, [150, 150], [30, 30], 8, 2, 64, 64, 16, torch.bfloat16)
+    s = wl.sched
+    s.block_tables[1, :3] = s.block_tables[0, :3]  # keys 0..47 shared
+    g = torch.Generator().manual_seed(12)
+    q, k, v = wl.q.cuda(), wl.k_cache.cuda(), wl.v_cache.cuda()
+    nq, hq, d = q.shape
+    dout = torch.randn(nq, hq, d, generator=g).to(q.dtype)
+    plan = pa.plan_for(wl)
+    out = torch.empty(nq, hq, d, dtype=q.dtype, device="cuda")
+    lse = torch.empty(nq, hq, dtype=torch.float32, device="cuda")
+    pa.pa_forward(plan, q, k, v, out, lse, wl.scale, True, 0)
+    dq = torch.empty((nq, hq, d), dtype=torch.float32, device="cuda")
+    dk = torch.zeros(k.shape, dtype=torch.float32, device="cuda")
+    dv = torch.zeros(v.shape, dtype=torch.float32, device="cuda")
+    pa.pa_backward(plan, q, k, v, out, lse, dout.cuda(), dq, dk, dv, wl.scale, True, 0)
+    assert pa.pa_plan_get_info(plan)["last_launches"] == 3
+    torch.cuda.synchronize()
+    plan.close()
+    rq, rk, rv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s.seq_lens, s.query_offsets,
+                                        s.block_tables, 16, wl.scale, True, 0)
+    close(dq.cpu(), rq, torch.bfloat16, "dq")
+    close(dk.cpu(), rk, torch.bfloat16, "dk")
+    close(dv.cpu(), rv, torch.bfloat16, "dv")
+
+
+def test_backward_tensor_core_deterministic():
+    """Without shared pages every gradient element is summed by one CTA in a fixed order: two runs
+    give the same bits."""
+    wl = W.make_gqa("det", 7, [400, 260], [60, 260], 16, 4, 128, 128, 64, torch.bfloat16)
+    runs = [run_backward(wl, torch.Generator().manual_seed(13)) for _ in range(2)]
+    for a, b in zip(runs[0][1:], runs[1][1:]):
+        assert torch.equal(torch.nan_to_num(a, nan=0.0), torch.nan_to_num(b, nan=0.0))
