@@ -302,7 +302,8 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
             ("fp16_decode", lambda sd: W.c2_decode_variant(sd, torch.float16, 128)),
             ("bf16_decode_d64", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 64)),
             ("bf16_decode_d256", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256)),
-            ("bf16_append_chunk", W.append_chunk), ("bf16_backward_chunk", W.backward_chunk)]
+            ("bf16_append_chunk", W.append_chunk), ("bf16_backward_chunk", W.backward_chunk),
+            ("bf16_mla_backward", W.mla_backward_small)]
     if only is not None:
         cfgs = [only]
     for name, fn in cfgs:
@@ -314,6 +315,9 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
             continue
         if name == "bf16_backward_chunk":
             res[name] = run_backward(args, pa, W, dev, tf_burst, peak_src)
+            continue
+        if name == "bf16_mla_backward":
+            res[name] = run_mla_backward(args, pa, W, dev, tf_burst, peak_src)
             continue
         try:
             wl = fn(args.seed)
@@ -453,6 +457,38 @@ def run_backward(args, pa, W, dev, tf_burst, peak_src):
         return {"error": str(e)[:300]}
 
 
+def run_mla_backward(args, pa, W, dev, tf_burst, peak_src):
+    """MLA backward of 4 decode sequences (128 heads, context U[256, 1024]): CUDA-core kernel, a warp
+    per (query, head) row, float32 atomics into the latent and rope gradient caches."""
+    try:
+        wl, d_out = W.mla_backward_small(args.seed)
+        plan = pa.plan_for(wl, device=dev.index)
+        ql, qr = wl.q_latent.to(dev), wl.q_rope.to(dev)
+        lat, rope = wl.latent_cache.to(dev), wl.rope_cache.to(dev)
+        d_out = d_out.to(dev)
+        out = torch.empty(ql.shape, dtype=ql.dtype, device=dev)
+        lse = torch.empty(ql.shape[:2], dtype=torch.float32, device=dev)
+        pa.pa_mla_forward(plan, ql, qr, lat, rope, out, lse, wl.scale, wl.causal, wl.window)
+        dql = torch.empty(ql.shape, dtype=torch.float32, device=dev)
+        dqr = torch.empty(qr.shape, dtype=torch.float32, device=dev)
+        dlat = torch.empty(lat.shape, dtype=torch.float32, device=dev)
+        drope = torch.empty(rope.shape, dtype=torch.float32, device=dev)
+
+        def zero():
+            dlat.zero_()
+            drope.zero_()
+        ms = event_median(lambda: pa.pa_mla_backward(plan, ql, qr, lat, rope, out, lse, d_out, dql, dqr, dlat, drope,
+                                                     wl.scale, wl.causal, wl.window), zero, max(args.extra_steps, 3), 2)
+        flops = W.mla_backward_flops(wl)
+        plan.close()
+        return {"ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                "frac_tensor_of_%s" % peak_src: round(flops / (ms * 1e-3) / 1e12 / tf_burst, 4),
+                "algorithmic_gflop": round(flops / 1e9, 2), "launches": 1,
+                "note": "CUDA-core float32 kernel with atomics (the MLA backward's first, correct version)"}
+    except Exception as e:  # a failing extra must not hide the headline
+        return {"error": str(e)[:300]}
+
+
 def run_single(args, ws, rank, local):
     """One of the other configurations as the only workload (profiling and tuning runs)."""
     import paged_kv_attention_39_b200 as pa
@@ -468,7 +504,8 @@ def run_single(args, ws, rank, local):
            "fp16_decode": lambda sd: W.c2_decode_variant(sd, torch.float16, 128),
            "bf16_decode_d64": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 64),
            "bf16_decode_d256": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256),
-           "bf16_append_chunk": W.append_chunk, "bf16_backward_chunk": W.backward_chunk}
+           "bf16_append_chunk": W.append_chunk, "bf16_backward_chunk": W.backward_chunk,
+           "bf16_mla_backward": W.mla_backward_small}
     res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
     r = res[args.workload]
     if args.workload in ("bf16_sparse_topk_decode", "bf16_append_chunk"):
@@ -554,7 +591,7 @@ def main():
                     choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode", "bf16_sparse_topk_decode",
                              "bf16_window_mixed_decode_part", "bf16_window_mixed_prefill_part",
                              "tiny_fp32_decode", "fp16_decode", "bf16_decode_d64", "bf16_decode_d256",
-                             "bf16_append_chunk", "bf16_backward_chunk"],
+                             "bf16_append_chunk", "bf16_backward_chunk", "bf16_mla_backward"],
                     help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -237,6 +237,35 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
                       float* d_k_cache, float* d_v_cache, pa_stream stream);
 
 /*
+ * pa_mla_backward -- gradients of MLA absorbed-latent attention (the backward the pages list for
+ * MLA beside GQA; ruDNN `mla_backward`, recompute-based). MLA is single-head attention with the key
+ * [latent | rope] and the value latent, so with P recomputed from the forward's lse:
+ *     dP_t = dO . latent_t,  D = dO . out,  dS_t = P_t (dP_t - D)
+ *     d_q_latent = scale sum_t dS_t latent_t,    d_q_rope = scale sum_t dS_t rope_t
+ *     d_latent_t += scale dS_t q_latent + P_t dO  (the latent is both key and value)
+ *     d_rope_t   += scale dS_t q_rope
+ * summed over every query head and query that sees key t (and every sequence sharing its page).
+ *
+ *   q_latent, q_rope, latent_cache, rope_cache   the forward's inputs (dtype; pa_mla_forward layouts)
+ *   out, lse                                     the forward's outputs
+ *   d_out            [N_q, num_heads, latent_dim] dtype
+ *   d_q_latent       [N_q, num_heads, latent_dim] float32, written
+ *   d_q_rope         [N_q, num_heads, rope_dim]   float32, written
+ *   d_latent_cache   [num_pages, page_size, 1, latent_dim] float32, ADDED INTO (zero it first)
+ *   d_rope_cache     [num_pages, page_size, 1, rope_dim]   float32, ADDED INTO (zero it first)
+ * A warp per (query, head) row on the CUDA cores, float32 throughout; the cache gradients are
+ * float32 atomics, so their summation order varies between runs. Shapes as pa_mla_forward;
+ * validation and errors as pa_backward (gradient outputs must not overlap each other or any
+ * input).
+ */
+pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rope,
+                          const void* latent_cache, const void* rope_cache, const void* out,
+                          const float* lse, const void* d_out, pa_dtype dtype, int32_t num_heads,
+                          int32_t latent_dim, int32_t rope_dim, float scale, int causal,
+                          int32_t window, float* d_q_latent, float* d_q_rope, float* d_latent_cache,
+                          float* d_rope_cache, pa_stream stream);
+
+/*
  * pa_forward_static_workspace -- pa_forward's split-KV decode without any memory allocation.
  * The pages describe no such call: it exists for callers that cannot allocate device memory
  * while they run attention (a serving loop that must not stall on the allocator mid-step, a

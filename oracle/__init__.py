@@ -140,6 +140,21 @@ class Oracle:
             raise ValueError(f"oracle rejected the schedule (code {rc})")
         return dq, dk, dvv
 
+    # -- backward of MLA absorbed-latent attention ---------------------------------------------
+    def mla_backward(self, q_latent, q_rope, latent_cache, rope_cache, d_out, seq_lens, query_offsets,
+                     block_tables, page_size, scale, causal=True, window=0, nthreads=None):
+        """(d_q_latent [Nq, H, R], d_q_rope [Nq, H, Pr], d_latent [P, ps, 1, R], d_rope [P, ps, 1, Pr])
+        float64. MLA is single-head GQA with the key [latent | rope] and the value latent (ruDNN
+        `mla` passes the latent as both K and V), so this is the GQA backward on the concatenated key
+        and query, split back by columns; the latent's gradient is the sum of its key part and its
+        value part."""
+        r = q_latent.shape[2]
+        q = torch.cat([q_latent, q_rope], dim=2)
+        k = torch.cat([latent_cache, rope_cache], dim=3)
+        dq, dk, dv = self.attention_backward(q, k, latent_cache, d_out, seq_lens, query_offsets, block_tables,
+                                             page_size, scale, causal, window, nthreads)
+        return dq[..., :r], dq[..., r:], dk[..., :r] + dv, dk[..., r:]
+
     # -- MLA absorbed-latent attention ------------------------------------------------------
     def mla(self, q_latent, q_rope, latent_cache, rope_cache, seq_lens, query_offsets,
             block_tables, page_size, scale, causal=True, window=0, key_begin=None, key_end=None,

@@ -30,6 +30,7 @@ STATUS = ["PA_OK", "PA_ERR_INVALID_ARGUMENT", "PA_ERR_SHAPE", "PA_ERR_DTYPE", "P
 # every entry point include/pa.h declares
 SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_prepare", "pa_forward",
            "pa_forward_ex", "pa_forward_static_workspace", "pa_mla_forward", "pa_mla_forward_ex", "pa_append", "pa_backward",
+           "pa_mla_backward",
            "pa_plan_device_status", "pa_sparse_select", "pa_sparse_forward", "pa_sparse_forward_ex",
            "pa_status_string", "pa_last_error_message", "pa_version"]
 PA_SPARSE_MAX_BLOCKS = 16384
@@ -97,6 +98,9 @@ def load_library(path: Optional[str] = None):
     lib.pa_backward.restype = ctypes.c_int
     lib.pa_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I, _I, _I, _I, ctypes.c_float, ctypes.c_int,
                                 _I, _P, _P, _P, _P]
+    lib.pa_mla_backward.restype = ctypes.c_int
+    lib.pa_mla_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int, _I, _I, _I, ctypes.c_float,
+                                    ctypes.c_int, _I, _P, _P, _P, _P, _P]
     lib.pa_plan_device_status.restype = ctypes.c_int
     lib.pa_plan_device_status.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
     lib.pa_sparse_select.restype = ctypes.c_int
@@ -302,6 +306,25 @@ def pa_append(plan: Plan, new_k: torch.Tensor, new_v: torch.Tensor, k_cache: tor
     _check(load_library().pa_append(plan.handle, _ptr(new_k), _ptr(new_v), _ptr(k_cache), _ptr(v_cache),
                                     _DTYPES[new_k.dtype], k_cache.shape[2], k_cache.shape[3], v_cache.shape[3],
                                     _stream_ptr(stream, plan.device)))
+
+
+def pa_mla_backward(plan: Plan, q_latent: torch.Tensor, q_rope: torch.Tensor, latent_cache: torch.Tensor,
+                    rope_cache: torch.Tensor, out: torch.Tensor, lse: torch.Tensor, d_out: torch.Tensor,
+                    d_q_latent: torch.Tensor, d_q_rope: torch.Tensor, d_latent_cache: torch.Tensor,
+                    d_rope_cache: torch.Tensor, scale: float, causal: bool = True, window: int = 0,
+                    stream=None) -> None:
+    """Gradients of pa_mla_forward: d_q_latent / d_q_rope written, d_latent_cache / d_rope_cache
+    (float32) accumulated."""
+    ts = (q_latent, q_rope, latent_cache, rope_cache, out, lse, d_out, d_q_latent, d_q_rope, d_latent_cache,
+          d_rope_cache)
+    for t in ts:
+        if not t.is_contiguous():
+            raise ValueError("pa_mla_backward takes contiguous tensors")
+    _check(load_library().pa_mla_backward(
+        plan.handle, _ptr(q_latent), _ptr(q_rope), _ptr(latent_cache), _ptr(rope_cache), _ptr(out), _ptr(lse),
+        _ptr(d_out), _DTYPES[q_latent.dtype], q_latent.shape[1], q_latent.shape[2], q_rope.shape[2], float(scale),
+        int(bool(causal)), int(window), _ptr(d_q_latent), _ptr(d_q_rope), _ptr(d_latent_cache), _ptr(d_rope_cache),
+        _stream_ptr(stream, plan.device)))
 
 
 def pa_backward(plan: Plan, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, out: torch.Tensor,

@@ -1177,6 +1177,61 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
     return ok();
 }
 
+pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rope, const void* latent_cache,
+                          const void* rope_cache, const void* out, const float* lse, const void* d_out, pa_dtype dtype,
+                          int32_t num_heads, int32_t latent_dim, int32_t rope_dim, float scale, int causal,
+                          int32_t window, float* d_q_latent, float* d_q_rope, float* d_latent_cache, float* d_rope_cache,
+                          pa_stream stream) {
+    if (!plan) return fail(PA_ERR_INVALID_ARGUMENT, "plan is NULL");
+    if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16) return fail(PA_ERR_DTYPE, "unknown dtype %d", (int)dtype);
+    if (num_heads <= 0) return fail(PA_ERR_SHAPE, "num_heads must be positive");
+    if (latent_dim <= 0 || latent_dim > 1024) return fail(PA_ERR_UNSUPPORTED, "latent_dim must be in [1, 1024]");
+    if (rope_dim <= 0 || rope_dim > 256) return fail(PA_ERR_UNSUPPORTED, "rope_dim must be in [1, 256]");
+    if (!std::isfinite(scale) || !(scale > 0.0f)) return fail(PA_ERR_INVALID_ARGUMENT, "scale must be finite and > 0");
+    if (causal != 0 && causal != 1) return fail(PA_ERR_INVALID_ARGUMENT, "causal must be 0 or 1");
+    if (window < 0) return fail(PA_ERR_INVALID_ARGUMENT, "window must be >= 0");
+    const int64_t es = (int64_t)dtype_size(dtype);
+    const int64_t nq = plan->Nq, pages = plan->num_pages, ps = plan->page_size;
+    int64_t n_ql, n_qr, n_lat, n_rope, n_o, n_l, n_dql, n_dqr, n_dlat, n_drope;
+    if (!product({nq, num_heads, latent_dim, es}, &n_ql) || !product({nq, num_heads, rope_dim, es}, &n_qr) ||
+        !product({pages, ps, latent_dim, es}, &n_lat) || !product({pages, ps, rope_dim, es}, &n_rope) ||
+        !product({nq, num_heads, latent_dim, es}, &n_o) || !product({nq, num_heads, 4}, &n_l) ||
+        !product({nq, num_heads, latent_dim, 4}, &n_dql) || !product({nq, num_heads, rope_dim, 4}, &n_dqr) ||
+        !product({pages, ps, latent_dim, 4}, &n_dlat) || !product({pages, ps, rope_dim, 4}, &n_drope))
+        return fail(PA_ERR_BOUNDS, "tensor size overflows 64-bit byte counts");
+    if (nq == 0) return ok();
+    if (!q_latent || !q_rope || !latent_cache || !rope_cache || !out || !lse || !d_out || !d_q_latent || !d_q_rope ||
+        !d_latent_cache || !d_rope_cache)
+        return fail(PA_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    for (const void* ptr : {q_latent, q_rope, latent_cache, rope_cache, out, (const void*)lse, d_out,
+                            (const void*)d_q_latent, (const void*)d_q_rope, (const void*)d_latent_cache,
+                            (const void*)d_rope_cache})
+        if ((uintptr_t)ptr % 16 != 0) return fail(PA_ERR_INVALID_ARGUMENT, "device pointers must be 16-byte aligned");
+    auto R = [](const void* p, int64_t n) { return Range{(uintptr_t)p, (uintptr_t)p + (uintptr_t)n}; };
+    const Range outs[4] = {R(d_q_latent, n_dql), R(d_q_rope, n_dqr), R(d_latent_cache, n_dlat), R(d_rope_cache, n_drope)};
+    const Range ins[7] = {R(q_latent, n_ql), R(q_rope, n_qr), R(latent_cache, n_lat), R(rope_cache, n_rope),
+                          R(out, n_o), R(lse, n_l), R(d_out, n_o)};
+    for (int a = 0; a < 4; ++a) {
+        for (int b = a + 1; b < 4; ++b)
+            if (overlap(outs[a], outs[b])) return fail(PA_ERR_ALIAS, "gradient outputs overlap");
+        for (const Range& r : ins)
+            if (overlap(outs[a], r)) return fail(PA_ERR_ALIAS, "a gradient output overlaps an input");
+    }
+    if (plan->device < 0) return fail(PA_ERR_INVALID_ARGUMENT, "host-only plan: no device to run on");
+    int cur = -1;
+    PA_CUDA_TRY(cudaGetDevice(&cur));
+    if (cur != plan->device)
+        return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
+    cudaError_t e = pa::launch_mla_backward(q_latent, q_rope, latent_cache, rope_cache, out, lse, d_out, d_q_latent,
+                                            d_q_rope, d_latent_cache, d_rope_cache, plan->d_seqs, plan->d_q2seq,
+                                            plan->d_bt, plan->table_width, plan->page_size, num_heads, latent_dim,
+                                            rope_dim, scale, causal, window, nq * num_heads, dtype, (cudaStream_t)stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "MLA backward kernel launch failed: %s", cudaGetErrorString(e));
+    plan->last_stream = (cudaStream_t)stream;
+    plan->last_launches = 1;
+    return ok();
+}
+
 pa_status pa_plan_device_status(const pa_plan* plan, int32_t* code) {
     if (!plan || !code) return fail(PA_ERR_INVALID_ARGUMENT, "plan or code is NULL");
     *code = 0;

@@ -111,6 +111,11 @@ cudaError_t launch_backward(const void* q, const void* k, const void* v, const v
                             const int32_t* block_tables, int32_t table_width, int32_t page_size, int32_t hq,
                             int32_t hkv, int32_t d, int32_t dv_dim, float scale, int causal, int32_t window,
                             int64_t rows, pa_dtype dt, cudaStream_t st);
+cudaError_t launch_mla_backward(const void* ql, const void* qr, const void* lat, const void* rope, const void* out,
+                                const float* lse, const void* dout, float* dql, float* dqr, float* dlat, float* drope,
+                                const SeqInfo* seqs, const int32_t* q2seq, const int32_t* block_tables,
+                                int32_t table_width, int32_t page_size, int32_t h, int32_t r, int32_t pr, float scale,
+                                int causal, int32_t window, int64_t rows, pa_dtype dt, cudaStream_t st);
 cudaError_t launch_append(const void* new_k, const void* new_v, void* k_cache, void* v_cache, const SeqInfo* seqs,
                           const int32_t* q2seq, const int32_t* block_tables, int32_t table_width, int32_t page_size,
                           int32_t hkv, int32_t k_row_bytes, int32_t v_row_bytes, int64_t rows, cudaStream_t st);

@@ -321,6 +321,22 @@ def backward_flops(wl) -> int:
     return visible_pairs(wl) * wl.num_q_heads * 2 * (3 * wl.head_dim + 2 * wl.v_head_dim)
 
 
+def mla_backward_small(seed: int = 0, batch: int = 4, lmin: int = 256, lmax: int = 1024):
+    """Backward of an MLA decode batch (128 heads, latent 512, rope 64, pages of 64, bf16), small
+    enough for the CUDA-core kernel: (workload, d_out [Nq, H, R])."""
+    lens = _uniform_ints(seed, 0xB5, batch, lmin, lmax)
+    wl = make_mla(f"bf16_mla_backward_b{batch}", seed, lens, [1] * batch, 128, 512, 64, 64, torch.bfloat16)
+    d_out = randn((wl.sched.num_queries, 128, 512), seed, 24, torch.bfloat16)
+    return wl, d_out
+
+
+def mla_backward_flops(wl) -> int:
+    """2 flops per multiply-add over visible pairs, every head: scores (R + Pr), dP (R), dV (R),
+    dQ (R + Pr) and dK (R + Pr)."""
+    k = wl.latent_dim + wl.rope_dim
+    return visible_pairs(wl) * wl.num_heads * 2 * (3 * k + 2 * wl.latent_dim)
+
+
 def sparse_bf16_decode(seed: int = 0, block_size: int = 64, topk: int = 16, pin: bool = False):
     """The bf16 decode batch (64 sequences, context U[512, 8192], Hq=32, Hkv=8, D=128, page 16)
     with sparse top-K attention over blocks of `block_size` keys: (workload, block_size, topk).

@@ -401,6 +401,40 @@ def pin_backward_finite_differences(orc):
         assert abs(fd - an) <= 1e-4 * max(1.0, abs(an)), (name, idx, fd, an)
 
 
+def pin_mla_backward_finite_differences(orc):
+    """Central differences of L = sum(out * dO) (MLA forward oracle) at entries of q_latent, q_rope,
+    the latent cache (a key and a value at once) and the rope cache."""
+    wl = W.make_mla("fdm", 35, [9, 6], [3, 2], 3, 8, 4, 4, torch.float32, causal=True, window=5)
+    s_ = wl.sched
+    g = torch.Generator().manual_seed(14)
+    dout = torch.randn(wl.q_latent.shape[0], 3, 8, generator=g).to(torch.float32)
+    dql, dqr, dlat, drope = orc.mla_backward(wl.q_latent, wl.q_rope, wl.latent_cache, wl.rope_cache, dout,
+                                             s_.seq_lens, s_.query_offsets, s_.block_tables, 4, wl.scale, True, 5)
+    names = ("ql", "qr", "lat", "rope")
+    base = {"ql": wl.q_latent, "qr": wl.q_rope, "lat": wl.latent_cache, "rope": wl.rope_cache}
+
+    def loss(a):
+        out, _ = orc.mla(a["ql"], a["qr"], a["lat"], a["rope"], s_.seq_lens, s_.query_offsets, s_.block_tables, 4,
+                         wl.scale, True, 5)
+        return float((out * dout.double()).sum())
+
+    probes = [("ql", (1, 2, 3)), ("ql", (4, 0, 7)), ("qr", (0, 1, 2)), ("qr", (3, 2, 0)),
+              ("lat", (int(s_.block_tables[0, 1]), 1, 0, 5)), ("lat", (int(s_.block_tables[1, 0]), 2, 0, 0)),
+              ("rope", (int(s_.block_tables[0, 0]), 3, 0, 1)), ("rope", (int(s_.block_tables[1, 1]), 0, 0, 3))]
+    grads = {"ql": dql, "qr": dqr, "lat": dlat, "rope": drope}
+    for name, idx in probes:
+        plus, minus = base[name].clone(), base[name].clone()
+        plus[idx] += 1e-2
+        minus[idx] -= 1e-2
+        h2 = float(plus[idx]) - float(minus[idx])
+        ap = dict(base); ap[name] = plus
+        am = dict(base); am[name] = minus
+        fd = (loss(ap) - loss(am)) / h2
+        an = float(grads[name][idx])
+        assert abs(fd - an) <= 1e-4 * max(1.0, abs(an)), (name, idx, fd, an)
+    assert names  # every input has at least one probe
+
+
 # ---- sparse top-K block selection (alice-llm `llama3_sparse_attention`) -------------------------
 
 def _sparse_cases():
@@ -573,6 +607,7 @@ ALL_PINS = [
     pin_page_permutation_invariance, pin_split_equals_unsplit, pin_chunked_equals_oneshot,
     pin_window_cases, pin_gqa_equals_mha_repeated, pin_mla_equals_gqa_concat,
     pin_half_precision_widening, pin_backward_vs_autograd, pin_backward_finite_differences,
+    pin_mla_backward_finite_differences,
     pin_sparse_bruteforce, pin_sparse_dense_fallback, pin_sparse_planted_block, pin_sparse_ties_lower_index,
     pin_sparse_alice_fixture,
 ]

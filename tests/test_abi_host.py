@@ -232,3 +232,40 @@ def test_sparse_validation(lib):
     assert pa.STATUS[st] == "PA_ERR_UNSUPPORTED"
     assert pa.STATUS[lib.pa_sparse_select(big.handle, q, k, 1, 4, 2, 64, ctypes.c_float(0.1), 1, 0, 32, 4, sel, 4,
                                           None, 0, None)] == "PA_ERR_INVALID_ARGUMENT"  # blocks of 32: fits
+
+
+def test_mla_backward_validation(lib):
+    """pa_mla_backward checks shapes, scalars, pointers and aliasing before the device: a host-only
+    plan gets past every check only to be refused for having no device."""
+    wl, plan = host_plan()
+    base = 1 << 36
+    ptr = [base + (i << 32) for i in range(11)]  # disjoint, 16-byte aligned fake ranges
+    f = ctypes.c_float
+
+    def call(r=512, pr=64, h=4, scale=0.1, causal=1, window=0, dt=1, p=None):
+        a = list(ptr if p is None else p)
+        st = lib.pa_mla_backward(plan.handle, a[0], a[1], a[2], a[3], a[4], a[5], a[6], dt, h, r, pr, f(scale), causal,
+                                 window, a[7], a[8], a[9], a[10], None)
+        return pa.STATUS[st]
+    assert call() == "PA_ERR_INVALID_ARGUMENT"  # host-only plan: every check passed
+    assert call(dt=7) == "PA_ERR_DTYPE"
+    assert call(h=0) == "PA_ERR_SHAPE"
+    assert call(r=2000) == "PA_ERR_UNSUPPORTED"
+    assert call(pr=0) == "PA_ERR_UNSUPPORTED"
+    assert call(pr=300) == "PA_ERR_UNSUPPORTED"
+    assert call(scale=float("nan")) == "PA_ERR_INVALID_ARGUMENT"
+    assert call(causal=2) == "PA_ERR_INVALID_ARGUMENT"
+    assert call(window=-1) == "PA_ERR_INVALID_ARGUMENT"
+    aliased = list(ptr)
+    aliased[9] = aliased[7]  # d_latent_cache on top of d_q_latent
+    assert call(p=aliased) == "PA_ERR_ALIAS"
+    over_input = list(ptr)
+    over_input[10] = over_input[2]  # d_rope_cache on the latent cache
+    assert call(p=over_input) == "PA_ERR_ALIAS"
+    misaligned = list(ptr)
+    misaligned[8] += 4
+    assert call(p=misaligned) == "PA_ERR_INVALID_ARGUMENT"
+    null = list(ptr)
+    null[6] = 0
+    assert call(p=null) == "PA_ERR_INVALID_ARGUMENT"
+    plan.close()

@@ -138,3 +138,40 @@ def test_backward_tensor_core_deterministic():
     runs = [run_backward(wl, torch.Generator().manual_seed(13)) for _ in range(2)]
     for a, b in zip(runs[0][1:], runs[1][1:]):
         assert torch.equal(torch.nan_to_num(a, nan=0.0), torch.nan_to_num(b, nan=0.0))
+
+
+@pytest.mark.parametrize("h,r,pr,ps,dtype,causal,window", [
+    (8, 64, 16, 16, torch.float32, True, 0),
+    (16, 512, 64, 64, torch.bfloat16, True, 0),
+    (4, 96, 32, 32, torch.float16, True, 40),
+    (8, 128, 64, 16, torch.bfloat16, False, 0),
+])
+def test_mla_backward_matches_oracle(orc, h, r, pr, ps, dtype, causal, window):
+    """pa_mla_backward against the oracle (the GQA backward on the key [latent | rope] with the latent
+    as value, the latent's key and value gradients summed), decode and chunked rows, ragged pages."""
+    wl = W.make_mla("mla_bwd", 9, [70, 200, 9, 130], [1, 40, 9, 3], h, r, pr, ps, dtype, causal=causal,
+                    window=window)
+    s = wl.sched
+    g = torch.Generator().manual_seed(15)
+    nq = s.num_queries
+    dout = torch.randn(nq, h, r, generator=g).to(dtype)
+    ql, qr = wl.q_latent.cuda(), wl.q_rope.cuda()
+    lat, rope = wl.latent_cache.cuda(), wl.rope_cache.cuda()
+    plan = pa.plan_for(wl)
+    out = torch.empty(nq, h, r, dtype=dtype, device="cuda")
+    lse = torch.empty(nq, h, dtype=torch.float32, device="cuda")
+    pa.pa_mla_forward(plan, ql, qr, lat, rope, out, lse, wl.scale, causal, window)
+    dql = torch.full((nq, h, r), float("nan"), dtype=torch.float32, device="cuda")
+    dqr = torch.full((nq, h, pr), float("nan"), dtype=torch.float32, device="cuda")
+    dlat = torch.zeros(lat.shape, dtype=torch.float32, device="cuda")
+    drope = torch.zeros(rope.shape, dtype=torch.float32, device="cuda")
+    pa.pa_mla_backward(plan, ql, qr, lat, rope, out, lse, dout.cuda(), dql, dqr, dlat, drope, wl.scale, causal,
+                       window)
+    torch.cuda.synchronize()
+    assert pa.pa_plan_device_status(plan) == 0
+    plan.close()
+    ref = orc.mla_backward(wl.q_latent, wl.q_rope, wl.latent_cache, wl.rope_cache, dout, s.seq_lens,
+                           s.query_offsets, s.block_tables, ps, wl.scale, causal, window)
+    tag = f"mla h{h} r{r} pr{pr} {dtype}"
+    for got, want, name in zip((dql, dqr, dlat, drope), ref, ("dq_latent", "dq_rope", "d_latent", "d_rope")):
+        close(got.cpu(), want, dtype, f"{name} {tag}")
