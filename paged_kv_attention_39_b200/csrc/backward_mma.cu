@@ -123,11 +123,27 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(const BwdParam
         for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
     const int kw = warp * 16;  // this warp's first key row in the tile
 
+    // lse and Drow of this thread's four rows (two per n-tile) of a block; the next block's are
+    // loaded while the current one computes
+    float lse_n[2][2], dr_n[2][2];
+    auto row_stats = [&](int rb) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int64_t R = (int64_t)rb * kRowBlock + nt * 8 + 2 * tq + c;
+                const bool in = R >= R_lo && R < R_hi;
+                const int64_t qr = in ? qrow_of(R) : 0;
+                lse_n[nt][c] = in ? p.lse[qr] : neg_inf();
+                dr_n[nt][c] = in ? p.drow[qr] : 0.f;
+            }
+    };
+    row_stats(rb0);
     for (int rb = rb0; rb < rb1; ++rb) {
         const int st = (rb - rb0) & 1;
         if (rb + 1 < rb1) load_rows(rb + 1, st ^ 1);
         cp_async_commit();
-        // this thread's four rows (two per n-tile): lse in base 2, Drow, position, liveness
+        // this block's rows: lse in base 2, Drow, position, liveness (a row without keys has lse -inf)
         float lse2[2][2], dr[2][2];
         int64_t pos[2][2];
         bool live[2][2];
@@ -136,14 +152,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(const BwdParam
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 const int64_t R = (int64_t)rb * kRowBlock + nt * 8 + 2 * tq + c;
-                live[nt][c] = R >= R_lo && R < R_hi;
-                const int64_t qr = live[nt][c] ? qrow_of(R) : 0;
-                const float l = live[nt][c] ? p.lse[qr] : 0.f;
-                live[nt][c] = live[nt][c] && l != neg_inf();
-                lse2[nt][c] = l * kLog2e;
-                dr[nt][c] = live[nt][c] ? p.drow[qr] : 0.f;
+                live[nt][c] = lse_n[nt][c] != neg_inf();
+                lse2[nt][c] = live[nt][c] ? lse_n[nt][c] * kLog2e : 0.f;
+                dr[nt][c] = dr_n[nt][c];
                 pos[nt][c] = base_pos + (live[nt][c] ? R / G : 0);
             }
+        if (rb + 1 < rb1) row_stats(rb + 1);
         cp_async_wait<1>();
         __syncthreads();
         const T* q_s = sQ + st * kRowBlock * D;
