@@ -42,3 +42,43 @@ def test_pins_reject_mutant(mutant, tmp_path):
         except AssertionError:
             failed.append(pin.__name__)
     assert failed, f"no pin caught {mutant}"
+
+
+# The MLA backward is composed in the oracle's Python front end (the GQA backward on the key
+# [latent | rope], value latent); its plausible mistakes are planted there, on the CPU.
+def _mla_bwd_drop_value_term(orc):
+    """The latent's gradient keeps only its key part (the value part P dO is dropped)."""
+    import torch
+
+    def bad(q_latent, q_rope, latent_cache, rope_cache, d_out, seq_lens, query_offsets, block_tables, page_size,
+            scale, causal=True, window=0, nthreads=None):
+        r = q_latent.shape[2]
+        dq, dk, _ = orc.attention_backward(torch.cat([q_latent, q_rope], 2), torch.cat([latent_cache, rope_cache], 3),
+                                           latent_cache, d_out, seq_lens, query_offsets, block_tables, page_size,
+                                           scale, causal, window, nthreads)
+        return dq[..., :r], dq[..., r:], dk[..., :r], dk[..., r:]
+    return bad
+
+
+def _mla_bwd_swapped_rope(orc):
+    """The rope gradient is taken from the latent columns (a wrong column split)."""
+    real = orc.mla_backward
+
+    def bad(*a, **k):
+        dql, dqr, dlat, drope = real(*a, **k)
+        pr = drope.shape[-1]
+        return dql, dql[..., :pr].clone(), dlat, dlat[..., :pr].clone()
+    return bad
+
+
+@pytest.mark.parametrize("plant", [_mla_bwd_drop_value_term, _mla_bwd_swapped_rope])
+def test_pins_reject_mla_backward_mistakes(plant):
+    orc = oracle.get()
+    bad = oracle.Oracle(orc.path) if hasattr(orc, "path") else orc
+    original = bad.mla_backward
+    bad.mla_backward = plant(bad)
+    try:
+        with pytest.raises(AssertionError):
+            oracle_pins.pin_mla_backward_finite_differences(bad)
+    finally:
+        bad.mla_backward = original
