@@ -12,7 +12,8 @@
 //   warp 4      TMA producer: Q (two boxes: 128 heads x all 8 latent column blocks, and the rope
 //               part), then per step the latent rows of 32 keys (one box with all 8 column
 //               blocks when a page holds the whole step) and the rope rows into a 2-stage ring,
-//               with an L2 prefetch a few steps ahead
+//               with an L2 prefetch a few steps ahead (one box per two steps when a page holds
+//               both)
 //   warps 5..8  S = Q K^T, nine of the 36 k-steps each into a partial score buffer (warp 5 also
 //               owns TMEM)
 //   warp 9      O_half += P V_half (2 k-steps); zeroes latent rows past the sequence's last key
@@ -78,7 +79,8 @@ template <typename T>
 __global__ void __launch_bounds__(kMlaThreads, 1)
     mla_tc_kernel(const __grid_constant__ CUtensorMap tm_ql, const __grid_constant__ CUtensorMap tm_qr,
                   const __grid_constant__ CUtensorMap tm_lat, const __grid_constant__ CUtensorMap tm_latw,
-                  const __grid_constant__ CUtensorMap tm_rope, const AttnParams p) {
+                  const __grid_constant__ CUtensorMap tm_rope, const __grid_constant__ CUtensorMap tm_latw2,
+                  const __grid_constant__ CUtensorMap tm_rope2, const AttnParams p) {
     using L_ = MlaSmem;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t IDESC_QK = idesc_f16(MBM, MBN, kBf16, false, false);
@@ -159,8 +161,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     my_row = key < si.L ? (int)((int64_t)bt[key / ps] * ps + key % ps) : 0;
                 }
                 // Warm L2 with the tile kPrefetchTiles ahead: with only two stages, a load issued
-                // when a stage frees up would otherwise pay the full HBM latency.
-                if (i + kPrefetchTiles < n_tiles) {
+                // when a stage frees up would otherwise pay the full HBM latency. Every TMA box
+                // costs the copy engine a fixed time, so when a page holds two whole tiles one box
+                // of 64 rows prefetches both (issued for the tile that starts the pair).
+                const bool pair_pf = bpt == 1 && ps % (2 * box) == 0;
+                if (pair_pf) {
+                    // one box of two tiles, issued for the tile that starts a page pair
+                    const int tp = i + kPrefetchTiles;
+                    if (tp < n_tiles && ((kt_start / box + tp) & 1) == 0) {
+                        const int prow = __shfl_sync(0xffffffffu, my_row, g0 + kPrefetchTiles - base_g);
+                        if (lane == 0) {
+                            tma_prefetch_l2_3d(&tm_latw2, 0, prow, 0);
+                            tma_prefetch_l2_3d(&tm_rope2, 0, 0, prow);
+                        }
+                    }
+                } else if (i + kPrefetchTiles < n_tiles) {
                     const int gp = g0 + kPrefetchTiles * bpt;
                     const int64_t ktp = kt0 + (int64_t)kPrefetchTiles * MBN;
                     for (int b = 0; b < bpt; ++b) {
@@ -471,7 +486,7 @@ cudaError_t mla_launch_t(const AttnParams& p, cudaStream_t st) {
     const int ps = p.page_size;
     const int box = ps < MBN ? ps : MBN;
     const uint64_t rows = (uint64_t)p.num_pages * ps;
-    CUtensorMap tql, tqr, tlat, tlatw, trope;
+    CUtensorMap tql, tqr, tlat, tlatw, trope, tlatw2, trope2;
     // Absorbed Q [Nq][H][R] seen as {64 elements, head, 64-column block, query}: one box brings the
     // 8 column blocks of 128 heads, laid out [block][head][64 elements] as the MMA reads them.
     const cuuint64_t qdims[4] = {64, (cuuint64_t)p.hq, MR / 64, (cuuint64_t)p.num_queries};
@@ -482,10 +497,12 @@ cudaError_t mla_launch_t(const AttnParams& p, cudaStream_t st) {
     const cuuint64_t ldims[3] = {64, rows, MR / 64};
     const cuuint64_t lstr[2] = {MR * 2, 128};
     const cuuint32_t lbox[3] = {64, (cuuint32_t)box, MR / 64};
+    const cuuint32_t lbox2[3] = {64, (cuuint32_t)(2 * box), MR / 64};
     if (!mla_encode(&tql, bf16, p.q, 4, qdims, qstr, qbox) ||
         !mla_map(&tqr, bf16, p.qr, MP, p.hq, (uint64_t)p.num_queries, MBM, 1) ||
         !mla_map(&tlat, bf16, p.k, MR, 1, rows, 1, box) || !mla_encode(&tlatw, bf16, p.k, 3, ldims, lstr, lbox) ||
-        !mla_map(&trope, bf16, p.kr, MP, 1, rows, 1, box))
+        !mla_map(&trope, bf16, p.kr, MP, 1, rows, 1, box) || !mla_encode(&tlatw2, bf16, p.k, 3, ldims, lstr, lbox2) ||
+        !mla_map(&trope2, bf16, p.kr, MP, 1, rows, 1, 2 * box))
         return cudaErrorInvalidValue;
     auto kern = mla_tc_kernel<T>;
     static unsigned long long configured = 0;
@@ -497,7 +514,7 @@ cudaError_t mla_launch_t(const AttnParams& p, cudaStream_t st) {
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<2 * p.num_units, kMlaThreads, MlaSmem::ALLOC, st>>>(tql, tqr, tlat, tlatw, trope, p);
+    kern<<<2 * p.num_units, kMlaThreads, MlaSmem::ALLOC, st>>>(tql, tqr, tlat, tlatw, trope, tlatw2, trope2, p);
     return cudaGetLastError();
 }
 
