@@ -1055,6 +1055,58 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
     return ok();
 }
 
+// Work lists of the tensor-core backward for one (group size, causal, window), longest first:
+// the 64-key tiles of every sequence that some query sees (cost: the rows that see them) for the
+// dK/dV kernel, and blocks of at most 16 rows (cost: the keys they see) for the dQ kernel. One
+// upload; the host blob stays with the plan.
+static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int32_t window, cudaStream_t st) {
+    const int KT = pa::backward_key_tile(), qpb = std::max(1, pa::backward_row_block() / G);
+    std::vector<std::pair<int64_t, pa::BwdKeyUnit>> ku;
+    std::vector<std::pair<int64_t, pa::BwdRowUnit>> ru;
+    for (int32_t si = 0; si < plan->S; ++si) {
+        const pa::SeqInfo& q_ = plan->seqs[si];
+        if (q_.n == 0) continue;
+        const int64_t base = (int64_t)q_.L - q_.n;  // position of query 0
+        for (int64_t k0 = 0; k0 < q_.L; k0 += KT) {
+            const int64_t kmax = std::min<int64_t>(k0 + KT, q_.L);
+            const int64_t jlo = causal ? std::max<int64_t>(0, k0 - base) : 0;
+            const int64_t jhi = window > 0 ? std::min<int64_t>(q_.n, kmax - 1 + window - base) : q_.n;
+            if (jhi <= jlo) continue;
+            ku.push_back({jhi - jlo, pa::BwdKeyUnit{si, (int32_t)k0}});
+        }
+        for (int32_t j0 = 0; j0 < q_.n; j0 += qpb) {
+            const int32_t j1 = std::min(q_.n, j0 + qpb);
+            int32_t lo = 0, hi = 0;
+            visible_union(q_.L, q_.n, j0, j1, causal != 0, window, &lo, &hi);
+            ru.push_back({(int64_t)hi - lo, pa::BwdRowUnit{si, j0, j1, 0}});
+        }
+    }
+    auto longer = [](const auto& a, const auto& b) { return a.first > b.first; };
+    std::stable_sort(ku.begin(), ku.end(), longer);
+    std::stable_sort(ru.begin(), ru.end(), longer);
+    const size_t row_off = (ku.size() * sizeof(pa::BwdKeyUnit) + 255) & ~size_t(255);
+    std::vector<char> blob(std::max<size_t>(16, row_off + ru.size() * sizeof(pa::BwdRowUnit)));
+    for (size_t i = 0; i < ku.size(); ++i)
+        std::memcpy(blob.data() + i * sizeof(pa::BwdKeyUnit), &ku[i].second, sizeof(pa::BwdKeyUnit));
+    for (size_t i = 0; i < ru.size(); ++i)
+        std::memcpy(blob.data() + row_off + i * sizeof(pa::BwdRowUnit), &ru[i].second, sizeof(pa::BwdRowUnit));
+    if (plan->bwd_dev) {
+        PA_CUDA_TRY(cudaFreeAsync(plan->bwd_dev, st));
+        plan->bwd_dev = nullptr;
+    }
+    PA_CUDA_TRY(lib_malloc(&plan->bwd_dev, blob.size(), st));
+    PA_CUDA_TRY(upload(plan->bwd_dev, blob.data(), blob.size(), st));
+    plan->bwd_host.push_back(std::move(blob));
+    plan->bwd_group = G;
+    plan->bwd_causal = causal;
+    plan->bwd_window = window;
+    plan->bwd_nkey = (int32_t)ku.size();
+    plan->bwd_nrow = (int32_t)ru.size();
+    plan->bwd_row_off = row_off;
+    plan->uploaded_bytes += (int64_t)plan->bwd_host.back().size();
+    return PA_OK;
+}
+
 pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache, const void* out,
                       const float* lse, const void* d_out, pa_dtype dtype, int32_t num_q_heads, int32_t num_kv_heads,
                       int32_t head_dim, int32_t v_head_dim, float scale, int causal, int32_t window, float* d_q,
@@ -1103,51 +1155,8 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
     if (pa::backward_mma_supported(dtype, head_dim, v_head_dim, G)) {
         std::lock_guard<std::mutex> lock(plan->mu);
         if (plan->bwd_group != G || plan->bwd_causal != causal || plan->bwd_window != window) {
-            // Work lists, longest first: 64-key tiles of every sequence (cost: the rows that see
-            // them) for dK/dV, and blocks of at most 16 rows (cost: the keys they see) for dQ.
-            const int KT = pa::backward_key_tile(), qpb = std::max(1, pa::backward_row_block() / G);
-            std::vector<std::pair<int64_t, pa::BwdKeyUnit>> ku;
-            std::vector<std::pair<int64_t, pa::BwdRowUnit>> ru;
-            for (int32_t si = 0; si < plan->S; ++si) {
-                const pa::SeqInfo& q_ = plan->seqs[si];
-                if (q_.n == 0) continue;
-                const int64_t base = (int64_t)q_.L - q_.n;
-                for (int64_t k0 = 0; k0 < q_.L; k0 += KT) {
-                    const int64_t kmax = std::min<int64_t>(k0 + KT, q_.L);
-                    const int64_t jlo = causal ? std::max<int64_t>(0, k0 - base) : 0;
-                    const int64_t jhi = window > 0 ? std::min<int64_t>(q_.n, kmax - 1 + window - base) : q_.n;
-                    if (jhi <= jlo) continue;
-                    ku.push_back({jhi - jlo, pa::BwdKeyUnit{si, (int32_t)k0}});
-                }
-                for (int32_t j0 = 0; j0 < q_.n; j0 += qpb) {
-                    const int32_t j1 = std::min(q_.n, j0 + qpb);
-                    int32_t lo = 0, hi = 0;
-                    visible_union(q_.L, q_.n, j0, j1, causal != 0, window, &lo, &hi);
-                    ru.push_back({(int64_t)hi - lo, pa::BwdRowUnit{si, j0, j1, 0}});
-                }
-            }
-            auto longer = [](const auto& a, const auto& b) { return a.first > b.first; };
-            std::stable_sort(ku.begin(), ku.end(), longer);
-            std::stable_sort(ru.begin(), ru.end(), longer);
-            const size_t row_off = (ku.size() * sizeof(pa::BwdKeyUnit) + 255) & ~size_t(255);
-            std::vector<char> blob(std::max<size_t>(16, row_off + ru.size() * sizeof(pa::BwdRowUnit)));
-            for (size_t i = 0; i < ku.size(); ++i) std::memcpy(blob.data() + i * sizeof(pa::BwdKeyUnit), &ku[i].second, sizeof(pa::BwdKeyUnit));
-            for (size_t i = 0; i < ru.size(); ++i)
-                std::memcpy(blob.data() + row_off + i * sizeof(pa::BwdRowUnit), &ru[i].second, sizeof(pa::BwdRowUnit));
-            if (plan->bwd_dev) {
-                PA_CUDA_TRY(cudaFreeAsync(plan->bwd_dev, st));
-                plan->bwd_dev = nullptr;
-            }
-            PA_CUDA_TRY(lib_malloc(&plan->bwd_dev, blob.size(), st));
-            PA_CUDA_TRY(upload(plan->bwd_dev, blob.data(), blob.size(), st));
-            plan->bwd_host.push_back(std::move(blob));
-            plan->bwd_group = G;
-            plan->bwd_causal = causal;
-            plan->bwd_window = window;
-            plan->bwd_nkey = (int32_t)ku.size();
-            plan->bwd_nrow = (int32_t)ru.size();
-            plan->bwd_row_off = row_off;
-            plan->uploaded_bytes += (int64_t)plan->bwd_host.back().size();
+            pa_status bs = build_backward_lists(plan, G, causal, window, st);
+            if (bs != PA_OK) return bs;
         }
         pa_status gs = grow_buffer(&plan->bwd_drow, &plan->bwd_drow_bytes, (size_t)nq * num_q_heads * sizeof(float), st);
         if (gs != PA_OK) return gs;
