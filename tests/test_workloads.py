@@ -51,3 +51,25 @@ def test_algorithmic_counts():
     # seq 0: one query at p=9 sees keys 7..9; seq 1: queries at 16..19 see 14..19
     assert W.algorithmic_kv_bytes(wl) == (3 + 6) * 2 * (8 + 8) * 2
     assert W.visible_pairs(wl) == 3 + 4 * 3
+
+
+def test_next_row_work_counts():
+    """The append, GQA backward and MLA backward numerators against per-pair brute force."""
+    wl = W.make_gqa("w", 5, [10, 6], [4, 6], 8, 2, 16, 8, 4, torch.bfloat16, causal=True, window=3)
+    s = wl.sched
+    pairs = 0
+    for i in range(s.num_seqs):
+        L, n = int(s.seq_lens[i]), int(s.query_offsets[i + 1] - s.query_offsets[i])
+        for j in range(n):
+            p = L - n + j
+            pairs += sum(1 for t in range(L) if t <= p and t + 3 > p)
+    assert W.backward_flops(wl) == pairs * 8 * 2 * (3 * 16 + 2 * 8)
+    assert W.append_bytes(wl) == 2 * s.num_queries * 2 * (16 + 8) * 2
+    ml = W.make_mla("m", 6, [9, 5], [2, 5], 4, 32, 8, 4, torch.float16, causal=False)
+    sm = ml.sched
+    mpairs = sum(int(sm.seq_lens[i]) * int(sm.query_offsets[i + 1] - sm.query_offsets[i]) for i in range(sm.num_seqs))
+    assert W.mla_backward_flops(ml) == mpairs * 4 * 2 * (3 * (32 + 8) + 2 * 32)
+    wb, d_out = W.backward_chunk(0, batch=2, hmax=64, chunk=16)
+    assert d_out.shape == (wb.sched.num_queries, 32, 128) and d_out.dtype == torch.bfloat16
+    wa, nk, nv = W.append_chunk(0)
+    assert nk.shape == (wa.sched.num_queries, 8, 128) and nv.shape == nk.shape
