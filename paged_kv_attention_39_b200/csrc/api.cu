@@ -1152,7 +1152,8 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
         return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
     const int32_t G = num_q_heads / num_kv_heads;
     cudaStream_t st = (cudaStream_t)stream;
-    if (pa::backward_mma_supported(dtype, head_dim, v_head_dim, G)) {
+    // the tensor-core kernels index a sequence's rows (queries x G) in 32 bits
+    if (pa::backward_mma_supported(dtype, head_dim, v_head_dim, G) && nq * (int64_t)G < ((int64_t)1 << 31)) {
         std::lock_guard<std::mutex> lock(plan->mu);
         if (plan->bwd_group != G || plan->bwd_causal != causal || plan->bwd_window != window) {
             pa_status bs = build_backward_lists(plan, G, causal, window, st);

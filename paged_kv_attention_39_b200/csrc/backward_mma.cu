@@ -101,7 +101,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(const BwdParam
     }
     const T* qg = static_cast<const T*>(p.q);
     const T* og = static_cast<const T*>(p.dout);
-    auto qrow_of = [&](int64_t R) { return (int64_t)(si.q_start + R / G) * p.hq + kvh * G + R % G; };
+    // rows of a sequence (queries x G) stay below 2^31 (the host checks), so row -> (query, head)
+    // is a 32-bit division
+    const uint32_t Gu = (uint32_t)G;
+    auto qrow_of = [&](int64_t R) {
+        const uint32_t r = (uint32_t)R, j = r / Gu;
+        return (int64_t)(si.q_start + (int64_t)j) * p.hq + kvh * G + (int)(r - j * Gu);
+    };
     auto load_rows = [&](int rb, int st) {
         for (int c = tid; c < 2 * kRowBlock * CH; c += kBwdWarps * 32) {
             const int which = c / (kRowBlock * CH), rc = c % (kRowBlock * CH);
@@ -155,8 +161,15 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(const BwdParam
                 live[nt][c] = lse_n[nt][c] != neg_inf();
                 lse2[nt][c] = live[nt][c] ? lse_n[nt][c] * kLog2e : 0.f;
                 dr[nt][c] = dr_n[nt][c];
-                pos[nt][c] = base_pos + (live[nt][c] ? R / G : 0);
+                pos[nt][c] = base_pos + (live[nt][c] ? (int64_t)((uint32_t)R / Gu) : 0);
             }
+        // every row of the block live and seeing every key of the tile: no per-element mask
+        const int64_t r_first = (int64_t)rb * kRowBlock, r_last = r_first + kRowBlock - 1;
+        const int64_t pmin = base_pos + (int64_t)((uint32_t)r_first / Gu);
+        const int64_t pmax = base_pos + (int64_t)((uint32_t)r_last / Gu);
+        const bool full = kmax == k0 + kKeyTile && r_first >= R_lo && r_last < R_hi && (!p.causal || kmax - 1 <= pmin) &&
+                          (p.window == 0 || k0 + p.window > pmax) &&
+                          __all_sync(0xffffffffu, live[0][0] && live[0][1] && live[1][0] && live[1][1]);
         if (rb + 1 < rb1) row_stats(rb + 1);
         cp_async_wait<1>();
         __syncthreads();
@@ -192,7 +205,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32) bwd_dkdv_kernel(const BwdParam
             for (int e = 0; e < 4; ++e) {
                 const int c = e & 1;
                 const int64_t t = k0 + kw + gq + 8 * (e >> 1);
-                const bool vis = live[nt][c] && t < kmax && key_visible(t, pos[nt][c], p.causal, p.window);
+                const bool vis =
+                    full || (live[nt][c] && t < kmax && key_visible(t, pos[nt][c], p.causal, p.window));
                 const float pr = vis ? fast_exp2(fmaf(s[nt][e], p.scale_log2, -lse2[nt][c])) : 0.f;
                 pv[e] = pr;
                 dsv[e] = pr * (dp[nt][e] - dr[nt][c]);
