@@ -1090,6 +1090,9 @@ static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int3
         std::memcpy(blob.data() + i * sizeof(pa::BwdKeyUnit), &ku[i].second, sizeof(pa::BwdKeyUnit));
     for (size_t i = 0; i < ru.size(); ++i)
         std::memcpy(blob.data() + row_off + i * sizeof(pa::BwdRowUnit), &ru[i].second, sizeof(pa::BwdRowUnit));
+    // the cached lists are invalid from here until the new ones are uploaded: a failure below
+    // leaves the plan to rebuild them on its next call
+    plan->bwd_group = 0;
     if (plan->bwd_dev) {
         PA_CUDA_TRY(cudaFreeAsync(plan->bwd_dev, st));
         plan->bwd_dev = nullptr;
