@@ -156,8 +156,9 @@ def test_binding_functions_compile_their_calls():
     """Every binding wrapper resolves the globals it loads (a typo would only show on a GPU)."""
     import builtins
     import dis
-    for name in ("pa_plan_prepare", "pa_forward", "pa_mla_forward", "pa_plan_create", "pa_plan_get_info",
-                 "plan_for", "trace_events"):
+    names = [n for n in dir(pa) if n.startswith("pa_") and callable(getattr(pa, n))] + ["plan_for", "trace_events"]
+    assert {"pa_backward", "pa_mla_backward", "pa_append", "pa_sparse_select", "pa_sparse_forward"} <= set(names)
+    for name in names:
         fn = getattr(pa, name)
         for ins in dis.get_instructions(fn):
             if ins.opname == "LOAD_GLOBAL":
@@ -268,4 +269,30 @@ def test_mla_backward_validation(lib):
     null = list(ptr)
     null[6] = 0
     assert call(p=null) == "PA_ERR_INVALID_ARGUMENT"
+    plan.close()
+
+
+def test_backward_wrappers_marshal_to_the_library():
+    """pa_backward / pa_mla_backward called through the Python binding with CPU tensors on a
+    host-only plan: every argument reaches the C entry point (a wrong argument list would raise in
+    ctypes), which passes its checks and refuses the plan for having no device."""
+    wl, plan = host_plan()
+    nq, hq, d = wl.q.shape
+    f32 = torch.float32
+    out = torch.zeros(nq, hq, d, dtype=wl.q.dtype)
+    lse = torch.zeros(nq, hq, dtype=f32)
+    with pytest.raises(pa.PaError) as ei:
+        pa.pa_backward(plan, wl.q, wl.k_cache, wl.v_cache, out, lse, out.clone(), torch.zeros(nq, hq, d, dtype=f32),
+                       torch.zeros(wl.k_cache.shape, dtype=f32), torch.zeros(wl.v_cache.shape, dtype=f32), 0.125)
+    assert pa.STATUS[ei.value.status] == "PA_ERR_INVALID_ARGUMENT" and "host-only" in str(ei.value)
+    h, r, pr = 4, 32, 16
+    pages, ps = wl.k_cache.shape[0], wl.k_cache.shape[1]
+    bf = torch.bfloat16
+    with pytest.raises(pa.PaError) as ei:
+        pa.pa_mla_backward(plan, torch.zeros(nq, h, r, dtype=bf), torch.zeros(nq, h, pr, dtype=bf),
+                           torch.zeros(pages, ps, 1, r, dtype=bf), torch.zeros(pages, ps, 1, pr, dtype=bf),
+                           torch.zeros(nq, h, r, dtype=bf), torch.zeros(nq, h, dtype=f32), torch.zeros(nq, h, r, dtype=bf),
+                           torch.zeros(nq, h, r, dtype=f32), torch.zeros(nq, h, pr, dtype=f32),
+                           torch.zeros(pages, ps, 1, r, dtype=f32), torch.zeros(pages, ps, 1, pr, dtype=f32), 0.1)
+    assert pa.STATUS[ei.value.status] == "PA_ERR_INVALID_ARGUMENT" and "host-only" in str(ei.value)
     plan.close()
