@@ -296,3 +296,14 @@ def test_backward_wrappers_marshal_to_the_library():
                            torch.zeros(pages, ps, 1, r, dtype=f32), torch.zeros(pages, ps, 1, pr, dtype=f32), 0.1)
     assert pa.STATUS[ei.value.status] == "PA_ERR_INVALID_ARGUMENT" and "host-only" in str(ei.value)
     plan.close()
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """Without the built library the binding raises: there is no CPU or oracle fallback."""
+    missing = str(tmp_path / "libpa_absent.so")
+    with pytest.raises(RuntimeError) as ei:
+        pa.load_library(missing)
+    assert "no fallback" in str(ei.value)
+    import paged_kv_attention_39_b200 as pkg
+    src = open(pkg.__file__).read()
+    assert "import oracle" not in src and "from oracle" not in src
