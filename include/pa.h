@@ -227,8 +227,12 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
  *   d_q                  [N_q, Hq, D] float32, written
  *   d_k_cache            [pages, page_size, Hkv, D] float32, ADDED INTO (zero it first)
  *   d_v_cache            [pages, page_size, Hkv, Dv] float32, ADDED INTO (zero it first)
- * Float32 atomics make the summation order of dK/dV vary between runs. Validation and errors as
- * pa_forward (gradient outputs must not overlap each other or any input).
+ * bf16 / fp16 with head_dim == v_head_dim in {64, 128} and at most 16 query heads per KV head run
+ * on the tensor cores: P and dS are rounded to the input type before the gradient products, every
+ * key's dK/dV row is summed by one CTA and added once, so the result repeats bit for bit unless two
+ * sequences share a page (three launches). Other shapes and fp32 run a float32 CUDA-core kernel
+ * whose dK/dV atomics make the summation order vary between runs (one launch). Validation and
+ * errors as pa_forward (gradient outputs must not overlap each other or any input).
  */
 pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
                       const void* out, const float* lse, const void* d_out, pa_dtype dtype,
