@@ -152,6 +152,13 @@ def kernel_traffic(kernel_file: str, key: str):
         return None
 
 
+def kernel_names(bits: int):
+    """The PA_KERNEL_* bits of a call as names."""
+    names = ["decode_tc", "prefill_tcgen05", "mla_tcgen05", "cuda_core", "merge", "sparse", "append",
+             "backward_tc", "backward_cuda_core"]
+    return [n for i, n in enumerate(names) if bits >> i & 1]
+
+
 def time_forward(pa, plan, args_fn, steps, warmup, trace=True, sampler=None, ws=1):
     """W untimed calls, then K calls bracketed by barrier + synchronize; per-call trace events."""
     for _ in range(warmup):
@@ -302,6 +309,7 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
             ("fp16_decode", lambda sd: W.c2_decode_variant(sd, torch.float16, 128)),
             ("bf16_decode_d64", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 64)),
             ("bf16_decode_d256", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256)),
+            ("bf16_chunked_prefill_d256", lambda sd: W.c3_prefill_variant(sd, torch.bfloat16, 256)),
             ("bf16_append_chunk", W.append_chunk), ("bf16_backward_chunk", W.backward_chunk),
             ("bf16_mla_backward", W.mla_backward_small)]
     if only is not None:
@@ -352,6 +360,7 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
                 "algorithmic_gflop": round(flops / 1e9, 2),
                 "algorithmic_kv_mb": round(kvb / 1e6, 1),
                 "launches": pa.pa_plan_get_info(plan)["last_launches"],
+                "kernels": kernel_names(pa.pa_plan_get_info(plan)["last_kernels"]),
             }
             plan.close()
             del wl
@@ -504,6 +513,7 @@ def run_single(args, ws, rank, local):
            "fp16_decode": lambda sd: W.c2_decode_variant(sd, torch.float16, 128),
            "bf16_decode_d64": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 64),
            "bf16_decode_d256": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256),
+           "bf16_chunked_prefill_d256": lambda sd: W.c3_prefill_variant(sd, torch.bfloat16, 256),
            "bf16_append_chunk": W.append_chunk, "bf16_backward_chunk": W.backward_chunk,
            "bf16_mla_backward": W.mla_backward_small}
     res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
@@ -591,6 +601,7 @@ def main():
                     choices=["bf16_decode", "bf16_chunked_prefill", "bf16_window_mixed", "bf16_mla_decode", "bf16_sparse_topk_decode",
                              "bf16_window_mixed_decode_part", "bf16_window_mixed_prefill_part",
                              "tiny_fp32_decode", "fp16_decode", "bf16_decode_d64", "bf16_decode_d256",
+                             "bf16_chunked_prefill_d256",
                              "bf16_append_chunk", "bf16_backward_chunk", "bf16_mla_backward"],
                     help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()

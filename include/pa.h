@@ -95,7 +95,12 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
 
 /* Free the plan's device memory, stream-ordered on the stream of its last call (or its upload
  * stream): work already queued there may still use it, work on other streams must be done.
- * The host does not wait. NULL is a no-op. */
+ * The host does not wait. NULL is a no-op. This is the release of what ruDNN's `DevicePlan`
+ * (paged_attention/mod.rs, the struct holding `host: Arc<HostPlan>` and the uploaded
+ * `metadata` tensor) owns, which Rust frees when the plan is dropped; the plan-owned split
+ * workspace (ruDNN `SplitWorkspace`) and work lists go with it. Returns PA_OK, or PA_ERR_CUDA
+ * if the release could not be queued on the stream (the memory is then freed after a stream
+ * synchronisation). */
 pa_status pa_plan_destroy(pa_plan* plan);
 
 /* Read-only facts about a plan. */
@@ -109,7 +114,19 @@ typedef struct pa_plan_info {
     int32_t last_launches;   /* kernels the last successful forward call launched */
     int64_t workspace_bytes; /* current size of the plan-owned split workspace */
     int64_t uploaded_bytes;  /* host-to-device bytes the plan has copied (schedule, work lists) */
+    int32_t last_kernels;    /* PA_KERNEL_* bits: which kernels the last successful call launched */
 } pa_plan_info;
+
+/* Bits of pa_plan_info.last_kernels (which code path served the last call). */
+#define PA_KERNEL_DECODE_TC 1u      /* split-KV decode on the tensor cores (mma.sync) */
+#define PA_KERNEL_PREFILL_TC 2u     /* chunked prefill on tcgen05 / TMEM / TMA */
+#define PA_KERNEL_MLA_TC 4u         /* MLA decode on tcgen05 / TMEM / TMA */
+#define PA_KERNEL_SIMT 8u           /* the CUDA-core kernel (fp32, other shapes, PA_PATH_SIMT) */
+#define PA_KERNEL_MERGE 16u         /* the split-part merge */
+#define PA_KERNEL_SPARSE 32u        /* sparse selection kernels (check, proxy scores, top-K) */
+#define PA_KERNEL_APPEND 64u        /* paged append */
+#define PA_KERNEL_BACKWARD_TC 128u  /* tensor-core GQA backward */
+#define PA_KERNEL_BACKWARD_SIMT 256u /* CUDA-core GQA or MLA backward */
 pa_status pa_plan_get_info(const pa_plan* plan, pa_plan_info* info);
 
 /* Path selection (testing and tuning). */
@@ -286,12 +303,20 @@ pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rop
  * split, > 0 keys per part). A batch whose work list or float32 split parts do not fit the array
  * returns PA_ERR_BOUNDS before anything is launched (a larger kv_chunk, or -1, needs fewer parts).
  *
+ * Limits of the array: at most 32768 work units (one per part of a sequence's keys), at most
+ * 16384 query rows whose keys are split, and float32 parts of at most the array's size minus
+ * 1.25 MiB of unit lists; beyond any of them the call returns PA_ERR_BOUNDS and launches
+ * nothing. A sequence whose keys would be cut into more than 1024 parts gets 1024 longer parts
+ * (as in pa_forward). The work list is written into the array by a small kernel from the plan's
+ * sequence table on the device, so the call makes no host-to-device copy (three launches: the
+ * list, the decode, the merge when some row is split).
+ *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress, once
  * per device, with that device current); make that first call before capturing the stream into
  * a CUDA graph. Every call shares the one array and leaves its contents behind; nothing in it
- * needs to start at zero (each call writes every part it later reads). Calls whose GPU work
- * overlaps -- issued on different streams of one process -- race on the array: order them on
- * one stream. Host threads are serialised inside the call.
+ * needs to start at zero (each call writes its unit lists and every part it later reads).
+ * Calls whose GPU work overlaps -- issued on different streams, or from different host threads
+ * on different streams -- race on the array: order them on one stream.
  * All other rules (validation before launch, no host synchronisation, errors) are pa_forward's.
  */
 #define PA_STATIC_WORKSPACE_BYTES (16u << 20)
@@ -398,10 +423,17 @@ pa_status pa_sparse_forward_ex(pa_plan* plan, const void* q, const void* k_cache
  */
 pa_status pa_plan_device_status(const pa_plan* plan, int32_t* code);
 
-/* Human-readable name of a status code (static string). */
+/* Human-readable name of a status code (static string, never NULL; "PA_ERR_UNKNOWN" for a
+ * value outside the enum). ruDNN (paged_attention/mod.rs) reports every failure as
+ * `PagedAttentionError(&'static str)`, whose `Display` prints that static text; in C the kind of
+ * failure becomes the pa_status code named here and the text goes to pa_last_error_message. */
 const char* pa_status_string(pa_status status);
 
-/* Message of the last failing call on this thread ("" if none); valid until the next call. */
+/* Message of the last failing call on this thread ("" if none or if the last call succeeded):
+ * the text ruDNN carries inside `PagedAttentionError` (paged_attention/mod.rs, e.g. "paged
+ * tensor exceeds U32 indexing"), here with the offending values filled in. A thread-local
+ * buffer owned by the library: valid until this thread's next call into the library; never
+ * free it. */
 const char* pa_last_error_message(void);
 
 /* Library version, e.g. "0.1.0". */

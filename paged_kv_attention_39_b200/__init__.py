@@ -34,6 +34,9 @@ SYMBOLS = ["pa_plan_create", "pa_plan_destroy", "pa_plan_get_info", "pa_plan_pre
            "pa_plan_device_status", "pa_sparse_select", "pa_sparse_forward", "pa_sparse_forward_ex",
            "pa_status_string", "pa_last_error_message", "pa_version"]
 PA_SPARSE_MAX_BLOCKS = 16384
+# bits of pa_plan_info.last_kernels
+PA_KERNEL_DECODE_TC, PA_KERNEL_PREFILL_TC, PA_KERNEL_MLA_TC, PA_KERNEL_SIMT = 1, 2, 4, 8
+PA_KERNEL_MERGE, PA_KERNEL_SPARSE, PA_KERNEL_APPEND, PA_KERNEL_BACKWARD_TC, PA_KERNEL_BACKWARD_SIMT = 16, 32, 64, 128, 256
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -55,7 +58,7 @@ class _Info(ctypes.Structure):
                 ("table_width", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32), ("device", ctypes.c_int32),
                 ("last_launches", ctypes.c_int32), ("workspace_bytes", ctypes.c_int64),
-                ("uploaded_bytes", ctypes.c_int64)]
+                ("uploaded_bytes", ctypes.c_int64), ("last_kernels", ctypes.c_int32)]
 
 
 _lib = None

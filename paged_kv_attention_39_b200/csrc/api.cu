@@ -197,6 +197,7 @@ struct pa_plan {
     size_t bwd_drow_bytes = 0;
     cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
     int32_t last_launches = 0;
+    int32_t last_kernels = 0;  // PA_KERNEL_* bits of the last call
     int64_t uploaded_bytes = 0;
     std::mutex mu;
 };
@@ -583,12 +584,14 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     cudaEvent_t* ev = (cudaEvent_t*)c.opts.trace_events;
     cudaError_t e;
     int launches = 0;
+    uint32_t kernels = 0;
     if (c.block_size > 0) {
         p.sel = P->sel_ws;
         p.sel_width = wout;
         p.block_size = c.block_size;
         if (wout > 0) {
             ++launches;
+            kernels |= PA_KERNEL_SPARSE;
             e = pa::launch_sparse_prep(c.selection, c.width, P->sel_ws, wout, P->d_seqs, P->d_q2seq, c.hkv,
                                        c.block_size, max_blocks(P, c.block_size), P->Nq, P->d_err, st);
             if (e != cudaSuccess) return fail(PA_ERR_CUDA, "selection check launch failed: %s", cudaGetErrorString(e));
@@ -597,6 +600,7 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     if (ev) PA_CUDA_TRY(cudaEventRecord(ev[0], st));
     if (S->n_tc > 0) {
         ++launches;
+        kernels |= PA_KERNEL_DECODE_TC;
         p.units = S->tc_units;
         p.num_units = S->n_tc;
         e = pa::launch_decode_mma(p, c.dtype, S->tc_rows_max, st);
@@ -604,11 +608,13 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     }
     if (S->n_pre > 0) {
         ++launches;
+        kernels |= PA_KERNEL_PREFILL_TC;
         e = pa::launch_prefill_tc(p, c.dtype, P->num_pages, st);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill kernel launch failed: %s", cudaGetErrorString(e));
     }
     if (S->n_mla > 0) {
         ++launches;
+        kernels |= PA_KERNEL_MLA_TC;
         p.units = S->mla_units;
         p.num_units = S->n_mla;
         e = pa::launch_mla_tc(p, c.dtype, st);
@@ -616,6 +622,7 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     }
     if (S->n_simt > 0) {
         ++launches;
+        kernels |= PA_KERNEL_SIMT;
         p.units = S->simt_units;
         p.num_units = S->n_simt;
         e = pa::launch_simt(p, c.dtype, st);
@@ -624,11 +631,13 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
     if (ev) PA_CUDA_TRY(cudaEventRecord(ev[1], st));
     if (S->n_comb > 0) {
         ++launches;
+        kernels |= PA_KERNEL_MERGE;
         e = pa::launch_combine(p, c.dtype, st);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "combine kernel launch failed: %s", cudaGetErrorString(e));
     }
     if (ev) PA_CUDA_TRY(cudaEventRecord(ev[2], st));
     P->last_launches = launches;
+    P->last_kernels = (int32_t)kernels;
     return ok();
 }
 
@@ -815,6 +824,7 @@ pa_status pa_plan_get_info(const pa_plan* plan, pa_plan_info* info) {
     info->last_launches = plan->last_launches;
     info->workspace_bytes = (int64_t)plan->ws_bytes;
     info->uploaded_bytes = plan->uploaded_bytes;
+    info->last_kernels = plan->last_kernels;
     return ok();
 }
 
@@ -965,6 +975,7 @@ pa_status pa_sparse_select(pa_plan* plan, const void* q, const void* k_cache, pa
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "top-k launch failed: %s", cudaGetErrorString(e));
     }
     P->last_launches = width > 0 ? 2 : 1;
+    P->last_kernels = PA_KERNEL_SPARSE;
     return ok();
 }
 
@@ -1052,6 +1063,7 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "append kernel launch failed: %s", cudaGetErrorString(e));
     plan->last_stream = (cudaStream_t)stream;
     plan->last_launches = 1;
+    plan->last_kernels = PA_KERNEL_APPEND;
     return ok();
 }
 
@@ -1178,6 +1190,7 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "backward kernel launch failed: %s", cudaGetErrorString(e));
         plan->last_stream = st;
         plan->last_launches = 1 + (plan->bwd_nkey > 0 ? 1 : 0) + (plan->bwd_nrow > 0 ? 1 : 0);
+        plan->last_kernels = PA_KERNEL_BACKWARD_TC;
         return ok();
     }
     cudaError_t e = pa::launch_backward(q, k_cache, v_cache, out, lse, d_out, d_q, d_k_cache, d_v_cache,
@@ -1187,6 +1200,7 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "backward kernel launch failed: %s", cudaGetErrorString(e));
     plan->last_stream = (cudaStream_t)stream;
     plan->last_launches = 1;
+    plan->last_kernels = PA_KERNEL_BACKWARD_SIMT;
     return ok();
 }
 
@@ -1242,6 +1256,7 @@ pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rop
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "MLA backward kernel launch failed: %s", cudaGetErrorString(e));
     plan->last_stream = (cudaStream_t)stream;
     plan->last_launches = 1;
+    plan->last_kernels = PA_KERNEL_BACKWARD_SIMT;
     return ok();
 }
 

@@ -1,9 +1,11 @@
 // Chunked-prefill paged attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
-// bf16 / fp16, head_dim 64 or 128, Dv == D.
+// bf16 / fp16, head_dim 64, 128 or 256, Dv == D.
 //
 // A unit is one 128-row tile: 128/G consecutive queries of a sequence times the G query heads
 // that share one KV head (so every K/V tile feeds all G heads), against the keys those queries
-// can see, 128 keys per step; it ends with the final output and lse. The kernel is persistent:
+// can see, BN keys per step (BN = 128; 64 at D = 256, where TMEM holds the two score buffers,
+// the 256 output columns and the two P buffers only at that width); it ends with the final
+// output and lse. The kernel is persistent:
 // one CTA per SM walks the units in strides of the grid, and its pipelines run on from one unit
 // into the next (the Q of the next unit loads as soon as the last score product of the current
 // one has completed; K/V loads and score products of the next unit overlap the current unit's
@@ -25,7 +27,8 @@
 //               the max grows by more than 2^8. The epilogue divides by the sum, rounds once
 //               and stores.
 //
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+D) P0, P1 (64 columns each) after O.
+// TMEM (512 columns): S0 [0,BN) S1 [BN,2BN) O [2BN,2BN+D) P0, P1 (BN/2 columns each) after O:
+// 448 columns at D = 128 (BN 128) and at D = 256 (BN 64).
 // QK of tile i+2 goes into score buffer i & 1 only after the softmax has marked P of tile i
 // ready (it has then read all of S of tile i). The QK and the P V chains come from two issuing
 // warps so that the tensor core overlaps them.
@@ -43,9 +46,6 @@ using namespace sm100;
 namespace {
 
 constexpr int BM = 128;  // rows per tile (queries x group heads)
-constexpr int BN = 128;  // keys per step
-constexpr int KST = 3;   // K stages
-constexpr int VST = 3;   // V stages
 constexpr int kSoftmaxWarps = 8;  // two per TMEM lane quadrant, each owning half of the columns
 constexpr int kTmaWarp = kSoftmaxWarps, kMmaWarp = kSoftmaxWarps + 1, kPvWarp = kSoftmaxWarps + 2;
 constexpr int kTmaVWarp = kSoftmaxWarps + 3;  // the V producer (kTmaWarp loads Q and K)
@@ -53,11 +53,19 @@ constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legal wait
 
+// Tile width and pipeline depth per head size. Shared memory: Q (D/64 boxes of 128 rows x
+// 128 bytes) plus KST K and VST V stages of BN rows x D columns: 112 KB at D = 64, 224 KB at
+// D = 128 (3 + 3 stages) and at D = 256 (64-key tiles, 3 + 2 stages), within the 227 KB of one
+// CTA.
 template <int D>
-struct PrefillSmem {
-    static constexpr int KH = D / 64;                 // 128-byte halves of a row
-    static constexpr int HALF_Q = BM * 128;           // bytes of one half of the Q tile
-    static constexpr int HALF_KV = BN * 128;          // bytes of one half of a K or V tile
+struct PrefillCfg {
+    static constexpr int BN = D == 256 ? 64 : 128;  // keys per step
+    static constexpr int KST = 3;                   // K stages
+    static constexpr int VST = D == 256 ? 2 : 3;    // V stages
+    static constexpr int NC = BN / 64;              // 32-column chunks of S per softmax warp
+    static constexpr int KH = D / 64;               // 128-byte halves of a row
+    static constexpr int HALF_Q = BM * 128;         // bytes of one half of the Q tile
+    static constexpr int HALF_KV = BN * 128;        // bytes of one half of a K or V tile
     static constexpr int Q = 0;
     static constexpr int K = Q + KH * HALF_Q;
     static constexpr int V = K + KST * KH * HALF_KV;
@@ -65,25 +73,30 @@ struct PrefillSmem {
     static constexpr int XCH = BAR + 256;  // 128 rows x 2 column halves of float: row statistics
     static constexpr int BYTES = XCH + 2 * BM * 4;
     static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
+    // TMEM columns: two score buffers, the output, two P buffers (16-bit pairs)
+    static constexpr int T_S1 = BN, T_O = 2 * BN, T_P0 = 2 * BN + D, T_P1 = T_P0 + BN / 2;
+    static_assert(T_P1 + BN / 2 <= 512, "TMEM holds S0, S1, O, P0 and P1");
+    static_assert(ALLOC <= 232448, "shared memory of one CTA");
+    // Barriers used once per tile in alternation come in pairs indexed by tile parity, so that no
+    // waiter can ever find its barrier two phases ahead of the phase it waits for.
+    static constexpr int B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
+                         B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_PFULL = B_SFULL + 2,
+                         B_ODONE = B_PFULL + 2, B_QEMPTY = B_ODONE + 2, B_COUNT = B_QEMPTY + 1;
+    static_assert(B_COUNT * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
 };
-
-// Barriers used once per tile in alternation come in pairs indexed by tile parity, so that no
-// waiter can ever find its barrier two phases ahead of the phase it waits for.
-enum BarId { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = B_KFULL + KST, B_VFULL = B_KEMPTY + KST,
-             B_VEMPTY = B_VFULL + VST, B_SFULL = B_VEMPTY + VST, B_PFULL = B_SFULL + 2, B_ODONE = B_PFULL + 2,
-             B_QEMPTY = B_ODONE + 2, B_COUNT = B_QEMPTY + 1 };
 
 }  // namespace
 
-// ---- softmax helpers: one thread owns one row of a 128-key score tile in TMEM -------------------
+// ---- softmax helpers: one thread owns one row of a score tile in TMEM ---------------------------
 // Column c of the tile is masked when c + off_lo < 0 or c + off_hi >= 0, where off_lo = kt0 - row_lo
 // and off_hi = kt0 - row_hi (the row's visible keys are [row_lo, row_hi)).
 
-// Each helper covers the 32-column chunks [c0, c0 + 2): one half of the tile's columns.
+// Each helper covers the 32-column chunks [c0, c0 + NC): one half of the tile's columns.
+template <int NC>
 __device__ __forceinline__ float tile_max_full(uint32_t taddr, int c0) {
     float m0 = neg_inf(), m1 = neg_inf(), m2 = neg_inf(), m3 = neg_inf();
 #pragma unroll 1
-    for (int c = c0; c < c0 + 2; ++c) {
+    for (int c = c0; c < c0 + NC; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -98,10 +111,11 @@ __device__ __forceinline__ float tile_max_full(uint32_t taddr, int c0) {
     return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
+template <int NC>
 __device__ __forceinline__ float tile_max_masked(uint32_t taddr, int c0, int off_lo, int off_hi) {
     float m0 = neg_inf(), m1 = neg_inf();
 #pragma unroll 1
-    for (int c = c0; c < c0 + 2; ++c) {
+    for (int c = c0; c < c0 + NC; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -143,12 +157,12 @@ __device__ __forceinline__ float exp_chunk(const uint32_t (&v)[32], int c, float
 }
 
 // Second pass of the two-pass path: probabilities against the (new) row max m.
-template <typename T, bool MASKED>
+template <typename T, bool MASKED, int NC>
 __device__ __forceinline__ float tile_exp(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
                                           int off_lo, int off_hi) {
     float sum = 0.f;
 #pragma unroll 1
-    for (int c = c0; c < c0 + 2; ++c) {
+    for (int c = c0; c < c0 + NC; ++c) {
         uint32_t v[32];
         tmem_ld32(taddr + c * 32, v);
         tmem_ld_wait(v);
@@ -161,8 +175,30 @@ __device__ __forceinline__ float tile_exp(uint32_t taddr, int c0, float scale, f
 // P buffer while the tile max of the raw scores is tracked; the caller keeps them when the max
 // grew by at most 2^8 (so p <= 256), and otherwise redoes the tile.
 template <typename T, bool MASKED>
-__device__ __forceinline__ float tile_fused(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
-                                            int off_lo, int off_hi, float& m_raw) {
+__device__ __forceinline__ float tile_fused1(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
+                                             int off_lo, int off_hi, float& m_raw) {
+    uint32_t v0[32];
+    tmem_ld32(taddr + c0 * 32, v0);
+    tmem_ld_wait(v0);
+    float m0 = neg_inf(), m1 = neg_inf();
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+        float x0 = __uint_as_float(v0[e]), x1 = __uint_as_float(v0[e + 1]);
+        if (MASKED) {
+            const int k0 = c0 * 32 + e;
+            x0 = (k0 + off_lo >= 0 && k0 + off_hi < 0) ? x0 : neg_inf();
+            x1 = (k0 + 1 + off_lo >= 0 && k0 + 1 + off_hi < 0) ? x1 : neg_inf();
+        }
+        m0 = fmaxf(m0, x0);
+        m1 = fmaxf(m1, x1);
+    }
+    m_raw = fmaxf(m0, m1);
+    return exp_chunk<T, MASKED>(v0, c0, scale, -m, p_taddr, off_lo, off_hi);
+}
+
+template <typename T, bool MASKED>
+__device__ __forceinline__ float tile_fused2(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
+                                             int off_lo, int off_hi, float& m_raw) {
     uint32_t v0[32], v1[32];
     tmem_ld32(taddr + c0 * 32, v0);  // both chunks in flight before the one wait
     tmem_ld32(taddr + (c0 + 1) * 32, v1);
@@ -188,12 +224,22 @@ __device__ __forceinline__ float tile_fused(uint32_t taddr, int c0, float scale,
            exp_chunk<T, MASKED>(v1, c0 + 1, scale, -m, p_taddr, off_lo, off_hi);
 }
 
+template <typename T, bool MASKED, int NC>
+__device__ __forceinline__ float tile_fused(uint32_t taddr, int c0, float scale, float m, uint32_t p_taddr,
+                                            int off_lo, int off_hi, float& m_raw) {
+    if constexpr (NC == 1) return tile_fused1<T, MASKED>(taddr, c0, scale, m, p_taddr, off_lo, off_hi, m_raw);
+    else return tile_fused2<T, MASKED>(taddr, c0, scale, m, p_taddr, off_lo, off_hi, m_raw);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const AttnParams p) {
-    using L_ = PrefillSmem<D>;
-    constexpr int KH = L_::KH;
+    using L_ = PrefillCfg<D>;
+    constexpr int KH = L_::KH, BN = L_::BN, KST = L_::KST, VST = L_::VST, NC = L_::NC;
+    constexpr int B_QFULL = L_::B_QFULL, B_KFULL = L_::B_KFULL, B_KEMPTY = L_::B_KEMPTY, B_VFULL = L_::B_VFULL,
+                  B_VEMPTY = L_::B_VEMPTY, B_SFULL = L_::B_SFULL, B_PFULL = L_::B_PFULL, B_ODONE = L_::B_ODONE,
+                  B_QEMPTY = L_::B_QEMPTY, B_COUNT = L_::B_COUNT;
     constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
     constexpr uint32_t IDESC_QK = idesc_f16(BM, BN, kBf16, false, false);
     constexpr uint32_t IDESC_PV = idesc_f16(BM, D, kBf16, false, true);
@@ -229,9 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s0 = tmem, t_s1 = tmem + 128;
-    const uint32_t t_o = tmem + 256;
-    const uint32_t t_p0 = t_o + D, t_p1 = t_o + D + 64;
+    const uint32_t t_s0 = tmem, t_s1 = tmem + L_::T_S1;
+    const uint32_t t_o = tmem + L_::T_O;
+    const uint32_t t_p0 = tmem + L_::T_P0, t_p1 = tmem + L_::T_P1;
     const uint32_t s_base = smem_u32(smem);
 
     // Units come longest first from the host. In round rr the CTA takes unit rr * grid + b, with b
@@ -370,8 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t dKs = desc_add(dK, ks * KH * L_::HALF_KV);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t off = (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;  // HALF_Q == HALF_KV
-                            mma_f16_ss(d_s, desc_add(dQ, off), desc_add(dKs, off), IDESC_QK, kk > 0);
+                            // k-step kk: 128-byte half kk / 4 of the rows, 32-byte slice kk % 4 of it
+                            const uint32_t off_q = (kk >> 2) * L_::HALF_Q + (kk & 3) * 32;
+                            const uint32_t off_k = (kk >> 2) * L_::HALF_KV + (kk & 3) * 32;
+                            mma_f16_ss(d_s, desc_add(dQ, off_q), desc_add(dKs, off_k), IDESC_QK, kk > 0);
                         }
                         mma_commit(&bars[B_SFULL + b]);
                         mma_commit(&bars[B_KEMPTY + ks]);
@@ -423,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int quad = warp & 3, half = warp >> 2;
         const int r = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        const int c0 = half * 2;  // first 32-column chunk of this warp's half
+        const int c0 = half * NC;  // first 32-column chunk of this warp's half
         float* xch = reinterpret_cast<float*>(smem + L_::XCH);
         auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;\n" ::"r"(1 + quad) : "memory"); };
         // max (or sum) of this row's two halves
@@ -476,15 +524,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float sum = 0.f;
                 if (__all_sync(0xffffffffu, m_run != neg_inf())) {
                     float m_raw;
-                    sum = full ? tile_fused<T, false>(t_sb, c0, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
-                               : tile_fused<T, true>(t_sb, c0, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
+                    sum = full ? tile_fused<T, false, NC>(t_sb, c0, p.scale_log2, m_run, t_pb, 0, 0, m_raw)
+                               : tile_fused<T, true, NC>(t_sb, c0, p.scale_log2, m_run, t_pb, off_lo, off_hi, m_raw);
                     m_raw = exchange(m_raw, true);
                     redo = __any_sync(0xffffffffu, m_raw * p.scale_log2 > m_run + 8.0f);
                 }
                 if (redo) {
                     // pass 1: tile max of the raw scores; the scale is positive, so it is applied to
                     // the max once. Edge tiles mask keys outside [row_lo, row_hi) first.
-                    float m_raw = full ? tile_max_full(t_sb, c0) : tile_max_masked(t_sb, c0, off_lo, off_hi);
+                    float m_raw = full ? tile_max_full<NC>(t_sb, c0) : tile_max_masked<NC>(t_sb, c0, off_lo, off_hi);
                     m_raw = exchange(m_raw, true);
                     const float m_tile = m_raw * p.scale_log2;
                     const float m_new = fmaxf(m_run, m_tile);
@@ -511,8 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const float m_use = m_run == neg_inf() ? 0.f : m_run;
                     // pass 2: probabilities p = 2^(s * scale - m) into the P buffer
-                    sum = full ? tile_exp<T, false>(t_sb, c0, p.scale_log2, m_use, t_pb, 0, 0)
-                               : tile_exp<T, true>(t_sb, c0, p.scale_log2, m_use, t_pb, off_lo, off_hi);
+                    sum = full ? tile_exp<T, false, NC>(t_sb, c0, p.scale_log2, m_use, t_pb, 0, 0)
+                               : tile_exp<T, true, NC>(t_sb, c0, p.scale_log2, m_use, t_pb, off_lo, off_hi);
                 }
                 tmem_st_wait();
                 l_part += sum;
@@ -581,6 +629,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+}  // namespace
+
 // 3-D map over a row-major [d2][d1][d0] tensor of 16-bit elements, box {64, b1, b2}, 128B swizzle.
 bool make_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1,
               uint32_t b2) {
@@ -596,9 +646,12 @@ bool make_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t
     return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <typename T, int D>
 cudaError_t launch_t(const AttnParams& p, int num_pages, cudaStream_t st) {
-    using L_ = PrefillSmem<D>;
+    using L_ = PrefillCfg<D>;
+    constexpr int BN = L_::BN;
     const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const int G = p.group, qpt = BM / G;
     const int ps = p.page_size;
@@ -634,18 +687,25 @@ cudaError_t launch_t(const AttnParams& p, int num_pages, cudaStream_t st) {
 }  // namespace
 
 bool prefill_tc_supported(pa_dtype dt, int d, int dv, int group, int page_size) {
-    if (dt == PA_F32 || d != dv || (d != 64 && d != 128)) return false;
+    if (dt == PA_F32 || d != dv || (d != 64 && d != 128 && d != 256)) return false;
     if (group < 1 || group > BM || BM % group != 0) return false;
     if (page_size % 16 != 0) return false;
-    if (page_size < BN ? (BN % page_size != 0) : (page_size % BN != 0)) return false;
+    const int bn = d == 256 ? PrefillCfg<256>::BN : PrefillCfg<128>::BN;  // a page box holds whole tiles, or a tile whole pages
+    if (page_size < bn ? (bn % page_size != 0) : (page_size % bn != 0)) return false;
     return true;
+}
+
+template <typename T>
+cudaError_t launch_d(const AttnParams& p, int num_pages, cudaStream_t st) {
+    if (p.d == 64) return launch_t<T, 64>(p, num_pages, st);
+    if (p.d == 256) return launch_t<T, 256>(p, num_pages, st);
+    return launch_t<T, 128>(p, num_pages, st);
 }
 
 cudaError_t launch_prefill_tc(const AttnParams& p, pa_dtype dt, int num_pages, cudaStream_t st) {
     if (p.num_punits == 0) return cudaSuccess;
-    if (dt == PA_BF16) return p.d == 64 ? launch_t<__nv_bfloat16, 64>(p, num_pages, st)
-                                        : launch_t<__nv_bfloat16, 128>(p, num_pages, st);
-    return p.d == 64 ? launch_t<__half, 64>(p, num_pages, st) : launch_t<__half, 128>(p, num_pages, st);
+    if (dt == PA_BF16) return launch_d<__nv_bfloat16>(p, num_pages, st);
+    return launch_d<__half>(p, num_pages, st);
 }
 
 }  // namespace pa

@@ -291,6 +291,17 @@ def c2_decode_variant(seed: int = 0, dtype: torch.dtype = torch.float16, d: int 
                     causal=True, window=0, pin=pin)
 
 
+def c3_prefill_variant(seed: int = 0, dtype: torch.dtype = torch.bfloat16, d: int = 256, batch: int = 8,
+                       pin: bool = False) -> GqaWorkload:
+    """The chunked-prefill batch's shape (8 sequences, history U[0, 4096] plus a 512-query chunk,
+    Hq=32, Hkv=8, page 64, causal) in another element type or head size (D = Dv = d)."""
+    hist = _uniform_ints(seed, 0xC3, batch, 0, 4096)
+    lens = [h + 512 for h in hist]
+    tag = {torch.float16: "fp16", torch.bfloat16: "bf16", torch.float32: "fp32"}[dtype]
+    return make_gqa(f"{tag}_chunked_prefill_d{d}_b{batch}", seed, lens, [512] * batch, 32, 8, d, d, 64, dtype,
+                    causal=True, window=0, pin=pin)
+
+
 def append_chunk(seed: int = 0):
     """Paged append of the chunked-prefill batch's new rows (8 sequences x 512 queries, Hkv=8,
     D=Dv=128, pages of 64, bf16): (workload, new_k [Nq, Hkv, D], new_v [Nq, Hkv, Dv])."""

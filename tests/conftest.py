@@ -20,3 +20,21 @@ def pytest_configure(config):
 def orc():
     import oracle
     return oracle.get()
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Measured errors of every GPU parity comparison of the session (gpu_helpers.MARGINS)."""
+    mod = sys.modules.get("gpu_helpers")
+    rows = getattr(mod, "MARGINS", None) if mod else None
+    if not rows:
+        return
+    tr = terminalreporter
+    tr.section("parity margins (measured error against the fp64 oracle; 'of bound' = error / allowed)")
+    tr.write_line(f"{'case':<58} {'dtype':<9} {'rows':>9} {'max|dout|':>11} {'of bound':>9} {'max|dlse|':>11} {'of bound':>9}")
+    worst = {}
+    for tag, dt, n, e, r, le, lr in rows:
+        tr.write_line(f"{tag[:58]:<58} {dt:<9} {n:>9} {e:>11.3e} {r:>9.3f} {le:>11.3e} {lr:>9.3f}")
+        w = worst.setdefault(dt, [0.0, 0.0])
+        w[0], w[1] = max(w[0], r), max(w[1], lr)
+    for dt, (r, lr) in sorted(worst.items()):
+        tr.write_line(f"worst {dt}: out at {r:.3f} of its bound, lse at {lr:.3f} of its bound")

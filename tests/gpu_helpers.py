@@ -5,12 +5,21 @@ Tolerances (fixed for the path in the design notes, checked here):
   fp32 inputs : max |out - ref| <= 1e-5 * max|ref|   and  |lse - ref| <= 1e-5 * max(1, |ref|)
   bf16 / fp16 : |out - ref| <= 1e-2 + 2e-2 * |ref| elementwise, and |lse - ref| <= 2e-3
 Rows the mask leaves empty must come back exactly as out = 0, lse = -inf.
+
+Every comparison records its measured error (largest |out - ref|, the largest ratio of
+|out - ref| to its allowed bound, largest lse error) in MARGINS; the session summary prints them
+(tests/conftest.py), so that a passing run still shows how much room each case has.
 """
 import math
+import os
 
 import torch
 
 import paged_kv_attention_39_b200 as pa
+
+# (tag, dtype, rows compared, max |dout|, max |dout| / allowed, max |dlse| (fp32: relative),
+#  max |dlse| / allowed), one entry per check() call
+MARGINS = []
 
 
 def to_dev(t):
@@ -65,17 +74,26 @@ def check(wl, out, lse, ref_out, ref_lse, rows=None, tag=""):
     assert torch.equal(l[empty], rl[empty]) and bool((o[empty] == 0).all()), f"{tag}: empty rows"
     o, l, ro, rl = o[~empty], l[~empty], ro[~empty], rl[~empty]
     assert torch.isfinite(o).all() and torch.isfinite(l).all(), f"{tag}: non-finite output"
+    cur = os.environ.get("PYTEST_CURRENT_TEST", "")
+    name = cur.split("::")[-1].split(" ")[0] if cur else ""
+    tag = f"{name} {tag}".strip()
     dt = out.dtype
+    diff = (o - ro).abs()
+    err = float(diff.max()) if ro.numel() else 0.0
     if dt == torch.float32:
         scale = max(float(ro.abs().max()) if ro.numel() else 1.0, 1e-30)
-        err = float((o - ro).abs().max()) if ro.numel() else 0.0
+        lrel = (l - rl).abs() / rl.abs().clamp_min(1.0)
+        lerr = float(lrel.max()) if rl.numel() else 0.0
+        MARGINS.append((tag, "fp32", int(o.shape[0]), err, err / (1e-5 * scale), lerr, lerr / 1e-5))
         assert err <= 1e-5 * scale, f"{tag}: out max err {err} > 1e-5 * {scale}"
-        lerr = (l - rl).abs() / rl.abs().clamp_min(1.0)
-        assert float(lerr.max()) <= 1e-5, f"{tag}: lse rel err {float(lerr.max())}"
+        assert lerr <= 1e-5, f"{tag}: lse rel err {lerr}"
     else:
-        bad = (o - ro).abs() > 1e-2 + 2e-2 * ro.abs()
-        assert not bool(bad.any()), f"{tag}: out err {float((o - ro).abs().max())} at {int(bad.sum())} elems"
+        bound = 1e-2 + 2e-2 * ro.abs()
+        ratio = float((diff / bound).max()) if ro.numel() else 0.0
         lerr = float((l - rl).abs().max()) if rl.numel() else 0.0
+        MARGINS.append((tag, str(dt).replace("torch.", ""), int(o.shape[0]), err, ratio, lerr, lerr / 2e-3))
+        bad = diff > bound
+        assert not bool(bad.any()), f"{tag}: out err {err} at {int(bad.sum())} elems"
         assert lerr <= 2e-3, f"{tag}: lse err {lerr}"
     return H
 

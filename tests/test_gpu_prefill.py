@@ -24,15 +24,76 @@ def status_ok(wl):
     return True
 
 
+def on_tensor_cores(plan):
+    """The last call ran the tcgen05 prefill kernel and no CUDA-core kernel."""
+    k = pa.pa_plan_get_info(plan)["last_kernels"]
+    return bool(k & pa.PA_KERNEL_PREFILL_TC) and not (k & pa.PA_KERNEL_SIMT)
+
+
 def test_prefill_basic(orc):
     wl = prefill_wl(1)
     ref = orc.run(wl)
     plan = pa.plan_for(wl)
     out, lse = run_gqa(wl, plan=plan)
     assert pa.pa_plan_get_info(plan)["last_launches"] == 1
+    assert on_tensor_cores(plan)
     assert pa.pa_plan_device_status(plan) == 0
     plan.close()
     check(wl, out, lse, *ref, tag="prefill basic")
+
+
+@pytest.mark.parametrize("dtype,hq,hkv,ps,window,causal", [
+    (torch.bfloat16, 32, 8, 64, 0, True),
+    (torch.float16, 32, 8, 64, 0, True),
+    (torch.bfloat16, 8, 8, 16, 0, True),      # G 1, pages of 16: four boxes per 64-key tile
+    (torch.bfloat16, 16, 8, 32, 100, True),   # G 2, sliding window
+    (torch.bfloat16, 64, 4, 128, 0, False),   # G 16, not causal, two tiles per page
+    (torch.float16, 32, 4, 256, 300, True),   # G 8, pages of 256, window
+    (torch.bfloat16, 32, 8, 64, 1, True),     # window 1: each row sees itself only
+])
+def test_prefill_head_dim_256(orc, dtype, hq, hkv, ps, window, causal):
+    """D = 256 on the tcgen05 prefill kernel (64-key tiles): ragged query tiles and histories from
+    empty to 700 keys, against the oracle element by element."""
+    wl = prefill_wl(11, hq=hq, hkv=hkv, d=256, ps=ps, dtype=dtype, hist=(0, 700), chunk=150, window=window,
+                    causal=causal)
+    ref = orc.run(wl)
+    plan = pa.plan_for(wl)
+    out, lse = run_gqa(wl, plan=plan)
+    assert on_tensor_cores(plan)
+    assert pa.pa_plan_device_status(plan) == 0
+    plan.close()
+    check(wl, out, lse, *ref, tag=f"d256 {dtype} G{hq // hkv} ps{ps} w{window} c{causal}")
+
+
+def test_prefill_head_dim_256_many_units_and_decode_rows(orc):
+    """Several hundred D = 256 tiles walked by each persistent CTA in turn, plus decode rows (the
+    D = 256 split-KV decode kernel) in the same call."""
+    hs = W._uniform_ints(12, 78, 40, 0, 600)
+    lens = [h + 70 for h in hs] + [3000, 1500]
+    qs = [70] * 40 + [1, 1]
+    wl = W.make_gqa("d256_many", 12, lens, qs, 16, 4, 256, 256, 64, torch.bfloat16, causal=True, window=0)
+    ref = orc.run(wl)
+    plan = pa.plan_for(wl)
+    out, lse = run_gqa(wl, plan=plan)
+    k = pa.pa_plan_get_info(plan)["last_kernels"]
+    assert k & pa.PA_KERNEL_PREFILL_TC and k & pa.PA_KERNEL_DECODE_TC and not k & pa.PA_KERNEL_SIMT
+    assert pa.pa_plan_device_status(plan) == 0
+    plan.close()
+    check(wl, out, lse, *ref, tag="d256 many units + decode")
+
+
+def test_prefill_head_dim_256_mask_bit_exact_by_counts():
+    for window, causal in ((0, True), (70, True), (33, False)):
+        wl = W.make_gqa("pmask256", 13, [200, 450, 64], [200, 130, 64], 16, 4, 256, 256, 64, torch.bfloat16,
+                        causal=causal, window=window)
+        wl.q.zero_()
+        out, lse = run_gqa(wl)
+        s = wl.sched
+        for si in range(s.num_seqs):
+            L = int(s.seq_lens[si]); q0 = int(s.query_offsets[si]); n = int(s.query_offsets[si + 1]) - q0
+            cnt = torch.tensor([visible_count(L, n, j, causal, window)[0] for j in range(n)])
+            got = torch.exp(lse[q0:q0 + n].double()).round().long()
+            assert bool((got == cnt.view(-1, 1)).all()), (window, causal, si)
 
 
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (64, 8), (32, 2), (128, 1)])
