@@ -95,7 +95,7 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
 
 /* Free the plan's device memory, stream-ordered on the stream of its last call (or its upload
  * stream): work already queued there may still use it, work on other streams must be done.
- * The host does not wait. NULL is a no-op. This is the release of what ruDNN's `DevicePlan`
+ * The host does not wait and nothing is queued on the stream but the frees. NULL is a no-op. This is the release of what ruDNN's `DevicePlan`
  * (paged_attention/mod.rs, the struct holding `host: Arc<HostPlan>` and the uploaded
  * `metadata` tensor) owns, which Rust frees when the plan is dropped; the plan-owned split
  * workspace (ruDNN `SplitWorkspace`) and work lists go with it. Returns PA_OK, or PA_ERR_CUDA
@@ -244,12 +244,17 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
  *   d_q                  [N_q, Hq, D] float32, written
  *   d_k_cache            [pages, page_size, Hkv, D] float32, ADDED INTO (zero it first)
  *   d_v_cache            [pages, page_size, Hkv, Dv] float32, ADDED INTO (zero it first)
- * bf16 / fp16 with head_dim == v_head_dim in {64, 128} and at most 16 query heads per KV head run
- * on the tensor cores: P and dS are rounded to the input type before the gradient products, every
- * key's dK/dV row is summed by one CTA and added once, so the result repeats bit for bit unless two
- * sequences share a page (three launches). Other shapes and fp32 run a float32 CUDA-core kernel
- * whose dK/dV atomics make the summation order vary between runs (one launch). Validation and
- * errors as pa_forward (gradient outputs must not overlap each other or any input).
+ * bf16 / fp16 with head_dim == v_head_dim in {64, 128} and G = num_q_heads / num_kv_heads dividing
+ * 128 and at most 16 run on the tensor cores: dK/dV key-major on tcgen05 (a CTA per 128 keys and KV
+ * head), dQ query-major on mma.sync; P and dS are rounded to the input type before the gradient
+ * products. Every key's dK/dV row is summed by one CTA and added once; where a page is referenced
+ * more than once in the plan (sequences sharing a prefix, a page listed twice), the rows of every key
+ * tile that touches it are summed per cache slot in (sequence, key) order by an ordered pass (ruDNN's
+ * atomic-free "ordered" history pass), so the result repeats bit for bit in every case (three
+ * launches, four with shared pages; the plan keeps the float32 scratch of those tiles). Other shapes
+ * and fp32 run a float32 CUDA-core kernel whose dK/dV atomics make the summation order vary between
+ * runs (one launch). Validation and errors as pa_forward (gradient outputs must not overlap each
+ * other or any input).
  */
 pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
                       const void* out, const float* lse, const void* d_out, pa_dtype dtype,

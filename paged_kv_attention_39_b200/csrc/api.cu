@@ -66,7 +66,7 @@ constexpr int kMaxSplits = 1024;           // parts one sequence's keys may be c
 // A copy from pageable memory makes the driver stage it itself (synchronously, and it may wait
 // for the stream); copies through page-locked slots are true asynchronous DMA. The slots are
 // allocated once per process and shared by every plan; a slot is reused once the event recorded
-// after its last copy has completed. Uploads larger than a slot go straight from pageable memory.
+// after its last copy has completed. Uploads larger than a slot go through several slots.
 constexpr int kStageSlots = 16;
 constexpr size_t kStageSlotBytes = 256 << 10;
 
@@ -120,11 +120,7 @@ cudaError_t lib_malloc(void** ptr, size_t bytes, cudaStream_t st) {
     return cudaMallocFromPoolAsync(ptr, bytes, pool, st);
 }
 
-cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
-    int dev = -1;
-    Staging* gp = bytes <= kStageSlotBytes && cudaGetDevice(&dev) == cudaSuccess ? staging(dev) : nullptr;
-    if (!gp) return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st);
-    Staging& g = *gp;
+cudaError_t upload_slot(Staging& g, void* dst, const void* src, size_t bytes, cudaStream_t st) {
     std::lock_guard<std::mutex> lock(g.mu);
     const int i = g.next;
     g.next = (g.next + 1) % kStageSlots;
@@ -142,6 +138,20 @@ cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     if ((e = cudaMemcpyAsync(dst, g.slot[i], bytes, cudaMemcpyHostToDevice, st)) != cudaSuccess) return e;
     g.used[i] = true;
     return cudaEventRecord(g.done[i], st);
+}
+
+// Every upload goes through the staging slots, in slot-sized pieces, so the host source may be
+// released as soon as this returns (nothing reads it later).
+cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+    int dev = -1;
+    Staging* gp = cudaGetDevice(&dev) == cudaSuccess ? staging(dev) : nullptr;
+    if (!gp) return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, st);
+    for (size_t off = 0; off < bytes; off += kStageSlotBytes) {
+        const size_t n = std::min(kStageSlotBytes, bytes - off);
+        cudaError_t e = upload_slot(*gp, static_cast<char*>(dst) + off, static_cast<const char*>(src) + off, n, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 constexpr int kTargetCtasPerSm = 8;        // automatic split size aims at this many CTAs/SM
 
@@ -192,9 +202,13 @@ struct pa_plan {
     void* bwd_dev = nullptr;
     int32_t bwd_group = 0, bwd_causal = -1, bwd_window = -1, bwd_nkey = 0, bwd_nrow = 0;
     size_t bwd_row_off = 0;
+    int32_t bwd_nord = 0, bwd_nsums = 0;  // ordered key tiles; cache rows of the ordered pass
+    size_t bwd_sums_off = 0, bwd_refs_off = 0;
     std::vector<std::vector<char>> bwd_host;  // host blobs of the uploads (kept with the plan)
     float* bwd_drow = nullptr;
     size_t bwd_drow_bytes = 0;
+    float* bwd_scratch = nullptr;  // finished dK then dV rows of ordered key tiles
+    size_t bwd_scratch_bytes = 0;
     cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
     int32_t last_launches = 0;
     int32_t last_kernels = 0;  // PA_KERNEL_* bits of the last call
@@ -385,9 +399,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     S->slots = slots;
     S->kv_chunk = (int32_t)std::min<int64_t>(chunk, INT32_MAX);
 
-    if (P->scheds.size() >= 8) {  // keep the plan's footprint bounded
-        // The host blob must outlive its copy: retire it only after the stream drains.
-        cudaStreamSynchronize(st);
+    if (P->scheds.size() >= 8) {  // keep the plan's footprint bounded (stream-ordered free)
         cudaFreeAsync(P->scheds.front()->dev, st);
         P->scheds.erase(P->scheds.begin());
     }
@@ -790,23 +802,20 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
 pa_status pa_plan_destroy(pa_plan* plan) {
     if (!plan) return ok();
     if (plan->device >= 0) {
-        // Stream-ordered frees after the plan's last queued use. The host blobs of pending
-        // uploads must outlive those copies, so the plan object is deleted by a host callback
-        // once the stream reaches this point.
+        // Stream-ordered frees after the plan's last queued use. Uploads read page-locked copies of
+        // the plan's host data, never the plan's own buffers, so the plan object goes at once (no
+        // host callback on the stream, which would hold back the work queued after it).
         cudaStream_t st = plan->last_stream;
         if (plan->ws) cudaFreeAsync(plan->ws, st);
         if (plan->sel_ws) cudaFreeAsync(plan->sel_ws, st);
         if (plan->score_ws) cudaFreeAsync(plan->score_ws, st);
         if (plan->bwd_dev) cudaFreeAsync(plan->bwd_dev, st);
         if (plan->bwd_drow) cudaFreeAsync(plan->bwd_drow, st);
+        if (plan->bwd_scratch) cudaFreeAsync(plan->bwd_scratch, st);
         for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
-        if (plan->d_meta) cudaFreeAsync(plan->d_meta, st);
-        cudaError_t e = cudaLaunchHostFunc(st, [](void* ud) { delete static_cast<pa_plan*>(ud); }, plan);
-        if (e != cudaSuccess) {
-            cudaStreamSynchronize(st);
-            delete plan;
-            return fail(PA_ERR_CUDA, "plan release failed: %s", cudaGetErrorString(e));
-        }
+        cudaError_t e = plan->d_meta ? cudaFreeAsync(plan->d_meta, st) : cudaSuccess;
+        delete plan;
+        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "plan release failed: %s", cudaGetErrorString(e));
         return ok();
     }
     delete plan;
@@ -1069,12 +1078,24 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
 
 // Work lists of the tensor-core backward for one (group size, causal, window), longest first:
 // the 64-key tiles of every sequence that some query sees (cost: the rows that see them) for the
-// dK/dV kernel, and blocks of at most 16 rows (cost: the keys they see) for the dQ kernel. One
-// upload; the host blob stays with the plan.
+// dK/dV kernel, and blocks of at most 16 rows (cost: the keys they see) for the dQ kernel. Key tiles
+// that touch a page referenced more than once in the plan (sequences sharing a prefix page, or a
+// page listed twice) are "ordered": their rows go to scratch, and the ordered pass's list gives
+// every cache row those tiles touch with its scratch rows in (sequence, key) order. One upload; the
+// host blob stays with the plan.
 static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int32_t window, cudaStream_t st) {
     const int KT = pa::backward_key_tile(), qpb = std::max(1, pa::backward_row_block() / G);
+    const int32_t ps = plan->page_size;
+    std::vector<int32_t> refs_per_page((size_t)std::max(1, plan->num_pages), 0);
+    for (int32_t si = 0; si < plan->S; ++si) {
+        const int64_t used = ((int64_t)plan->seqs[si].L + ps - 1) / ps;
+        for (int64_t b = 0; b < used; ++b) ++refs_per_page[plan->bt[(size_t)si * plan->table_width + b]];
+    }
+    auto page_of = [&](int32_t si, int64_t t) { return plan->bt[(size_t)si * plan->table_width + t / ps]; };
     std::vector<std::pair<int64_t, pa::BwdKeyUnit>> ku;
     std::vector<std::pair<int64_t, pa::BwdRowUnit>> ru;
+    std::vector<std::pair<int64_t, int32_t>> slot_refs;  // (cache row, scratch row) of ordered tiles
+    int32_t n_ord = 0;
     for (int32_t si = 0; si < plan->S; ++si) {
         const pa::SeqInfo& q_ = plan->seqs[si];
         if (q_.n == 0) continue;
@@ -1084,7 +1105,16 @@ static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int3
             const int64_t jlo = causal ? std::max<int64_t>(0, k0 - base) : 0;
             const int64_t jhi = window > 0 ? std::min<int64_t>(q_.n, kmax - 1 + window - base) : q_.n;
             if (jhi <= jlo) continue;
-            ku.push_back({jhi - jlo, pa::BwdKeyUnit{si, (int32_t)k0}});
+            bool shared = false;
+            for (int64_t t = k0; t < kmax && !shared; t += std::min<int64_t>(ps - t % ps, kmax - t))
+                shared = refs_per_page[page_of(si, t)] > 1;
+            int32_t ord = -1;
+            if (shared) {
+                ord = n_ord++;
+                for (int64_t t = k0; t < kmax; ++t)
+                    slot_refs.push_back({(int64_t)page_of(si, t) * ps + t % ps, ord * KT + (int32_t)(t - k0)});
+            }
+            ku.push_back({jhi - jlo, pa::BwdKeyUnit{si, (int32_t)k0, ord, 0}});
         }
         for (int32_t j0 = 0; j0 < q_.n; j0 += qpb) {
             const int32_t j1 = std::min(q_.n, j0 + qpb);
@@ -1096,12 +1126,28 @@ static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int3
     auto longer = [](const auto& a, const auto& b) { return a.first > b.first; };
     std::stable_sort(ku.begin(), ku.end(), longer);
     std::stable_sort(ru.begin(), ru.end(), longer);
-    const size_t row_off = (ku.size() * sizeof(pa::BwdKeyUnit) + 255) & ~size_t(255);
-    std::vector<char> blob(std::max<size_t>(16, row_off + ru.size() * sizeof(pa::BwdRowUnit)));
+    // ordered pass: group the scratch rows by cache row, keeping (sequence, key) order within a row
+    std::stable_sort(slot_refs.begin(), slot_refs.end(),
+                     [](const auto& a, const auto& b) { return a.first < b.first; });
+    std::vector<pa::BwdSlotSum> sums;
+    std::vector<int32_t> refs(slot_refs.size());
+    for (size_t i = 0; i < slot_refs.size(); ++i) {
+        if (i == 0 || slot_refs[i].first != slot_refs[i - 1].first)
+            sums.push_back(pa::BwdSlotSum{slot_refs[i].first, (int32_t)i, 0});
+        ++sums.back().count;
+        refs[i] = slot_refs[i].second;
+    }
+    auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t row_off = align(ku.size() * sizeof(pa::BwdKeyUnit));
+    const size_t sums_off = align(row_off + ru.size() * sizeof(pa::BwdRowUnit));
+    const size_t refs_off = align(sums_off + sums.size() * sizeof(pa::BwdSlotSum));
+    std::vector<char> blob(std::max<size_t>(16, refs_off + refs.size() * sizeof(int32_t)));
     for (size_t i = 0; i < ku.size(); ++i)
         std::memcpy(blob.data() + i * sizeof(pa::BwdKeyUnit), &ku[i].second, sizeof(pa::BwdKeyUnit));
     for (size_t i = 0; i < ru.size(); ++i)
         std::memcpy(blob.data() + row_off + i * sizeof(pa::BwdRowUnit), &ru[i].second, sizeof(pa::BwdRowUnit));
+    if (!sums.empty()) std::memcpy(blob.data() + sums_off, sums.data(), sums.size() * sizeof(pa::BwdSlotSum));
+    if (!refs.empty()) std::memcpy(blob.data() + refs_off, refs.data(), refs.size() * sizeof(int32_t));
     // the cached lists are invalid from here until the new ones are uploaded: a failure below
     // leaves the plan to rebuild them on its next call
     plan->bwd_group = 0;
@@ -1118,6 +1164,10 @@ static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int3
     plan->bwd_nkey = (int32_t)ku.size();
     plan->bwd_nrow = (int32_t)ru.size();
     plan->bwd_row_off = row_off;
+    plan->bwd_nord = n_ord;
+    plan->bwd_nsums = (int32_t)sums.size();
+    plan->bwd_sums_off = sums_off;
+    plan->bwd_refs_off = refs_off;
     plan->uploaded_bytes += (int64_t)plan->bwd_host.back().size();
     return PA_OK;
 }
@@ -1176,20 +1226,31 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
         }
         pa_status gs = grow_buffer(&plan->bwd_drow, &plan->bwd_drow_bytes, (size_t)nq * num_q_heads * sizeof(float), st);
         if (gs != PA_OK) return gs;
+        const size_t half = (size_t)plan->bwd_nord * num_kv_heads * pa::backward_key_tile() * head_dim;
+        if (half > 0) {
+            gs = grow_buffer(&plan->bwd_scratch, &plan->bwd_scratch_bytes, 2 * half * sizeof(float), st);
+            if (gs != PA_OK) return gs;
+        }
         pa::BwdParams2 bp{};
         bp.q = q; bp.k = k_cache; bp.v = v_cache; bp.out = out; bp.lse = lse; bp.dout = d_out;
         bp.drow = plan->bwd_drow; bp.dq = d_q; bp.dk = d_k_cache; bp.dv = d_v_cache;
         bp.seqs = plan->d_seqs; bp.block_tables = plan->d_bt;
         bp.key_units = (const pa::BwdKeyUnit*)plan->bwd_dev;
         bp.row_units = (const pa::BwdRowUnit*)((const char*)plan->bwd_dev + plan->bwd_row_off);
+        bp.scratch_k = half > 0 ? plan->bwd_scratch : nullptr;
+        bp.scratch_v = half > 0 ? plan->bwd_scratch + half : nullptr;
+        bp.slot_sums = (const pa::BwdSlotSum*)((const char*)plan->bwd_dev + plan->bwd_sums_off);
+        bp.slot_refs = (const int32_t*)((const char*)plan->bwd_dev + plan->bwd_refs_off);
         bp.table_width = plan->table_width; bp.page_size = plan->page_size;
         bp.hq = num_q_heads; bp.hkv = num_kv_heads; bp.group = G; bp.d = head_dim;
         bp.scale = scale; bp.scale_log2 = scale * 1.4426950408889634f;
         bp.causal = causal; bp.window = window;
-        cudaError_t e = pa::launch_backward_mma(bp, dtype, plan->bwd_nkey, plan->bwd_nrow, nq * num_q_heads, st);
+        bp.err = plan->d_err;
+        cudaError_t e = pa::launch_backward_mma(bp, dtype, plan->bwd_nkey, plan->bwd_nrow, nq * num_q_heads,
+                                                plan->bwd_nsums, st);
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "backward kernel launch failed: %s", cudaGetErrorString(e));
         plan->last_stream = st;
-        plan->last_launches = 1 + (plan->bwd_nkey > 0 ? 1 : 0) + (plan->bwd_nrow > 0 ? 1 : 0);
+        plan->last_launches = 1 + (plan->bwd_nkey > 0 ? 1 : 0) + (plan->bwd_nrow > 0 ? 1 : 0) + (plan->bwd_nsums > 0 ? 1 : 0);
         plan->last_kernels = PA_KERNEL_BACKWARD_TC;
         return ok();
     }

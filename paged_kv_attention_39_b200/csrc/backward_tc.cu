@@ -1,0 +1,390 @@
+// dK and dV of paged GQA attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
+// bf16 / fp16, head_dim == v_head_dim in {64, 128}, G dividing 128 (boostr
+// `standard_attention_bwd`; ruDNN's recompute-based backward). With P recomputed from Q, K and the
+// forward's lse (natural log), for every visible (row, key):
+//     P = exp(scale q.k - lse),  dP = dO . v,  dS = P (dP - Drow),  Drow = dO . O
+//     dV_k += P dO,   dK_k += scale dS q
+//
+// Key-major: a CTA owns 128 keys of one sequence and one KV head and walks the blocks of 128 rows
+// (128 / G queries x the G heads of the KV head, the prefill kernels' tile) that see those keys:
+//   S^T  = K Q^T       (M = 128 keys, N = 128 rows, K = D)   -> TMEM columns [0, 128)
+//   dP^T = V dO^T                                            -> TMEM columns [128, 256)
+//   P^T, dS^T in float32 by the four compute warps (thread = key), rounded to 16 bits and written
+//   over the first 64 columns of their own buffers
+//   dV  += P^T dO      (A = P^T from TMEM, B = dO, MN-major)  -> TMEM columns [256, 256 + D)
+//   dK  += dS^T Q      (A = dS^T from TMEM, B = Q)            -> TMEM columns [256 + D, 256 + 2D)
+// and at the end adds its finished rows once into the float32 gradient caches (the only writer of
+// those rows), or, for a tile the host marked ordered (it touches a shared page), writes them to
+// the scratch the ordered pass sums. dQ comes from the query-major mma.sync kernel.
+//
+//   warps 0..3  compute: row statistics from shared memory, masks, P and dS, the epilogue
+//   warp 4      loads: the K and V rows of the tile once (cp.async, straight from the pages, zeros
+//               past the sequence's end), then per row block the Q and dO rows (TMA, two stages)
+//               and the block's lse, Drow and visible key ranges (into shared memory)
+//   warp 5      TMEM owner and MMA issuer (one thread)
+//
+// Every wait on an mbarrier is bounded (Watchdog): a stalled pipeline sets the plan's error word and
+// the CTA leaves through its normal exit, freeing TMEM.
+#include <cudaTypedefs.h>
+
+#include "sm100.cuh"
+
+namespace pa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int KT = 128;  // keys per CTA
+constexpr int RB = 128;  // rows per block
+constexpr int QST = 2;   // Q / dO stages
+constexpr int kLoadWarp = 4, kMmaWarp = 5, kThreadsB = 6 * 32;
+constexpr uint32_t kTmemColsB = 512;
+constexpr uint64_t kWaitLimitNsB = 2000000000ull;
+constexpr float kLog2eB = 1.4426950408889634f;
+
+template <int D>
+struct BtcCfg {
+    static constexpr int KH = D / 64;       // 128-byte halves of a row
+    static constexpr int HALF = 128 * 128;  // bytes of one half of a 128-row tile
+    static constexpr int K = 0;
+    static constexpr int V = K + KH * HALF;
+    static constexpr int Q = V + KH * HALF;          // stage s: Q at Q + s * 2 * KH * HALF, dO after it
+    static constexpr int ROWS = Q + QST * 2 * KH * HALF;  // stage s: lse2, drow, lo, hi (128 each) + 2 ints
+    static constexpr int ROWS_STAGE = 4 * RB * 4 + 16;
+    static constexpr int BAR = ROWS + QST * ROWS_STAGE;
+    static constexpr int BYTES = BAR + 256;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(ALLOC <= 232448, "shared memory of one CTA");
+    static constexpr int T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D;
+    static constexpr int B_KV = 0, B_QFULL = 1, B_QEMPTY = B_QFULL + QST, B_SFULL = B_QEMPTY + QST,
+                         B_PFULL = B_SFULL + 1, B_DONE = B_PFULL + 1, B_COUNT = B_DONE + 1;
+};
+
+__device__ __forceinline__ int btc_swz(int row, int chunk) { return chunk ^ (row & 7); }
+
+}  // namespace
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreadsB, 1)
+    bwd_tc_dkdv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
+                       const BwdParams2 p) {
+    using L_ = BtcCfg<D>;
+    constexpr int KH = L_::KH;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr uint32_t IDESC_S = idesc_f16(KT, RB, kBf16, false, false);
+    constexpr uint32_t IDESC_G = idesc_f16(KT, D, kBf16, false, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L_::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L_::B_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Watchdog wd{abort_flag, p.err, kWaitLimitNsB};
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const BwdKeyUnit u = p.key_units[blockIdx.x];
+    const int kvh = blockIdx.y;
+    const SeqInfo si = p.seqs[u.seq];
+    const int G = p.group, qpt = RB / G;
+    const int64_t k0 = u.k0;
+    const int64_t kmax = min64(k0 + KT, si.L);       // keys [k0, kmax) exist
+    const int64_t base_pos = (int64_t)si.L - si.n;   // position of query 0
+    // queries that see at least one key of the tile: [j_lo, j_hi), in blocks of qpt
+    const int64_t j_lo = p.causal ? max64(0, k0 - base_pos) : 0;
+    const int64_t j_hi = p.window > 0 ? min64(si.n, kmax - 1 + p.window - base_pos) : si.n;
+    const int rb0 = (int)(j_lo / qpt);
+    const int nblk = j_hi > j_lo ? (int)((j_hi + qpt - 1) / qpt) - rb0 : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < L_::B_COUNT; ++i) {
+            uint32_t cnt = 1;
+            if (i == L_::B_KV) cnt = 32;        // every lane of the load warp (cp.async arrivals)
+            if (i == L_::B_PFULL) cnt = 128;    // the compute warps
+            mbar_init(&bars[i], cnt);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemColsB);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t s_base = smem_u32(smem);
+
+    if (warp == kLoadWarp) {
+        // ===================== loads =====================
+        if (lane == 0) {
+            tma_prefetch(&tmq);
+            tma_prefetch(&tmo);
+        }
+        // the row block's Q and dO rows (TMA) and its row statistics (plain loads) into stage s
+        auto load_block = [&](int i, int s) {
+            const int j0 = (rb0 + i) * qpt;
+            uint8_t* rows = smem + L_::ROWS + s * L_::ROWS_STAGE;
+            float* lse2 = reinterpret_cast<float*>(rows);
+            float* drow = lse2 + RB;
+            int* lo = reinterpret_cast<int*>(drow + RB);
+            int* hi = lo + RB;
+            int lo_max = 0, hi_min = INT32_MAX;
+            for (int r = lane; r < RB; r += 32) {
+                const int j = j0 + r / G;
+                const bool live = j < si.n;
+                const int64_t qr = (int64_t)(si.q_start + (live ? j : 0)) * p.hq + kvh * G + r % G;
+                const float l = live ? p.lse[qr] : neg_inf();
+                const bool has = live && l != neg_inf();
+                const int64_t pos = base_pos + j;
+                const int64_t a = p.window > 0 ? max64(0, pos - p.window + 1) : 0;
+                const int64_t b = p.causal ? min64(si.L, pos + 1) : si.L;
+                lse2[r] = has ? l * kLog2eB : 0.f;
+                drow[r] = has ? p.drow[qr] : 0.f;
+                lo[r] = has ? (int)a : 0;
+                hi[r] = has ? (int)b : 0;
+                lo_max = max(lo_max, lo[r]);
+                hi_min = min(hi_min, hi[r]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                lo_max = max(lo_max, __shfl_xor_sync(0xffffffffu, lo_max, o));
+                hi_min = min(hi_min, __shfl_xor_sync(0xffffffffu, hi_min, o));
+            }
+            if (lane == 0) {
+                hi[RB] = lo_max;  // every row sees [lo_max, hi_min)
+                hi[RB + 1] = hi_min;
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars[L_::B_QFULL + s], 2 * KH * L_::HALF);
+                uint8_t* qs = smem + L_::Q + s * 2 * KH * L_::HALF;
+                for (int h = 0; h < KH; ++h) {
+                    tma_load_3d(qs + h * L_::HALF, &tmq, &bars[L_::B_QFULL + s], h * 64, kvh * G, si.q_start + j0);
+                    tma_load_3d(qs + (KH + h) * L_::HALF, &tmo, &bars[L_::B_QFULL + s], h * 64, kvh * G,
+                                si.q_start + j0);
+                }
+            }
+            __syncwarp();
+        };
+        bool ok = true;
+        for (int i = 0; i < nblk && i < QST; ++i) load_block(i, i);
+        // the tile's K and V rows, 16-byte pieces straight from their pages (zeros past the end),
+        // 128-byte swizzled like the TMA boxes
+        {
+            const T* kc = static_cast<const T*>(p.k);
+            const T* vc = static_cast<const T*>(p.v);
+            const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+            const int ps = p.page_size;
+            const int64_t rstride = (int64_t)p.hkv * D;
+            for (int idx = lane; idx < KT * (D / 8); idx += 32) {
+                const int r = idx / (D / 8), c = idx % (D / 8);
+                const int64_t t = k0 + r;
+                const bool valid = t < kmax;
+                const int64_t off = valid ? ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D : 0;
+                const int h = c >> 3, ch = c & 7;
+                const int dst = h * L_::HALF + r * 128 + btc_swz(r, ch) * 16;
+                cp_async_16(smem + L_::K + dst, kc + off + c * 8, valid);
+                cp_async_16(smem + L_::V + dst, vc + off + c * 8, valid);
+            }
+            cp_async_wait<0>();
+            fence_proxy_async_smem();  // the pieces are read by the tensor core
+            mbar_arrive(&bars[L_::B_KV]);
+        }
+        for (int i = QST; ok && i < nblk; ++i) {
+            const int s = i % QST;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_QEMPTY + s], ((i / QST) - 1) & 1, wd, 21));
+            if (ok) load_block(i, s);
+        }
+        if (lane == 0 && *abort_flag) {
+            const uint64_t t0 = globaltimer_ns();
+            for (int i = max(0, nblk - QST); i < nblk; ++i)
+                while (!mbar_try_wait(&bars[L_::B_QFULL + i % QST], (i / QST) & 1) && globaltimer_ns() - t0 < kWaitLimitNsB) {}
+        }
+    } else if (warp == kMmaWarp) {
+        // ===================== MMA issuer =====================
+        const uint64_t dK = sdesc_sw128(s_base + L_::K, 16, 1024);
+        const uint64_t dV = sdesc_sw128(s_base + L_::V, 16, 1024);
+        bool ok = nblk == 0 || __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_KV], 0, wd, 22));
+        for (int i = 0; ok && i < nblk; ++i) {
+            const int s = i % QST;
+            // S^T and dP^T of this block overwrite P^T / dS^T of the previous one: its products are done
+            if (i > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_DONE], (i - 1) & 1, wd, 23));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_QFULL + s], (i / QST) & 1, wd, 24));
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t qs = s_base + L_::Q + s * 2 * KH * L_::HALF;
+            const uint32_t os = qs + KH * L_::HALF;
+            if (lane == 0) {
+                const uint64_t dQk = sdesc_sw128(qs, 16, 1024), dOk = sdesc_sw128(os, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L_::HALF + (kk & 3) * 32;
+                    mma_f16_ss(tmem + L_::T_ST, desc_add(dK, off), desc_add(dQk, off), IDESC_S, kk > 0);
+                    mma_f16_ss(tmem + L_::T_DPT, desc_add(dV, off), desc_add(dOk, off), IDESC_S, kk > 0);
+                }
+                mma_commit(&bars[L_::B_SFULL]);
+            }
+            __syncwarp();
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL], i & 1, wd, 25));
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                // rows are the contraction: 16 rows = 8 TMEM columns of P^T / dS^T, 2 KB of dO / Q
+                const uint64_t dOn = sdesc_sw128(os, L_::HALF, 1024), dQn = sdesc_sw128(qs, L_::HALF, 1024);
+#pragma unroll
+                for (int kk = 0; kk < RB / 16; ++kk) {
+                    const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+                    mma_f16_ts(tmem + L_::T_DV, tmem + L_::T_ST + kk * 8, desc_add(dOn, kk * 16 * 128), IDESC_G, acc);
+                    mma_f16_ts(tmem + L_::T_DK, tmem + L_::T_DPT + kk * 8, desc_add(dQn, kk * 16 * 128), IDESC_G, acc);
+                }
+                mma_commit(&bars[L_::B_DONE]);
+                mma_commit(&bars[L_::B_QEMPTY + s]);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ===================== compute: thread = key =====================
+        const int r0 = warp * 32;  // this warp's TMEM lanes (keys k0 + r0 ..)
+        const uint32_t lane_off = (uint32_t)r0 << 16;
+        const int64_t t = k0 + r0 + lane;  // this thread's key
+        const int64_t tw0 = k0 + r0, tw1 = k0 + r0 + 31;
+        bool ok = true;
+        for (int i = 0; i < nblk; ++i) {
+            const int s = i % QST;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_QFULL + s], (i / QST) & 1, wd, 26)) && ok;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_SFULL], i & 1, wd, 27)) && ok;
+            tc_fence_after();
+            const uint8_t* rows = smem + L_::ROWS + s * L_::ROWS_STAGE;
+            const float* lse2 = reinterpret_cast<const float*>(rows);
+            const float* drow = lse2 + RB;
+            const int* lo = reinterpret_cast<const int*>(drow + RB);
+            const int* hi = lo + RB;
+            // every key of the warp seen by every row of the block: no per-element mask
+            const bool full = tw1 < kmax && tw0 >= hi[RB] && tw1 < hi[RB + 1];
+#pragma unroll 1
+            for (int c = 0; c < RB / 32; ++c) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tmem + L_::T_ST + lane_off + c * 32, sv);
+                tmem_ld32(tmem + L_::T_DPT + lane_off + c * 32, dv);
+                tmem_ld_wait(sv);
+                tmem_regs_ready(dv);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float pr[2], ds[2];
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        const int r = c * 32 + 2 * e + x;
+                        const bool vis = full || (t < kmax && t >= lo[r] && t < hi[r]);
+                        const float pv = fast_exp2(fmaf(__uint_as_float(sv[2 * e + x]), p.scale_log2, -lse2[r]));
+                        pr[x] = vis ? pv : 0.f;
+                        ds[x] = vis ? pv * (__uint_as_float(dv[2 * e + x]) - drow[r]) : 0.f;
+                    }
+                    pk[e] = pack2<T>(pr[0], pr[1]);
+                    dk[e] = pack2<T>(ds[0], ds[1]);
+                }
+                // 32 row-columns -> 16 TMEM columns, over columns already read
+                tmem_st16(tmem + L_::T_ST + lane_off + c * 16, pk);
+                tmem_st16(tmem + L_::T_DPT + lane_off + c * 16, dk);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[L_::B_PFULL]);
+        }
+        // ---- epilogue: the tile's finished dK / dV rows ----
+        if (nblk > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_DONE], (nblk - 1) & 1, wd, 28));
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        if (ok && nblk > 0) {
+            float* dk_row = nullptr;
+            float* dv_row = nullptr;
+            if (u.ord >= 0) {
+                const int64_t srow = ((int64_t)u.ord * p.hkv + kvh) * KT + r0 + lane;
+                dk_row = p.scratch_k + srow * D;
+                dv_row = p.scratch_v + srow * D;
+            } else if (t < kmax) {
+                const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+                const int64_t row = (((int64_t)bt[t / p.page_size] * p.page_size + t % p.page_size) * p.hkv + kvh) * D;
+                dk_row = p.dk + row;
+                dv_row = p.dv + row;
+            }
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32], b[32];
+                tmem_ld32(tmem + L_::T_DV + lane_off + c * 32, a);
+                tmem_ld32(tmem + L_::T_DK + lane_off + c * 32, b);
+                tmem_ld_wait(a);
+                tmem_regs_ready(b);
+                if (!dk_row) continue;
+                float4* kd = reinterpret_cast<float4*>(dk_row + c * 32);
+                float4* vd = reinterpret_cast<float4*>(dv_row + c * 32);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float4 kv4 = make_float4(__uint_as_float(b[4 * e]) * p.scale, __uint_as_float(b[4 * e + 1]) * p.scale,
+                                                   __uint_as_float(b[4 * e + 2]) * p.scale, __uint_as_float(b[4 * e + 3]) * p.scale);
+                    const float4 vv4 = make_float4(__uint_as_float(a[4 * e]), __uint_as_float(a[4 * e + 1]),
+                                                   __uint_as_float(a[4 * e + 2]), __uint_as_float(a[4 * e + 3]));
+                    if (u.ord >= 0) {  // scratch rows: written, summed by the ordered pass
+                        kd[e] = kv4;
+                        vd[e] = vv4;
+                    } else {  // this CTA is the row's only writer: one add onto the caller's zeroed cache
+                        float4 k_old = kd[e], v_old = vd[e];
+                        kd[e] = make_float4(k_old.x + kv4.x, k_old.y + kv4.y, k_old.z + kv4.z, k_old.w + kv4.w);
+                        vd[e] = make_float4(v_old.x + vv4.x, v_old.y + vv4.y, v_old.z + vv4.z, v_old.w + vv4.w);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemColsB);
+    }
+}
+
+namespace {
+
+template <typename T, int D>
+cudaError_t launch_btc(const BwdParams2& p, int num_key_units, int64_t num_queries, cudaStream_t st) {
+    using L_ = BtcCfg<D>;
+    const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+    const int G = p.group, qpt = RB / G;
+    CUtensorMap tq, to;  // Q and dO, boxes of 128 rows (qpt queries x G heads) and 64 columns
+    if (!make_map(&tq, bf16, p.q, D, p.hq, (uint64_t)num_queries, G, qpt) ||
+        !make_map(&to, bf16, p.dout, D, p.hq, (uint64_t)num_queries, G, qpt))
+        return cudaErrorInvalidValue;
+    auto kern = bwd_tc_dkdv_kernel<T, D>;
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !(configured >> dev & 1ull)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L_::ALLOC);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured |= 1ull << dev;
+    }
+    kern<<<dim3(num_key_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int backward_tc_key_tile() { return KT; }
+
+cudaError_t launch_backward_tc_dkdv(const BwdParams2& p, pa_dtype dt, int num_key_units, int64_t num_queries,
+                                    cudaStream_t st) {
+    if (num_key_units == 0) return cudaSuccess;
+    if (dt == PA_BF16)
+        return p.d == 64 ? launch_btc<__nv_bfloat16, 64>(p, num_key_units, num_queries, st)
+                         : launch_btc<__nv_bfloat16, 128>(p, num_key_units, num_queries, st);
+    return p.d == 64 ? launch_btc<__half, 64>(p, num_key_units, num_queries, st)
+                     : launch_btc<__half, 128>(p, num_key_units, num_queries, st);
+}
+
+}  // namespace pa

@@ -40,8 +40,16 @@ struct PrefillUnit {
 
 // Backward on the tensor cores: a 64-key tile of sequence `seq` starting at key k0 (dK/dV
 // kernel), and queries j0 .. j1-1 of a sequence, at most 16 rows per KV head (dQ kernel).
+// ord >= 0: the tile touches a page that another key of the plan shares; its finished rows go
+// to scratch tile `ord` and the ordered pass adds them (in sequence order) instead of the tile.
 struct BwdKeyUnit {
-    int32_t seq, k0;
+    int32_t seq, k0, ord, pad;
+};
+// Ordered pass: cache row `slot` (page * page_size + slot in page) receives the scratch rows
+// refs[begin .. begin + count) (scratch tile * 64 + row), summed in that order.
+struct BwdSlotSum {
+    int64_t slot;
+    int32_t begin, count;
 };
 struct BwdRowUnit {
     int32_t seq, j0, j1, pad;
@@ -62,9 +70,14 @@ struct BwdParams2 {
     const int32_t* block_tables;
     const BwdKeyUnit* key_units;
     const BwdRowUnit* row_units;
+    float* scratch_k;             // [ordered tiles, Hkv, 64, D] finished rows of ordered tiles
+    float* scratch_v;
+    const BwdSlotSum* slot_sums;  // ordered pass work list
+    const int32_t* slot_refs;
     int32_t table_width, page_size, hq, hkv, group, d;
     float scale, scale_log2;
     int32_t causal, window;
+    int* err;  // device error word of the plan (bounded waits of the tcgen05 kernel)
 };
 
 // Everything a kernel needs; passed by value.
@@ -124,8 +137,13 @@ cudaError_t launch_append(const void* new_k, const void* new_v, void* k_cache, v
 bool backward_mma_supported(pa_dtype dt, int d, int dv, int group);
 int backward_key_tile();
 int backward_row_block();
+// tcgen05 dK/dV kernel (backward_tc.cu): keys per CTA and launch; its 128-row blocks are read
+// through TMA maps over Q and dO of num_queries rows.
+int backward_tc_key_tile();
+cudaError_t launch_backward_tc_dkdv(const BwdParams2& p, pa_dtype dt, int num_key_units, int64_t num_queries,
+                                    cudaStream_t st);
 cudaError_t launch_backward_mma(const BwdParams2& p, pa_dtype dt, int num_key_units, int num_row_units, int64_t rows,
-                                cudaStream_t st);
+                                int num_slot_sums, cudaStream_t st);
 // Sparse top-K block selection (sparse.cu).
 cudaError_t launch_sparse_scores(const void* q, const void* k, float* scores, int32_t sw, const SeqInfo* seqs,
                                  const int32_t* q2seq, const int32_t* block_tables, int32_t table_width,

@@ -229,4 +229,10 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16, bool a
 }
 
 }  // namespace sm100
+
+// Host: a 3-D TMA map over a row-major [d2][d1][d0] tensor of 16-bit elements with boxes of
+// {64, b1, b2} and the 128-byte swizzle (defined in prefill.cu).
+bool make_map(CUtensorMap* m, bool bf16, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b1,
+              uint32_t b2);
+
 }  // namespace pa

@@ -103,9 +103,10 @@ def test_backward_tensor_core_shapes(orc, hq, hkv, d, ps, causal, window, dtype)
 
 
 def test_backward_tensor_core_shared_pages_and_launches(orc):
-    """bf16 on the tensor-core path with two sequences sharing their first pages: each CTA adds its
-    finished key rows once, so the shared slots receive both sequences' gradients. The path runs
-    three kernels (Drow, dK/dV, dQ)."""
+    """bf16 on the tensor-core path with two sequences sharing their first pages: the key tiles that
+    touch the shared pages hand their rows to the ordered pass, which adds each shared slot's rows
+    in sequence order, so the shared slots receive both sequences' gradients. The path runs four
+    kernels (Drow, dK/dV, the ordered pass, dQ)."""
     wl = W.make_gqa("share_tc", 6, [150, 150], [30, 30], 8, 2, 64, 64, 16, torch.bfloat16)
     s = wl.sched
     s.block_tables[1, :3] = s.block_tables[0, :3]  # keys 0..47 shared
@@ -121,7 +122,7 @@ def test_backward_tensor_core_shared_pages_and_launches(orc):
     dk = torch.zeros(k.shape, dtype=torch.float32, device="cuda")
     dv = torch.zeros(v.shape, dtype=torch.float32, device="cuda")
     pa.pa_backward(plan, q, k, v, out, lse, dout.cuda(), dq, dk, dv, wl.scale, True, 0)
-    assert pa.pa_plan_get_info(plan)["last_launches"] == 3
+    assert pa.pa_plan_get_info(plan)["last_launches"] == 4
     torch.cuda.synchronize()
     plan.close()
     rq, rk, rv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s.seq_lens, s.query_offsets,
@@ -129,6 +130,29 @@ def test_backward_tensor_core_shared_pages_and_launches(orc):
     close(dq.cpu(), rq, torch.bfloat16, "dq")
     close(dk.cpu(), rk, torch.bfloat16, "dk")
     close(dv.cpu(), rv, torch.bfloat16, "dv")
+
+
+@pytest.mark.parametrize("ps,shared_pages", [(16, 5), (64, 2), (128, 1)])
+def test_backward_tensor_core_shared_pages_same_bits(orc, ps, shared_pages):
+    """Three sequences share a prefix of pages (a common prompt) and one more lists a page twice:
+    every shared cache slot is summed by the ordered pass in sequence order, so two runs give the
+    same bits, and the gradients match the oracle."""
+    wl = W.make_gqa("share_bits", 8, [400, 260, 333, 200], [60, 130, 1, 40], 16, 4, 128, 128, ps, torch.bfloat16)
+    s = wl.sched
+    for j in (1, 2):
+        s.block_tables[j, :shared_pages] = s.block_tables[0, :shared_pages]
+    used = (200 + ps - 1) // ps
+    if used >= 2:
+        s.block_tables[3, used - 1] = s.block_tables[3, 0]  # keys of its first and last page share slots
+    runs = [run_backward(wl, torch.Generator().manual_seed(21)) for _ in range(2)]
+    for a, b in zip(runs[0][1:], runs[1][1:]):
+        assert torch.equal(torch.nan_to_num(a, nan=0.0), torch.nan_to_num(b, nan=0.0))
+    dout, dq, dk, dv = runs[0]
+    rq, rk, rv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s.seq_lens, s.query_offsets,
+                                        s.block_tables, ps, wl.scale, True, 0)
+    close(dq, rq, torch.bfloat16, f"dq ps{ps}")
+    close(dk, rk, torch.bfloat16, f"dk ps{ps}")
+    close(dv, rv, torch.bfloat16, f"dv ps{ps}")
 
 
 def test_backward_tensor_core_deterministic():

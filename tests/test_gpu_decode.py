@@ -63,6 +63,40 @@ def test_decode_head_dim_256(orc, hq, hkv, qn):
         check(wl, out, lse, *ref, tag=f"d256 G{hq // hkv} n{qn} chunk {kv_chunk}")
 
 
+def test_split_rows_plan_reused(orc):
+    """One plan, five calls with other queries and split sizes (the workspace and the cached work
+    lists reused across calls), each against the oracle; split rows go through the merge kernel."""
+    wl = small_decode(5, batch=12, lmin=200, lmax=3000)
+    s = wl.sched
+    plan = pa.plan_for(wl)
+    for i, kv_chunk in enumerate((64, 64, 100, 0, 64)):
+        q = W.randn(tuple(wl.q.shape), 100 + i, 1, wl.q.dtype)
+        ref = orc.attention(q, wl.k_cache, wl.v_cache, s.seq_lens, s.query_offsets, s.block_tables, s.page_size,
+                            wl.scale, wl.causal, wl.window)
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk, plan=plan, q=q)
+        k = pa.pa_plan_get_info(plan)["last_kernels"]
+        assert k & pa.PA_KERNEL_DECODE_TC and (kv_chunk == 0 or k & pa.PA_KERNEL_MERGE), k
+        check(wl, out, lse, *ref, tag=f"call {i} chunk {kv_chunk}")
+    assert pa.pa_plan_device_status(plan) == 0
+    plan.close()
+
+
+def test_split_rows_of_both_decode_kernels_in_one_call(orc):
+    """Rows of the tensor-core decode kernel and of the CUDA-core kernel (5 queries x 4 heads per
+    KV head, pages of 48 that the tcgen05 prefill kernel does not take) split in the same call and
+    merged by one merge launch."""
+    lens = [700, 1300, 450, 900, 1000]
+    qs = [1, 5, 1, 5, 1]
+    wl = W.make_gqa("two_merges", 6, lens, qs, 32, 8, 128, 128, 48, torch.bfloat16)
+    ref = orc.run(wl)
+    plan = pa.plan_for(wl)
+    out, lse = run_gqa(wl, kv_chunk=96, plan=plan)
+    k = pa.pa_plan_get_info(plan)["last_kernels"]
+    assert k & pa.PA_KERNEL_DECODE_TC and k & pa.PA_KERNEL_SIMT and k & pa.PA_KERNEL_MERGE, k
+    plan.close()
+    check(wl, out, lse, *ref, tag="tensor-core and CUDA-core splits")
+
+
 @pytest.mark.parametrize("window", [1, 7, 100, 5000])
 def test_decode_window(orc, window):
     wl = small_decode(3, window=window, qn=2, hq=16, hkv=4, lmin=2, lmax=900)
