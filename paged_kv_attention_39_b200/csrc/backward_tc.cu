@@ -65,6 +65,53 @@ __device__ __forceinline__ int btc_swz(int row, int chunk) { return chunk ^ (row
 
 }  // namespace
 
+// P^T and dS^T of one key (thread = TMEM lane) against the 128 rows of a block, 16-bit, written
+// over the first 64 columns of the S^T and dP^T buffers. The rows' statistics come from shared
+// memory four at a time (one 16-byte load per statistic for four rows); MASKED adds each row's
+// visible key range [lo, hi) (a row without keys has lo = hi = 0).
+template <typename T, bool MASKED>
+__device__ __forceinline__ void btc_probs(uint32_t t_lane, const float* lse2, const float* drow, const int* lo,
+                                          const int* hi, int64_t t, float scale_log2) {
+#pragma unroll 1
+    for (int c = 0; c < RB / 32; ++c) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(t_lane + BtcCfg<64>::T_ST + c * 32, sv);
+        tmem_ld32(t_lane + BtcCfg<64>::T_DPT + c * 32, dv);
+        tmem_ld_wait(sv);
+        tmem_regs_ready(dv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // rows c*32 + 4q .. + 3
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + c * 32 + 4 * q);
+            const float4 d4 = *reinterpret_cast<const float4*>(drow + c * 32 + 4 * q);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dr[4] = {d4.x, d4.y, d4.z, d4.w};
+            bool vis[4] = {true, true, true, true};
+            if (MASKED) {
+                const int4 a4 = *reinterpret_cast<const int4*>(lo + c * 32 + 4 * q);
+                const int4 b4 = *reinterpret_cast<const int4*>(hi + c * 32 + 4 * q);
+                vis[0] = t >= a4.x && t < b4.x;
+                vis[1] = t >= a4.y && t < b4.y;
+                vis[2] = t >= a4.z && t < b4.z;
+                vis[3] = t >= a4.w && t < b4.w;
+            }
+            float pr[4], ds[4];
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float pv = fast_exp2(fmaf(__uint_as_float(sv[4 * q + x]), scale_log2, -lv[x]));
+                pr[x] = vis[x] ? pv : 0.f;
+                ds[x] = vis[x] ? pv * (__uint_as_float(dv[4 * q + x]) - dr[x]) : 0.f;
+            }
+            pk[2 * q] = pack2<T>(pr[0], pr[1]);
+            pk[2 * q + 1] = pack2<T>(pr[2], pr[3]);
+            dk[2 * q] = pack2<T>(ds[0], ds[1]);
+            dk[2 * q + 1] = pack2<T>(ds[2], ds[3]);
+        }
+        // 32 row-columns -> 16 TMEM columns, over columns already read
+        tmem_st16(t_lane + BtcCfg<64>::T_ST + c * 16, pk);
+        tmem_st16(t_lane + BtcCfg<64>::T_DPT + c * 16, dk);
+    }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreadsB, 1)
     bwd_tc_dkdv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
@@ -262,34 +309,13 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             const float* drow = lse2 + RB;
             const int* lo = reinterpret_cast<const int*>(drow + RB);
             const int* hi = lo + RB;
-            // every key of the warp seen by every row of the block: no per-element mask
+            // every key of the warp seen by every row of the block: no per-element mask (keys past the
+            // sequence's end are outside every row's range, so they always take the masked path)
             const bool full = tw1 < kmax && tw0 >= hi[RB] && tw1 < hi[RB + 1];
-#pragma unroll 1
-            for (int c = 0; c < RB / 32; ++c) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tmem + L_::T_ST + lane_off + c * 32, sv);
-                tmem_ld32(tmem + L_::T_DPT + lane_off + c * 32, dv);
-                tmem_ld_wait(sv);
-                tmem_regs_ready(dv);
-                uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    float pr[2], ds[2];
-#pragma unroll
-                    for (int x = 0; x < 2; ++x) {
-                        const int r = c * 32 + 2 * e + x;
-                        const bool vis = full || (t < kmax && t >= lo[r] && t < hi[r]);
-                        const float pv = fast_exp2(fmaf(__uint_as_float(sv[2 * e + x]), p.scale_log2, -lse2[r]));
-                        pr[x] = vis ? pv : 0.f;
-                        ds[x] = vis ? pv * (__uint_as_float(dv[2 * e + x]) - drow[r]) : 0.f;
-                    }
-                    pk[e] = pack2<T>(pr[0], pr[1]);
-                    dk[e] = pack2<T>(ds[0], ds[1]);
-                }
-                // 32 row-columns -> 16 TMEM columns, over columns already read
-                tmem_st16(tmem + L_::T_ST + lane_off + c * 16, pk);
-                tmem_st16(tmem + L_::T_DPT + lane_off + c * 16, dk);
-            }
+            if (__all_sync(0xffffffffu, full))
+                btc_probs<T, false>(tmem + lane_off, lse2, drow, lo, hi, t, p.scale_log2);
+            else
+                btc_probs<T, true>(tmem + lane_off, lse2, drow, lo, hi, t, p.scale_log2);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars[L_::B_PFULL]);
