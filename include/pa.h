@@ -245,9 +245,9 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
  *   d_k_cache            [pages, page_size, Hkv, D] float32, ADDED INTO (zero it first)
  *   d_v_cache            [pages, page_size, Hkv, Dv] float32, ADDED INTO (zero it first)
  * bf16 / fp16 with head_dim == v_head_dim in {64, 128} and G = num_q_heads / num_kv_heads dividing
- * 128 and at most 16 run on the tensor cores: dK/dV key-major on tcgen05 (a CTA per 128 keys and KV
- * head), dQ query-major on mma.sync; P and dS are rounded to the input type before the gradient
- * products. Every key's dK/dV row is summed by one CTA and added once; where a page is referenced
+ * 128 run on the tensor cores (tcgen05): dK/dV key-major (a CTA per 128 keys and KV head), dQ
+ * query-major (a CTA per 128 rows = 128 / G queries x G heads and KV head); P and dS are rounded to
+ * the input type before the gradient products. Every key's dK/dV row is summed by one CTA and added once; where a page is referenced
  * more than once in the plan (sequences sharing a prefix, a page listed twice), the rows of every key
  * tile that touches it are summed per cache slot in (sequence, key) order by an ordered pass (ruDNN's
  * atomic-free "ordered" history pass), so the result repeats bit for bit in every case (three

@@ -1077,8 +1077,8 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
 }
 
 // Work lists of the tensor-core backward for one (group size, causal, window), longest first:
-// the 64-key tiles of every sequence that some query sees (cost: the rows that see them) for the
-// dK/dV kernel, and blocks of at most 16 rows (cost: the keys they see) for the dQ kernel. Key tiles
+// the 128-key tiles of every sequence that some query sees (cost: the rows that see them) for the
+// dK/dV kernel, and blocks of at most 128 rows (cost: the keys they see) for the dQ kernel. Key tiles
 // that touch a page referenced more than once in the plan (sequences sharing a prefix page, or a
 // page listed twice) are "ordered": their rows go to scratch, and the ordered pass's list gives
 // every cache row those tiles touch with its scratch rows in (sequence, key) order. One upload; the

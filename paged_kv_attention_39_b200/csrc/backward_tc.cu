@@ -1,4 +1,4 @@
-// dK and dV of paged GQA attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
+// dK, dV and dQ of paged GQA attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA),
 // bf16 / fp16, head_dim == v_head_dim in {64, 128}, G dividing 128 (boostr
 // `standard_attention_bwd`; ruDNN's recompute-based backward). With P recomputed from Q, K and the
 // forward's lse (natural log), for every visible (row, key):
@@ -15,7 +15,7 @@
 //   dK  += dS^T Q      (A = dS^T from TMEM, B = Q)            -> TMEM columns [256 + D, 256 + 2D)
 // and at the end adds its finished rows once into the float32 gradient caches (the only writer of
 // those rows), or, for a tile the host marked ordered (it touches a shared page), writes them to
-// the scratch the ordered pass sums. dQ comes from the query-major mma.sync kernel.
+// the scratch the ordered pass sums. dQ comes from the query-major kernel at the end of this file.
 //
 //   warps 0..3  compute: row statistics from shared memory, masks, P and dS, the epilogue
 //   warp 4      loads: the K and V rows of the tile once (cp.async, straight from the pages, zeros
@@ -374,6 +374,294 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// dQ on tcgen05, query-major: a CTA owns one 128-row block (128/G queries x the G heads of a KV
+// head) and walks the keys its rows see, 64 per step:
+//   S  = Q K^T,  dP = dO V^T   (M = 128 rows, N = 64 keys)  -> TMEM, two buffers each (step & 1)
+//   dS = P (dP - Drow), P = exp2(S scale_log2 - lse2)       by the compute warps (thread = row; the
+//        row's lse, Drow and visible key range live in registers), 16-bit into a shared-memory
+//        buffer of its own (step & 1)
+//   dQ += dS K                 (A = dS from shared memory, B = K, MN-major) -> TMEM [256, 256 + D)
+// The score products of a step go into the buffer the step before last used (its dS is already in
+// shared memory), so they overlap the compute warps' work on the previous step, and the dQ product
+// of a step runs while the compute warps work on the next one. The finished rows are scaled and
+// written once.
+//   warps 0..3  compute and the epilogue
+//   warp 4      loads: Q and dO of the block (TMA), the K and V rows of each step (cp.async, one page
+//               lookup per row, zeros past the sequence's end) into a ring of stages
+//   warp 5      TMEM owner and MMA issuer
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+constexpr int QKB = 64;   // keys per step of the dQ kernel
+constexpr int QKVST = 3;  // K/V stages
+
+template <int D>
+struct BqCfg {
+    static constexpr int KH = D / 64;
+    static constexpr int HALF_R = 128 * 128;  // one 64-column half of the 128-row Q / dO tiles
+    static constexpr int HALF_K = QKB * 128;  // one 64-column half of a 64-key K / V tile
+    static constexpr int Q = 0;
+    static constexpr int O = Q + KH * HALF_R;
+    static constexpr int K = O + KH * HALF_R;                 // stage s: K at K + s * 2 * KH * HALF_K, V after
+    static constexpr int DS = K + QKVST * 2 * KH * HALF_K;    // two dS buffers: 128 rows x 64 keys, 16-bit
+    static constexpr int BAR = DS + 2 * 128 * 128;
+    static constexpr int BYTES = BAR + 256;
+    static constexpr int ALLOC = BYTES + 1024;
+    static_assert(ALLOC <= 232448, "shared memory of one CTA");
+    static constexpr int T_S = 0, T_DP = 128, T_DQ = 256;    // S_b at b * 64, dP_b at 128 + b * 64
+    static constexpr int B_QFULL = 0, B_KVFULL = 1, B_KVEMPTY = B_KVFULL + QKVST, B_SFULL = B_KVEMPTY + QKVST,
+                         B_PFULL = B_SFULL + 2, B_DSFREE = B_PFULL + 2, B_DQFULL = B_DSFREE + 2,
+                         B_COUNT = B_DQFULL + 1;
+};
+
+}  // namespace
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreadsB, 1)
+    bwd_tc_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
+                     const BwdParams2 p) {
+    using L_ = BqCfg<D>;
+    constexpr int KH = L_::KH;
+    constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+    constexpr uint32_t IDESC_S = idesc_f16(128, QKB, kBf16, false, false);
+    constexpr uint32_t IDESC_DQ = idesc_f16(128, D, kBf16, false, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L_::BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + L_::B_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const Watchdog wd{abort_flag, p.err, kWaitLimitNsB};
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const BwdRowUnit u = p.row_units[blockIdx.x];
+    const int kvh = blockIdx.y;
+    const SeqInfo si = p.seqs[u.seq];
+    const int G = p.group;
+    const int64_t base_pos = (int64_t)si.L - si.n;
+    // keys any of the block's rows can see: [lo, hi), in steps of QKB
+    const int64_t p_first = base_pos + u.j0, p_last = base_pos + u.j1 - 1;
+    const int64_t lo = p.window > 0 ? max64(0, p_first - p.window + 1) : 0;
+    const int64_t hi = p.causal ? min64(si.L, p_last + 1) : si.L;
+    const int nsteps = hi > lo ? (int)((hi - lo + QKB - 1) / QKB) : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < L_::B_COUNT; ++i) {
+            uint32_t cnt = 1;
+            if (i >= L_::B_KVFULL && i < L_::B_KVFULL + QKVST) cnt = 32;  // every lane of the load warp
+            if (i == L_::B_PFULL || i == L_::B_PFULL + 1) cnt = 128;  // the compute warps
+            mbar_init(&bars[i], cnt);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+        fence_proxy_async_smem();
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemColsB);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t s_base = smem_u32(smem);
+
+    if (warp == kLoadWarp) {
+        // ===================== loads =====================
+        if (nsteps > 0 && lane == 0) {
+            tma_prefetch(&tmq);
+            tma_prefetch(&tmo);
+            mbar_arrive_expect_tx(&bars[L_::B_QFULL], 2 * KH * L_::HALF_R);
+            for (int h = 0; h < KH; ++h) {
+                tma_load_3d(smem + L_::Q + h * L_::HALF_R, &tmq, &bars[L_::B_QFULL], h * 64, kvh * G,
+                            si.q_start + u.j0);
+                tma_load_3d(smem + L_::O + h * L_::HALF_R, &tmo, &bars[L_::B_QFULL], h * 64, kvh * G,
+                            si.q_start + u.j0);
+            }
+        }
+        const T* kc = static_cast<const T*>(p.k);
+        const T* vc = static_cast<const T*>(p.v);
+        const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+        const int ps = p.page_size;
+        const int64_t rstride = (int64_t)p.hkv * D;
+        bool ok = true;
+        // step j's rows go into stage j % QKVST; the stage of the step before is handed over once its
+        // copies have landed (every lane waits for its own, fences them for the tensor core, arrives)
+        for (int j = 0; ok && j < nsteps; ++j) {
+            const int st = j % QKVST;
+            if (j >= QKVST)
+                ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_KVEMPTY + st], ((j / QKVST) - 1) & 1, wd, 31));
+            if (!ok) break;
+            uint8_t* ks = smem + L_::K + st * 2 * KH * L_::HALF_K;
+            uint8_t* vs = ks + KH * L_::HALF_K;
+            for (int r = lane; r < QKB; r += 32) {
+                const int64_t t = lo + (int64_t)j * QKB + r;
+                const bool valid = t < hi;
+                const int64_t off = valid ? ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D : 0;
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    const int h = c >> 3, ch = c & 7;
+                    const int dst = h * L_::HALF_K + r * 128 + btc_swz(r, ch) * 16;
+                    cp_async_16(ks + dst, kc + off + c * 8, valid);
+                    cp_async_16(vs + dst, vc + off + c * 8, valid);
+                }
+            }
+            cp_async_commit();
+            if (j >= 1) {
+                cp_async_wait<1>();
+                fence_proxy_async_smem();
+                mbar_arrive(&bars[L_::B_KVFULL + (j - 1) % QKVST]);
+            }
+        }
+        if (ok && nsteps > 0) {
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&bars[L_::B_KVFULL + (nsteps - 1) % QKVST]);
+        } else {
+            cp_async_wait<0>();
+        }
+        if (lane == 0 && *abort_flag && nsteps > 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars[L_::B_QFULL], 0) && globaltimer_ns() - t0 < kWaitLimitNsB) {}
+        }
+    } else if (warp == kMmaWarp) {
+        // ===================== MMA issuer =====================
+        const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
+        const uint64_t dO = sdesc_sw128(s_base + L_::O, 16, 1024);
+        bool ok = nsteps == 0 || __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_QFULL], 0, wd, 32));
+        // dQ += dS_j K_j (dS of step j in buffer j & 1, K in stage j % QKVST)
+        auto issue_dq = [&](int j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL + (j & 1)], (j >> 1) & 1, wd, 33));
+            if (!ok) return;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t ks = s_base + L_::K + (j % QKVST) * 2 * KH * L_::HALF_K;
+                const uint64_t dA = sdesc_sw128(s_base + L_::DS + (j & 1) * 128 * 128, 16, 1024);
+                const uint64_t dB = sdesc_sw128(ks, L_::HALF_K, 1024);  // K as (keys x D), MN-major
+#pragma unroll
+                for (int kk = 0; kk < QKB / 16; ++kk)
+                    mma_f16_ss(tmem + L_::T_DQ, desc_add(dA, kk * 32), desc_add(dB, kk * 16 * 128), IDESC_DQ,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars[L_::B_DSFREE + (j & 1)]);
+                mma_commit(&bars[L_::B_KVEMPTY + j % QKVST]);
+                if (j == nsteps - 1) mma_commit(&bars[L_::B_DQFULL]);
+            }
+            __syncwarp();
+        };
+        for (int j = 0; ok && j < nsteps; ++j) {
+            const int st = j % QKVST, b = j & 1;
+            // buffer b held S and dP of step j - 2, read by the compute warps before they marked P
+            if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL + b], ((j - 2) >> 1) & 1, wd, 34));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_KVFULL + st], (j / QKVST) & 1, wd, 35));
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t ks = s_base + L_::K + st * 2 * KH * L_::HALF_K;
+                const uint64_t dK = sdesc_sw128(ks, 16, 1024), dV = sdesc_sw128(ks + KH * L_::HALF_K, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off_r = (kk >> 2) * L_::HALF_R + (kk & 3) * 32;
+                    const uint32_t off_k = (kk >> 2) * L_::HALF_K + (kk & 3) * 32;
+                    mma_f16_ss(tmem + L_::T_S + b * QKB, desc_add(dQ, off_r), desc_add(dK, off_k), IDESC_S, kk > 0);
+                    mma_f16_ss(tmem + L_::T_DP + b * QKB, desc_add(dO, off_r), desc_add(dV, off_k), IDESC_S, kk > 0);
+                }
+                mma_commit(&bars[L_::B_SFULL + b]);
+            }
+            __syncwarp();
+            if (j >= 1) issue_dq(j - 1);  // the previous step's dQ, while this step's scores run
+        }
+        if (ok && nsteps > 0) issue_dq(nsteps - 1);
+    } else {
+        // ===================== compute: thread = row =====================
+        const int r = warp * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const int R = (u.j1 - u.j0) * G;  // live rows
+        const bool live = r < R;
+        const int64_t qrow = (int64_t)(si.q_start + u.j0 + (live ? r / G : 0)) * p.hq + kvh * G + (live ? r % G : 0);
+        const float l = live ? p.lse[qrow] : neg_inf();
+        const bool has = live && l != neg_inf();
+        const float lse2 = has ? l * kLog2eB : 0.f;
+        const float drow = has ? p.drow[qrow] : 0.f;
+        const int64_t pos = base_pos + u.j0 + (live ? r / G : 0);
+        const int64_t row_lo = has ? (p.window > 0 ? max64(0, pos - p.window + 1) : 0) : 0;
+        const int64_t row_hi = has ? (p.causal ? min64(si.L, pos + 1) : si.L) : 0;
+        uint8_t* dsbuf = smem + L_::DS;
+        bool ok = true;
+        for (int j = 0; j < nsteps; ++j) {
+            const int b = j & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_SFULL + b], (j >> 1) & 1, wd, 36)) && ok;
+            tc_fence_after();
+            const int64_t t0 = lo + (int64_t)j * QKB;
+            // columns outside [row_lo, row_hi) are masked: off_lo = t0 - row_lo, off_hi = t0 - row_hi
+            const int off_lo = (int)max64(min64(t0 - row_lo, 1 << 20), -(1 << 20));
+            const int off_hi = (int)max64(min64(t0 - row_hi, 1 << 20), -(1 << 20));
+            uint32_t dk[32];
+#pragma unroll
+            for (int c = 0; c < QKB / 32; ++c) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tmem + L_::T_S + b * QKB + lane_off + c * 32, sv);
+                tmem_ld32(tmem + L_::T_DP + b * QKB + lane_off + c * 32, dv);
+                tmem_ld_wait(sv);
+                tmem_regs_ready(dv);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    float ds[2];
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        const int k = c * 32 + 2 * e + x;
+                        const bool vis = k + off_lo >= 0 && k + off_hi < 0;
+                        const float pv = fast_exp2(fmaf(__uint_as_float(sv[2 * e + x]), p.scale_log2, -lse2));
+                        ds[x] = vis ? pv * (__uint_as_float(dv[2 * e + x]) - drow) : 0.f;
+                    }
+                    dk[c * 16 + e] = pack2<T>(ds[0], ds[1]);
+                }
+            }
+            // the dS buffer was last read by the dQ product of step j - 2
+            if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_DSFREE + b], ((j - 2) >> 1) & 1, wd, 37)) && ok;
+            // row r of dS: 64 keys = 128 bytes, 16-byte chunk ch at position ch ^ (r & 7)
+            uint8_t* row = dsbuf + b * 128 * 128 + r * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(row + (btc_swz(r, ch) << 4)) =
+                    make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[L_::B_PFULL + b]);
+        }
+        // ---- epilogue: the block's dQ rows, scaled, written once ----
+        if (nsteps > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_DQFULL], 0, wd, 38));
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        float* dst = p.dq + qrow * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            if (ok && nsteps > 0) {
+                tmem_ld32(tmem + L_::T_DQ + lane_off + c * 32, v);
+                tmem_ld_wait(v);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0u;
+            }
+            if (live && ok) {
+                float4* d4 = reinterpret_cast<float4*>(dst + c * 32);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    d4[e] = make_float4(__uint_as_float(v[4 * e]) * p.scale, __uint_as_float(v[4 * e + 1]) * p.scale,
+                                        __uint_as_float(v[4 * e + 2]) * p.scale, __uint_as_float(v[4 * e + 3]) * p.scale);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemColsB);
+    }
+}
+
 namespace {
 
 template <typename T, int D>
@@ -401,7 +689,31 @@ cudaError_t launch_btc(const BwdParams2& p, int num_key_units, int64_t num_queri
 
 }  // namespace
 
+template <typename T, int D>
+cudaError_t launch_bq(const BwdParams2& p, int num_row_units, int64_t num_queries, cudaStream_t st) {
+    using L_ = BqCfg<D>;
+    const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
+    const int G = p.group, qpt = RB / G;
+    CUtensorMap tq, to;
+    if (!make_map(&tq, bf16, p.q, D, p.hq, (uint64_t)num_queries, G, qpt) ||
+        !make_map(&to, bf16, p.dout, D, p.hq, (uint64_t)num_queries, G, qpt))
+        return cudaErrorInvalidValue;
+    auto kern = bwd_tc_dq_kernel<T, D>;
+    static unsigned long long configured = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !(configured >> dev & 1ull)) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L_::ALLOC);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) configured |= 1ull << dev;
+    }
+    kern<<<dim3(num_row_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, p);
+    return cudaGetLastError();
+}
+
 int backward_tc_key_tile() { return KT; }
+int backward_tc_row_block() { return RB; }
 
 cudaError_t launch_backward_tc_dkdv(const BwdParams2& p, pa_dtype dt, int num_key_units, int64_t num_queries,
                                     cudaStream_t st) {
@@ -411,6 +723,17 @@ cudaError_t launch_backward_tc_dkdv(const BwdParams2& p, pa_dtype dt, int num_ke
                          : launch_btc<__nv_bfloat16, 128>(p, num_key_units, num_queries, st);
     return p.d == 64 ? launch_btc<__half, 64>(p, num_key_units, num_queries, st)
                      : launch_btc<__half, 128>(p, num_key_units, num_queries, st);
+}
+
+
+cudaError_t launch_backward_tc_dq(const BwdParams2& p, pa_dtype dt, int num_row_units, int64_t num_queries,
+                                  cudaStream_t st) {
+    if (num_row_units == 0) return cudaSuccess;
+    if (dt == PA_BF16)
+        return p.d == 64 ? launch_bq<__nv_bfloat16, 64>(p, num_row_units, num_queries, st)
+                         : launch_bq<__nv_bfloat16, 128>(p, num_row_units, num_queries, st);
+    return p.d == 64 ? launch_bq<__half, 64>(p, num_row_units, num_queries, st)
+                     : launch_bq<__half, 128>(p, num_row_units, num_queries, st);
 }
 
 }  // namespace pa

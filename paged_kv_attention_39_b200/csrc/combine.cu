@@ -4,15 +4,17 @@
 // Parts without keys carry lse_i = -inf and weight 0; a row whose parts are all empty gets
 // out = 0 and lse = -inf.
 //
-// One warp per (query, head). The weights go to shared memory first; then each lane owns four
-// consecutive output columns (float4) and walks the parts four at a time, so that every lane
-// keeps several independent loads in flight -- the merge is a short, latency-bound HBM read.
+// One warp per (query, head, 128 output columns). The weights go to shared memory first; then each
+// lane owns four consecutive output columns (float4) and walks the parts eight at a time, so that
+// every lane keeps several independent loads in flight -- the merge is a short, latency-bound read
+// of parts the attention kernel has just written (mostly L2 hits).
 #include "device_common.cuh"
 
 namespace pa {
 
 constexpr int kCombineWarps = 4;
 constexpr int kCombineMaxSplits = 1024;
+constexpr int kCombineCols = 128;  // output columns per warp (wider rows spread over more CTAs)
 
 template <typename T>
 __device__ __forceinline__ void store4(T* dst, float4 v);
@@ -49,31 +51,49 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y * kCombineWarps + warp;
     if (h >= p.hq) return;
+    const int c_lo = blockIdx.z * kCombineCols;  // this warp's output columns [c_lo, c_hi)
+    const int c_hi = min(p.dv, c_lo + kCombineCols);
     const int n = cu.nsplit;
     const float* ls = p.ws_lse + (int64_t)cu.part_base * p.hq + h;
-    float m = neg_inf();
-    for (int i = lane; i < n; i += 32) m = fmaxf(m, ls[(int64_t)i * p.hq]);
+    const float kLog2e = 1.4426950408889634f;
+    // Up to 32 parts: each lane keeps its part's logsumexp, so the max and the sum need one round
+    // of loads; more parts are read again for the sum.
+    const float my_l = lane < n ? ls[(int64_t)lane * p.hq] : neg_inf();
+    float m = my_l;
+    for (int i = lane + 32; i < n; i += 32) m = fmaxf(m, ls[(int64_t)i * p.hq]);
     m = warp_max(m);
     const int64_t row = (int64_t)cu.query * p.hq + h;
     T* o = static_cast<T*>(p.out) + row * p.dv;
     if (m == neg_inf()) {
-        for (int c = lane; c < p.dv; c += 32) o[c] = from_f32<T>(0.f);
-        if (lane == 0) p.lse[row] = m;
+        for (int c = c_lo + lane; c < c_hi; c += 32) o[c] = from_f32<T>(0.f);
+        if (lane == 0 && blockIdx.z == 0) p.lse[row] = m;
         return;
     }
-    const float kLog2e = 1.4426950408889634f;
-    float sum = 0.f;
-    for (int i = lane; i < n; i += 32) sum += fast_exp2((ls[(int64_t)i * p.hq] - m) * kLog2e);
+    float sum = lane < n ? fast_exp2((my_l - m) * kLog2e) : 0.f;
+    for (int i = lane + 32; i < n; i += 32) sum += fast_exp2((ls[(int64_t)i * p.hq] - m) * kLog2e);
     sum = warp_sum(sum);
     const float lse = m + __logf(sum);
-    for (int i = lane; i < n; i += 32) wts[warp][i] = fast_exp2((ls[(int64_t)i * p.hq] - lse) * kLog2e);
+    if (lane < n) wts[warp][lane] = fast_exp2((my_l - lse) * kLog2e);
+    for (int i = lane + 32; i < n; i += 32) wts[warp][i] = fast_exp2((ls[(int64_t)i * p.hq] - lse) * kLog2e);
     __syncwarp();
     const float* op = p.ws_o + ((int64_t)cu.part_base * p.hq + h) * p.dv;
     const int64_t step = (int64_t)p.hq * p.dv;
     if ((p.dv & 3) == 0) {
-        for (int c = lane * 4; c < p.dv; c += 128) {
+        for (int c = c_lo + lane * 4; c < c_hi; c += 128) {
             float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
             int i = 0;
+            for (; i + 8 <= n; i += 8) {  // eight parts in flight
+                float4 b[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) b[x] = *reinterpret_cast<const float4*>(op + (i + x) * step + c);
+#pragma unroll
+                for (int x = 0; x < 8; x += 4) {
+                    fma4(a0, wts[warp][i + x + 0], b[x + 0]);
+                    fma4(a1, wts[warp][i + x + 1], b[x + 1]);
+                    fma4(a2, wts[warp][i + x + 2], b[x + 2]);
+                    fma4(a3, wts[warp][i + x + 3], b[x + 3]);
+                }
+            }
             for (; i + 4 <= n; i += 4) {
                 const float4 b0 = *reinterpret_cast<const float4*>(op + (i + 0) * step + c);
                 const float4 b1 = *reinterpret_cast<const float4*>(op + (i + 1) * step + c);
@@ -90,18 +110,19 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
             store4<T>(o + c, r);
         }
     } else {
-        for (int c = lane; c < p.dv; c += 32) {
+        for (int c = c_lo + lane; c < c_hi; c += 32) {
             float acc = 0.f;
             for (int i = 0; i < n; ++i) acc += wts[warp][i] * op[i * step + c];
             o[c] = from_f32<T>(acc);
         }
     }
-    if (lane == 0) p.lse[row] = lse;
+    if (lane == 0 && blockIdx.z == 0) p.lse[row] = lse;
 }
 
 cudaError_t launch_combine(const AttnParams& p, pa_dtype dt, cudaStream_t st) {
     if (p.num_cunits == 0) return cudaSuccess;
-    const dim3 grid(p.num_cunits, (p.hq + kCombineWarps - 1) / kCombineWarps), block(kCombineWarps * 32);
+    const dim3 grid(p.num_cunits, (p.hq + kCombineWarps - 1) / kCombineWarps, (p.dv + kCombineCols - 1) / kCombineCols);
+    const dim3 block(kCombineWarps * 32);
     switch (dt) {
         case PA_F32: combine_kernel<float><<<grid, block, 0, st>>>(p); break;
         case PA_BF16: combine_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(p); break;

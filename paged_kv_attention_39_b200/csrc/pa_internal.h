@@ -38,8 +38,8 @@ struct PrefillUnit {
     int32_t kvh, pad0, pad1, pad2;
 };
 
-// Backward on the tensor cores: a 64-key tile of sequence `seq` starting at key k0 (dK/dV
-// kernel), and queries j0 .. j1-1 of a sequence, at most 16 rows per KV head (dQ kernel).
+// Backward on the tensor cores: a 128-key tile of sequence `seq` starting at key k0 (dK/dV
+// kernel), and queries j0 .. j1-1 of a sequence, at most 128 rows per KV head (dQ kernel).
 // ord >= 0: the tile touches a page that another key of the plan shares; its finished rows go
 // to scratch tile `ord` and the ordered pass adds them (in sequence order) instead of the tile.
 struct BwdKeyUnit {
@@ -142,6 +142,10 @@ int backward_row_block();
 int backward_tc_key_tile();
 cudaError_t launch_backward_tc_dkdv(const BwdParams2& p, pa_dtype dt, int num_key_units, int64_t num_queries,
                                     cudaStream_t st);
+// tcgen05 dQ kernel (backward_tc.cu): rows per CTA (128: 128 / G queries x G heads) and launch.
+int backward_tc_row_block();
+cudaError_t launch_backward_tc_dq(const BwdParams2& p, pa_dtype dt, int num_row_units, int64_t num_queries,
+                                  cudaStream_t st);
 cudaError_t launch_backward_mma(const BwdParams2& p, pa_dtype dt, int num_key_units, int num_row_units, int64_t rows,
                                 int num_slot_sums, cudaStream_t st);
 // Sparse top-K block selection (sparse.cu).

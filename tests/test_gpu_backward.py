@@ -1,5 +1,5 @@
 """GPU backward against the fp64 oracle's backward: the tensor-core path (bf16 / fp16, D in {64, 128},
-at most 16 heads per group; deterministic dK/dV) and the float32 CUDA-core kernel (other shapes)."""
+G dividing 128; deterministic dK/dV) and the float32 CUDA-core kernel (other shapes)."""
 import pytest
 import torch
 
@@ -85,10 +85,11 @@ def test_backward_shared_prefix_page_accumulates(orc):
     (16, 1, 64, 32, True, 100, torch.bfloat16),  # sixteen heads per group, window
     (8, 2, 128, 16, False, 0, torch.bfloat16),
     (8, 4, 64, 128, True, 0, torch.float16),
+    (32, 1, 64, 16, True, 0, torch.bfloat16),   # 32 heads per group: 4 queries per 128-row block
 ])
 def test_backward_tensor_core_shapes(orc, hq, hkv, d, ps, causal, window, dtype):
-    """The tensor-core backward (key-major dK/dV, query-major dQ): chunked prefills with history,
-    a prefill from empty history, many 64-key tiles and 16-row blocks, ragged ends."""
+    """The tensor-core backward (key-major dK/dV, query-major dQ, both on tcgen05): chunked prefills
+    with history, a prefill from empty history, many 128-key tiles and 128-row blocks, ragged ends."""
     wl = W.make_gqa("bwd_tc", 5, [300, 513, 64, 1000], [100, 200, 64, 17], hq, hkv, d, d, ps, dtype,
                     causal=causal, window=window)
     g = torch.Generator().manual_seed(11)
