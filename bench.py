@@ -217,18 +217,26 @@ def run_ours(args, ws, rank, local):
     traffic = kernel_traffic("decode.cu", "decode_mma_kernel")
 
     # ---- end to end through the public API with host buffers -------------------------------
-    # A decode loop as a serving engine runs it: every step copies its queries in from pinned
-    # host memory, uploads its own plan (a new schedule per step: lengths grow, pages move), runs
-    # pa_forward and reads out and lse back, and the host waits for that result before the next
-    # step; the next step's plan is built (pa_plan_create + pa_plan_prepare: validation, work
-    # list, their uploads queued on the stream) while the current step runs on the GPU. The K
-    # steps are timed as one region on the stream, so every copy, upload and host gap between
-    # steps is inside it.
+    # A decode loop as a serving engine with asynchronous scheduling runs it: every step copies
+    # its queries in from pinned host memory, uploads its own plan (a new schedule per step:
+    # lengths grow, pages move), runs pa_forward and reads out and lse back into pinned host
+    # memory. Two steps are in flight: step i+1's query upload (on a copy stream) and plan build
+    # (pa_plan_create + pa_plan_prepare: validation, work list, their uploads queued on the
+    # compute stream) overlap step i's attention, and step i's download (on the copy stream)
+    # overlaps step i+1's attention; the host waits for step i's result before it issues step
+    # i+2. Device buffers are double-buffered so no copy touches a buffer a running step uses.
+    # The K steps are timed as one region on the compute stream, joined with the copy stream at
+    # the end, so every copy, upload and host gap is inside it.
     q_host = wl.q.pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lse_host = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+    lse_host = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+    q_dev = [q, torch.empty_like(q)]
+    out_dev = [out, torch.empty_like(out)]
+    lse_dev = [lse, torch.empty_like(lse)]
     e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 200))
     uploaded = 0
+    main = torch.cuda.current_stream(dev)
+    copy_stream = torch.cuda.Stream(dev)
 
     def next_plan():
         pn = pa.plan_for(wl, device=local)
@@ -238,20 +246,34 @@ def run_ours(args, ws, rank, local):
     def e2e_loop(n):
         nonlocal uploaded
         cur = next_plan()
-        done = torch.cuda.Event()
+        h2d = [torch.cuda.Event(), torch.cuda.Event()]
+        fwd = [torch.cuda.Event(), torch.cuda.Event()]
+        d2h = [torch.cuda.Event(), torch.cuda.Event()]
         for i in range(n):
-            q.copy_(q_host, non_blocking=True)
-            pa.pa_forward(cur, q, k, v, out, lse, wl.scale, wl.causal, wl.window)
-            out_host.copy_(out, non_blocking=True)
-            lse_host.copy_(lse, non_blocking=True)
-            done.record()
-            # host work overlapping this step's GPU work: the next plan, and this plan's release
-            # (its frees are ordered on the stream after the step)
+            b = i & 1
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(fwd[b])  # step i-2 has finished reading q_dev[b]
+                q_dev[b].copy_(q_host, non_blocking=True)
+                h2d[b].record(copy_stream)
+            main.wait_event(h2d[b])
+            pa.pa_forward(cur, q_dev[b], k, v, out_dev[b], lse_dev[b], wl.scale, wl.causal, wl.window)
+            fwd[b].record(main)
+            with torch.cuda.stream(copy_stream):
+                copy_stream.wait_event(fwd[b])
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                lse_host[b].copy_(lse_dev[b], non_blocking=True)
+                d2h[b].record(copy_stream)
+            # host work overlapping the GPU: the next plan, and this plan's release (its frees are
+            # ordered on the compute stream after the step)
             nxt = next_plan() if i + 1 < n else None
             uploaded = pa.pa_plan_get_info(cur)["uploaded_bytes"]
             cur.close()
-            done.synchronize()  # the step's result is on the host
+            if i >= 1:
+                d2h[b ^ 1].synchronize()  # step i-1's result is on the host
             cur = nxt
+        d2h[(n - 1) & 1].synchronize()
+        main.wait_stream(copy_stream)
 
     e2e_ms = float("nan")
     if e2e_steps:
@@ -313,12 +335,13 @@ def run_ours(args, ws, rank, local):
             "value": round(e2e_val, 2),
             "unit": "GB/s",
             "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size() + uploaded),
-            "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size() + lse_host.numel() * 4),
+            "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4),
             "ms_per_step": round(e2e_ms, 4),
-            "includes": "per step: H2D of Q from pinned memory, a new plan (pa_plan_create + pa_plan_prepare: "
-                        "schedule and work-list uploads), pa_forward, D2H of out and lse into pinned memory, host "
-                        "waits for the result; the next step's plan is built on the host while the step runs; K "
-                        "steps timed as one region",
+            "includes": "per step: H2D of Q from pinned memory (copy stream), a new plan (pa_plan_create + "
+                        "pa_plan_prepare: schedule and work-list uploads), pa_forward, D2H of out and lse into "
+                        "pinned memory (copy stream); two steps in flight (step i+1's upload and plan build "
+                        "overlap step i, step i's download overlaps step i+1; the host waits for step i's "
+                        "result before issuing step i+2); K steps timed as one region",
         },
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,

@@ -244,10 +244,14 @@ pa_status pa_append(pa_plan* plan, const void* new_k, const void* new_v, void* k
  *   d_q                  [N_q, Hq, D] float32, written
  *   d_k_cache            [pages, page_size, Hkv, D] float32, ADDED INTO (zero it first)
  *   d_v_cache            [pages, page_size, Hkv, Dv] float32, ADDED INTO (zero it first)
- * bf16 / fp16 with head_dim == v_head_dim in {64, 128} and G = num_q_heads / num_kv_heads dividing
- * 128 run on the tensor cores (tcgen05): dK/dV key-major (a CTA per 128 keys and KV head), dQ
- * query-major (a CTA per 128 rows = 128 / G queries x G heads and KV head); P and dS are rounded to
- * the input type before the gradient products. Every key's dK/dV row is summed by one CTA and added once; where a page is referenced
+ * bf16 / fp16 with head_dim == v_head_dim in {64, 128}, G = num_q_heads / num_kv_heads dividing
+ * 128, a page size that is a multiple of 16 and divides 128 or is a multiple of 128, fewer than 2^31
+ * cache rows and 16-byte aligned q, k_cache, v_cache, d_out, d_k_cache and d_v_cache run on the
+ * tensor cores (tcgen05, every operand moved by TMA, K / V one page box at a time): dK/dV key-major
+ * (a CTA per 128 keys and KV head, its finished rows added by TMA reduce-adds), dQ query-major (a CTA
+ * per 128 rows = 128 / G queries x G heads and KV head, on a second stream of the library that
+ * forks from and joins back into `stream`); P and dS are rounded to the input type before the
+ * gradient products. Every key's dK/dV row is summed by one CTA and added once; where a page is referenced
  * more than once in the plan (sequences sharing a prefix, a page listed twice), the rows of every key
  * tile that touches it are summed per cache slot in (sequence, key) order by an ordered pass (ruDNN's
  * atomic-free "ordered" history pass), so the result repeats bit for bit in every case (three

@@ -329,7 +329,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
         const int32_t base = nsplit > 1 ? (int32_t)slots : -1;
         if (nsplit > 1) {
             for (int32_t j = b.j0; j < b.j1; ++j)
-                cu.push_back({P->seqs[b.seq].q_start + j, base + (j - b.j0) * nsplit, nsplit, 0});
+                    cu.push_back({P->seqs[b.seq].q_start + j, base + (j - b.j0) * nsplit, nsplit, 0});
             slots += (int64_t)(b.j1 - b.j0) * nsplit;
         }
         for (int32_t i = 0; i < nsplit; ++i) {
@@ -1217,8 +1217,17 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
         return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
     const int32_t G = num_q_heads / num_kv_heads;
     cudaStream_t st = (cudaStream_t)stream;
-    // the tensor-core kernels index a sequence's rows (queries x G) in 32 bits
-    if (pa::backward_mma_supported(dtype, head_dim, v_head_dim, G) && nq * (int64_t)G < ((int64_t)1 << 31)) {
+    // The tensor-core kernels index a sequence's rows (queries x G) and the cache rows in 32 bits,
+    // load K / V one page box at a time (a page size that divides the 128-key tile or is a multiple
+    // of it) and move every operand by TMA (16-byte aligned bases).
+    const int64_t cache_rows = (int64_t)plan->num_pages * plan->page_size;
+    auto al16 = [](const void* x) { return ((uintptr_t)x & 15u) == 0; };
+    const bool tc_layout = plan->page_size % 16 == 0 &&
+                           (pa::backward_key_tile() % plan->page_size == 0 ||
+                            plan->page_size % pa::backward_key_tile() == 0) &&
+                           cache_rows < ((int64_t)1 << 31) && al16(q) && al16(k_cache) && al16(v_cache) &&
+                           al16(d_out) && al16(d_k_cache) && al16(d_v_cache);
+    if (pa::backward_mma_supported(dtype, head_dim, v_head_dim, G) && tc_layout && nq * (int64_t)G < ((int64_t)1 << 31)) {
         std::lock_guard<std::mutex> lock(plan->mu);
         if (plan->bwd_group != G || plan->bwd_causal != causal || plan->bwd_window != window) {
             pa_status bs = build_backward_lists(plan, G, causal, window, st);
@@ -1245,6 +1254,7 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
         bp.hq = num_q_heads; bp.hkv = num_kv_heads; bp.group = G; bp.d = head_dim;
         bp.scale = scale; bp.scale_log2 = scale * 1.4426950408889634f;
         bp.causal = causal; bp.window = window;
+        bp.num_pages = plan->num_pages;
         bp.err = plan->d_err;
         cudaError_t e = pa::launch_backward_mma(bp, dtype, plan->bwd_nkey, plan->bwd_nrow, nq * num_q_heads,
                                                 plan->bwd_nsums, st);

@@ -11,6 +11,8 @@
 //                      than once sums the scratch rows that map to it in sequence order and adds
 //                      the sum once, so shared pages give the same bits on every run.
 //   (backward_tc.cu)   dQ: query-major, each 128-row block's dQ summed in TMEM and written once.
+#include <mutex>
+
 #include "device_common.cuh"
 #include "pa_internal.h"
 
@@ -57,6 +59,40 @@ __global__ void __launch_bounds__(128) bwd_ordered_kernel(const BwdParams2 p, in
 // ---------------------------------------------------------------------------------------------
 namespace {
 
+// A non-blocking side stream of the library per device, with the two events of a fork/join.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+std::mutex& side_mutex() {
+    static std::mutex m;
+    return m;
+}
+
+// Called with side_mutex() held. Created on first use per device, kept for the process's life.
+cudaError_t side_stream(SideStream** out) {
+    static SideStream per_device[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    SideStream& s = per_device[dev];
+    if (!s.stream) {
+        e = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming);
+        if (e != cudaSuccess) {
+            if (s.fork) cudaEventDestroy(s.fork);
+            if (s.stream) cudaStreamDestroy(s.stream);
+            s = SideStream{};
+            return e;
+        }
+    }
+    *out = &s;
+    return cudaSuccess;
+}
+
 template <typename T, int D>
 cudaError_t bwd_launch_d(const BwdParams2& p, int num_key_units, int num_row_units, int64_t rows, int num_sums,
                          cudaStream_t st) {
@@ -65,18 +101,37 @@ cudaError_t bwd_launch_d(const BwdParams2& p, int num_key_units, int num_row_uni
                                                                    static_cast<const T*>(p.dout), p.drow, rows, D);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (num_key_units > 0) {
+    // dK/dV (then the ordered pass) on the caller's stream and dQ on a side stream, so that the
+    // second kernel's CTAs fill the SMs the first one's last wave leaves idle; both only read
+    // what the Drow kernel and the caller wrote. The side stream forks from and joins back into
+    // the caller's stream through events, so the call stays stream-ordered (and capturable).
+    const bool fork = num_key_units > 0 && num_row_units > 0;
+    std::unique_lock<std::mutex> lk(side_mutex(), std::defer_lock);
+    SideStream* side = nullptr;
+    if (fork) {
+        lk.lock();  // one fork/join at a time: each wait pairs with its own record
+        e = side_stream(&side);
+        if (e != cudaSuccess) return e;
+        e = cudaEventRecord(side->fork, st);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+        if (e != cudaSuccess) return e;
+    }
+    if (num_key_units > 0)
         e = launch_backward_tc_dkdv(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, num_key_units,
                                     rows / p.hq, st);
-        if (e != cudaSuccess) return e;
-    }
-    if (num_sums > 0)
+    if (e == cudaSuccess && num_sums > 0) {
         bwd_ordered_kernel<D><<<dim3((num_sums + 3) / 4, p.hkv), 128, 0, st>>>(p, num_sums, backward_tc_key_tile());
-    if (num_row_units > 0) {
-        e = launch_backward_tc_dq(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, num_row_units,
-                                  rows / p.hq, st);
-        if (e != cudaSuccess) return e;
+        e = cudaGetLastError();
     }
+    if (e == cudaSuccess && num_row_units > 0)
+        e = launch_backward_tc_dq(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, num_row_units,
+                                  rows / p.hq, fork ? side->stream : st);
+    if (fork) {  // joined on every path, so that a capture on the caller's stream never ends unjoined
+        cudaError_t j = cudaEventRecord(side->join, side->stream);
+        if (j == cudaSuccess) j = cudaStreamWaitEvent(st, side->join, 0);
+        if (e == cudaSuccess) e = j;
+    }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

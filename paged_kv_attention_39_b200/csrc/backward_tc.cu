@@ -56,6 +56,7 @@ struct BtcCfg {
     static constexpr int BYTES = BAR + 256;
     static constexpr int ALLOC = BYTES + 1024;
     static_assert(ALLOC <= 232448, "shared memory of one CTA");
+    static_assert(2 * (D / 32) * 128 * 128 <= QST * 2 * KH * HALF, "dK / dV staging fits over the Q / dO stages");
     static constexpr int T_ST = 0, T_DPT = 128, T_DV = 256, T_DK = 256 + D;
     static constexpr int B_KV = 0, B_QFULL = 1, B_QEMPTY = B_QFULL + QST, B_SFULL = B_QEMPTY + QST,
                          B_PFULL = B_SFULL + 1, B_DONE = B_PFULL + 1, B_COUNT = B_DONE + 1;
@@ -115,6 +116,8 @@ __device__ __forceinline__ void btc_probs(uint32_t t_lane, const float* lse2, co
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreadsB, 1)
     bwd_tc_dkdv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
+                       const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                       const __grid_constant__ CUtensorMap tmdk, const __grid_constant__ CUtensorMap tmdv,
                        const BwdParams2 p) {
     using L_ = BtcCfg<D>;
     constexpr int KH = L_::KH;
@@ -146,7 +149,6 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     if (tid == 0) {
         for (int i = 0; i < L_::B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i == L_::B_KV) cnt = 32;        // every lane of the load warp (cp.async arrivals)
             if (i == L_::B_PFULL) cnt = 128;    // the compute warps
             mbar_init(&bars[i], cnt);
         }
@@ -216,37 +218,44 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             }
             __syncwarp();
         };
+        // the tile's K and V rows: one TMA box per page (and 64-column half), landing 128-byte
+        // swizzled at rows b * kbox .. of the tile. Boxes past the sequence's last page are not
+        // loaded: those keys are masked (P and dS select zero), and their dK / dV rows are zero.
+        const int ps = p.page_size, kbox = ps < KT ? ps : KT;
+        const int nbox = (int)((kmax - k0 + kbox - 1) / kbox);  // at most KT / 16 boxes
+        {
+            const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+            int my_row = 0;
+            if (lane < nbox) {
+                const int64_t key = k0 + (int64_t)lane * kbox;
+                my_row = bt[key / ps] * ps + (int)(key % ps);
+            }
+            if (lane == 0) {
+                tma_prefetch(&tmk);
+                tma_prefetch(&tmv);
+                mbar_arrive_expect_tx(&bars[L_::B_KV], (uint32_t)(nbox * kbox * 128 * KH * 2));
+            }
+            for (int b = 0; b < nbox; ++b) {
+                const int row = __shfl_sync(0xffffffffu, my_row, b);
+                if (lane == 0)
+                    for (int h = 0; h < KH; ++h) {
+                        tma_load_3d(smem + L_::K + h * L_::HALF + b * kbox * 128, &tmk, &bars[L_::B_KV], h * 64, kvh, row);
+                        tma_load_3d(smem + L_::V + h * L_::HALF + b * kbox * 128, &tmv, &bars[L_::B_KV], h * 64, kvh, row);
+                    }
+            }
+            __syncwarp();
+        }
         bool ok = true;
         for (int i = 0; i < nblk && i < QST; ++i) load_block(i, i);
-        // the tile's K and V rows, 16-byte pieces straight from their pages (zeros past the end),
-        // 128-byte swizzled like the TMA boxes
-        {
-            const T* kc = static_cast<const T*>(p.k);
-            const T* vc = static_cast<const T*>(p.v);
-            const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
-            const int ps = p.page_size;
-            const int64_t rstride = (int64_t)p.hkv * D;
-            for (int idx = lane; idx < KT * (D / 8); idx += 32) {
-                const int r = idx / (D / 8), c = idx % (D / 8);
-                const int64_t t = k0 + r;
-                const bool valid = t < kmax;
-                const int64_t off = valid ? ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D : 0;
-                const int h = c >> 3, ch = c & 7;
-                const int dst = h * L_::HALF + r * 128 + btc_swz(r, ch) * 16;
-                cp_async_16(smem + L_::K + dst, kc + off + c * 8, valid);
-                cp_async_16(smem + L_::V + dst, vc + off + c * 8, valid);
-            }
-            cp_async_wait<0>();
-            fence_proxy_async_smem();  // the pieces are read by the tensor core
-            mbar_arrive(&bars[L_::B_KV]);
-        }
         for (int i = QST; ok && i < nblk; ++i) {
             const int s = i % QST;
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_QEMPTY + s], ((i / QST) - 1) & 1, wd, 21));
             if (ok) load_block(i, s);
         }
         if (lane == 0 && *abort_flag) {
+            // leave no copy in flight into this CTA's shared memory (bounded, ignoring the flag)
             const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&bars[L_::B_KV], 0) && globaltimer_ns() - t0 < kWaitLimitNsB) {}
             for (int i = max(0, nblk - QST); i < nblk; ++i)
                 while (!mbar_try_wait(&bars[L_::B_QFULL + i % QST], (i / QST) & 1) && globaltimer_ns() - t0 < kWaitLimitNsB) {}
         }
@@ -324,19 +333,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (nblk > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_DONE], (nblk - 1) & 1, wd, 28));
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
-        if (ok && nblk > 0) {
-            float* dk_row = nullptr;
-            float* dv_row = nullptr;
-            if (u.ord >= 0) {
-                const int64_t srow = ((int64_t)u.ord * p.hkv + kvh) * KT + r0 + lane;
-                dk_row = p.scratch_k + srow * D;
-                dv_row = p.scratch_v + srow * D;
-            } else if (t < kmax) {
-                const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
-                const int64_t row = (((int64_t)bt[t / p.page_size] * p.page_size + t % p.page_size) * p.hkv + kvh) * D;
-                dk_row = p.dk + row;
-                dv_row = p.dv + row;
-            }
+        if (ok && nblk > 0 && u.ord >= 0) {
+            // a tile touching a shared page: its rows go to scratch, summed later by the ordered pass
+            const int64_t srow = ((int64_t)u.ord * p.hkv + kvh) * KT + r0 + lane;
+            float* dk_row = p.scratch_k + srow * D;
+            float* dv_row = p.scratch_v + srow * D;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t a[32], b[32];
@@ -344,25 +345,61 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                 tmem_ld32(tmem + L_::T_DK + lane_off + c * 32, b);
                 tmem_ld_wait(a);
                 tmem_regs_ready(b);
-                if (!dk_row) continue;
                 float4* kd = reinterpret_cast<float4*>(dk_row + c * 32);
                 float4* vd = reinterpret_cast<float4*>(dv_row + c * 32);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const float4 kv4 = make_float4(__uint_as_float(b[4 * e]) * p.scale, __uint_as_float(b[4 * e + 1]) * p.scale,
-                                                   __uint_as_float(b[4 * e + 2]) * p.scale, __uint_as_float(b[4 * e + 3]) * p.scale);
-                    const float4 vv4 = make_float4(__uint_as_float(a[4 * e]), __uint_as_float(a[4 * e + 1]),
-                                                   __uint_as_float(a[4 * e + 2]), __uint_as_float(a[4 * e + 3]));
-                    if (u.ord >= 0) {  // scratch rows: written, summed by the ordered pass
-                        kd[e] = kv4;
-                        vd[e] = vv4;
-                    } else {  // this CTA is the row's only writer: one add onto the caller's zeroed cache
-                        float4 k_old = kd[e], v_old = vd[e];
-                        kd[e] = make_float4(k_old.x + kv4.x, k_old.y + kv4.y, k_old.z + kv4.z, k_old.w + kv4.w);
-                        vd[e] = make_float4(v_old.x + vv4.x, v_old.y + vv4.y, v_old.z + vv4.z, v_old.w + vv4.w);
-                    }
+                    kd[e] = make_float4(__uint_as_float(b[4 * e]) * p.scale, __uint_as_float(b[4 * e + 1]) * p.scale,
+                                        __uint_as_float(b[4 * e + 2]) * p.scale, __uint_as_float(b[4 * e + 3]) * p.scale);
+                    vd[e] = make_float4(__uint_as_float(a[4 * e]), __uint_as_float(a[4 * e + 1]),
+                                        __uint_as_float(a[4 * e + 2]), __uint_as_float(a[4 * e + 3]));
                 }
             }
+        } else if (ok && nblk > 0) {
+            // This CTA is the only writer of its rows: stage them in shared memory (over the Q / dO
+            // stages, idle now) as 128-byte swizzled 32-column blocks of the 128 rows, then add them
+            // onto the caller's cache with TMA reduce-adds, one box per page and column block (one
+            // add per element; keys past the sequence's end add zeros to their own page's rows).
+            constexpr int CB = 128 * 128;  // one 32-column block of the 128 rows, float32
+            uint8_t* stg_v = smem + L_::Q;
+            uint8_t* stg_k = stg_v + (D / 32) * CB;
+            const int r = r0 + lane;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32], b[32];
+                tmem_ld32(tmem + L_::T_DV + lane_off + c * 32, a);
+                tmem_ld32(tmem + L_::T_DK + lane_off + c * 32, b);
+                tmem_ld_wait(a);
+                tmem_regs_ready(b);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const int off = c * CB + r * 128 + (btc_swz(r, ch) << 4);
+                    *reinterpret_cast<float4*>(stg_v + off) =
+                        make_float4(__uint_as_float(a[4 * ch]), __uint_as_float(a[4 * ch + 1]),
+                                    __uint_as_float(a[4 * ch + 2]), __uint_as_float(a[4 * ch + 3]));
+                    *reinterpret_cast<float4*>(stg_k + off) =
+                        make_float4(__uint_as_float(b[4 * ch]) * p.scale, __uint_as_float(b[4 * ch + 1]) * p.scale,
+                                    __uint_as_float(b[4 * ch + 2]) * p.scale, __uint_as_float(b[4 * ch + 3]) * p.scale);
+                }
+            }
+            fence_proxy_async_smem();  // the staged rows are read by the TMA engine
+            __syncwarp();
+            if (lane == 0) {
+                const int ps = p.page_size, rbox = ps < 32 ? ps : 32;
+                const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
+                for (int b0 = 0; b0 < 32; b0 += rbox) {  // this warp's 32 rows, one box per page
+                    const int64_t key = k0 + r0 + b0;
+                    if (key >= kmax) break;
+                    const int row = bt[key / ps] * ps + (int)(key % ps);
+                    for (int c = 0; c < D / 32; ++c) {
+                        tma_reduce_add_3d(&tmdv, stg_v + c * CB + (r0 + b0) * 128, c * 32, kvh, row);
+                        tma_reduce_add_3d(&tmdk, stg_k + c * CB + (r0 + b0) * 128, c * 32, kvh, row);
+                    }
+                }
+                bulk_commit_group();
+                bulk_wait_all();
+            }
+            __syncwarp();
         }
     }
 
@@ -420,6 +457,7 @@ struct BqCfg {
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreadsB, 1)
     bwd_tc_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
+                     const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const BwdParams2 p) {
     using L_ = BqCfg<D>;
     constexpr int KH = L_::KH;
@@ -440,16 +478,24 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const SeqInfo si = p.seqs[u.seq];
     const int G = p.group;
     const int64_t base_pos = (int64_t)si.L - si.n;
-    // keys any of the block's rows can see: [lo, hi), in steps of QKB
+    // keys any of the block's rows can see: [lo, hi), walked in steps of QKB from lo rounded down to
+    // a multiple of QKB (so that every step starts on a page box)
     const int64_t p_first = base_pos + u.j0, p_last = base_pos + u.j1 - 1;
-    const int64_t lo = p.window > 0 ? max64(0, p_first - p.window + 1) : 0;
+    const int64_t lo = (p.window > 0 ? max64(0, p_first - p.window + 1) : 0) / QKB * QKB;
     const int64_t hi = p.causal ? min64(si.L, p_last + 1) : si.L;
     const int nsteps = hi > lo ? (int)((hi - lo + QKB - 1) / QKB) : 0;
+    const int ps = p.page_size, qbox = ps < QKB ? ps : QKB;  // rows of a K / V box
+    // key rows of step j a box brings in: those of the boxes holding a key < hi; rows past that, or
+    // past the sequence's end, hold arbitrary bytes (zeroed before dQ += dS K reads them)
+    auto loaded_rows = [&](int j) {
+        const int64_t t0 = lo + (int64_t)j * QKB;
+        const int nb = (int)((min64(t0 + QKB, hi) - t0 + qbox - 1) / qbox);
+        return (int)min64(nb * qbox, si.L - t0);
+    };
 
     if (tid == 0) {
         for (int i = 0; i < L_::B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i >= L_::B_KVFULL && i < L_::B_KVFULL + QKVST) cnt = 32;  // every lane of the load warp
             if (i == L_::B_PFULL || i == L_::B_PFULL + 1) cnt = 128;  // the compute warps
             mbar_init(&bars[i], cnt);
         }
@@ -480,50 +526,51 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                             si.q_start + u.j0);
             }
         }
-        const T* kc = static_cast<const T*>(p.k);
-        const T* vc = static_cast<const T*>(p.v);
+        // step j's K and V rows go into stage j % QKVST, one TMA box per page (and 64-column half)
+        // holding a key < hi; lane l keeps the cache row of box base_g + l
         const int32_t* bt = p.block_tables + (int64_t)u.seq * p.table_width;
-        const int ps = p.page_size;
-        const int64_t rstride = (int64_t)p.hkv * D;
+        const int bps = QKB / qbox;
+        int base_g = -(1 << 30), my_row = 0;
+        if (lane == 0) {
+            tma_prefetch(&tmk);
+            tma_prefetch(&tmv);
+        }
         bool ok = true;
-        // step j's rows go into stage j % QKVST; the stage of the step before is handed over once its
-        // copies have landed (every lane waits for its own, fences them for the tensor core, arrives)
         for (int j = 0; ok && j < nsteps; ++j) {
             const int st = j % QKVST;
+            const int64_t t0 = lo + (int64_t)j * QKB;
+            const int nb = (int)((min64(t0 + QKB, hi) - t0 + qbox - 1) / qbox);
+            const int g0 = j * bps;
+            if (g0 + nb > base_g + 32) {
+                base_g = g0;
+                const int64_t key = lo + (int64_t)(base_g + lane) * qbox;
+                my_row = key < si.L ? bt[key / ps] * ps + (int)(key % ps) : 0;
+            }
             if (j >= QKVST)
                 ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_KVEMPTY + st], ((j / QKVST) - 1) & 1, wd, 31));
             if (!ok) break;
             uint8_t* ks = smem + L_::K + st * 2 * KH * L_::HALF_K;
             uint8_t* vs = ks + KH * L_::HALF_K;
-            for (int r = lane; r < QKB; r += 32) {
-                const int64_t t = lo + (int64_t)j * QKB + r;
-                const bool valid = t < hi;
-                const int64_t off = valid ? ((int64_t)bt[t / ps] * ps + t % ps) * rstride + (int64_t)kvh * D : 0;
-#pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    const int h = c >> 3, ch = c & 7;
-                    const int dst = h * L_::HALF_K + r * 128 + btc_swz(r, ch) * 16;
-                    cp_async_16(ks + dst, kc + off + c * 8, valid);
-                    cp_async_16(vs + dst, vc + off + c * 8, valid);
-                }
+            if (lane == 0) mbar_arrive_expect_tx(&bars[L_::B_KVFULL + st], (uint32_t)(nb * qbox * 128 * KH * 2));
+            for (int b = 0; b < nb; ++b) {
+                const int row = __shfl_sync(0xffffffffu, my_row, g0 + b - base_g);
+                if (lane == 0)
+                    for (int h = 0; h < KH; ++h) {
+                        tma_load_3d(ks + h * L_::HALF_K + b * qbox * 128, &tmk, &bars[L_::B_KVFULL + st], h * 64, kvh,
+                                    row);
+                        tma_load_3d(vs + h * L_::HALF_K + b * qbox * 128, &tmv, &bars[L_::B_KVFULL + st], h * 64, kvh,
+                                    row);
+                    }
             }
-            cp_async_commit();
-            if (j >= 1) {
-                cp_async_wait<1>();
-                fence_proxy_async_smem();
-                mbar_arrive(&bars[L_::B_KVFULL + (j - 1) % QKVST]);
-            }
-        }
-        if (ok && nsteps > 0) {
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[L_::B_KVFULL + (nsteps - 1) % QKVST]);
-        } else {
-            cp_async_wait<0>();
+            __syncwarp();
         }
         if (lane == 0 && *abort_flag && nsteps > 0) {
+            // leave no copy in flight into this CTA's shared memory (bounded, ignoring the flag)
             const uint64_t t0 = globaltimer_ns();
             while (!mbar_try_wait(&bars[L_::B_QFULL], 0) && globaltimer_ns() - t0 < kWaitLimitNsB) {}
+            for (int j = max(0, nsteps - QKVST); j < nsteps; ++j)
+                while (!mbar_try_wait(&bars[L_::B_KVFULL + j % QKVST], (j / QKVST) & 1) &&
+                       globaltimer_ns() - t0 < kWaitLimitNsB) {}
         }
     } else if (warp == kMmaWarp) {
         // ===================== MMA issuer =====================
@@ -535,6 +582,19 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL + (j & 1)], (j >> 1) & 1, wd, 33));
             if (!ok) return;
             tc_fence_after();
+            // K rows the step's boxes did not bring (or past the sequence's end) hold arbitrary bytes,
+            // and dS is zero there: make them zero too, so that 0 * garbage cannot reach dQ. S and dP of
+            // the step, which read them as well, are complete.
+            const int nz = loaded_rows(j);
+            if (nz < QKB) {
+                uint8_t* ks = smem + L_::K + (j % QKVST) * 2 * KH * L_::HALF_K;
+                for (int h = 0; h < KH; ++h) {
+                    uint4* base = reinterpret_cast<uint4*>(ks + h * L_::HALF_K);
+                    for (int c = nz * 8 + lane; c < QKB * 8; c += 32) base[c] = make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+            }
             if (lane == 0) {
                 const uint32_t ks = s_base + L_::K + (j % QKVST) * 2 * KH * L_::HALF_K;
                 const uint64_t dA = sdesc_sw128(s_base + L_::DS + (j & 1) * 128 * 128, 16, 1024);
@@ -669,9 +729,17 @@ cudaError_t launch_btc(const BwdParams2& p, int num_key_units, int64_t num_queri
     using L_ = BtcCfg<D>;
     const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const int G = p.group, qpt = RB / G;
-    CUtensorMap tq, to;  // Q and dO, boxes of 128 rows (qpt queries x G heads) and 64 columns
+    const int ps = p.page_size;
+    const uint64_t cache_rows = (uint64_t)p.num_pages * ps;
+    // Q and dO: boxes of 128 rows (qpt queries x G heads) and 64 columns; K and V: one page (at
+    // most the tile) of one KV head; the float32 gradient caches: 32 rows of one KV head
+    CUtensorMap tq, to, tk, tv, tdk, tdv;
     if (!make_map(&tq, bf16, p.q, D, p.hq, (uint64_t)num_queries, G, qpt) ||
-        !make_map(&to, bf16, p.dout, D, p.hq, (uint64_t)num_queries, G, qpt))
+        !make_map(&to, bf16, p.dout, D, p.hq, (uint64_t)num_queries, G, qpt) ||
+        !make_map(&tk, bf16, p.k, D, p.hkv, cache_rows, 1, ps < KT ? ps : KT) ||
+        !make_map(&tv, bf16, p.v, D, p.hkv, cache_rows, 1, ps < KT ? ps : KT) ||
+        !make_map_f32(&tdk, p.dk, D, p.hkv, cache_rows, 1, ps < 32 ? ps : 32) ||
+        !make_map_f32(&tdv, p.dv, D, p.hkv, cache_rows, 1, ps < 32 ? ps : 32))
         return cudaErrorInvalidValue;
     auto kern = bwd_tc_dkdv_kernel<T, D>;
     static unsigned long long configured = 0;
@@ -683,7 +751,7 @@ cudaError_t launch_btc(const BwdParams2& p, int num_key_units, int64_t num_queri
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<dim3(num_key_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, p);
+    kern<<<dim3(num_key_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, tk, tv, tdk, tdv, p);
     return cudaGetLastError();
 }
 
@@ -694,9 +762,13 @@ cudaError_t launch_bq(const BwdParams2& p, int num_row_units, int64_t num_querie
     using L_ = BqCfg<D>;
     const bool bf16 = std::is_same<T, __nv_bfloat16>::value;
     const int G = p.group, qpt = RB / G;
-    CUtensorMap tq, to;
+    const int ps = p.page_size;
+    const uint64_t cache_rows = (uint64_t)p.num_pages * ps;
+    CUtensorMap tq, to, tk, tv;  // Q, dO as in the dK/dV kernel; K, V: one page (at most a step) of a KV head
     if (!make_map(&tq, bf16, p.q, D, p.hq, (uint64_t)num_queries, G, qpt) ||
-        !make_map(&to, bf16, p.dout, D, p.hq, (uint64_t)num_queries, G, qpt))
+        !make_map(&to, bf16, p.dout, D, p.hq, (uint64_t)num_queries, G, qpt) ||
+        !make_map(&tk, bf16, p.k, D, p.hkv, cache_rows, 1, ps < QKB ? ps : QKB) ||
+        !make_map(&tv, bf16, p.v, D, p.hkv, cache_rows, 1, ps < QKB ? ps : QKB))
         return cudaErrorInvalidValue;
     auto kern = bwd_tc_dq_kernel<T, D>;
     static unsigned long long configured = 0;
@@ -708,7 +780,7 @@ cudaError_t launch_bq(const BwdParams2& p, int num_row_units, int64_t num_querie
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<dim3(num_row_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, p);
+    kern<<<dim3(num_row_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, tk, tv, p);
     return cudaGetLastError();
 }
 

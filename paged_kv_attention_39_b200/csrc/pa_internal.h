@@ -77,6 +77,7 @@ struct BwdParams2 {
     int32_t table_width, page_size, hq, hkv, group, d;
     float scale, scale_log2;
     int32_t causal, window;
+    int32_t num_pages;
     int* err;  // device error word of the plan (bounded waits of the tcgen05 kernel)
 };
 

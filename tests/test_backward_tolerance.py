@@ -86,7 +86,8 @@ def _cases():
                                                    (16, 1, 64, 32, True, 100, torch.bfloat16),
                                                    (8, 2, 128, 16, False, 0, torch.bfloat16),
                                                    (8, 4, 64, 128, True, 0, torch.float16),
-                                                   (32, 1, 64, 16, True, 0, torch.bfloat16)]:
+                                                   (32, 1, 64, 16, True, 0, torch.bfloat16),
+                                                   (8, 2, 128, 256, True, 0, torch.bfloat16)]:
         wl = W.make_gqa("bwd_tc", 5, [300, 513, 64, 1000], [100, 200, 64, 17], hq, hkv, d, d, ps, dtype,
                         causal=causal, window=window)
         g = torch.Generator().manual_seed(11)

@@ -86,6 +86,7 @@ def test_backward_shared_prefix_page_accumulates(orc):
     (8, 2, 128, 16, False, 0, torch.bfloat16),
     (8, 4, 64, 128, True, 0, torch.float16),
     (32, 1, 64, 16, True, 0, torch.bfloat16),   # 32 heads per group: 4 queries per 128-row block
+    (8, 2, 128, 256, True, 0, torch.bfloat16),  # pages longer than a key tile: boxes inside a page
 ])
 def test_backward_tensor_core_shapes(orc, hq, hkv, d, ps, causal, window, dtype):
     """The tensor-core backward (key-major dK/dV, query-major dQ, both on tcgen05): chunked prefills
@@ -101,6 +102,33 @@ def test_backward_tensor_core_shapes(orc, hq, hkv, d, ps, causal, window, dtype)
     close(dq, rq, dtype, "dq " + tag)
     close(dk, rk, dtype, "dk " + tag)
     close(dv, rv, dtype, "dv " + tag)
+
+
+def test_backward_page_size_outside_the_box_layout_runs_the_cuda_core_kernel(orc):
+    """A page of 48 rows neither divides the 128-key tile nor is a multiple of it, so the tensor-core
+    kernels (one TMA box per page) do not take it: the CUDA-core kernel does, and matches."""
+    wl = W.make_gqa("bwd_ps48", 9, [300, 100], [40, 5], 8, 2, 64, 64, 48, torch.bfloat16)
+    g = torch.Generator().manual_seed(13)
+    s = wl.sched
+    q, k, v = wl.q.cuda(), wl.k_cache.cuda(), wl.v_cache.cuda()
+    nq, hq, d = q.shape
+    dout = torch.randn(nq, hq, d, generator=g).to(q.dtype)
+    plan = pa.plan_for(wl)
+    out = torch.empty(nq, hq, d, dtype=q.dtype, device="cuda")
+    lse = torch.empty(nq, hq, dtype=torch.float32, device="cuda")
+    pa.pa_forward(plan, q, k, v, out, lse, wl.scale, True, 0)
+    dq = torch.empty((nq, hq, d), dtype=torch.float32, device="cuda")
+    dk = torch.zeros(k.shape, dtype=torch.float32, device="cuda")
+    dv = torch.zeros(v.shape, dtype=torch.float32, device="cuda")
+    pa.pa_backward(plan, q, k, v, out, lse, dout.cuda(), dq, dk, dv, wl.scale, True, 0)
+    assert pa.pa_plan_get_info(plan)["last_kernels"] == pa.PA_KERNEL_BACKWARD_SIMT
+    torch.cuda.synchronize()
+    plan.close()
+    rq, rk, rv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s.seq_lens, s.query_offsets,
+                                        s.block_tables, 48, wl.scale, True, 0)
+    close(dq.cpu(), rq, torch.bfloat16, "dq")
+    close(dk.cpu(), rk, torch.bfloat16, "dk")
+    close(dv.cpu(), rv, torch.bfloat16, "dv")
 
 
 def test_backward_tensor_core_shared_pages_and_launches(orc):
