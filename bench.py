@@ -18,6 +18,7 @@ sample of the same workload per step.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -139,6 +140,31 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+_E2E = None
+
+
+def e2e_library():
+    """libpa_e2e.so (the end-to-end decode loop in C over the public C ABI), built beside libpa.so."""
+    global _E2E
+    if _E2E is None:
+        P, I = ctypes.c_void_p, ctypes.c_int32
+        lib = ctypes.CDLL(os.path.join(ROOT, "paged_kv_attention_39_b200", "libpa_e2e.so"))
+        lib.pa_e2e_create.restype = P
+        lib.pa_e2e_create.argtypes = [P, P, I, P, I, I, I, ctypes.c_int, P, ctypes.c_size_t, P, P, P, ctypes.c_int,
+                                      I, I, I, I, ctypes.c_float, ctypes.c_int, I, P, P, ctypes.c_size_t,
+                                      ctypes.c_size_t]
+        lib.pa_e2e_run.restype = ctypes.c_int
+        lib.pa_e2e_run.argtypes = [P, ctypes.c_int, P]
+        lib.pa_e2e_destroy.restype = None
+        lib.pa_e2e_destroy.argtypes = [P]
+        lib.pa_e2e_uploaded_bytes.restype = ctypes.c_longlong
+        lib.pa_e2e_uploaded_bytes.argtypes = [P]
+        lib.pa_e2e_host_times.restype = None
+        lib.pa_e2e_host_times.argtypes = [P, ctypes.POINTER(ctypes.c_double)]
+        _E2E = lib
+    return _E2E
+
+
 def kernel_traffic(kernel_file: str, key: str):
     """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
     try:
@@ -208,7 +234,10 @@ def run_ours(args, ws, rank, local):
         pa.pa_forward(plan, q, k, v, out, lse, wl.scale, wl.causal, wl.window, trace=tr)
 
     sampler = ClockSampler(local) if rank == 0 else None
-    ms, kern_ms, comb_ms, clocks = time_forward(pa, plan, step, args.steps, args.warmup, True, sampler, ws)
+    # the timed steps carry no instrumentation; a second, traced pass (events between the kernels of
+    # each call) splits a step into the attention kernel and the merge for the roofline
+    ms, _, _, clocks = time_forward(pa, plan, step, args.steps, args.warmup, False, sampler, ws)
+    _, kern_ms, comb_ms, _ = time_forward(pa, plan, step, max(1, min(args.steps, 200)), 3, True, None, ws)
     launches_per_step = pa.pa_plan_get_info(plan)["last_launches"]
     ms_max = allreduce_max(ms, ws)
     total_bytes = allreduce_sum(kv_bytes, ws)
@@ -217,63 +246,36 @@ def run_ours(args, ws, rank, local):
     traffic = kernel_traffic("decode.cu", "decode_mma_kernel")
 
     # ---- end to end through the public API with host buffers -------------------------------
-    # A decode loop as a serving engine with asynchronous scheduling runs it: every step copies
-    # its queries in from pinned host memory, uploads its own plan (a new schedule per step:
-    # lengths grow, pages move), runs pa_forward and reads out and lse back into pinned host
-    # memory. Two steps are in flight: step i+1's query upload (on a copy stream) and plan build
-    # (pa_plan_create + pa_plan_prepare: validation, work list, their uploads queued on the
-    # compute stream) overlap step i's attention, and step i's download (on the copy stream)
-    # overlaps step i+1's attention; the host waits for step i's result before it issues step
-    # i+2. Device buffers are double-buffered so no copy touches a buffer a running step uses.
-    # The K steps are timed as one region on the compute stream, joined with the copy stream at
-    # the end, so every copy, upload and host gap is inside it.
-    q_host = wl.q.pin_memory()
-    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    lse_host = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
+    # A decode loop as a serving engine with asynchronous scheduling runs it, written in C over the
+    # public C ABI (paged_kv_attention_39_b200/e2e/e2e_loop.cu, libpa_e2e.so): every step builds and
+    # uploads its own plan (pa_plan_create + pa_plan_prepare: a new schedule per step, as lengths grow
+    # and pages move) and copies its queries in from pinned host memory on an upload stream, runs
+    # pa_forward, and copies out and lse back into pinned host memory on a download stream; two
+    # steps are in flight, and the host waits for step i's result before it issues step i+2. The K
+    # steps are timed as one region on the compute stream (the call returns once every result is on
+    # the host), so every copy, upload and host gap is inside it.
+    s = wl.sched
+    lib = e2e_library()
     q_dev = [q, torch.empty_like(q)]
     out_dev = [out, torch.empty_like(out)]
     lse_dev = [lse, torch.empty_like(lse)]
     e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 200))
-    uploaded = 0
+    sl, qo, bt = pa._i32(s.seq_lens), pa._i32(s.query_offsets), pa._i32(s.block_tables)
+    q_src = wl.q.contiguous()
     main = torch.cuda.current_stream(dev)
-    copy_stream = torch.cuda.Stream(dev)
-
-    def next_plan():
-        pn = pa.plan_for(wl, device=local)
-        pa.pa_plan_prepare(pn, q.dtype, hq, wl.num_kv_heads, d, d, wl.causal, wl.window)
-        return pn
+    ptr2 = lambda ts: (ctypes.c_void_p * 2)(*(t.data_ptr() for t in ts))
+    out_bytes, lse_bytes = out.numel() * out.element_size(), lse.numel() * 4
+    loop = lib.pa_e2e_create(sl.data_ptr(), qo.data_ptr(), sl.numel(), bt.data_ptr(), bt.shape[1], s.page_size,
+                             s.num_pages, local, q_src.data_ptr(), q_src.numel() * q_src.element_size(), ptr2(q_dev),
+                             k.data_ptr(), v.data_ptr(), pa._DTYPES[q.dtype], hq, wl.num_kv_heads, d, d, wl.scale,
+                             int(wl.causal), wl.window, ptr2(out_dev), ptr2(lse_dev), out_bytes, lse_bytes)
+    if not loop:
+        raise RuntimeError("end-to-end loop set-up failed")
 
     def e2e_loop(n):
-        nonlocal uploaded
-        cur = next_plan()
-        h2d = [torch.cuda.Event(), torch.cuda.Event()]
-        fwd = [torch.cuda.Event(), torch.cuda.Event()]
-        d2h = [torch.cuda.Event(), torch.cuda.Event()]
-        for i in range(n):
-            b = i & 1
-            with torch.cuda.stream(copy_stream):
-                if i >= 2:
-                    copy_stream.wait_event(fwd[b])  # step i-2 has finished reading q_dev[b]
-                q_dev[b].copy_(q_host, non_blocking=True)
-                h2d[b].record(copy_stream)
-            main.wait_event(h2d[b])
-            pa.pa_forward(cur, q_dev[b], k, v, out_dev[b], lse_dev[b], wl.scale, wl.causal, wl.window)
-            fwd[b].record(main)
-            with torch.cuda.stream(copy_stream):
-                copy_stream.wait_event(fwd[b])
-                out_host[b].copy_(out_dev[b], non_blocking=True)
-                lse_host[b].copy_(lse_dev[b], non_blocking=True)
-                d2h[b].record(copy_stream)
-            # host work overlapping the GPU: the next plan, and this plan's release (its frees are
-            # ordered on the compute stream after the step)
-            nxt = next_plan() if i + 1 < n else None
-            uploaded = pa.pa_plan_get_info(cur)["uploaded_bytes"]
-            cur.close()
-            if i >= 1:
-                d2h[b ^ 1].synchronize()  # step i-1's result is on the host
-            cur = nxt
-        d2h[(n - 1) & 1].synchronize()
-        main.wait_stream(copy_stream)
+        rc = lib.pa_e2e_run(loop, n, main.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"end-to-end loop failed with code {rc}")
 
     e2e_ms = float("nan")
     if e2e_steps:
@@ -289,6 +291,10 @@ def run_ours(args, ws, rank, local):
         e2e_ms = e0.elapsed_time(e1) / e2e_steps
     e2e_ms = allreduce_max(e2e_ms, ws)
     e2e_val = total_bytes / (e2e_ms * 1e-3) / 1e9
+    host_us = (ctypes.c_double * 6)()
+    lib.pa_e2e_host_times(loop, host_us)
+    uploaded = lib.pa_e2e_uploaded_bytes(loop)
+    lib.pa_e2e_destroy(loop)
     plan.close()
 
     extra = {}
@@ -334,14 +340,17 @@ def run_ours(args, ws, rank, local):
         "e2e": {
             "value": round(e2e_val, 2),
             "unit": "GB/s",
-            "h2d_bytes_per_step": int(q_host.numel() * q_host.element_size() + uploaded),
-            "d2h_bytes_per_step": int(out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4),
+            "h2d_bytes_per_step": int(q_src.numel() * q_src.element_size() + uploaded),
+            "d2h_bytes_per_step": int(out_bytes + lse_bytes),
+            "host_us_per_step": {name: round(host_us[i] / max(1, e2e_steps), 1) for i, name in enumerate(
+                ("plan_create", "plan_prepare", "copies", "forward", "plan_release", "wait"))},
             "ms_per_step": round(e2e_ms, 4),
-            "includes": "per step: H2D of Q from pinned memory (copy stream), a new plan (pa_plan_create + "
-                        "pa_plan_prepare: schedule and work-list uploads), pa_forward, D2H of out and lse into "
-                        "pinned memory (copy stream); two steps in flight (step i+1's upload and plan build "
-                        "overlap step i, step i's download overlaps step i+1; the host waits for step i's "
-                        "result before issuing step i+2); K steps timed as one region",
+            "includes": "a C loop over the public C ABI (libpa_e2e.so); per step: a new plan (pa_plan_create + "
+                        "pa_plan_prepare: schedule and work-list uploads) and the H2D of Q from pinned memory on "
+                        "an upload stream, pa_forward, the D2H of out and lse into pinned memory on a download "
+                        "stream; two steps in flight (step i+1's plan and upload overlap step i, step i's "
+                        "download overlaps step i+1; the host waits for step i's result before issuing step "
+                        "i+2); K steps timed as one region",
         },
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -400,8 +409,8 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
 
                 def step(tr):
                     pa.pa_forward(plan, q, k, v, out, lse, wl.scale, wl.causal, wl.window, trace=tr)
-            ms, kern, comb, _ = time_forward(pa, plan, step, args.extra_steps, args.warmup if only else 3, True,
-                                             None, 1)
+            ms, _, _, _ = time_forward(pa, plan, step, args.extra_steps, args.warmup if only else 3, False, None, 1)
+            _, kern, comb, _ = time_forward(pa, plan, step, args.extra_steps, 1, True, None, 1)
             res[name] = {
                 "ms_per_step": round(ms, 4),
                 "attention_kernels_ms": round(kern, 4),

@@ -122,7 +122,7 @@ typedef struct pa_plan_info {
 #define PA_KERNEL_PREFILL_TC 2u     /* chunked prefill on tcgen05 / TMEM / TMA */
 #define PA_KERNEL_MLA_TC 4u         /* MLA decode on tcgen05 / TMEM / TMA */
 #define PA_KERNEL_SIMT 8u           /* the CUDA-core kernel (fp32, other shapes, PA_PATH_SIMT) */
-#define PA_KERNEL_MERGE 16u         /* the split-part merge */
+#define PA_KERNEL_MERGE 16u         /* the split-part merge kernel (CUDA-core, MLA and sparse parts) */
 #define PA_KERNEL_SPARSE 32u        /* sparse selection kernels (check, proxy scores, top-K) */
 #define PA_KERNEL_APPEND 64u        /* paged append */
 #define PA_KERNEL_BACKWARD_TC 128u  /* tensor-core GQA backward */
@@ -158,8 +158,10 @@ typedef struct pa_forward_options {
  * Shapes: num_kv_heads >= 1, num_q_heads % num_kv_heads == 0, 1 <= head_dim, v_head_dim
  * <= 1024 (ruDNN's limit). N_q == 0 returns PA_OK without launching anything.
  * Long contexts are split over several CTAs whose float32 partial results (o_i, lse_i) go to
- * the plan-owned workspace and are merged by a second kernel (ruDNN "split the visible
- * history over multiple planes and merge FP32 statistics"). The workspace grows on demand
+ * the plan-owned workspace and are merged (ruDNN "split the visible history over multiple planes
+ * and merge FP32 statistics"): on the tensor-core decode path by the CTA that completes a row
+ * last (plan-owned arrival counters, zero between calls), elsewhere by a second kernel; either
+ * way the parts are summed in a fixed order. The workspace grows on demand
  * with stream-ordered allocation on `stream`; calls on one plan must therefore be ordered
  * (one stream, or explicit events). The first call with a new head configuration builds and
  * uploads that configuration's work list once (also available as pa_plan_prepare); make it

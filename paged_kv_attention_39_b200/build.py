@@ -41,6 +41,7 @@ def _deps_mtime() -> float:
 
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
+        build_e2e(force)
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
@@ -66,7 +67,33 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     os.replace(tmp, LIB)
+    build_e2e(True)
     return LIB
+
+
+E2E_SRC = os.path.join(HERE, "e2e", "e2e_loop.cu")
+E2E_LIB = os.path.join(HERE, "libpa_e2e.so")
+
+
+def build_e2e(force: bool = False) -> str:
+    """libpa_e2e.so: the end-to-end decode loop bench.py times (host code over the public C ABI,
+    linked against libpa.so next to it)."""
+    if not force and os.path.exists(E2E_LIB) and os.path.getmtime(E2E_LIB) >= max(
+            os.path.getmtime(E2E_SRC), os.path.getmtime(LIB), os.path.getmtime(__file__)):
+        return E2E_LIB
+    cc = nvcc()
+    obj = os.path.join(BUILD, "e2e_loop.o")
+    os.makedirs(BUILD, exist_ok=True)
+    r = subprocess.run([cc] + _flags() + ["-c", E2E_SRC, "-o", obj], capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {E2E_SRC}:\n{r.stdout}\n{r.stderr}")
+    tmp = E2E_LIB + f".tmp{os.getpid()}"
+    r = subprocess.run([cc] + ARCH + ["-shared", "-o", tmp, obj, "-L", HERE, "-lpa", "-Xlinker", "-rpath,$ORIGIN",
+                                       "-cudart", "static"], capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+    os.replace(tmp, E2E_LIB)
+    return E2E_LIB
 
 
 if __name__ == "__main__":

@@ -153,7 +153,7 @@ cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     }
     return cudaSuccess;
 }
-constexpr int kTargetCtasPerSm = 8;        // automatic split size aims at this many CTAs/SM
+constexpr int kUnitKeys = 2048;            // automatic split: keys per unit (per KV head), at most
 
 struct SchedKey {
     int mla, dtype, hq, hkv, d, dv, pr, causal, window, path, kv_chunk;
@@ -209,6 +209,8 @@ struct pa_plan {
     size_t bwd_drow_bytes = 0;
     float* bwd_scratch = nullptr;  // finished dK then dV rows of ordered key tiles
     size_t bwd_scratch_bytes = 0;
+    int* merge_ctr = nullptr;  // arrival counters of the decode kernel's own merge, zero between calls
+    size_t merge_ctr_n = 0;
     cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
     int32_t last_launches = 0;
     int32_t last_kernels = 0;  // PA_KERNEL_* bits of the last call
@@ -304,14 +306,17 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     int64_t chunk;
     if (k.kv_chunk > 0) chunk = k.sparse_bs > 0 ? ((int64_t)k.kv_chunk + 15) / 16 * 16 : k.kv_chunk;
     else if (k.kv_chunk < 0) chunk = INT32_MAX;
-    else {
+    else if (tc_mla) {
         // The tensor-core MLA kernel runs one CTA per SM, two per unit: aim at one unit per SM.
-        const int64_t target = tc_mla ? (int64_t)P->num_sms : (int64_t)P->num_sms * kTargetCtasPerSm;
-        chunk = (total + target - 1) / std::max<int64_t>(1, target);
-        chunk = ((chunk + 63) / 64) * 64;
-        // Sparse rows are short runs of selected blocks: whole rows up to 1024 keys per unit (no
-        // merge) beat finer splits; dense decode rows are split down to 256 keys.
-        chunk = std::max<int64_t>(chunk, k.sparse_bs > 0 ? 1024 : 256);
+        chunk = (total + P->num_sms - 1) / std::max<int64_t>(1, P->num_sms);
+        chunk = std::max<int64_t>(((chunk + 63) / 64) * 64, 256);
+    } else {
+        // Long units amortise each CTA's start (first loads in flight) and end (merging its warps,
+        // writing its part, merging the row): units of at most kUnitKeys keys, short enough that
+        // there are about 7 units per 4 SMs, and never below 256 keys. Sparse rows are short runs
+        // of selected blocks: whole rows up to 1024 keys per unit (no merge) beat finer splits.
+        chunk = std::min<int64_t>(kUnitKeys, total * 4 / std::max<int64_t>(1, 7 * (int64_t)P->num_sms));
+        chunk = std::max<int64_t>(((chunk + 63) / 64) * 64, k.sparse_bs > 0 ? 1024 : 256);
     }
 
     std::vector<pa::KvUnit> tcu, simtu, mlau;
@@ -325,10 +330,18 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
             c = (len + kMaxSplits - 1) / kMaxSplits;
             if (k.sparse_bs > 0) c = (c + 15) / 16 * 16;  // tiles of 16 keys stay inside one block
             nsplit = ceil_div(len, c);
+        } else if (nsplit > 1 && k.kv_chunk == 0 && !tc_mla) {
+            // automatic split: parts of (nearly) equal length, multiples of 64 keys, rather than
+            // full parts and a short last one
+            c = (ceil_div(len, nsplit) + 63) / 64 * 64;
+            nsplit = ceil_div(len, c);
         }
         const int32_t base = nsplit > 1 ? (int32_t)slots : -1;
         if (nsplit > 1) {
-            for (int32_t j = b.j0; j < b.j1; ++j)
+            // the tensor-core decode kernel merges its own split rows (dense keys only); the merge
+            // kernel takes the other kernels' rows
+            if (!(b.kind == 1 && k.sparse_bs == 0))
+                for (int32_t j = b.j0; j < b.j1; ++j)
                     cu.push_back({P->seqs[b.seq].q_start + j, base + (j - b.j0) * nsplit, nsplit, 0});
             slots += (int64_t)(b.j1 - b.j0) * nsplit;
         }
@@ -609,6 +622,22 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
             if (e != cudaSuccess) return fail(PA_ERR_CUDA, "selection check launch failed: %s", cudaGetErrorString(e));
         }
     }
+    if (S->n_tc > 0 && S->slots > 0 && c.block_size == 0) {
+        // counters of the decode kernel's own merge: zeroed when allocated, and put back to zero by
+        // the kernel after each merge, so every call finds them zero
+        const size_t n = (size_t)S->slots * c.hkv;
+        if (n > P->merge_ctr_n) {
+            if (P->merge_ctr) PA_CUDA_TRY(cudaFreeAsync(P->merge_ctr, st));
+            P->merge_ctr = nullptr;
+            P->merge_ctr_n = 0;
+            void* m = nullptr;
+            PA_CUDA_TRY(lib_malloc(&m, n * sizeof(int), st));
+            PA_CUDA_TRY(cudaMemsetAsync(m, 0, n * sizeof(int), st));
+            P->merge_ctr = (int*)m;
+            P->merge_ctr_n = n;
+        }
+        p.merge_ctr = P->merge_ctr;
+    }
     if (ev) PA_CUDA_TRY(cudaEventRecord(ev[0], st));
     if (S->n_tc > 0) {
         ++launches;
@@ -812,6 +841,7 @@ pa_status pa_plan_destroy(pa_plan* plan) {
         if (plan->bwd_dev) cudaFreeAsync(plan->bwd_dev, st);
         if (plan->bwd_drow) cudaFreeAsync(plan->bwd_drow, st);
         if (plan->bwd_scratch) cudaFreeAsync(plan->bwd_scratch, st);
+        if (plan->merge_ctr) cudaFreeAsync(plan->merge_ctr, st);
         for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
         cudaError_t e = plan->d_meta ? cudaFreeAsync(plan->d_meta, st) : cudaSuccess;
         delete plan;

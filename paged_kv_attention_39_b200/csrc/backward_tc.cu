@@ -17,11 +17,12 @@
 // those rows), or, for a tile the host marked ordered (it touches a shared page), writes them to
 // the scratch the ordered pass sums. dQ comes from the query-major kernel at the end of this file.
 //
-//   warps 0..3  compute: row statistics from shared memory, masks, P and dS, the epilogue
-//   warp 4      loads: the K and V rows of the tile once (cp.async, straight from the pages, zeros
-//               past the sequence's end), then per row block the Q and dO rows (TMA, two stages)
-//               and the block's lse, Drow and visible key ranges (into shared memory)
-//   warp 5      TMEM owner and MMA issuer (one thread)
+//   warps 0..7  compute: row statistics from shared memory, masks, P and dS, the epilogue (two
+//               warps per 32 keys, each taking half of the block's rows and of the dK/dV columns)
+//   warp 8      loads: the K and V rows of the tile once (TMA, one box per page), then per row
+//               block the Q and dO rows (TMA, two stages) and the block's lse, Drow and visible
+//               key ranges (into shared memory)
+//   warp 9      TMEM owner and MMA issuer (one thread)
 //
 // Every wait on an mbarrier is bounded (Watchdog): a stalled pipeline sets the plan's error word and
 // the CTA leaves through its normal exit, freeing TMEM.
@@ -38,7 +39,9 @@ namespace {
 constexpr int KT = 128;  // keys per CTA
 constexpr int RB = 128;  // rows per block
 constexpr int QST = 2;   // Q / dO stages
-constexpr int kLoadWarp = 4, kMmaWarp = 5, kThreadsB = 6 * 32;
+// warps 0..7 compute (two per TMEM lane quadrant: warp w reaches lanes 32 (w % 4) .. and takes
+// half w / 4 of the block's columns), warp 8 loads, warp 9 owns TMEM and issues the MMAs
+constexpr int kComputeWarpsB = 8, kLoadWarp = 8, kMmaWarp = 9, kThreadsB = 10 * 32;
 constexpr uint32_t kTmemColsB = 512;
 constexpr uint64_t kWaitLimitNsB = 2000000000ull;
 constexpr float kLog2eB = 1.4426950408889634f;
@@ -64,17 +67,23 @@ struct BtcCfg {
 
 __device__ __forceinline__ int btc_swz(int row, int chunk) { return chunk ^ (row & 7); }
 
+// TMEM column of row `row` of a block's packed P^T / dS^T (two 16-bit rows per column; the second
+// half of the rows sits over the third quarter of the buffer)
+__host__ __device__ constexpr int packed_col(int row) { return row / 2 + (row >= RB / 2 ? RB / 4 : 0); }
+
 }  // namespace
 
-// P^T and dS^T of one key (thread = TMEM lane) against the 128 rows of a block, 16-bit, written
-// over the first 64 columns of the S^T and dP^T buffers. The rows' statistics come from shared
+// P^T and dS^T of one key (thread = TMEM lane) against rows [32 c0, 32 c1) of a block, 16-bit,
+// packed two rows per column over columns of the S^T and dP^T buffers that this warp has read
+// (rows [0, 64) -> columns [0, 32), rows [64, 128) -> columns [64, 96): the two warps of a lane
+// quadrant each read and write only their own half of a buffer). The rows' statistics come from shared
 // memory four at a time (one 16-byte load per statistic for four rows); MASKED adds each row's
 // visible key range [lo, hi) (a row without keys has lo = hi = 0).
 template <typename T, bool MASKED>
 __device__ __forceinline__ void btc_probs(uint32_t t_lane, const float* lse2, const float* drow, const int* lo,
-                                          const int* hi, int64_t t, float scale_log2) {
+                                          const int* hi, int64_t t, float scale_log2, int c0, int c1) {
 #pragma unroll 1
-    for (int c = 0; c < RB / 32; ++c) {
+    for (int c = c0; c < c1; ++c) {
         uint32_t sv[32], dv[32];
         tmem_ld32(t_lane + BtcCfg<64>::T_ST + c * 32, sv);
         tmem_ld32(t_lane + BtcCfg<64>::T_DPT + c * 32, dv);
@@ -108,8 +117,9 @@ __device__ __forceinline__ void btc_probs(uint32_t t_lane, const float* lse2, co
             dk[2 * q + 1] = pack2<T>(ds[2], ds[3]);
         }
         // 32 row-columns -> 16 TMEM columns, over columns already read
-        tmem_st16(t_lane + BtcCfg<64>::T_ST + c * 16, pk);
-        tmem_st16(t_lane + BtcCfg<64>::T_DPT + c * 16, dk);
+        const int pc = packed_col(c * 32);
+        tmem_st16(t_lane + BtcCfg<64>::T_ST + pc, pk);
+        tmem_st16(t_lane + BtcCfg<64>::T_DPT + pc, dk);
     }
 }
 
@@ -149,7 +159,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     if (tid == 0) {
         for (int i = 0; i < L_::B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i == L_::B_PFULL) cnt = 128;    // the compute warps
+            if (i == L_::B_PFULL) cnt = kComputeWarpsB * 32;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -293,8 +303,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 #pragma unroll
                 for (int kk = 0; kk < RB / 16; ++kk) {
                     const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16_ts(tmem + L_::T_DV, tmem + L_::T_ST + kk * 8, desc_add(dOn, kk * 16 * 128), IDESC_G, acc);
-                    mma_f16_ts(tmem + L_::T_DK, tmem + L_::T_DPT + kk * 8, desc_add(dQn, kk * 16 * 128), IDESC_G, acc);
+                    mma_f16_ts(tmem + L_::T_DV, tmem + L_::T_ST + packed_col(kk * 16), desc_add(dOn, kk * 16 * 128),
+                               IDESC_G, acc);
+                    mma_f16_ts(tmem + L_::T_DK, tmem + L_::T_DPT + packed_col(kk * 16), desc_add(dQn, kk * 16 * 128),
+                               IDESC_G, acc);
                 }
                 mma_commit(&bars[L_::B_DONE]);
                 mma_commit(&bars[L_::B_QEMPTY + s]);
@@ -303,7 +315,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
     } else {
         // ===================== compute: thread = key =====================
-        const int r0 = warp * 32;  // this warp's TMEM lanes (keys k0 + r0 ..)
+        const int hf = warp >> 2;        // this warp's half of the block's rows / of the dK, dV columns
+        const int r0 = (warp & 3) * 32;  // this warp's TMEM lanes (keys k0 + r0 ..)
         const uint32_t lane_off = (uint32_t)r0 << 16;
         const int64_t t = k0 + r0 + lane;  // this thread's key
         const int64_t tw0 = k0 + r0, tw1 = k0 + r0 + 31;
@@ -322,9 +335,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             // sequence's end are outside every row's range, so they always take the masked path)
             const bool full = tw1 < kmax && tw0 >= hi[RB] && tw1 < hi[RB + 1];
             if (__all_sync(0xffffffffu, full))
-                btc_probs<T, false>(tmem + lane_off, lse2, drow, lo, hi, t, p.scale_log2);
+                btc_probs<T, false>(tmem + lane_off, lse2, drow, lo, hi, t, p.scale_log2, hf * RB / 64, (hf + 1) * RB / 64);
             else
-                btc_probs<T, true>(tmem + lane_off, lse2, drow, lo, hi, t, p.scale_log2);
+                btc_probs<T, true>(tmem + lane_off, lse2, drow, lo, hi, t, p.scale_log2, hf * RB / 64, (hf + 1) * RB / 64);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars[L_::B_PFULL]);
@@ -339,7 +352,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             float* dk_row = p.scratch_k + srow * D;
             float* dv_row = p.scratch_v + srow * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {
                 uint32_t a[32], b[32];
                 tmem_ld32(tmem + L_::T_DV + lane_off + c * 32, a);
                 tmem_ld32(tmem + L_::T_DK + lane_off + c * 32, b);
@@ -360,12 +373,13 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             // stages, idle now) as 128-byte swizzled 32-column blocks of the 128 rows, then add them
             // onto the caller's cache with TMA reduce-adds, one box per page and column block (one
             // add per element; keys past the sequence's end add zeros to their own page's rows).
+            // Each warp takes its 32 rows and its half of the column blocks.
             constexpr int CB = 128 * 128;  // one 32-column block of the 128 rows, float32
             uint8_t* stg_v = smem + L_::Q;
             uint8_t* stg_k = stg_v + (D / 32) * CB;
             const int r = r0 + lane;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {
                 uint32_t a[32], b[32];
                 tmem_ld32(tmem + L_::T_DV + lane_off + c * 32, a);
                 tmem_ld32(tmem + L_::T_DK + lane_off + c * 32, b);
@@ -391,7 +405,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                     const int64_t key = k0 + r0 + b0;
                     if (key >= kmax) break;
                     const int row = bt[key / ps] * ps + (int)(key % ps);
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {
                         tma_reduce_add_3d(&tmdv, stg_v + c * CB + (r0 + b0) * 128, c * 32, kvh, row);
                         tma_reduce_add_3d(&tmdk, stg_k + c * CB + (r0 + b0) * 128, c * 32, kvh, row);
                     }
@@ -423,15 +437,16 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 // shared memory), so they overlap the compute warps' work on the previous step, and the dQ product
 // of a step runs while the compute warps work on the next one. The finished rows are scaled and
 // written once.
-//   warps 0..3  compute and the epilogue
-//   warp 4      loads: Q and dO of the block (TMA), the K and V rows of each step (cp.async, one page
-//               lookup per row, zeros past the sequence's end) into a ring of stages
-//   warp 5      TMEM owner and MMA issuer
+//   warps 0..7  compute and the epilogue (two warps per 32 rows, each taking half of a step's keys
+//               and of the dQ columns)
+//   warp 8      loads: Q and dO of the block (TMA), the K and V rows of each step (TMA, one box per
+//               page) into a ring of stages
+//   warp 9      TMEM owner and MMA issuer
 // ---------------------------------------------------------------------------------------------
 namespace {
 
 constexpr int QKB = 64;   // keys per step of the dQ kernel
-constexpr int QKVST = 3;  // K/V stages
+constexpr int QKVST = 4;  // K/V stages (the fourth lets the loads run a step further ahead of dQ += dS K)
 
 template <int D>
 struct BqCfg {
@@ -496,7 +511,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     if (tid == 0) {
         for (int i = 0; i < L_::B_COUNT; ++i) {
             uint32_t cnt = 1;
-            if (i == L_::B_PFULL || i == L_::B_PFULL + 1) cnt = 128;  // the compute warps
+            if (i == L_::B_PFULL || i == L_::B_PFULL + 1) cnt = kComputeWarpsB * 32;
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -633,9 +648,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         }
         if (ok && nsteps > 0) issue_dq(nsteps - 1);
     } else {
-        // ===================== compute: thread = row =====================
-        const int r = warp * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // ===================== compute: thread = row, half hf of the keys / dQ columns =====================
+        const int hf = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const int R = (u.j1 - u.j0) * G;  // live rows
         const bool live = r < R;
         const int64_t qrow = (int64_t)(si.q_start + u.j0 + (live ? r / G : 0)) * p.hq + kvh * G + (live ? r % G : 0);
@@ -656,9 +672,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             // columns outside [row_lo, row_hi) are masked: off_lo = t0 - row_lo, off_hi = t0 - row_hi
             const int off_lo = (int)max64(min64(t0 - row_lo, 1 << 20), -(1 << 20));
             const int off_hi = (int)max64(min64(t0 - row_hi, 1 << 20), -(1 << 20));
-            uint32_t dk[32];
-#pragma unroll
-            for (int c = 0; c < QKB / 32; ++c) {
+            uint32_t dk[16];
+            {
+                const int c = hf;  // keys 32 hf .. 32 hf + 31 of the step
                 uint32_t sv[32], dv[32];
                 tmem_ld32(tmem + L_::T_S + b * QKB + lane_off + c * 32, sv);
                 tmem_ld32(tmem + L_::T_DP + b * QKB + lane_off + c * 32, dv);
@@ -674,17 +690,18 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                         const float pv = fast_exp2(fmaf(__uint_as_float(sv[2 * e + x]), p.scale_log2, -lse2));
                         ds[x] = vis ? pv * (__uint_as_float(dv[2 * e + x]) - drow) : 0.f;
                     }
-                    dk[c * 16 + e] = pack2<T>(ds[0], ds[1]);
+                    dk[e] = pack2<T>(ds[0], ds[1]);
                 }
             }
             // the dS buffer was last read by the dQ product of step j - 2
             if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_DSFREE + b], ((j - 2) >> 1) & 1, wd, 37)) && ok;
-            // row r of dS: 64 keys = 128 bytes, 16-byte chunk ch at position ch ^ (r & 7)
+            // row r of dS: 64 keys = 128 bytes, 16-byte chunk ch at position ch ^ (r & 7); this warp
+            // writes chunks 4 hf .. 4 hf + 3
             uint8_t* row = dsbuf + b * 128 * 128 + r * 128;
 #pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(row + (btc_swz(r, ch) << 4)) =
-                    make_uint4(dk[4 * ch], dk[4 * ch + 1], dk[4 * ch + 2], dk[4 * ch + 3]);
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4*>(row + (btc_swz(r, 4 * hf + q4) << 4)) =
+                    make_uint4(dk[4 * q4], dk[4 * q4 + 1], dk[4 * q4 + 2], dk[4 * q4 + 3]);
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[L_::B_PFULL + b]);
@@ -695,7 +712,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tc_fence_after();
         float* dst = p.dq + qrow * D;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = hf * (D / 64); c < (hf + 1) * (D / 64); ++c) {
             uint32_t v[32];
             if (ok && nsteps > 0) {
                 tmem_ld32(tmem + L_::T_DQ + lane_off + c * 32, v);

@@ -42,6 +42,98 @@ __device__ __forceinline__ int swz(int row, int chunk) { return chunk ^ (row & 7
 
 }  // namespace
 
+// The merge of a split (row set, KV head), run by the CTA whose part completes it last (ruDNN
+// "merge FP32 statistics"; alice-llm `lse_combine`): for each of the R rows, lse = logsumexp_i
+// lse_i over its parts and out = sum_i exp(lse_i - lse) o_i, parts taken in index order, so the
+// result does not depend on which CTA merges. A row whose parts are all empty gets out = 0 and
+// lse = -inf. Every CTA publishes its part (fence, then one counted arrival); the CTA that sees
+// the count complete reads the parts from L2 and puts the counter back to zero.
+template <typename T, int D>
+__device__ __forceinline__ void merge_own_parts(const AttnParams& p, const KvUnit& u, const SeqInfo& si, int kvh,
+                                                int R) {
+    __shared__ int s_last;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const float kLog2e = 1.4426950408889634f;
+    int* ctr = p.merge_ctr + (int64_t)u.part_base * p.hkv + kvh;
+    __threadfence();  // this CTA's part is visible before its arrival is counted
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(ctr, 1) == u.nsplit - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();  // the parts counted before this arrival are visible to this CTA
+    const int G = p.group;
+    const int64_t step = (int64_t)p.hq * D;
+    for (int r = warp; r < R; r += kWarps) {
+        const int j = u.j0 + r / G, h = kvh * G + r % G;
+        const int64_t base = (int64_t)u.part_base + (int64_t)(j - u.j0) * u.nsplit;
+        const float* ls = p.ws_lse + base * p.hq + h;  // part i at ls[i * hq]
+        const float* op = p.ws_o + (base * p.hq + h) * D;
+        const int64_t qrow = (int64_t)(si.q_start + j) * p.hq + h;
+        T* o = static_cast<T*>(p.out) + qrow * D;
+        // up to 32 parts: lane i keeps part i's lse and weight, handed out by shuffles; more parts
+        // are read again per use
+        const int n = u.nsplit;
+        const float my_l = lane < n ? __ldcg(ls + (int64_t)lane * p.hq) : neg_inf();
+        float m = my_l;
+        for (int i = lane + 32; i < n; i += 32) m = fmaxf(m, __ldcg(ls + (int64_t)i * p.hq));
+        m = warp_max(m);
+        if (m == neg_inf()) {
+            for (int d = lane; d < D; d += 32) o[d] = from_f32<T>(0.f);
+            if (lane == 0) p.lse[qrow] = m;
+            continue;
+        }
+        float sum = lane < n ? fast_exp2((my_l - m) * kLog2e) : 0.f;
+        for (int i = lane + 32; i < n; i += 32) sum += fast_exp2((__ldcg(ls + (int64_t)i * p.hq) - m) * kLog2e);
+        sum = warp_sum(sum);
+        const float lse = m + __logf(sum);
+        const float my_w = lane < n ? fast_exp2((my_l - lse) * kLog2e) : 0.f;
+        auto weight = [&](int i) {
+            return i < 32 ? __shfl_sync(0xffffffffu, my_w, i)
+                          : fast_exp2((__ldcg(ls + (int64_t)i * p.hq) - lse) * kLog2e);
+        };
+        for (int d0 = 0; d0 < D; d0 += 128) {
+            const int d = d0 + lane * 4;
+            const bool on = d < D;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            int i = 0;
+            for (; i + 4 <= n; i += 4) {  // four parts in flight, added in part order
+                float4 b[4];
+                float w[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    w[x] = weight(i + x);
+                    b[x] = on ? __ldcg(reinterpret_cast<const float4*>(op + (i + x) * step + d))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    acc.x = fmaf(w[x], b[x].x, acc.x);
+                    acc.y = fmaf(w[x], b[x].y, acc.y);
+                    acc.z = fmaf(w[x], b[x].z, acc.z);
+                    acc.w = fmaf(w[x], b[x].w, acc.w);
+                }
+            }
+            for (; i < n; ++i) {
+                const float w = weight(i);
+                const float4 b = on ? __ldcg(reinterpret_cast<const float4*>(op + i * step + d))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                acc.x = fmaf(w, b.x, acc.x);
+                acc.y = fmaf(w, b.y, acc.y);
+                acc.z = fmaf(w, b.z, acc.z);
+                acc.w = fmaf(w, b.w, acc.w);
+            }
+            if (on) {
+                uint2 v;
+                v.x = pack2<T>(acc.x, acc.y);
+                v.y = pack2<T>(acc.z, acc.w);
+                *reinterpret_cast<uint2*>(o + d) = v;
+            }
+        }
+        if (lane == 0) p.lse[qrow] = lse;
+    }
+    if (threadIdx.x == 0) *ctr = 0;  // ready for the next call
+}
+
 template <typename T, int D, int NT, int MT, int STAGES, bool SPARSE>
 __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParams p) {
     using C = DecodeCfg<D, MT, STAGES>;
@@ -330,6 +422,9 @@ __global__ void __launch_bounds__(kWarps * 32) decode_mma_kernel(const AttnParam
             p.ws_o[(slot * p.hq + h) * D + d] = val;
             if (d == 0) p.ws_lse[slot * p.hq + h] = lse;
         }
+    }
+    if constexpr (!SPARSE) {
+        if (p.merge_ctr != nullptr && u.nsplit > 1) merge_own_parts<T, D>(p, u, si, kvh, R);
     }
 }
 

@@ -110,6 +110,10 @@ struct AttnParams {
     // block_size + v % block_size of the sequence (entries of -1 hold no keys).
     const int32_t* sel;  // [Nq, Hkv, sel_width] checked, compacted selection
     int32_t sel_width, block_size;
+    // Tensor-core decode only: when set, split rows are merged by the kernel itself: the CTA that
+    // finishes a (row set, KV head) last, counted at merge_ctr[part_base * hkv + kvh], merges its
+    // parts and puts the counter back to zero (the counters are zero between calls).
+    int* merge_ctr;
 };
 
 // Kernel launchers (one per .cu file). Each returns the launch's cudaError_t.

@@ -64,8 +64,9 @@ def test_decode_head_dim_256(orc, hq, hkv, qn):
 
 
 def test_split_rows_plan_reused(orc):
-    """One plan, five calls with other queries and split sizes (the workspace and the cached work
-    lists reused across calls), each against the oracle; split rows go through the merge kernel."""
+    """One plan, five calls with other queries and split sizes (the workspace, the cached work lists
+    and the merge counters reused across calls), each against the oracle; the tensor-core decode
+    kernel merges its own split rows (no merge launch)."""
     wl = small_decode(5, batch=12, lmin=200, lmax=3000)
     s = wl.sched
     plan = pa.plan_for(wl)
@@ -75,7 +76,7 @@ def test_split_rows_plan_reused(orc):
                             wl.scale, wl.causal, wl.window)
         out, lse = run_gqa(wl, kv_chunk=kv_chunk, plan=plan, q=q)
         k = pa.pa_plan_get_info(plan)["last_kernels"]
-        assert k & pa.PA_KERNEL_DECODE_TC and (kv_chunk == 0 or k & pa.PA_KERNEL_MERGE), k
+        assert k & pa.PA_KERNEL_DECODE_TC and not k & pa.PA_KERNEL_MERGE, k
         check(wl, out, lse, *ref, tag=f"call {i} chunk {kv_chunk}")
     assert pa.pa_plan_device_status(plan) == 0
     plan.close()
