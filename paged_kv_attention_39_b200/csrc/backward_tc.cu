@@ -434,19 +434,21 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 //        buffer of its own (step & 1)
 //   dQ += dS K                 (A = dS from shared memory, B = K, MN-major) -> TMEM [256, 256 + D)
 // The score products of a step go into the buffer the step before last used (its dS is already in
-// shared memory), so they overlap the compute warps' work on the previous step, and the dQ product
-// of a step runs while the compute warps work on the next one. The finished rows are scaled and
-// written once.
+// shared memory), so they overlap the compute warps' work on the previous step; the dQ products come
+// from a second issuing warp, so they run beside the next step's score products rather than queue
+// behind them. The finished rows are scaled and written once.
 //   warps 0..7  compute and the epilogue (two warps per 32 rows, each taking half of a step's keys
 //               and of the dQ columns)
 //   warp 8      loads: Q and dO of the block (TMA), the K and V rows of each step (TMA, one box per
 //               page) into a ring of stages
-//   warp 9      TMEM owner and MMA issuer
+//   warp 9      TMEM owner and issuer of the score products
+//   warp 10     issuer of dQ += dS K (a second chain, which the tensor core overlaps with the first)
 // ---------------------------------------------------------------------------------------------
 namespace {
 
 constexpr int QKB = 64;   // keys per step of the dQ kernel
 constexpr int QKVST = 4;  // K/V stages (the fourth lets the loads run a step further ahead of dQ += dS K)
+constexpr int kDqWarp = 10, kThreadsDq = 11 * 32;  // warp 10 issues dQ += dS K
 
 template <int D>
 struct BqCfg {
@@ -470,7 +472,7 @@ struct BqCfg {
 }  // namespace
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kThreadsB, 1)
+__global__ void __launch_bounds__(kThreadsDq, 1)
     bwd_tc_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmo,
                      const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
                      const BwdParams2 p) {
@@ -588,18 +590,44 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                        globaltimer_ns() - t0 < kWaitLimitNsB) {}
         }
     } else if (warp == kMmaWarp) {
-        // ===================== MMA issuer =====================
+        // ===================== issuer of the score products =====================
         const uint64_t dQ = sdesc_sw128(s_base + L_::Q, 16, 1024);
         const uint64_t dO = sdesc_sw128(s_base + L_::O, 16, 1024);
         bool ok = nsteps == 0 || __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_QFULL], 0, wd, 32));
-        // dQ += dS_j K_j (dS of step j in buffer j & 1, K in stage j % QKVST)
-        auto issue_dq = [&](int j) {
+        for (int j = 0; ok && j < nsteps; ++j) {
+            const int st = j % QKVST, b = j & 1;
+            // buffer b held S and dP of step j - 2, read by the compute warps before they marked P
+            if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL + b], ((j - 2) >> 1) & 1, wd, 34));
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_KVFULL + st], (j / QKVST) & 1, wd, 35));
+            if (!ok) break;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t ks = s_base + L_::K + st * 2 * KH * L_::HALF_K;
+                const uint64_t dK = sdesc_sw128(ks, 16, 1024), dV = sdesc_sw128(ks + KH * L_::HALF_K, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off_r = (kk >> 2) * L_::HALF_R + (kk & 3) * 32;
+                    const uint32_t off_k = (kk >> 2) * L_::HALF_K + (kk & 3) * 32;
+                    mma_f16_ss(tmem + L_::T_S + b * QKB, desc_add(dQ, off_r), desc_add(dK, off_k), IDESC_S, kk > 0);
+                    mma_f16_ss(tmem + L_::T_DP + b * QKB, desc_add(dO, off_r), desc_add(dV, off_k), IDESC_S, kk > 0);
+                }
+                mma_commit(&bars[L_::B_SFULL + b]);
+            }
+            __syncwarp();
+        }
+    } else if (warp == kDqWarp) {
+        // ===================== issuer of dQ += dS_j K_j =====================
+        // dS of step j in buffer j & 1, K in stage j % QKVST; a chain of its own, so that the tensor
+        // core runs it beside the next step's score products instead of behind them
+        bool ok = true;
+        for (int j = 0; ok && j < nsteps; ++j) {
             ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL + (j & 1)], (j >> 1) & 1, wd, 33));
-            if (!ok) return;
+            if (!ok) break;
             tc_fence_after();
             // K rows the step's boxes did not bring (or past the sequence's end) hold arbitrary bytes,
             // and dS is zero there: make them zero too, so that 0 * garbage cannot reach dQ. S and dP of
-            // the step, which read them as well, are complete.
+            // the step, which read them as well, are complete (the compute warps saw them before
+            // marking P).
             const int nz = loaded_rows(j);
             if (nz < QKB) {
                 uint8_t* ks = smem + L_::K + (j % QKVST) * 2 * KH * L_::HALF_K;
@@ -623,30 +651,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                 if (j == nsteps - 1) mma_commit(&bars[L_::B_DQFULL]);
             }
             __syncwarp();
-        };
-        for (int j = 0; ok && j < nsteps; ++j) {
-            const int st = j % QKVST, b = j & 1;
-            // buffer b held S and dP of step j - 2, read by the compute warps before they marked P
-            if (j >= 2) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_PFULL + b], ((j - 2) >> 1) & 1, wd, 34));
-            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars[L_::B_KVFULL + st], (j / QKVST) & 1, wd, 35));
-            if (!ok) break;
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t ks = s_base + L_::K + st * 2 * KH * L_::HALF_K;
-                const uint64_t dK = sdesc_sw128(ks, 16, 1024), dV = sdesc_sw128(ks + KH * L_::HALF_K, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off_r = (kk >> 2) * L_::HALF_R + (kk & 3) * 32;
-                    const uint32_t off_k = (kk >> 2) * L_::HALF_K + (kk & 3) * 32;
-                    mma_f16_ss(tmem + L_::T_S + b * QKB, desc_add(dQ, off_r), desc_add(dK, off_k), IDESC_S, kk > 0);
-                    mma_f16_ss(tmem + L_::T_DP + b * QKB, desc_add(dO, off_r), desc_add(dV, off_k), IDESC_S, kk > 0);
-                }
-                mma_commit(&bars[L_::B_SFULL + b]);
-            }
-            __syncwarp();
-            if (j >= 1) issue_dq(j - 1);  // the previous step's dQ, while this step's scores run
         }
-        if (ok && nsteps > 0) issue_dq(nsteps - 1);
     } else {
         // ===================== compute: thread = row, half hf of the keys / dQ columns =====================
         const int hf = warp >> 2;
@@ -797,7 +802,7 @@ cudaError_t launch_bq(const BwdParams2& p, int num_row_units, int64_t num_querie
         if (e != cudaSuccess) return e;
         if (dev < 64) configured |= 1ull << dev;
     }
-    kern<<<dim3(num_row_units, p.hkv), kThreadsB, L_::ALLOC, st>>>(tq, to, tk, tv, p);
+    kern<<<dim3(num_row_units, p.hkv), kThreadsDq, L_::ALLOC, st>>>(tq, to, tk, tv, p);
     return cudaGetLastError();
 }
 
