@@ -373,7 +373,8 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
             ("bf16_decode_d256", lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256)),
             ("bf16_chunked_prefill_d256", lambda sd: W.c3_prefill_variant(sd, torch.bfloat16, 256)),
             ("bf16_append_chunk", W.append_chunk), ("bf16_backward_chunk", W.backward_chunk),
-            ("bf16_mla_backward", W.mla_backward_small)]
+            ("bf16_mla_backward", W.mla_backward_small),
+            ("bf16_mla_backward_decode_batch", W.mla_backward_decode_batch)]
     if only is not None:
         cfgs = [only]
     for name, fn in cfgs:
@@ -386,8 +387,9 @@ def run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=None):
         if name == "bf16_backward_chunk":
             res[name] = run_backward(args, pa, W, dev, tf_burst, peak_src)
             continue
-        if name == "bf16_mla_backward":
-            res[name] = run_mla_backward(args, pa, W, dev, tf_burst, peak_src)
+        if name in ("bf16_mla_backward", "bf16_mla_backward_decode_batch"):
+            res[name] = run_mla_backward(args, pa, W, dev, tf_burst, peak_src,
+                                         "small" if name == "bf16_mla_backward" else "decode_batch")
             continue
         try:
             wl = fn(args.seed)
@@ -528,11 +530,12 @@ def run_backward(args, pa, W, dev, tf_burst, peak_src):
         return {"error": str(e)[:300]}
 
 
-def run_mla_backward(args, pa, W, dev, tf_burst, peak_src):
-    """MLA backward of 4 decode sequences (128 heads, context U[256, 1024]): CUDA-core kernel, a warp
-    per (query, head) row, float32 atomics into the latent and rope gradient caches."""
+def run_mla_backward(args, pa, W, dev, tf_burst, peak_src, batch="small"):
+    """MLA backward of a decode batch: 4 sequences with context U[256, 1024] ("small"), or the MLA
+    decode batch (32 sequences, context U[1024, 16384]); 128 heads, latent 512, rope 64. The gradient
+    caches are zeroed before each timed call, outside the timed region."""
     try:
-        wl, d_out = W.mla_backward_small(args.seed)
+        wl, d_out = W.mla_backward_small(args.seed) if batch == "small" else W.mla_backward_decode_batch(args.seed)
         plan = pa.plan_for(wl, device=dev.index)
         ql, qr = wl.q_latent.to(dev), wl.q_rope.to(dev)
         lat, rope = wl.latent_cache.to(dev), wl.rope_cache.to(dev)
@@ -551,11 +554,16 @@ def run_mla_backward(args, pa, W, dev, tf_burst, peak_src):
         ms = event_median(lambda: pa.pa_mla_backward(plan, ql, qr, lat, rope, out, lse, d_out, dql, dqr, dlat, drope,
                                                      wl.scale, wl.causal, wl.window), zero, max(args.extra_steps, 3), 2)
         flops = W.mla_backward_flops(wl)
+        info = pa.pa_plan_get_info(plan)
         plan.close()
+        tc = bool(info["last_kernels"] & pa.PA_KERNEL_BACKWARD_TC)
         return {"ms_per_step": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
                 "frac_tensor_of_%s" % peak_src: round(flops / (ms * 1e-3) / 1e12 / tf_burst, 4),
-                "algorithmic_gflop": round(flops / 1e9, 2), "launches": 1,
-                "note": "CUDA-core float32 kernel with atomics (the MLA backward's first, correct version)"}
+                "algorithmic_gflop": round(flops / 1e9, 2), "launches": info["last_launches"],
+                "kernels": kernel_names(info["last_kernels"]),
+                "note": ("Drow kernel, key tiles on tcgen05 (CTA pairs over the latent's column halves, TMA "
+                         "reduce-adds), dQ per 64-column chunk on tcgen05" if tc else
+                         "CUDA-core float32 kernel with atomics")}
     except Exception as e:  # a failing extra must not hide the headline
         return {"error": str(e)[:300]}
 
@@ -577,7 +585,8 @@ def run_single(args, ws, rank, local):
            "bf16_decode_d256": lambda sd: W.c2_decode_variant(sd, torch.bfloat16, 256),
            "bf16_chunked_prefill_d256": lambda sd: W.c3_prefill_variant(sd, torch.bfloat16, 256),
            "bf16_append_chunk": W.append_chunk, "bf16_backward_chunk": W.backward_chunk,
-           "bf16_mla_backward": W.mla_backward_small}
+           "bf16_mla_backward": W.mla_backward_small,
+           "bf16_mla_backward_decode_batch": W.mla_backward_decode_batch}
     res = run_extra(args, pa, W, dev, hbm, tf_burst, peak_src, only=(args.workload, fns[args.workload]))
     r = res[args.workload]
     if args.workload in ("bf16_sparse_topk_decode", "bf16_append_chunk"):
@@ -664,7 +673,8 @@ def main():
                              "bf16_window_mixed_decode_part", "bf16_window_mixed_prefill_part",
                              "tiny_fp32_decode", "fp16_decode", "bf16_decode_d64", "bf16_decode_d256",
                              "bf16_chunked_prefill_d256",
-                             "bf16_append_chunk", "bf16_backward_chunk", "bf16_mla_backward"],
+                             "bf16_append_chunk", "bf16_backward_chunk", "bf16_mla_backward",
+                             "bf16_mla_backward_decode_batch"],
                     help="the headline is bf16_decode; the others run alone for profiling")
     args = ap.parse_args()
     if args.warmup < 3:

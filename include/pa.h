@@ -285,10 +285,17 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
  *   d_q_rope         [N_q, num_heads, rope_dim]   float32, written
  *   d_latent_cache   [num_pages, page_size, 1, latent_dim] float32, ADDED INTO (zero it first)
  *   d_rope_cache     [num_pages, page_size, 1, rope_dim]   float32, ADDED INTO (zero it first)
- * A warp per (query, head) row on the CUDA cores, float32 throughout; the cache gradients are
- * float32 atomics, so their summation order varies between runs. Shapes as pa_mla_forward;
- * validation and errors as pa_backward (gradient outputs must not overlap each other or any
- * input).
+ * bf16 / fp16 with latent_dim 512 and rope_dim 64, every sequence's rows (its queries x num_heads)
+ * at most 128, a page size that is a multiple of 16 and divides 128 or is a multiple of 128, fewer
+ * than 2^31 cache rows, and no page used by two keys of the plan run on the tensor cores (tcgen05,
+ * every operand moved by TMA): a Drow kernel, a key-major kernel (a CTA pair per 128 keys, each
+ * owning half of the latent's columns and adding its finished rows once by TMA reduce-adds: the
+ * result repeats bit for bit), and a dQ kernel (a CTA per sequence and 64-column chunk of
+ * [latent | rope]); P and scale * dS are rounded to the input type before the gradient products.
+ * Other shapes, fp32 and plans that share pages run a warp per (query, head) row on the CUDA cores,
+ * float32 throughout, with float32 atomics into the cache gradients, so their summation order varies
+ * between runs. Shapes as pa_mla_forward; validation and errors as pa_backward (gradient outputs
+ * must not overlap each other or any input).
  */
 pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rope,
                           const void* latent_cache, const void* rope_cache, const void* out,

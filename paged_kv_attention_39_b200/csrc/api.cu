@@ -211,6 +211,15 @@ struct pa_plan {
     size_t bwd_scratch_bytes = 0;
     int* merge_ctr = nullptr;  // arrival counters of the decode kernel's own merge, zero between calls
     size_t merge_ctr_n = 0;
+    // tensor-core MLA backward: key tiles and dQ units for one (heads, causal, window), the dS' scratch
+    void* mla_bwd_dev = nullptr;
+    int32_t mla_bwd_h = 0, mla_bwd_causal = -1, mla_bwd_window = -1, mla_ntiles = 0, mla_ndq = 0;
+    size_t mla_dq_off = 0;
+    int64_t mla_ds_cols = 0;
+    std::vector<char> mla_bwd_host;
+    void* mla_ds = nullptr;
+    size_t mla_ds_bytes = 0;
+    int shared_pages = -1;  // -1 unknown, 0 every used page belongs to one sequence once, 1 some page is shared
     cudaStream_t last_stream = nullptr;  // stream of the last call: frees are ordered on it
     int32_t last_launches = 0;
     int32_t last_kernels = 0;  // PA_KERNEL_* bits of the last call
@@ -842,6 +851,8 @@ pa_status pa_plan_destroy(pa_plan* plan) {
         if (plan->bwd_drow) cudaFreeAsync(plan->bwd_drow, st);
         if (plan->bwd_scratch) cudaFreeAsync(plan->bwd_scratch, st);
         if (plan->merge_ctr) cudaFreeAsync(plan->merge_ctr, st);
+        if (plan->mla_bwd_dev) cudaFreeAsync(plan->mla_bwd_dev, st);
+        if (plan->mla_ds) cudaFreeAsync(plan->mla_ds, st);
         for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
         cudaError_t e = plan->d_meta ? cudaFreeAsync(plan->d_meta, st) : cudaSuccess;
         delete plan;
@@ -1305,6 +1316,68 @@ pa_status pa_backward(pa_plan* plan, const void* q, const void* k_cache, const v
     return ok();
 }
 
+// Whether some page is used by more than one key of the plan (a shared prefix, a page listed twice).
+static bool plan_has_shared_pages(pa_plan* plan) {
+    if (plan->shared_pages < 0) {
+        std::vector<int32_t> refs((size_t)std::max(1, plan->num_pages), 0);
+        bool shared = false;
+        for (int32_t si = 0; si < plan->S && !shared; ++si) {
+            const int64_t used = ((int64_t)plan->seqs[si].L + plan->page_size - 1) / plan->page_size;
+            for (int64_t b = 0; b < used && !shared; ++b)
+                shared = ++refs[plan->bt[(size_t)si * plan->table_width + b]] > 1;
+        }
+        plan->shared_pages = shared ? 1 : 0;
+    }
+    return plan->shared_pages == 1;
+}
+
+// Work lists of the tensor-core MLA backward for one (heads, causal, window): the 128-key tiles of
+// every sequence that some of its rows see (each with its columns in the dS' scratch), and one dQ
+// unit per sequence with rows, over the same tiles. One upload; the host blob stays with the plan.
+static pa_status build_mla_backward_lists(pa_plan* plan, int32_t H, int causal, int32_t window, cudaStream_t st) {
+    const int KT = pa::kMlaBwdKeyTile;
+    std::vector<pa::MlaKeyTile> tiles;
+    std::vector<pa::MlaDqUnit> units;
+    int64_t cols = 0;
+    for (int32_t si = 0; si < plan->S; ++si) {
+        const pa::SeqInfo& q_ = plan->seqs[si];
+        if (q_.n == 0) continue;
+        // keys any row sees: from the first query's window start to the end of the sequence
+        const int64_t first = (int64_t)q_.L - q_.n;
+        const int64_t lo = window > 0 ? std::max<int64_t>(0, first - window + 1) : 0;
+        const int64_t k0 = lo / KT * KT;
+        const int64_t n_t = q_.L > k0 ? (q_.L - k0 + KT - 1) / KT : 0;
+        units.push_back({si, (int32_t)k0, (int32_t)(k0 + n_t * KT), (int32_t)cols});
+        for (int64_t i = 0; i < n_t; ++i) {
+            tiles.push_back({si, (int32_t)(k0 + i * KT), (int32_t)cols, 0});
+            cols += KT;
+        }
+    }
+    if (cols > INT32_MAX) return fail(PA_ERR_BOUNDS, "MLA backward scratch too wide");
+    (void)causal;
+    auto align = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t dq_off = align(tiles.size() * sizeof(pa::MlaKeyTile));
+    const size_t bytes = std::max<size_t>(256, align(dq_off + units.size() * sizeof(pa::MlaDqUnit)));
+    plan->mla_bwd_host.assign(bytes, 0);
+    if (!tiles.empty()) std::memcpy(plan->mla_bwd_host.data(), tiles.data(), tiles.size() * sizeof(pa::MlaKeyTile));
+    if (!units.empty())
+        std::memcpy(plan->mla_bwd_host.data() + dq_off, units.data(), units.size() * sizeof(pa::MlaDqUnit));
+    if (plan->mla_bwd_dev) PA_CUDA_TRY(cudaFreeAsync(plan->mla_bwd_dev, st));
+    plan->mla_bwd_dev = nullptr;
+    plan->mla_bwd_h = 0;
+    PA_CUDA_TRY(lib_malloc(&plan->mla_bwd_dev, bytes, st));
+    PA_CUDA_TRY(upload(plan->mla_bwd_dev, plan->mla_bwd_host.data(), bytes, st));
+    plan->uploaded_bytes += (int64_t)bytes;
+    plan->mla_ntiles = (int32_t)tiles.size();
+    plan->mla_ndq = (int32_t)units.size();
+    plan->mla_dq_off = dq_off;
+    plan->mla_ds_cols = std::max<int64_t>(cols, KT);
+    plan->mla_bwd_h = H;
+    plan->mla_bwd_causal = causal;
+    plan->mla_bwd_window = window;
+    return PA_OK;
+}
+
 pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rope, const void* latent_cache,
                           const void* rope_cache, const void* out, const float* lse, const void* d_out, pa_dtype dtype,
                           int32_t num_heads, int32_t latent_dim, int32_t rope_dim, float scale, int causal,
@@ -1350,6 +1423,50 @@ pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rop
     PA_CUDA_TRY(cudaGetDevice(&cur));
     if (cur != plan->device)
         return fail(PA_ERR_INVALID_ARGUMENT, "current device %d is not the plan's device %d", cur, plan->device);
+    cudaStream_t st = (cudaStream_t)stream;
+    // The tensor-core path: bf16 / fp16, latent 512, rope 64, every sequence's rows (queries x heads)
+    // within one block of 128, pages of a size the key tiles take whole, no page used twice (each
+    // cache row then has one writer), 32-bit cache rows.
+    bool tc = pa::mla_backward_tc_supported(dtype, latent_dim, rope_dim, num_heads) && ps % 16 == 0 &&
+              (pa::kMlaBwdKeyTile % ps == 0 || ps % pa::kMlaBwdKeyTile == 0) && pages * ps < ((int64_t)1 << 31) &&
+              nq * num_heads < ((int64_t)1 << 31);
+    for (int32_t si = 0; tc && si < plan->S; ++si) tc = (int64_t)plan->seqs[si].n * num_heads <= 128;
+    if (tc) {
+        std::lock_guard<std::mutex> lock(plan->mu);
+        tc = !plan_has_shared_pages(plan);
+        if (tc) {
+            if (plan->mla_bwd_h != num_heads || plan->mla_bwd_causal != causal || plan->mla_bwd_window != window) {
+                pa_status bs = build_mla_backward_lists(plan, num_heads, causal, window, st);
+                if (bs != PA_OK) return bs;
+            }
+            pa_status gs = grow_buffer(&plan->bwd_drow, &plan->bwd_drow_bytes, (size_t)nq * num_heads * sizeof(float), st);
+            if (gs != PA_OK) return gs;
+            gs = grow_buffer(&plan->mla_ds, &plan->mla_ds_bytes, (size_t)128 * plan->mla_ds_cols * 2, st);
+            if (gs != PA_OK) return gs;
+            cudaError_t e = pa::launch_bwd_dot(out, d_out, plan->bwd_drow, nq * num_heads, latent_dim, dtype, st);
+            if (e == cudaSuccess) {
+                pa::MlaBwdTcParams mp{};
+                mp.ql = q_latent; mp.qr = q_rope; mp.lat = latent_cache; mp.rope = rope_cache; mp.dout = d_out;
+                mp.lse = lse; mp.drow = plan->bwd_drow;
+                mp.dql = d_q_latent; mp.dqr = d_q_rope; mp.dlat = d_latent_cache; mp.drope = d_rope_cache;
+                mp.ds = plan->mla_ds; mp.ds_cols = plan->mla_ds_cols;
+                mp.seqs = plan->d_seqs; mp.block_tables = plan->d_bt;
+                mp.tiles = (const pa::MlaKeyTile*)plan->mla_bwd_dev;
+                mp.dq_units = (const pa::MlaDqUnit*)((const char*)plan->mla_bwd_dev + plan->mla_dq_off);
+                mp.table_width = plan->table_width; mp.page_size = plan->page_size; mp.h = num_heads;
+                mp.num_pages = plan->num_pages;
+                mp.scale = scale; mp.scale_log2 = scale * 1.4426950408889634f;
+                mp.causal = causal; mp.window = window;
+                mp.err = plan->d_err;
+                e = pa::launch_mla_backward_tc(mp, dtype, plan->mla_ntiles, plan->mla_ndq, nq, st);
+            }
+            if (e != cudaSuccess) return fail(PA_ERR_CUDA, "MLA backward kernel launch failed: %s", cudaGetErrorString(e));
+            plan->last_stream = st;
+            plan->last_launches = 1 + (plan->mla_ntiles > 0 ? 1 : 0) + (plan->mla_ndq > 0 ? 1 : 0);
+            plan->last_kernels = PA_KERNEL_BACKWARD_TC;
+            return ok();
+        }
+    }
     cudaError_t e = pa::launch_mla_backward(q_latent, q_rope, latent_cache, rope_cache, out, lse, d_out, d_q_latent,
                                             d_q_rope, d_latent_cache, d_rope_cache, plan->d_seqs, plan->d_q2seq,
                                             plan->d_bt, plan->table_width, plan->page_size, num_heads, latent_dim,

@@ -137,6 +137,19 @@ cudaError_t bwd_launch_d(const BwdParams2& p, int num_key_units, int num_row_uni
 
 }  // namespace
 
+cudaError_t launch_bwd_dot(const void* out, const void* dout, float* drow, int64_t rows, int dv, pa_dtype dt,
+                           cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((rows + 3) / 4);
+    if (dt == PA_BF16)
+        bwd_dot_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(out),
+                                                             static_cast<const __nv_bfloat16*>(dout), drow, rows, dv);
+    else
+        bwd_dot_kernel<__half><<<grid, 128, 0, st>>>(static_cast<const __half*>(out), static_cast<const __half*>(dout),
+                                                      drow, rows, dv);
+    return cudaGetLastError();
+}
+
 bool backward_mma_supported(pa_dtype dt, int d, int dv, int group) {
     // both tcgen05 passes walk 128-row blocks: 128 / G queries x the G heads of a KV head
     return (dt == PA_BF16 || dt == PA_F16) && d == dv && (d == 64 || d == 128) && group >= 1 && 128 % group == 0;

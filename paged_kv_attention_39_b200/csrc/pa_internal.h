@@ -153,6 +153,46 @@ cudaError_t launch_backward_tc_dq(const BwdParams2& p, pa_dtype dt, int num_row_
                                   cudaStream_t st);
 cudaError_t launch_backward_mma(const BwdParams2& p, pa_dtype dt, int num_key_units, int num_row_units, int64_t rows,
                                 int num_slot_sums, cudaStream_t st);
+// Drow = dO . O per row (backward_mma.cu), for the other backward paths.
+cudaError_t launch_bwd_dot(const void* out, const void* dout, float* drow, int64_t rows, int dv, pa_dtype dt,
+                           cudaStream_t st);
+
+// Tensor-core MLA backward (mla_backward_tc.cu): latent 512, rope 64, every sequence's rows
+// (queries x heads) within one block of 128. Key tiles of 128 keys (two CTAs each: the latent's
+// column halves), then dQ per (sequence, 64-column chunk of [latent | rope]).
+struct MlaKeyTile {
+    int32_t seq, k0, koff, pad;  // keys [k0, k0 + 128) of sequence seq; scratch key column koff + (t - k0)
+};
+struct MlaDqUnit {
+    int32_t seq, k0, k1, koff;   // the sequence's key tiles cover [k0, k1); scratch columns from koff
+};
+struct MlaBwdTcParams {
+    const void* ql;      // [Nq, H, 512]
+    const void* qr;      // [Nq, H, 64]
+    const void* lat;     // [P, ps, 1, 512]
+    const void* rope;    // [P, ps, 1, 64]
+    const void* dout;    // [Nq, H, 512]
+    const float* lse;    // [Nq, H]
+    const float* drow;   // [Nq, H] dO . O
+    float* dql;          // [Nq, H, 512] written
+    float* dqr;          // [Nq, H, 64] written
+    float* dlat;         // [P, ps, 1, 512] added into
+    float* drope;        // [P, ps, 1, 64] added into
+    void* ds;            // [128][ds_cols] 16-bit scale * dS, row = the sequence's row (query x head)
+    int64_t ds_cols;
+    const SeqInfo* seqs;
+    const int32_t* block_tables;
+    const MlaKeyTile* tiles;
+    const MlaDqUnit* dq_units;
+    int32_t table_width, page_size, h, num_pages;
+    float scale, scale_log2;
+    int32_t causal, window;
+    int* err;
+};
+constexpr int kMlaBwdKeyTile = 128;
+bool mla_backward_tc_supported(pa_dtype dt, int latent_dim, int rope_dim, int num_heads);
+cudaError_t launch_mla_backward_tc(const MlaBwdTcParams& p, pa_dtype dt, int num_tiles, int num_dq_units,
+                                   int64_t num_queries, cudaStream_t st);
 // Sparse top-K block selection (sparse.cu).
 cudaError_t launch_sparse_scores(const void* q, const void* k, float* scores, int32_t sw, const SeqInfo* seqs,
                                  const int32_t* q2seq, const int32_t* block_tables, int32_t table_width,

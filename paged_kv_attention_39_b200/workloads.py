@@ -333,11 +333,19 @@ def backward_flops(wl) -> int:
 
 
 def mla_backward_small(seed: int = 0, batch: int = 4, lmin: int = 256, lmax: int = 1024):
-    """Backward of an MLA decode batch (128 heads, latent 512, rope 64, pages of 64, bf16), small
-    enough for the CUDA-core kernel: (workload, d_out [Nq, H, R])."""
+    """Backward of a small MLA decode batch (128 heads, latent 512, rope 64, pages of 64, bf16):
+    (workload, d_out [Nq, H, R])."""
     lens = _uniform_ints(seed, 0xB5, batch, lmin, lmax)
     wl = make_mla(f"bf16_mla_backward_b{batch}", seed, lens, [1] * batch, 128, 512, 64, 64, torch.bfloat16)
     d_out = randn((wl.sched.num_queries, 128, 512), seed, 24, torch.bfloat16)
+    return wl, d_out
+
+
+def mla_backward_decode_batch(seed: int = 0):
+    """Backward of the MLA decode batch (32 sequences, context U[1024, 16384], 128 heads, latent
+    512, rope 64, pages of 64, bf16): (workload, d_out [Nq, H, R])."""
+    wl = c5_mla_decode(seed)
+    d_out = randn((wl.sched.num_queries, 128, 512), seed, 25, torch.bfloat16)
     return wl, d_out
 
 

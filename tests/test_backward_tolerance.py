@@ -93,6 +93,20 @@ def _cases():
         g = torch.Generator().manual_seed(11)
         dout = torch.randn(wl.sched.num_queries, hq, d, generator=g).to(dtype)
         out.append((f"tensor_core_shapes hq{hq} hkv{hkv} d{d} ps{ps} c{causal} w{window}", wl, dout))
+    # the tensor-core MLA backward's shapes, as the GQA backward they are: one KV head, the key
+    # [latent | rope] (576 columns), the value the latent (512), every query head in the group
+    for h, lens, qs, ps, dtype, causal, window in [
+            (128, [700, 2000, 130, 4100], [1, 1, 1, 1], 64, torch.bfloat16, True, 0),
+            (16, [300, 513, 64, 1000], [8, 3, 1, 5], 16, torch.float16, True, 300),
+            (128, [90, 1500, 257], [1, 1, 1], 128, torch.bfloat16, False, 0),
+            (64, [1024, 777], [2, 1], 32, torch.bfloat16, True, 0)]:
+        m = W.make_mla("mla_bwd_tc", 19, lens, qs, h, 512, 64, ps, dtype, causal=causal, window=window)
+        wl = W.GqaWorkload("mla_as_gqa", m.sched, torch.cat([m.q_latent, m.q_rope], dim=-1),
+                           torch.cat([m.latent_cache, m.rope_cache], dim=-1), m.latent_cache, h, 1, 576, 512,
+                           m.scale, causal, window)
+        g = torch.Generator().manual_seed(21)
+        dout = torch.randn(m.sched.num_queries, h, 512, generator=g).to(dtype)
+        out.append((f"mla tensor core h{h} ps{ps} {dtype} c{causal} w{window}", wl, dout))
     wl = W.make_gqa("share_tc", 6, [150, 150], [30, 30], 8, 2, 64, 64, 16, torch.bfloat16)
     wl.sched.block_tables[1, :3] = wl.sched.block_tables[0, :3]
     g = torch.Generator().manual_seed(12)

@@ -228,3 +228,72 @@ def test_mla_backward_matches_oracle(orc, h, r, pr, ps, dtype, causal, window):
     tag = f"mla h{h} r{r} pr{pr} {dtype}"
     for got, want, name in zip((dql, dqr, dlat, drope), ref, ("dq_latent", "dq_rope", "d_latent", "d_rope")):
         close(got.cpu(), want, dtype, f"{name} {tag}")
+
+
+def _mla_backward_run(wl, causal, window, seed):
+    s = wl.sched
+    g = torch.Generator().manual_seed(seed)
+    nq, h, r, pr = s.num_queries, wl.num_heads, wl.latent_dim, wl.rope_dim
+    dtype = wl.q_latent.dtype
+    dout = torch.randn(nq, h, r, generator=g).to(dtype)
+    ql, qr = wl.q_latent.cuda(), wl.q_rope.cuda()
+    lat, rope = wl.latent_cache.cuda(), wl.rope_cache.cuda()
+    plan = pa.plan_for(wl)
+    out = torch.empty(nq, h, r, dtype=dtype, device="cuda")
+    lse = torch.empty(nq, h, dtype=torch.float32, device="cuda")
+    pa.pa_mla_forward(plan, ql, qr, lat, rope, out, lse, wl.scale, causal, window)
+    dql = torch.full((nq, h, r), float("nan"), dtype=torch.float32, device="cuda")
+    dqr = torch.full((nq, h, pr), float("nan"), dtype=torch.float32, device="cuda")
+    dlat = torch.zeros(lat.shape, dtype=torch.float32, device="cuda")
+    drope = torch.zeros(rope.shape, dtype=torch.float32, device="cuda")
+    pa.pa_mla_backward(plan, ql, qr, lat, rope, out, lse, dout.cuda(), dql, dqr, dlat, drope, wl.scale, causal,
+                       window)
+    torch.cuda.synchronize()
+    assert pa.pa_plan_device_status(plan) == 0
+    kernels = pa.pa_plan_get_info(plan)["last_kernels"]
+    plan.close()
+    return dout, (dql.cpu(), dqr.cpu(), dlat.cpu(), drope.cpu()), kernels
+
+
+@pytest.mark.parametrize("h,lens,qs,ps,dtype,causal,window", [
+    (128, [700, 2000, 130, 4100], [1, 1, 1, 1], 64, torch.bfloat16, True, 0),   # decode, many key tiles
+    (16, [300, 513, 64, 1000], [8, 3, 1, 5], 16, torch.float16, True, 300),     # 16 heads x up to 8 queries, window
+    (128, [90, 1500, 257], [1, 1, 1], 128, torch.bfloat16, False, 0),           # a tile shorter than 128 keys
+    (64, [1024, 777], [2, 1], 32, torch.bfloat16, True, 0),                     # 2 queries x 64 heads = 128 rows
+])
+def test_mla_backward_tensor_core(orc, h, lens, qs, ps, dtype, causal, window):
+    """The tensor-core MLA backward (latent 512, rope 64, every sequence's rows within one block of
+    128): key tiles in CTA pairs over the latent's column halves, dQ per 64-column chunk; against the
+    oracle, and on the tensor-core path."""
+    wl = W.make_mla("mla_bwd_tc", 19, lens, qs, h, 512, 64, ps, dtype, causal=causal, window=window)
+    dout, got, kernels = _mla_backward_run(wl, causal, window, 21)
+    assert kernels == pa.PA_KERNEL_BACKWARD_TC, kernels
+    s = wl.sched
+    ref = orc.mla_backward(wl.q_latent, wl.q_rope, wl.latent_cache, wl.rope_cache, dout, s.seq_lens,
+                           s.query_offsets, s.block_tables, ps, wl.scale, causal, window)
+    tag = f"mla tc h{h} ps{ps} {dtype} c{causal} w{window}"
+    for g, want, name in zip(got, ref, ("dq_latent", "dq_rope", "d_latent", "d_rope")):
+        close(g, want, dtype, f"{name} {tag}")
+
+
+def test_mla_backward_shared_pages_take_the_cuda_core_kernel(orc):
+    """Sequences sharing a page would give its cache rows two writers: the CUDA-core kernel (float32
+    atomics) takes such plans, and the shared slots get both sequences' gradients."""
+    wl = W.make_mla("mla_bwd_share", 23, [200, 200], [1, 1], 128, 512, 64, 64, torch.bfloat16)
+    s = wl.sched
+    s.block_tables[1, :2] = s.block_tables[0, :2]  # keys 0..127 shared
+    dout, got, kernels = _mla_backward_run(wl, True, 0, 24)
+    assert kernels == pa.PA_KERNEL_BACKWARD_SIMT, kernels
+    ref = orc.mla_backward(wl.q_latent, wl.q_rope, wl.latent_cache, wl.rope_cache, dout, s.seq_lens,
+                           s.query_offsets, s.block_tables, 64, wl.scale, True, 0)
+    for g, want, name in zip(got, ref, ("dq_latent", "dq_rope", "d_latent", "d_rope")):
+        close(g, want, torch.bfloat16, f"{name} shared pages")
+
+
+def test_mla_backward_tensor_core_deterministic():
+    """Every cache row of the tensor-core MLA backward has one writer: two runs give the same bits."""
+    wl = W.make_mla("mla_bwd_det", 25, [900, 300], [1, 1], 128, 512, 64, 64, torch.bfloat16)
+    a = _mla_backward_run(wl, True, 0, 26)[1]
+    b = _mla_backward_run(wl, True, 0, 26)[1]
+    for x, y in zip(a, b):
+        assert torch.equal(torch.nan_to_num(x, nan=0.0), torch.nan_to_num(y, nan=0.0))
