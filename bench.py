@@ -161,6 +161,8 @@ def e2e_library():
         lib.pa_e2e_uploaded_bytes.argtypes = [P]
         lib.pa_e2e_host_times.restype = None
         lib.pa_e2e_host_times.argtypes = [P, ctypes.POINTER(ctypes.c_double)]
+        lib.pa_e2e_gpu_times.restype = None
+        lib.pa_e2e_gpu_times.argtypes = [P, ctypes.POINTER(ctypes.c_double)]
         _E2E = lib
     return _E2E
 
@@ -293,6 +295,8 @@ def run_ours(args, ws, rank, local):
     e2e_val = total_bytes / (e2e_ms * 1e-3) / 1e9
     host_us = (ctypes.c_double * 6)()
     lib.pa_e2e_host_times(loop, host_us)
+    gpu_us = (ctypes.c_double * 2)()
+    lib.pa_e2e_gpu_times(loop, gpu_us)
     uploaded = lib.pa_e2e_uploaded_bytes(loop)
     lib.pa_e2e_destroy(loop)
     plan.close()
@@ -344,6 +348,10 @@ def run_ours(args, ws, rank, local):
             "d2h_bytes_per_step": int(out_bytes + lse_bytes),
             "host_us_per_step": {name: round(host_us[i] / max(1, e2e_steps), 1) for i, name in enumerate(
                 ("plan_create", "plan_prepare", "copies", "forward", "plan_release", "wait"))},
+            # device side of the same steps: the forward's kernels, and the compute stream idle
+            # before each forward (waiting for the step's uploads or for the host to issue it)
+            "gpu_us_per_step": {"forward": round(gpu_us[0] / max(1, e2e_steps - 1), 1),
+                                "idle_before_forward": round(gpu_us[1] / max(1, e2e_steps - 2), 1)},
             "ms_per_step": round(e2e_ms, 4),
             "includes": "a C loop over the public C ABI (libpa_e2e.so); per step: a new plan (pa_plan_create + "
                         "pa_plan_prepare: schedule and work-list uploads) and the H2D of Q from pinned memory on "

@@ -5,10 +5,12 @@
 //
 // Proxy scores. Block b of sequence s holds keys [b * bs, min((b + 1) * bs, L_s)). For query i
 // and KV head h the proxy query is query head h * G; the block's score is the largest
-// scale * q_proxy . k_t over the keys t of the block the query sees, -inf if none. One warp
-// scores one block: four lanes share a key row (each loads a 16-byte chunk of every 64 bytes,
-// so a row is read as whole 32-byte sectors), eight rows per step, float32 dot products of the
-// stored values, then a max over the warp. The kernel is an HBM stream of the K rows.
+// scale * q_proxy . k_t over the keys t of the block the query sees, -inf if none. The pass is an
+// HBM stream of the K rows with float32 dot products of the stored values. When a cache slot (the
+// Hkv rows of one key) fits one warp at 64 bytes per lane, a CTA scores one (query, block) for
+// every KV head and each warp reads whole slots; otherwise one warp scores one (query, KV head,
+// block), four lanes sharing a key row, or, for rows that are not a multiple of 64 bytes, one lane
+// per key row.
 //
 // Top-K. One CTA per (query, KV head) row sorts (score, index) pairs packed into 64-bit keys
 // (descending score, then ascending index) with a bitonic sort in shared memory, keeps the first
@@ -161,6 +163,86 @@ __global__ void __launch_bounds__(kProxyWarps * 32) proxy_scores_generic_kernel(
     if (lane == 0) out[b] = m == neg_inf() ? m : canonical_zero(m * p.scale);
 }
 
+// Every KV head of one (query, block) in one CTA: a key's cache slot (its Hkv rows, contiguous) is
+// read by one warp in one pass, lane l taking 64 bytes of row l / LPR (LPR = row bytes / 64 lanes
+// per row), so each load instruction of a warp covers whole 128-byte lines. Warp w takes keys
+// lo + w, lo + w + kProxyAllWarps, ..., kProxyUnroll of them per step with all their loads in flight;
+// the LPR partial dot products of a row meet by shuffles, and the warps' maxima in shared memory.
+// Page arithmetic in 32 bits (positions are below 2^31).
+constexpr int kProxyAllWarps = 4;
+constexpr int kProxyUnroll = 4;
+
+template <typename T, int LPR>
+__global__ void __launch_bounds__(kProxyAllWarps * 32) proxy_scores_slot_kernel(const ProxyParams p) {
+    constexpr int EPC = 16 / (int)sizeof(T);  // elements per 16-byte chunk
+    constexpr int CPL = 4;                    // chunks per lane: 64 bytes
+    __shared__ float wmax[kProxyAllWarps][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.x;
+    const int64_t qi = blockIdx.y;
+    const int32_t s = p.q2seq[qi];
+    const SeqInfo si = p.seqs[s];
+    const int nb = (si.L + p.block_size - 1) / p.block_size;
+    const int64_t pos = (int64_t)si.L - si.n + (qi - si.q_start);
+    const int h = lane / LPR, part = lane % LPR;
+    const bool head_lane = h < p.hkv;
+    float* out = p.scores + qi * p.hkv * (int64_t)p.sw + b;  // + head * sw
+    int64_t lo64 = 0, hi64 = 0;
+    if (b < nb) block_visible(si, pos, b, p.block_size, p.causal, p.window, &lo64, &hi64);
+    if (lo64 >= hi64) {
+        if (warp == 0 && part == 0 && head_lane) out[(int64_t)h * p.sw] = neg_inf();
+        return;
+    }
+    const int lo = (int)lo64, hi = (int)hi64;
+    float qf[CPL][EPC];
+    const T* qp = static_cast<const T*>(p.q) + (qi * p.hq + (int64_t)(head_lane ? h : 0) * p.group) * p.d + part * CPL * EPC;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) widen16<T>(*reinterpret_cast<const uint4*>(qp + j * EPC), qf[j]);
+    const T* kc = static_cast<const T*>(p.k) + (int64_t)(head_lane ? h : 0) * p.d + part * CPL * EPC;
+    const int32_t* bt = p.block_tables + (int64_t)s * p.table_width;
+    const int ps = p.page_size;
+    const int64_t slot_elems = (int64_t)p.hkv * p.d;
+    float m = neg_inf();
+    for (int t0 = lo + warp; t0 < hi; t0 += kProxyAllWarps * kProxyUnroll) {
+        uint4 raw[kProxyUnroll][CPL];
+#pragma unroll
+        for (int u = 0; u < kProxyUnroll; ++u) {
+            const int t = t0 + u * kProxyAllWarps;
+            if (t < hi && head_lane) {
+                const int64_t slot = (int64_t)bt[t / ps] * ps + t % ps;
+                const T* kp = kc + slot * slot_elems;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) raw[u][j] = __ldg(reinterpret_cast<const uint4*>(kp + j * EPC));
+            } else {
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) raw[u][j] = make_uint4(0, 0, 0, 0);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kProxyUnroll; ++u) {
+            float dot = 0.f;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                float kf[EPC];
+                widen16<T>(raw[u][j], kf);
+#pragma unroll
+                for (int e = 0; e < EPC; ++e) dot = fmaf(qf[j][e], kf[e], dot);
+            }
+#pragma unroll
+            for (int o = 1; o < LPR; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            if (t0 + u * kProxyAllWarps < hi) m = fmaxf(m, dot);
+        }
+    }
+    wmax[warp][lane] = m;
+    __syncthreads();
+    if (warp == 0 && part == 0 && head_lane) {
+        float mm = wmax[0][lane];
+#pragma unroll
+        for (int w = 1; w < kProxyAllWarps; ++w) mm = fmaxf(mm, wmax[w][lane]);
+        out[(int64_t)h * p.sw] = canonical_zero(mm * p.scale);  // scale > 0: the max commutes with it
+    }
+}
+
 // (score, index) -> key that sorts ascending as (score descending, index ascending).
 __device__ __forceinline__ unsigned long long rank_key(float score, int idx) {
     const uint32_t u = __float_as_uint(canonical_zero(score));
@@ -267,6 +349,18 @@ __global__ void __launch_bounds__(kPrepThreads)
 template <typename T>
 cudaError_t proxy_launch_t(const ProxyParams& p, int64_t rows, cudaStream_t st) {
     const int64_t row_bytes = (int64_t)p.d * (int64_t)sizeof(T);
+    // whole cache slots per warp when a slot's rows fit one warp at 64 bytes per lane
+    const int lpr = row_bytes % 64 == 0 ? (int)(row_bytes / 64) : 0;
+    if ((lpr == 1 || lpr == 2 || lpr == 4 || lpr == 8) && (int64_t)p.hkv * lpr <= 32) {
+        const dim3 g((unsigned)p.sw, (unsigned)(rows / p.hkv));
+        switch (lpr) {
+            case 1: proxy_scores_slot_kernel<T, 1><<<g, kProxyAllWarps * 32, 0, st>>>(p); break;
+            case 2: proxy_scores_slot_kernel<T, 2><<<g, kProxyAllWarps * 32, 0, st>>>(p); break;
+            case 4: proxy_scores_slot_kernel<T, 4><<<g, kProxyAllWarps * 32, 0, st>>>(p); break;
+            default: proxy_scores_slot_kernel<T, 8><<<g, kProxyAllWarps * 32, 0, st>>>(p); break;
+        }
+        return cudaGetLastError();
+    }
     const dim3 grid((unsigned)((p.sw + kProxyWarps - 1) / kProxyWarps), (unsigned)rows);
     const int cpr = row_bytes % 16 == 0 ? (int)(row_bytes / 16) : 0;  // 16-byte chunks per row
     switch (cpr % 4 == 0 ? cpr / 4 : 0) {

@@ -41,8 +41,10 @@ struct E2eLoop {
     float* lse_host[2] = {};
     cudaStream_t up = nullptr, down = nullptr;
     cudaEvent_t h2d[2] = {}, fwd[2] = {}, d2h[2] = {}, ready[2] = {};
+    cudaEvent_t fs[4] = {}, fe[4] = {};  // timing: start / end of step i's forward on the compute stream, ring of 4
     long long uploaded = 0;
     double host_us[6] = {};  // plan create, plan prepare, copies, forward, release, waits
+    double gpu_us[2] = {};   // device time of the forward kernels, compute stream idle before them
 
     ~E2eLoop() {
         for (int b = 0; b < 2; ++b) {
@@ -50,6 +52,10 @@ struct E2eLoop {
             if (fwd[b]) cudaEventDestroy(fwd[b]);
             if (d2h[b]) cudaEventDestroy(d2h[b]);
             if (ready[b]) cudaEventDestroy(ready[b]);
+            for (int r = 2 * b; r < 2 * b + 2; ++r) {
+                if (fs[r]) cudaEventDestroy(fs[r]);
+                if (fe[r]) cudaEventDestroy(fe[r]);
+            }
             if (out_host[b]) cudaFreeHost(out_host[b]);
             if (lse_host[b]) cudaFreeHost(lse_host[b]);
         }
@@ -99,6 +105,10 @@ void* pa_e2e_create(const int32_t* seq_lens, const int32_t* query_offsets, int32
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->d2h[b], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L->ready[b], cudaEventDisableTiming);
     }
+    for (int r = 0; r < 4 && e == cudaSuccess; ++r) {
+        e = cudaEventCreate(&L->fs[r]);
+        if (e == cudaSuccess) e = cudaEventCreate(&L->fe[r]);
+    }
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->up, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&L->down, cudaStreamNonBlocking);
     if (e != cudaSuccess) {
@@ -116,6 +126,11 @@ long long pa_e2e_uploaded_bytes(const void* loop) { return static_cast<const E2e
 void pa_e2e_host_times(const void* loop, double* us6) {
     for (int i = 0; i < 6; ++i) us6[i] = static_cast<const E2eLoop*>(loop)->host_us[i];
 }
+// Device time of the forwards of the last run (summed over its steps but the last) and the time the
+// compute stream sat idle before each of them (from the end of the previous step's forward).
+void pa_e2e_gpu_times(const void* loop, double* us2) {
+    for (int i = 0; i < 2; ++i) us2[i] = static_cast<const E2eLoop*>(loop)->gpu_us[i];
+}
 
 // Runs `steps` steps on `stream` (the compute stream) and returns once every step's result is on
 // the host. Returns 0, a pa_status (> 0) from a library call, or -(cudaError_t) from a runtime call.
@@ -124,6 +139,7 @@ int pa_e2e_run(void* loop, int steps, void* stream) {
     if (steps <= 0) return 0;
     cudaStream_t main = static_cast<cudaStream_t>(stream);
     for (double& t : L.host_us) t = 0.0;
+    for (double& t : L.gpu_us) t = 0.0;
     pa_plan* cur = nullptr;
     pa_plan* nxt = nullptr;
     int rc = 0;
@@ -158,8 +174,10 @@ int pa_e2e_run(void* loop, int steps, void* stream) {
         ok = ok && cu_ok(cudaStreamWaitEvent(main, L.ready[b], 0));  // the plan's uploads
         L.host_us[2] += since_us(t0);
         t0 = std::chrono::steady_clock::now();
+        ok = ok && cu_ok(cudaEventRecord(L.fs[i & 3], main));
         ok = ok && pa_ok(pa_forward(cur, L.q_dev[b], L.k_cache, L.v_cache, L.dtype, L.hq, L.hkv, L.d, L.dv, L.scale,
                                     L.causal, L.window, L.out_dev[b], L.lse_dev[b], main));
+        ok = ok && cu_ok(cudaEventRecord(L.fe[i & 3], main));
         ok = ok && cu_ok(cudaEventRecord(L.fwd[b], main));
         L.host_us[3] += since_us(t0);
         t0 = std::chrono::steady_clock::now();
@@ -179,6 +197,12 @@ int pa_e2e_run(void* loop, int steps, void* stream) {
         t0 = std::chrono::steady_clock::now();
         if (ok && i >= 1) ok = cu_ok(cudaEventSynchronize(L.d2h[b ^ 1]));  // step i-1's result is on the host
         L.host_us[5] += since_us(t0);
+        if (ok && i >= 1) {
+            float ms = 0.f;
+            if (cudaEventElapsedTime(&ms, L.fs[(i - 1) & 3], L.fe[(i - 1) & 3]) == cudaSuccess) L.gpu_us[0] += 1e3 * ms;
+            if (i >= 2 && cudaEventElapsedTime(&ms, L.fe[(i - 2) & 3], L.fs[(i - 1) & 3]) == cudaSuccess)
+                L.gpu_us[1] += 1e3 * ms;
+        }
         cur = nxt;
         nxt = nullptr;
     }
