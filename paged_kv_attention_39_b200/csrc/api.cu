@@ -9,8 +9,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <deque>
 #include <memory>
 #include <mutex>
+#include <unordered_map>
 #include <vector>
 
 #include "pa_internal.h"
@@ -88,10 +90,9 @@ Staging* staging(int dev) {  // one set of slots per device (events belong to a 
 }
 
 // Device memory of plans (metadata, work lists, workspaces) comes from a pool of the library's
-// own per device that keeps freed memory cached (release threshold at its maximum): a plan per
-// decode step then allocates without going back to the driver, and the process's default pool
-// is left as the caller configured it.
-cudaError_t lib_malloc(void** ptr, size_t bytes, cudaStream_t st) {
+// own per device that keeps freed memory cached (release threshold at its maximum), and the
+// process's default pool is left as the caller configured it.
+cudaError_t pool_malloc(void** ptr, size_t bytes, cudaStream_t st) {
     static std::mutex mu;
     static cudaMemPool_t pools[kStageDevices] = {};
     static bool tried[kStageDevices] = {};
@@ -118,6 +119,107 @@ cudaError_t lib_malloc(void** ptr, size_t bytes, cudaStream_t st) {
     }
     if (!pool) return cudaMallocAsync(ptr, bytes, st);
     return cudaMallocFromPoolAsync(ptr, bytes, pool, st);
+}
+
+// Freed plan memory first waits in a per-device list, with an event recorded on the stream that
+// freed it; an allocation takes the oldest listed block of a fitting size (at most twice the
+// request) whose event has completed, so that a new plan per decode step reuses an earlier step's
+// memory without a driver call. (The pool's own reuse of memory freed on another stream -- plans
+// allocate on their upload stream and free on their call stream -- may map more memory instead,
+// which cost up to 1.5 ms per plan on some hosts.) The list keeps at most kRecycleBytes; older
+// blocks go back to the pool, stream-ordered after their event. Calls on a capturing stream use
+// the pool directly.
+struct Recycled {
+    void* p;
+    size_t bytes;
+    cudaEvent_t ev;
+};
+struct Recycler {
+    std::mutex mu;
+    std::unordered_map<void*, size_t> sizes;  // every block handed out by lib_malloc, rounded size
+    std::deque<Recycled> list;                // freed blocks, oldest first
+    size_t held = 0;
+    std::vector<cudaEvent_t> spare;           // completed events, for reuse
+};
+constexpr size_t kRecycleBytes = size_t(256) << 20;
+constexpr size_t kRecycleGrain = size_t(64) << 10;
+Recycler* recycler(int dev) {
+    static std::mutex mu;
+    static Recycler* per_dev[kStageDevices] = {};  // never destroyed: outlive any plan released at exit
+    if (dev < 0 || dev >= kStageDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!per_dev[dev]) per_dev[dev] = new Recycler();
+    return per_dev[dev];
+}
+bool capturing(cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    return cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs != cudaStreamCaptureStatusNone;
+}
+
+cudaError_t lib_malloc(void** ptr, size_t bytes, cudaStream_t st) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    Recycler* R = capturing(st) ? nullptr : recycler(dev);
+    if (!R) return pool_malloc(ptr, bytes, st);
+    const size_t want = (std::max<size_t>(bytes, 1) + kRecycleGrain - 1) / kRecycleGrain * kRecycleGrain;
+    std::lock_guard<std::mutex> lock(R->mu);
+    for (auto it = R->list.begin(); it != R->list.end(); ++it) {
+        if (it->bytes < want || it->bytes > 2 * want) continue;
+        const cudaError_t q = cudaEventQuery(it->ev);
+        if (q == cudaErrorNotReady) continue;  // its last user is still queued
+        if (q != cudaSuccess) return q;
+        *ptr = it->p;
+        R->spare.push_back(it->ev);
+        R->held -= it->bytes;
+        R->list.erase(it);
+        return cudaSuccess;
+    }
+    e = pool_malloc(ptr, want, st);
+    if (e == cudaSuccess) R->sizes[*ptr] = want;
+    return e;
+}
+
+// Release a block from lib_malloc after the work queued on `st` so far (device `dev`).
+cudaError_t lib_free(void* p, int dev, cudaStream_t st) {
+    if (!p) return cudaSuccess;
+    Recycler* R = capturing(st) ? nullptr : recycler(dev);
+    if (!R) return cudaFreeAsync(p, st);
+    std::lock_guard<std::mutex> lock(R->mu);
+    auto f = R->sizes.find(p);
+    if (f == R->sizes.end()) return cudaFreeAsync(p, st);
+    const size_t bytes = f->second;
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return e;
+    if (cur != dev && (e = cudaSetDevice(dev)) != cudaSuccess) return e;
+    cudaEvent_t ev = nullptr;
+    if (!R->spare.empty()) {
+        ev = R->spare.back();
+        R->spare.pop_back();
+    } else {
+        e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev, st);
+    if (e == cudaSuccess) {
+        R->list.push_back({p, bytes, ev});
+        R->held += bytes;
+        while (R->held > kRecycleBytes && e == cudaSuccess) {
+            const Recycled old = R->list.front();
+            R->list.pop_front();
+            R->held -= old.bytes;
+            R->sizes.erase(old.p);
+            R->spare.push_back(old.ev);
+            e = cudaStreamWaitEvent(st, old.ev, 0);
+            if (e == cudaSuccess) e = cudaFreeAsync(old.p, st);
+        }
+    } else {
+        if (ev) R->spare.push_back(ev);
+        R->sizes.erase(f);
+        e = cudaFreeAsync(p, st);
+    }
+    if (cur != dev) cudaSetDevice(cur);
+    return e;
 }
 
 cudaError_t upload_slot(Staging& g, void* dst, const void* src, size_t bytes, cudaStream_t st) {
@@ -403,7 +505,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     PA_CUDA_TRY(lib_malloc(&S->dev, S->host.size(), st));
     cudaError_t e = upload(S->dev, S->host.data(), S->host.size(), st);
     if (e != cudaSuccess) {
-        cudaFreeAsync(S->dev, st);
+        lib_free(S->dev, P->device, st);
         return fail(PA_ERR_CUDA, "schedule upload failed: %s", cudaGetErrorString(e));
     }
     P->uploaded_bytes += (int64_t)S->host.size();
@@ -422,7 +524,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     S->kv_chunk = (int32_t)std::min<int64_t>(chunk, INT32_MAX);
 
     if (P->scheds.size() >= 8) {  // keep the plan's footprint bounded (stream-ordered free)
-        cudaFreeAsync(P->scheds.front()->dev, st);
+        lib_free(P->scheds.front()->dev, P->device, st);
         P->scheds.erase(P->scheds.begin());
     }
     P->scheds.push_back(std::move(S));
@@ -433,7 +535,7 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
 pa_status ensure_workspace(pa_plan* P, size_t bytes, cudaStream_t st) {
     if (bytes <= P->ws_bytes) return PA_OK;
     if (P->ws) {
-        PA_CUDA_TRY(cudaFreeAsync(P->ws, st));
+        PA_CUDA_TRY(lib_free(P->ws, P->device, st));
         P->ws = nullptr;
         P->ws_bytes = 0;
     }
@@ -448,7 +550,9 @@ template <typename P_>
 pa_status grow_buffer(P_** buf, size_t* have, size_t bytes, cudaStream_t st) {
     if (bytes <= *have) return PA_OK;
     if (*buf) {
-        PA_CUDA_TRY(cudaFreeAsync(*buf, st));
+        int dev = -1;
+        PA_CUDA_TRY(cudaGetDevice(&dev));
+        PA_CUDA_TRY(lib_free(*buf, dev, st));
         *buf = nullptr;
         *have = 0;
     }
@@ -636,7 +740,7 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
         // the kernel after each merge, so every call finds them zero
         const size_t n = (size_t)S->slots * c.hkv;
         if (n > P->merge_ctr_n) {
-            if (P->merge_ctr) PA_CUDA_TRY(cudaFreeAsync(P->merge_ctr, st));
+            if (P->merge_ctr) PA_CUDA_TRY(lib_free(P->merge_ctr, P->device, st));
             P->merge_ctr = nullptr;
             P->merge_ctr_n = 0;
             void* m = nullptr;
@@ -825,7 +929,7 @@ pa_status pa_plan_create(const int32_t* seq_lens, const int32_t* query_offsets, 
         P->last_stream = (cudaStream_t)upload_stream;
         P->uploaded_bytes = (int64_t)total;
         if (e != cudaSuccess) {
-            cudaFreeAsync(P->d_meta, (cudaStream_t)upload_stream);
+            lib_free(P->d_meta, device, (cudaStream_t)upload_stream);
             return fail(PA_ERR_CUDA, "plan upload failed: %s", cudaGetErrorString(e));
         }
         P->d_seqs = (pa::SeqInfo*)P->d_meta;
@@ -844,17 +948,18 @@ pa_status pa_plan_destroy(pa_plan* plan) {
         // the plan's host data, never the plan's own buffers, so the plan object goes at once (no
         // host callback on the stream, which would hold back the work queued after it).
         cudaStream_t st = plan->last_stream;
-        if (plan->ws) cudaFreeAsync(plan->ws, st);
-        if (plan->sel_ws) cudaFreeAsync(plan->sel_ws, st);
-        if (plan->score_ws) cudaFreeAsync(plan->score_ws, st);
-        if (plan->bwd_dev) cudaFreeAsync(plan->bwd_dev, st);
-        if (plan->bwd_drow) cudaFreeAsync(plan->bwd_drow, st);
-        if (plan->bwd_scratch) cudaFreeAsync(plan->bwd_scratch, st);
-        if (plan->merge_ctr) cudaFreeAsync(plan->merge_ctr, st);
-        if (plan->mla_bwd_dev) cudaFreeAsync(plan->mla_bwd_dev, st);
-        if (plan->mla_ds) cudaFreeAsync(plan->mla_ds, st);
-        for (auto& s : plan->scheds) cudaFreeAsync(s->dev, st);
-        cudaError_t e = plan->d_meta ? cudaFreeAsync(plan->d_meta, st) : cudaSuccess;
+        const int dv = plan->device;
+        lib_free(plan->ws, dv, st);
+        lib_free(plan->sel_ws, dv, st);
+        lib_free(plan->score_ws, dv, st);
+        lib_free(plan->bwd_dev, dv, st);
+        lib_free(plan->bwd_drow, dv, st);
+        lib_free(plan->bwd_scratch, dv, st);
+        lib_free(plan->merge_ctr, dv, st);
+        lib_free(plan->mla_bwd_dev, dv, st);
+        lib_free(plan->mla_ds, dv, st);
+        for (auto& s : plan->scheds) lib_free(s->dev, dv, st);
+        cudaError_t e = lib_free(plan->d_meta, dv, st);
         delete plan;
         if (e != cudaSuccess) return fail(PA_ERR_CUDA, "plan release failed: %s", cudaGetErrorString(e));
         return ok();
@@ -1193,7 +1298,7 @@ static pa_status build_backward_lists(pa_plan* plan, int32_t G, int causal, int3
     // leaves the plan to rebuild them on its next call
     plan->bwd_group = 0;
     if (plan->bwd_dev) {
-        PA_CUDA_TRY(cudaFreeAsync(plan->bwd_dev, st));
+        PA_CUDA_TRY(lib_free(plan->bwd_dev, plan->device, st));
         plan->bwd_dev = nullptr;
     }
     PA_CUDA_TRY(lib_malloc(&plan->bwd_dev, blob.size(), st));
@@ -1362,7 +1467,7 @@ static pa_status build_mla_backward_lists(pa_plan* plan, int32_t H, int causal, 
     if (!tiles.empty()) std::memcpy(plan->mla_bwd_host.data(), tiles.data(), tiles.size() * sizeof(pa::MlaKeyTile));
     if (!units.empty())
         std::memcpy(plan->mla_bwd_host.data() + dq_off, units.data(), units.size() * sizeof(pa::MlaDqUnit));
-    if (plan->mla_bwd_dev) PA_CUDA_TRY(cudaFreeAsync(plan->mla_bwd_dev, st));
+    if (plan->mla_bwd_dev) PA_CUDA_TRY(lib_free(plan->mla_bwd_dev, plan->device, st));
     plan->mla_bwd_dev = nullptr;
     plan->mla_bwd_h = 0;
     PA_CUDA_TRY(lib_malloc(&plan->mla_bwd_dev, bytes, st));

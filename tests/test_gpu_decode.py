@@ -53,6 +53,17 @@ def test_decode_groups_and_multi_query(orc, hq, hkv, qn):
         check(wl, out, lse, *ref, tag=f"G{hq // hkv} n{qn} chunk {kv_chunk}")
 
 
+@pytest.mark.parametrize("hq,hkv,qn", [(16, 1, 1), (8, 2, 4), (4, 4, 1), (32, 8, 1)])
+def test_decode_head_dim_64(orc, hq, hkv, qn):
+    """head_dim 64 (32-key warp tiles) with 1 to 16 rows per KV head, parts that start off the
+    32-key grid (chunk 100) and ragged lengths."""
+    wl = small_decode(5, hq=hq, hkv=hkv, d=64, qn=qn, lmin=qn, lmax=700)
+    ref = orc.run(wl)
+    for kv_chunk in (0, 100, -1):
+        out, lse = run_gqa(wl, kv_chunk=kv_chunk)
+        check(wl, out, lse, *ref, tag=f"d64 G{hq // hkv} n{qn} chunk {kv_chunk}")
+
+
 @pytest.mark.parametrize("hq,hkv,qn", [(16, 1, 1), (8, 2, 4), (4, 4, 1)])
 def test_decode_head_dim_256(orc, hq, hkv, qn):
     """head_dim 256 on the tensor-core decode kernel, up to 16 rows per KV head (two n-tiles)."""
@@ -80,6 +91,31 @@ def test_split_rows_plan_reused(orc):
         check(wl, out, lse, *ref, tag=f"call {i} chunk {kv_chunk}")
     assert pa.pa_plan_device_status(plan) == 0
     plan.close()
+
+
+def test_plan_memory_recycled_across_steps(orc):
+    """Forty decode steps, each with a new plan (other lengths, so other work lists, part counts and
+    workspace sizes) created on an upload stream and released as soon as its forward is queued,
+    without synchronising: the library may hand a released plan's device memory to a later plan
+    only once the work queued before the release has completed. Every step matches the oracle."""
+    up = torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+    steps = []
+    for i in range(40):
+        wl = small_decode(200 + i, batch=3 + i % 6, lmin=17, lmax=300 + 60 * i)
+        plan = pa.plan_for(wl, device=0, stream=up)
+        pa.pa_plan_prepare(plan, wl.q.dtype, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.v_head_dim,
+                           wl.causal, wl.window, stream=up)
+        main.wait_stream(up)
+        qd, kd, vd = wl.q.to("cuda"), wl.k_cache.to("cuda"), wl.v_cache.to("cuda")
+        out = torch.full((qd.shape[0], wl.num_q_heads, wl.v_head_dim), float("nan"), dtype=qd.dtype, device="cuda")
+        lse = torch.full((qd.shape[0], wl.num_q_heads), float("nan"), dtype=torch.float32, device="cuda")
+        pa.pa_forward(plan, qd, kd, vd, out, lse, wl.scale, wl.causal, wl.window, kv_chunk=64 if i % 2 else 0)
+        plan.close()
+        steps.append((wl, (qd, kd, vd), out, lse))
+    torch.cuda.synchronize()
+    for i, (wl, _, out, lse) in enumerate(steps):
+        check(wl, out.cpu(), lse.cpu(), *orc.run(wl), tag=f"step {i}")
 
 
 def test_split_rows_of_both_decode_kernels_in_one_call(orc):
