@@ -124,9 +124,9 @@ cudaError_t pool_malloc(void** ptr, size_t bytes, cudaStream_t st) {
 // Freed plan memory first waits in a per-device list, with an event recorded on the stream that
 // freed it; an allocation takes the oldest listed block of a fitting size (at most twice the
 // request) whose event has completed, so that a new plan per decode step reuses an earlier step's
-// memory without a driver call. (The pool's own reuse of memory freed on another stream -- plans
-// allocate on their upload stream and free on their call stream -- may map more memory instead,
-// which cost up to 1.5 ms per plan on some hosts.) The list keeps at most kRecycleBytes; older
+// memory without a driver call. (Plans allocate on their upload stream and free on their call
+// stream, so the pool can reuse such memory only through a cross-stream dependency or maps more;
+// its allocations were measured at 3-52 us per plan.) The list keeps at most kRecycleBytes; older
 // blocks go back to the pool, stream-ordered after their event. Calls on a capturing stream use
 // the pool directly.
 struct Recycled {
