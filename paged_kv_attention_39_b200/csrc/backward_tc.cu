@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         for (int i = 0; i < L_::B_COUNT; ++i) {
             uint32_t cnt = 1;
             if (i == L_::B_PFULL) cnt = kComputeWarpsB * 32;
+            if (i >= L_::B_QFULL && i < L_::B_QFULL + QST) cnt = 2;  // tile bytes + row statistics
             mbar_init(&bars[i], cnt);
         }
         *abort_flag = 0;
@@ -185,6 +186,17 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         // the row block's Q and dO rows (TMA) and its row statistics (plain loads) into stage s
         auto load_block = [&](int i, int s) {
             const int j0 = (rb0 + i) * qpt;
+            // the tiles first: their landing is what the block waits for; the row statistics are
+            // gathered while they are in flight and reported by a second arrival
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&bars[L_::B_QFULL + s], 2 * KH * L_::HALF);
+                uint8_t* qs = smem + L_::Q + s * 2 * KH * L_::HALF;
+                for (int h = 0; h < KH; ++h) {
+                    tma_load_3d(qs + h * L_::HALF, &tmq, &bars[L_::B_QFULL + s], h * 64, kvh * G, si.q_start + j0);
+                    tma_load_3d(qs + (KH + h) * L_::HALF, &tmo, &bars[L_::B_QFULL + s], h * 64, kvh * G,
+                                si.q_start + j0);
+                }
+            }
             uint8_t* rows = smem + L_::ROWS + s * L_::ROWS_STAGE;
             float* lse2 = reinterpret_cast<float*>(rows);
             float* drow = lse2 + RB;
@@ -217,15 +229,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                 hi[RB + 1] = hi_min;
             }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&bars[L_::B_QFULL + s], 2 * KH * L_::HALF);
-                uint8_t* qs = smem + L_::Q + s * 2 * KH * L_::HALF;
-                for (int h = 0; h < KH; ++h) {
-                    tma_load_3d(qs + h * L_::HALF, &tmq, &bars[L_::B_QFULL + s], h * 64, kvh * G, si.q_start + j0);
-                    tma_load_3d(qs + (KH + h) * L_::HALF, &tmo, &bars[L_::B_QFULL + s], h * 64, kvh * G,
-                                si.q_start + j0);
-                }
-            }
+            if (lane == 0) mbar_arrive(&bars[L_::B_QFULL + s]);  // the statistics are written
             __syncwarp();
         };
         // the tile's K and V rows: one TMA box per page (and 64-column half), landing 128-byte
