@@ -330,8 +330,7 @@ pa_status pa_mla_backward(pa_plan* plan, const void* q_latent, const void* q_rop
  * list, the decode, the merge when some row is split).
  *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress, once
- * per device, with that device current); make that first call before capturing the stream into
- * a CUDA graph. Every call shares the one array and leaves its contents behind; nothing in it
+ * per device, with that device current). Every call shares the one array and leaves its contents behind; nothing in it
  * needs to start at zero (each call writes its unit lists and every part it later reads).
  * Calls whose GPU work overlaps -- issued on different streams, or from different host threads
  * on different streams -- race on the array: order them on one stream.

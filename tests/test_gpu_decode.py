@@ -244,6 +244,40 @@ def test_plan_reuse_and_workspace_growth(orc):
     plan.close()
 
 
+def test_forward_replayed_from_a_cuda_graph(orc):
+    """pa_forward on decode rows (parts merged by the decode kernel's last CTA) and a prefill chunk
+    (two launches), captured into a CUDA graph after a first call has built the plan's work list
+    and workspace, then replayed with three other sets of queries written into the captured input
+    buffer: every replay matches the oracle on its own queries (the merge counters are back at
+    zero after each replay)."""
+    wl = W.make_gqa("graph", 41, [3000, 700, 1400, 900], [1, 1, 200, 1], 32, 8, 128, 128, 64, torch.bfloat16)
+    s = wl.sched
+    plan = pa.plan_for(wl)
+    qd, kd, vd = wl.q.to("cuda"), wl.k_cache.to("cuda"), wl.v_cache.to("cuda")
+    out = torch.empty((qd.shape[0], wl.num_q_heads, wl.v_head_dim), dtype=qd.dtype, device="cuda")
+    lse = torch.empty((qd.shape[0], wl.num_q_heads), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        pa.pa_forward(plan, qd, kd, vd, out, lse, wl.scale, wl.causal, wl.window, kv_chunk=256)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        pa.pa_forward(plan, qd, kd, vd, out, lse, wl.scale, wl.causal, wl.window, kv_chunk=256)
+    kernels = pa.pa_plan_get_info(plan)["last_kernels"]
+    assert kernels & pa.PA_KERNEL_DECODE_TC and kernels & pa.PA_KERNEL_PREFILL_TC, kernels
+    for i in range(3):
+        q = W.randn(tuple(wl.q.shape), 300 + i, 1, wl.q.dtype)
+        qd.copy_(q.to("cuda"))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = orc.attention(q, wl.k_cache, wl.v_cache, s.seq_lens, s.query_offsets, s.block_tables, s.page_size,
+                            wl.scale, wl.causal, wl.window)
+        check(wl, out.cpu(), lse.cpu(), *ref, tag=f"graph replay {i}")
+    assert pa.pa_plan_device_status(plan) == 0
+    del graph
+    plan.close()
+
+
 @pytest.mark.slow
 def test_full_size_bf16_decode_sampled(orc):
     """The full decode workload (batch 64, context U[512, 8192], Hq 32, Hkv 8, D 128, pages of
