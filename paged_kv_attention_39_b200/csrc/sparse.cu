@@ -78,8 +78,8 @@ template <typename T, int CPL>
 __global__ void __launch_bounds__(kProxyWarps * 32) proxy_scores_kernel(const ProxyParams p) {
     constexpr int EPC = 16 / (int)sizeof(T);  // elements per chunk
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.y;
-    const int b = blockIdx.x * kProxyWarps + warp;
+    const int64_t row = blockIdx.x;
+    const int b = blockIdx.y * kProxyWarps + warp;
     if (b >= p.sw) return;
     const int64_t qi = row / p.hkv;
     const int kvh = (int)(row % p.hkv);
@@ -136,8 +136,8 @@ __global__ void __launch_bounds__(kProxyWarps * 32) proxy_scores_kernel(const Pr
 template <typename T>
 __global__ void __launch_bounds__(kProxyWarps * 32) proxy_scores_generic_kernel(const ProxyParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.y;
-    const int b = blockIdx.x * kProxyWarps + warp;
+    const int64_t row = blockIdx.x;
+    const int b = blockIdx.y * kProxyWarps + warp;
     if (b >= p.sw) return;
     const int64_t qi = row / p.hkv;
     const int kvh = (int)(row % p.hkv);
@@ -178,8 +178,8 @@ __global__ void __launch_bounds__(kProxyAllWarps * 32) proxy_scores_slot_kernel(
     constexpr int CPL = 4;                    // chunks per lane: 64 bytes
     __shared__ float wmax[kProxyAllWarps][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.x;
-    const int64_t qi = blockIdx.y;
+    const int64_t qi = blockIdx.x;  // rows on x (no 65535 limit), blocks on y (at most 16384)
+    const int b = blockIdx.y;
     const int32_t s = p.q2seq[qi];
     const SeqInfo si = p.seqs[s];
     const int nb = (si.L + p.block_size - 1) / p.block_size;
@@ -352,7 +352,7 @@ cudaError_t proxy_launch_t(const ProxyParams& p, int64_t rows, cudaStream_t st) 
     // whole cache slots per warp when a slot's rows fit one warp at 64 bytes per lane
     const int lpr = row_bytes % 64 == 0 ? (int)(row_bytes / 64) : 0;
     if ((lpr == 1 || lpr == 2 || lpr == 4 || lpr == 8) && (int64_t)p.hkv * lpr <= 32) {
-        const dim3 g((unsigned)p.sw, (unsigned)(rows / p.hkv));
+        const dim3 g((unsigned)(rows / p.hkv), (unsigned)p.sw);
         switch (lpr) {
             case 1: proxy_scores_slot_kernel<T, 1><<<g, kProxyAllWarps * 32, 0, st>>>(p); break;
             case 2: proxy_scores_slot_kernel<T, 2><<<g, kProxyAllWarps * 32, 0, st>>>(p); break;
@@ -361,7 +361,7 @@ cudaError_t proxy_launch_t(const ProxyParams& p, int64_t rows, cudaStream_t st) 
         }
         return cudaGetLastError();
     }
-    const dim3 grid((unsigned)((p.sw + kProxyWarps - 1) / kProxyWarps), (unsigned)rows);
+    const dim3 grid((unsigned)rows, (unsigned)((p.sw + kProxyWarps - 1) / kProxyWarps));
     const int cpr = row_bytes % 16 == 0 ? (int)(row_bytes / 16) : 0;  // 16-byte chunks per row
     switch (cpr % 4 == 0 ? cpr / 4 : 0) {
         case 1: proxy_scores_kernel<T, 1><<<grid, kProxyWarps * 32, 0, st>>>(p); break;

@@ -132,6 +132,20 @@ def test_select_scores_and_topk(orc, name, wl, bs, topk):
     compare_selection(wl, bs, topk, sel, ref_sc, ref_sel)
 
 
+def test_select_more_rows_than_a_grid_dimension_holds(orc):
+    """4200 queries x 16 KV heads = 67200 (query, KV head) rows, more than the 65535 a grid's second
+    dimension holds (the proxy kernels put rows on the first): scores and selection against the
+    oracle."""
+    wl = W.make_gqa("rows", 69, [2200, 2150], [2100, 2100], 16, 16, 128, 128, 64, torch.bfloat16)
+    s = wl.sched
+    sc, sel = gpu_select(wl, 64, 4)
+    ref_sc = orc.sparse_block_scores(wl.q, wl.k_cache, s.seq_lens, s.query_offsets, s.block_tables, s.page_size,
+                                     wl.scale, 64, wl.causal, wl.window)
+    check_scores(sc, ref_sc, "67200 rows")
+    ref_sel = orc.sparse_topk(ref_sc, s.seq_lens, s.query_offsets, 64, 4, width=sel.shape[2])
+    compare_selection(wl, 64, 4, sel, ref_sc, ref_sel)
+
+
 @pytest.mark.parametrize("topk", [1, 3, 0])
 def test_select_exact_on_integer_inputs(orc, topk):
     """Small-integer Q and K with scale 1/8: exact scores, so ties decide alike on both sides."""
