@@ -107,6 +107,13 @@ def _cases():
         g = torch.Generator().manual_seed(21)
         dout = torch.randn(m.sched.num_queries, h, 512, generator=g).to(dtype)
         out.append((f"mla tensor core h{h} ps{ps} {dtype} c{causal} w{window}", wl, dout))
+    # the bf16 shapes of test_backward_limits (CUDA-core kernel: no 16-bit rounding of P or dS, so
+    # its error stays below this emulation's; the 128-head group on the tensor cores)
+    for name, hq, hkv, d, dv, ps in [("d256", 16, 4, 256, 256, 16), ("d192v128", 8, 2, 192, 128, 16),
+                                     ("g128", 128, 1, 128, 128, 64)]:
+        wl = W.make_gqa("bwd_lim_" + name, 71, [300, 45, 700], [60, 9, 3], hq, hkv, d, dv, ps, torch.bfloat16)
+        g = torch.Generator().manual_seed(17)
+        out.append((f"limits {name}", wl, torch.randn(wl.sched.num_queries, hq, dv, generator=g).to(torch.bfloat16)))
     wl = W.make_gqa("share_tc", 6, [150, 150], [30, 30], 8, 2, 64, 64, 16, torch.bfloat16)
     wl.sched.block_tables[1, :3] = wl.sched.block_tables[0, :3]
     g = torch.Generator().manual_seed(12)

@@ -104,6 +104,42 @@ def test_backward_tensor_core_shapes(orc, hq, hkv, d, ps, causal, window, dtype)
     close(dv, rv, dtype, "dv " + tag)
 
 
+@pytest.mark.parametrize("name,hq,hkv,d,dv,ps,dtype,path", [
+    ("d256", 16, 4, 256, 256, 16, torch.bfloat16, "simt"),         # head dim beyond the tensor-core kernels
+    ("d192v128", 8, 2, 192, 128, 16, torch.bfloat16, "simt"),      # key and value widths differ
+    ("d512f32", 8, 2, 512, 512, 16, torch.float32, "simt"),        # float32, wide rows
+    ("g128", 128, 1, 128, 128, 64, torch.bfloat16, "tc"),          # 128 heads on one KV head: one query per block
+])
+def test_backward_limits(orc, name, hq, hkv, d, dv, ps, dtype, path):
+    """The backward at the edges of its shapes, each against the oracle, on the kernel the shape is
+    meant for (the CUDA-core kernel for head dims outside {64, 128}, unequal widths and float32; the
+    tensor-core kernels for a 128-head group)."""
+    wl = W.make_gqa("bwd_lim_" + name, 71, [300, 45, 700], [60, 9, 3], hq, hkv, d, dv, ps, dtype)
+    s = wl.sched
+    g = torch.Generator().manual_seed(17)
+    q, k, v = wl.q.cuda(), wl.k_cache.cuda(), wl.v_cache.cuda()
+    nq = q.shape[0]
+    dout = torch.randn(nq, hq, dv, generator=g).to(dtype)
+    plan = pa.plan_for(wl)
+    out = torch.empty(nq, hq, dv, dtype=dtype, device="cuda")
+    lse = torch.empty(nq, hq, dtype=torch.float32, device="cuda")
+    pa.pa_forward(plan, q, k, v, out, lse, wl.scale, True, 0)
+    dq = torch.full((nq, hq, d), float("nan"), dtype=torch.float32, device="cuda")
+    dk = torch.zeros(k.shape, dtype=torch.float32, device="cuda")
+    dv_ = torch.zeros(v.shape, dtype=torch.float32, device="cuda")
+    pa.pa_backward(plan, q, k, v, out, lse, dout.cuda(), dq, dk, dv_, wl.scale, True, 0)
+    kernels = pa.pa_plan_get_info(plan)["last_kernels"]
+    torch.cuda.synchronize()
+    plan.close()
+    expect = pa.PA_KERNEL_BACKWARD_SIMT if path == "simt" else pa.PA_KERNEL_BACKWARD_TC
+    assert kernels == expect, (name, kernels)
+    rq, rk, rv = orc.attention_backward(wl.q, wl.k_cache, wl.v_cache, dout, s.seq_lens, s.query_offsets,
+                                        s.block_tables, ps, wl.scale, True, 0)
+    close(dq.cpu(), rq, dtype, "dq " + name)
+    close(dk.cpu(), rk, dtype, "dk " + name)
+    close(dv_.cpu(), rv, dtype, "dv " + name)
+
+
 def test_backward_page_size_outside_the_box_layout_runs_the_cuda_core_kernel(orc):
     """A page of 48 rows neither divides the 128-key tile nor is a multiple of it, so the tensor-core
     kernels (one TMA box per page) do not take it: the CUDA-core kernel does, and matches."""
