@@ -26,7 +26,7 @@ def test_mla_decode(orc, kv_chunk):
     check(wl, out, lse, *ref, tag=f"mla chunk {kv_chunk}")
 
 
-@pytest.mark.parametrize("h", [16, 64, 100])
+@pytest.mark.parametrize("h", [1, 16, 64, 100])
 def test_mla_fewer_heads(orc, h):
     wl = mla_wl(2, h=h)
     ref = orc.run(wl)
@@ -34,7 +34,7 @@ def test_mla_fewer_heads(orc, h):
     check(wl, out, lse, *ref, tag=f"mla H{h}")
 
 
-@pytest.mark.parametrize("ps", [16, 32, 128])
+@pytest.mark.parametrize("ps", [16, 32, 128, 256])
 def test_mla_page_sizes(orc, ps):
     wl = mla_wl(3, ps=ps, lmax=1500)
     ref = orc.run(wl)
