@@ -4,17 +4,18 @@
 // Parts without keys carry lse_i = -inf and weight 0; a row whose parts are all empty gets
 // out = 0 and lse = -inf.
 //
-// One warp per (query, head, 128 output columns). The weights go to shared memory first; then each
-// lane owns four consecutive output columns (float4) and walks the parts eight at a time, so that
-// every lane keeps several independent loads in flight -- the merge is a short, latency-bound read
-// of parts the attention kernel has just written (mostly L2 hits).
+// One warp per (query, head, up to 512 output columns): the weights go to shared memory once per
+// row; then each lane owns four consecutive columns (float4) of each of the row's (up to four)
+// 128-column chunks and walks the parts four at a time, so that a lane keeps up to sixteen
+// independent loads in flight -- the merge is a short, latency-bound read of parts the attention
+// kernel has just written (mostly L2 hits).
 #include "device_common.cuh"
 
 namespace pa {
 
 constexpr int kCombineWarps = 4;
 constexpr int kCombineMaxSplits = 1024;
-constexpr int kCombineCols = 128;  // output columns per warp (wider rows spread over more CTAs)
+constexpr int kCombineCols = 512;  // output columns per warp at most (wider rows spread over more CTAs)
 
 template <typename T>
 __device__ __forceinline__ void store4(T* dst, float4 v);
@@ -44,7 +45,7 @@ __device__ __forceinline__ void fma4(float4& a, float w, const float4 b) {
     a.w = fmaf(w, b.w, a.w);
 }
 
-template <typename T>
+template <typename T, int NJ>
 __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnParams p) {
     __shared__ float wts[kCombineWarps][kCombineMaxSplits];
     const CombineUnit cu = p.cunits[blockIdx.x];
@@ -79,36 +80,40 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
     const float* op = p.ws_o + ((int64_t)cu.part_base * p.hq + h) * p.dv;
     const int64_t step = (int64_t)p.hq * p.dv;
     if ((p.dv & 3) == 0) {
-        for (int c = c_lo + lane * 4; c < c_hi; c += 128) {
-            float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0, a2 = a0, a3 = a0;
-            int i = 0;
-            for (; i + 8 <= n; i += 8) {  // eight parts in flight
-                float4 b[8];
+        // chunk j: columns c_lo + 128 j + 4 lane .. + 3 (when inside [c_lo, c_hi))
+        bool on[NJ];
+        float4 acc[NJ];
 #pragma unroll
-                for (int x = 0; x < 8; ++x) b[x] = *reinterpret_cast<const float4*>(op + (i + x) * step + c);
-#pragma unroll
-                for (int x = 0; x < 8; x += 4) {
-                    fma4(a0, wts[warp][i + x + 0], b[x + 0]);
-                    fma4(a1, wts[warp][i + x + 1], b[x + 1]);
-                    fma4(a2, wts[warp][i + x + 2], b[x + 2]);
-                    fma4(a3, wts[warp][i + x + 3], b[x + 3]);
-                }
-            }
-            for (; i + 4 <= n; i += 4) {
-                const float4 b0 = *reinterpret_cast<const float4*>(op + (i + 0) * step + c);
-                const float4 b1 = *reinterpret_cast<const float4*>(op + (i + 1) * step + c);
-                const float4 b2 = *reinterpret_cast<const float4*>(op + (i + 2) * step + c);
-                const float4 b3 = *reinterpret_cast<const float4*>(op + (i + 3) * step + c);
-                fma4(a0, wts[warp][i + 0], b0);
-                fma4(a1, wts[warp][i + 1], b1);
-                fma4(a2, wts[warp][i + 2], b2);
-                fma4(a3, wts[warp][i + 3], b3);
-            }
-            for (; i < n; ++i) fma4(a0, wts[warp][i], *reinterpret_cast<const float4*>(op + i * step + c));
-            const float4 r = make_float4(a0.x + a1.x + a2.x + a3.x, a0.y + a1.y + a2.y + a3.y,
-                                         a0.z + a1.z + a2.z + a3.z, a0.w + a1.w + a2.w + a3.w);
-            store4<T>(o + c, r);
+        for (int j = 0; j < NJ; ++j) {
+            on[j] = c_lo + 128 * j + lane * 4 < c_hi;
+            acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
+        const float* base = op + c_lo + lane * 4;
+        int i = 0;
+        for (; i + 4 <= n; i += 4) {  // four parts x NJ chunks in flight, added in part order
+            float4 b[4][NJ];
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int j = 0; j < NJ; ++j)
+                    b[x][j] = on[j] ? *reinterpret_cast<const float4*>(base + (i + x) * step + 128 * j)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float w = wts[warp][i + x];
+#pragma unroll
+                for (int j = 0; j < NJ; ++j) fma4(acc[j], w, b[x][j]);
+            }
+        }
+        for (; i < n; ++i) {
+            const float w = wts[warp][i];
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+                if (on[j]) fma4(acc[j], w, *reinterpret_cast<const float4*>(base + i * step + 128 * j));
+        }
+#pragma unroll
+        for (int j = 0; j < NJ; ++j)
+            if (on[j]) store4<T>(o + c_lo + 128 * j + lane * 4, acc[j]);
     } else {
         for (int c = c_lo + lane; c < c_hi; c += 32) {
             float acc = 0.f;
@@ -119,14 +124,22 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
     if (lane == 0 && blockIdx.z == 0) p.lse[row] = lse;
 }
 
+template <typename T>
+void combine_launch_t(const AttnParams& p, dim3 grid, dim3 block, cudaStream_t st) {
+    const int cols = min(p.dv, kCombineCols);  // columns per warp
+    if (cols <= 128) combine_kernel<T, 1><<<grid, block, 0, st>>>(p);
+    else if (cols <= 256) combine_kernel<T, 2><<<grid, block, 0, st>>>(p);
+    else combine_kernel<T, 4><<<grid, block, 0, st>>>(p);
+}
+
 cudaError_t launch_combine(const AttnParams& p, pa_dtype dt, cudaStream_t st) {
     if (p.num_cunits == 0) return cudaSuccess;
     const dim3 grid(p.num_cunits, (p.hq + kCombineWarps - 1) / kCombineWarps, (p.dv + kCombineCols - 1) / kCombineCols);
     const dim3 block(kCombineWarps * 32);
     switch (dt) {
-        case PA_F32: combine_kernel<float><<<grid, block, 0, st>>>(p); break;
-        case PA_BF16: combine_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(p); break;
-        default: combine_kernel<__half><<<grid, block, 0, st>>>(p); break;
+        case PA_F32: combine_launch_t<float>(p, grid, block, st); break;
+        case PA_BF16: combine_launch_t<__nv_bfloat16>(p, grid, block, st); break;
+        default: combine_launch_t<__half>(p, grid, block, st); break;
     }
     return cudaGetLastError();
 }
