@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstring>
 #include <deque>
+#include <functional>
 #include <memory>
 #include <mutex>
 #include <unordered_map>
@@ -256,6 +257,7 @@ cudaError_t upload(void* dst, const void* src, size_t bytes, cudaStream_t st) {
     return cudaSuccess;
 }
 constexpr int kUnitKeys = 2048;            // automatic split: keys per unit (per KV head), at most
+constexpr int64_t kMlaUnitCost = 256;      // an MLA unit's fixed start and end, in keys of streaming
 
 struct SchedKey {
     int mla, dtype, hq, hkv, d, dv, pr, causal, window, path, kv_chunk;
@@ -349,6 +351,41 @@ void visible_union(int32_t L, int32_t n, int32_t j0, int32_t j1, bool causal, in
 
 int32_t ceil_div(int64_t a, int64_t b) { return (int32_t)((a + b - 1) / b); }
 
+// Part length for the tensor-core MLA kernel. It runs one CTA per SM and two CTAs per unit, and
+// the block scheduler hands the units (sorted longest first) to SM pairs as they free up. A unit
+// costs about its keys plus kMlaUnitCost (loading the query rows, writing and merging its part),
+// so among the lengths that fill one to eight waves of pairs this takes the one whose greedy
+// longest-first hand-out is estimated to finish first (the shortest on a tie). Lengths are
+// multiples of 64 keys, at least 256, and cut a range into at most kMaxSplits parts, like the
+// units the schedule then builds.
+int64_t mla_part_length(const std::vector<int64_t>& lens, int64_t total, int pairs) {
+    pairs = std::max(1, pairs);
+    int64_t best = 0, best_end = INT64_MAX;
+    std::vector<int64_t> units, busy;
+    for (int waves = 1; waves <= 8; ++waves) {
+        int64_t c = (total + (int64_t)waves * pairs - 1) / ((int64_t)waves * pairs);
+        c = std::max<int64_t>((c + 63) / 64 * 64, 256);
+        units.clear();
+        for (int64_t len : lens) {
+            int64_t cc = c;
+            if (len > cc * kMaxSplits) cc = (len + kMaxSplits - 1) / kMaxSplits;
+            if (len <= 0) { units.push_back(0); continue; }
+            for (int64_t t = 0; t < len; t += cc) units.push_back(std::min(cc, len - t));
+        }
+        std::sort(units.begin(), units.end(), std::greater<int64_t>());
+        busy.assign(pairs, 0);  // min-heap of the times at which each pair frees up
+        int64_t end = 0;
+        for (int64_t u : units) {
+            std::pop_heap(busy.begin(), busy.end(), std::greater<int64_t>());
+            busy.back() += u + kMlaUnitCost;
+            end = std::max(end, busy.back());
+            std::push_heap(busy.begin(), busy.end(), std::greater<int64_t>());
+        }
+        if (end < best_end || (end == best_end && c < best)) { best_end = end; best = c; }
+    }
+    return best;
+}
+
 pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedule** out) {
     for (auto& s : P->scheds)
         if (s->key == k) { *out = s.get(); return PA_OK; }
@@ -418,9 +455,10 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
     if (k.kv_chunk > 0) chunk = k.sparse_bs > 0 ? ((int64_t)k.kv_chunk + 15) / 16 * 16 : k.kv_chunk;
     else if (k.kv_chunk < 0) chunk = INT32_MAX;
     else if (tc_mla) {
-        // The tensor-core MLA kernel runs one CTA per SM, two per unit: aim at one unit per SM.
-        chunk = (total + P->num_sms - 1) / std::max<int64_t>(1, P->num_sms);
-        chunk = std::max<int64_t>(((chunk + 63) / 64) * 64, 256);
+        std::vector<int64_t> lens;
+        lens.reserve(blocks.size());
+        for (const Block& b : blocks) lens.push_back(b.hi - b.lo);
+        chunk = mla_part_length(lens, total, P->num_sms / 2);
     } else {
         // Long units amortise each CTA's start (first loads in flight) and end (merging its warps,
         // writing its part, merging the row): units of at most kUnitKeys keys, short enough that
