@@ -5,10 +5,10 @@
 // out = 0 and lse = -inf.
 //
 // One warp per (query, head, up to 512 output columns): the weights go to shared memory once per
-// row; then each lane owns four consecutive columns (float4) of each of the row's (up to four)
-// 128-column chunks and walks the parts four at a time, so that a lane keeps up to sixteen
-// independent loads in flight -- the merge is a short, latency-bound read of parts the attention
-// kernel has just written (mostly L2 hits).
+// row; each lane owns four consecutive columns (float4) of each of the row's (up to four)
+// 128-column chunks and walks the parts two or four at a time (eight loads in flight). The merge is
+// a short, latency-bound read of parts the attention kernel has just written: the first parts'
+// rows are requested before the weights are known, and the registers stay low enough for one wave.
 #include "device_common.cuh"
 
 namespace pa {
@@ -46,7 +46,11 @@ __device__ __forceinline__ void fma4(float4& a, float w, const float4 b) {
 }
 
 template <typename T, int NJ>
-__global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kCombineWarps * 32, 7) combine_kernel(const AttnParams p) {
+    // parts in flight per lane: four with one 128-column chunk, two with two or four chunks (at
+    // most eight float4 loads), so that the kernel fits 72 registers and seven CTAs per SM, and the
+    // usual grids one wave
+    constexpr int PF = NJ >= 2 ? 2 : 4;
     __shared__ float wts[kCombineWarps][kCombineMaxSplits];
     const CombineUnit cu = p.cunits[blockIdx.x];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -56,9 +60,28 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
     const int c_hi = min(p.dv, c_lo + kCombineCols);
     const int n = cu.nsplit;
     const float* ls = p.ws_lse + (int64_t)cu.part_base * p.hq + h;
+    const float* op = p.ws_o + ((int64_t)cu.part_base * p.hq + h) * p.dv;
+    const int64_t step = (int64_t)p.hq * p.dv;
     const float kLog2e = 1.4426950408889634f;
-    // Up to 32 parts: each lane keeps its part's logsumexp, so the max and the sum need one round
-    // of loads; more parts are read again for the sum.
+    const bool vec = (p.dv & 3) == 0;
+    // chunk j: columns c_lo + 128 j + 4 lane .. + 3 (when inside [c_lo, c_hi))
+    bool on[NJ];
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) on[j] = vec && c_lo + 128 * j + lane * 4 < c_hi;
+    const float* base = op + c_lo + lane * 4;
+    float4 b[PF][NJ];
+    auto load = [&](int i0) {
+#pragma unroll
+        for (int x = 0; x < PF; ++x)
+#pragma unroll
+            for (int j = 0; j < NJ; ++j)
+                b[x][j] = on[j] && i0 + x < n ? *reinterpret_cast<const float4*>(base + (i0 + x) * step + 128 * j)
+                                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    // the first parts' rows are requested together with the logsumexps: they do not depend on
+    // the weights. Up to 32 parts: each lane keeps its part's logsumexp, so the max and the sum
+    // need one round of loads; more parts are read again for the sum.
+    load(0);
     const float my_l = lane < n ? ls[(int64_t)lane * p.hq] : neg_inf();
     float m = my_l;
     for (int i = lane + 32; i < n; i += 32) m = fmaxf(m, ls[(int64_t)i * p.hq]);
@@ -77,39 +100,19 @@ __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const AttnP
     if (lane < n) wts[warp][lane] = fast_exp2((my_l - lse) * kLog2e);
     for (int i = lane + 32; i < n; i += 32) wts[warp][i] = fast_exp2((ls[(int64_t)i * p.hq] - lse) * kLog2e);
     __syncwarp();
-    const float* op = p.ws_o + ((int64_t)cu.part_base * p.hq + h) * p.dv;
-    const int64_t step = (int64_t)p.hq * p.dv;
-    if ((p.dv & 3) == 0) {
-        // chunk j: columns c_lo + 128 j + 4 lane .. + 3 (when inside [c_lo, c_hi))
-        bool on[NJ];
+    if (vec) {
         float4 acc[NJ];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-            on[j] = c_lo + 128 * j + lane * 4 < c_hi;
-            acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        const float* base = op + c_lo + lane * 4;
-        int i = 0;
-        for (; i + 4 <= n; i += 4) {  // four parts x NJ chunks in flight, added in part order
-            float4 b[4][NJ];
+        for (int j = 0; j < NJ; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < n; i += PF) {  // PF parts x NJ chunks in flight, added in part order
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
+            for (int x = 0; x < PF; ++x)
+                if (i + x < n) {
+                    const float w = wts[warp][i + x];
 #pragma unroll
-                for (int j = 0; j < NJ; ++j)
-                    b[x][j] = on[j] ? *reinterpret_cast<const float4*>(base + (i + x) * step + 128 * j)
-                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const float w = wts[warp][i + x];
-#pragma unroll
-                for (int j = 0; j < NJ; ++j) fma4(acc[j], w, b[x][j]);
-            }
-        }
-        for (; i < n; ++i) {
-            const float w = wts[warp][i];
-#pragma unroll
-            for (int j = 0; j < NJ; ++j)
-                if (on[j]) fma4(acc[j], w, *reinterpret_cast<const float4*>(base + i * step + 128 * j));
+                    for (int j = 0; j < NJ; ++j) fma4(acc[j], w, b[x][j]);
+                }
+            if (i + PF < n) load(i + PF);
         }
 #pragma unroll
         for (int j = 0; j < NJ; ++j)
