@@ -70,8 +70,13 @@ struct PrefillCfg {
     static constexpr int K = Q + KH * HALF_Q;
     static constexpr int V = K + KST * KH * HALF_KV;
     static constexpr int BAR = V + VST * KH * HALF_KV;
-    static constexpr int XCH = BAR + 256;  // 128 rows x 2 column halves of float: row statistics
-    static constexpr int BYTES = XCH + 2 * BM * 4;
+    // row statistics: slots of 128 rows x 2 column halves of float. Two alternating slots (one
+    // barrier per exchange) at D = 64; at D = 128 and 256 one slot and two barriers per exchange,
+    // which measured faster there (and the second slot's kilobyte does not fit beside 224 KB of
+    // tiles and the alignment room).
+    static constexpr int XSLOTS = D == 64 ? 2 : 1;
+    static constexpr int XCH = BAR + 256;
+    static constexpr int BYTES = XCH + XSLOTS * 2 * BM * 4;
     static constexpr int ALLOC = BYTES + 1024;        // room to align the base to 1024
     // TMEM columns: two score buffers, the output, two P buffers (16-bit pairs)
     static constexpr int T_S1 = BN, T_O = 2 * BN, T_P0 = 2 * BN + D, T_P1 = T_P0 + BN / 2;
@@ -474,12 +479,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c0 = half * NC;  // first 32-column chunk of this warp's half
         float* xch = reinterpret_cast<float*>(smem + L_::XCH);
         auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;\n" ::"r"(1 + quad) : "memory"); };
-        // max (or sum) of this row's two halves
+        // max (or sum) of this row's two halves. Both warps of a row make the same exchanges in the
+        // same order. With two slots exchange x uses slot x & 1, so a slot is written again only
+        // after the next exchange's barrier, which the partner reaches after reading it: one
+        // barrier each. With one slot a second barrier keeps the next write behind the partner's read.
+        uint32_t n_xch = 0;
         auto exchange = [&](float mine, bool is_max) {
-            xch[half * BM + r] = mine;
+            float* slot = xch + (L_::XSLOTS == 2 ? (n_xch++ & 1u) * 2 * BM : 0u);
+            slot[half * BM + r] = mine;
             pair_sync();
-            const float other = xch[(1 - half) * BM + r];
-            pair_sync();  // the slot may be written again only after the partner has read it
+            const float other = slot[(1 - half) * BM + r];
+            if (L_::XSLOTS == 1) pair_sync();
             return is_max ? fmaxf(mine, other) : mine + other;
         };
         int gt = 0;
