@@ -6,11 +6,12 @@
 // Proxy scores. Block b of sequence s holds keys [b * bs, min((b + 1) * bs, L_s)). For query i
 // and KV head h the proxy query is query head h * G; the block's score is the largest
 // scale * q_proxy . k_t over the keys t of the block the query sees, -inf if none. The pass is an
-// HBM stream of the K rows with float32 dot products of the stored values. When a cache slot (the
-// Hkv rows of one key) fits one warp at 64 bytes per lane, a CTA scores one (query, block) for
-// every KV head and each warp reads whole slots; otherwise one warp scores one (query, KV head,
-// block), four lanes sharing a key row, or, for rows that are not a multiple of 64 bytes, one lane
-// per key row.
+// HBM stream of the K rows with float32 dot products of the stored values. 16-bit rows of 64, 128
+// or 256 elements (at most 32 KV heads) take the products on the tensor cores (mma.sync, float32
+// accumulation), a CTA per (query, block) for every KV head. Otherwise, when a cache slot (the Hkv
+// rows of one key) fits one warp at 64 bytes per lane, a CTA scores one (query, block) for every
+// KV head and each warp reads whole slots; else one warp scores one (query, KV head, block), four
+// lanes sharing a key row, or, for rows that are not a multiple of 64 bytes, one lane per key row.
 //
 // Top-K. One CTA per (query, KV head) row sorts (score, index) pairs packed into 64-bit keys
 // (descending score, then ascending index) with a bitonic sort in shared memory, keeps the first
@@ -346,9 +347,108 @@ __global__ void __launch_bounds__(kPrepThreads)
     if (bad && err) atomicCAS(err, 0, 64);
 }
 
+// Every KV head of one (query, block) in one CTA, the dot products on the tensor cores (16-bit
+// keys, D = 64, 128 or 256, at most kProxyMmaHeads KV heads). The warps take (KV head, 512 / D * 8
+// keys) pieces of the block; for every 16 keys a warp issues D / 16 mma.m16n8k16 with the keys as
+// M (fragment rows g and g + 8 of lane 4 g + t) and the proxy query copied into all 8 columns of N.
+// A dot product does not depend on the order of its terms, so each lane loads the 16-byte chunks
+// 4 c + t of its keys' rows and of the query straight from global memory (the four lanes of a key
+// cover 64 contiguous bytes per load) and feeds words 0, 1 of chunk c as one k-step and words 2, 3
+// as the next, on both operands alike. Keys outside [lo, hi) are not loaded and do not enter the
+// max; the warps' maxima meet in shared memory.
+constexpr int kProxyMmaHeads = 32;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kProxyAllWarps * 32) proxy_scores_mma_kernel(const ProxyParams p) {
+    constexpr int CH = D / 32;   // 16-byte chunks of a row per lane
+    constexpr int R = 512 / D;   // fragment rows per lane per piece: 8 R keys (64 registers of keys)
+    __shared__ float wmax[kProxyAllWarps][kProxyMmaHeads];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t qi = blockIdx.x;  // rows on x (no 65535 limit), blocks on y (at most 16384)
+    const int b = blockIdx.y;
+    const int32_t s = p.q2seq[qi];
+    const SeqInfo si = p.seqs[s];
+    const int nb = (si.L + p.block_size - 1) / p.block_size;
+    const int64_t pos = (int64_t)si.L - si.n + (qi - si.q_start);
+    float* out = p.scores + qi * p.hkv * (int64_t)p.sw + b;  // + head * sw
+    int64_t lo64 = 0, hi64 = 0;
+    if (b < nb) block_visible(si, pos, b, p.block_size, p.causal, p.window, &lo64, &hi64);
+    if (lo64 >= hi64) {
+        for (int h = threadIdx.x; h < p.hkv; h += blockDim.x) out[(int64_t)h * p.sw] = neg_inf();
+        return;
+    }
+    const int lo = (int)lo64, hi = (int)hi64;
+    for (int h = lane; h < p.hkv; h += 32) wmax[warp][h] = neg_inf();
+    __syncwarp();
+    const int pieces = (hi - lo + 8 * R - 1) / (8 * R);
+    const T* kc = static_cast<const T*>(p.k) + t * 8;
+    const int32_t* bt = p.block_tables + (int64_t)s * p.table_width;
+    const int ps = p.page_size;
+    const int64_t slot_elems = (int64_t)p.hkv * D;
+    for (int it = warp; it < p.hkv * pieces; it += kProxyAllWarps) {
+        const int h = it % p.hkv, t0 = lo + (it / p.hkv) * 8 * R;
+        const T* qp = static_cast<const T*>(p.q) + (qi * p.hq + (int64_t)h * p.group) * D + t * 8;
+        uint4 qf[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) qf[c] = __ldg(reinterpret_cast<const uint4*>(qp + c * 32));
+        uint4 kf[R][CH];
+        bool vis[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {  // fragment row r: key t0 + 8 r + g
+            const int tk = t0 + 8 * r + g;
+            vis[r] = tk < hi;
+            if (vis[r]) {
+                const int64_t slot = (int64_t)bt[tk / ps] * ps + tk % ps;
+                const T* kp = kc + slot * slot_elems + (int64_t)h * D;
+#pragma unroll
+                for (int c = 0; c < CH; ++c) kf[r][c] = __ldg(reinterpret_cast<const uint4*>(kp + c * 32));
+            } else {
+#pragma unroll
+                for (int c = 0; c < CH; ++c) kf[r][c] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        float m = neg_inf();
+#pragma unroll
+        for (int gr = 0; gr < R / 2; ++gr) {  // 16 keys: rows 2 gr (keys g) and 2 gr + 1 (keys g + 8)
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+                const uint4 ka = kf[2 * gr][c], kb = kf[2 * gr + 1][c];
+                const uint32_t a0[4] = {ka.x, kb.x, ka.y, kb.y};
+                mma16816<T>(d, a0, qf[c].x, qf[c].y);
+                const uint32_t a1[4] = {ka.z, kb.z, ka.w, kb.w};
+                mma16816<T>(d, a1, qf[c].z, qf[c].w);
+            }
+            if (vis[2 * gr]) m = fmaxf(m, d[0]);
+            if (vis[2 * gr + 1]) m = fmaxf(m, d[2]);
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        if (lane == 0) wmax[warp][h] = fmaxf(wmax[warp][h], m);
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < p.hkv; h += blockDim.x) {
+        float mm = wmax[0][h];
+#pragma unroll
+        for (int w = 1; w < kProxyAllWarps; ++w) mm = fmaxf(mm, wmax[w][h]);
+        out[(int64_t)h * p.sw] = canonical_zero(mm * p.scale);  // scale > 0: the max commutes with it
+    }
+}
+
 template <typename T>
 cudaError_t proxy_launch_t(const ProxyParams& p, int64_t rows, cudaStream_t st) {
     const int64_t row_bytes = (int64_t)p.d * (int64_t)sizeof(T);
+    if constexpr (sizeof(T) == 2) {  // dot products on the tensor cores
+        if ((p.d == 64 || p.d == 128 || p.d == 256) && p.hkv <= kProxyMmaHeads) {
+            const dim3 g((unsigned)(rows / p.hkv), (unsigned)p.sw);
+            if (p.d == 64) proxy_scores_mma_kernel<T, 64><<<g, kProxyAllWarps * 32, 0, st>>>(p);
+            else if (p.d == 128) proxy_scores_mma_kernel<T, 128><<<g, kProxyAllWarps * 32, 0, st>>>(p);
+            else proxy_scores_mma_kernel<T, 256><<<g, kProxyAllWarps * 32, 0, st>>>(p);
+            return cudaGetLastError();
+        }
+    }
     // whole cache slots per warp when a slot's rows fit one warp at 64 bytes per lane
     const int lpr = row_bytes % 64 == 0 ? (int)(row_bytes / 64) : 0;
     if ((lpr == 1 || lpr == 2 || lpr == 4 || lpr == 8) && (int64_t)p.hkv * lpr <= 32) {

@@ -111,10 +111,16 @@ def sparse_cases():
                                         window=100), 16, 5),
         ("bf16_noncausal_g16", W.make_gqa("sp5", 65, [260], [2], 16, 1, 128, 128, 16, torch.bfloat16,
                                           causal=False), 32, 3),
-        # slots wider than one warp's 32 lanes x 64 bytes (16 KV heads of 256-byte rows): the proxy
-        # pass scores one (query, KV head) row per warp
-        ("bf16_hkv16_row_proxy", W.make_gqa("sp6", 67, [333, 70], [1, 1], 32, 16, 128, 128, 16,
+        # 16 KV heads of 256-byte rows: the proxy pass on the tensor cores, warps over (head, keys)
+        ("bf16_hkv16_mma_proxy", W.make_gqa("sp6", 67, [333, 70], [1, 1], 32, 16, 128, 128, 16,
                                             torch.bfloat16), 32, 3),
+        # slots wider than one warp's 32 lanes x 64 bytes (16 KV heads of 512-byte float32 rows):
+        # the proxy pass scores one (query, KV head) row per warp
+        ("fp32_hkv16_row_proxy", W.make_gqa("sp8", 70, [200, 90], [1, 1], 16, 16, 128, 128, 16,
+                                            torch.float32), 32, 3),
+        # head dim 256: the tensor-core proxy with two fragment rows per piece
+        ("bf16_d256_mma_proxy", W.make_gqa("sp9", 71, [300, 513], [1, 1], 16, 4, 256, 256, 16,
+                                           torch.bfloat16), 64, 3),
         # rows of 80 bytes: the proxy pass's scalar kernel
         ("bf16_d40_scalar_proxy", W.make_gqa("sp7", 68, [150, 77], [1, 2], 4, 2, 40, 40, 16, torch.bfloat16),
          16, 2),
