@@ -461,10 +461,12 @@ pa_status build_schedule(pa_plan* P, const SchedKey& k, cudaStream_t st, Schedul
         chunk = mla_part_length(lens, total, P->num_sms / 2);
     } else {
         // Long units amortise each CTA's start (first loads in flight) and end (merging its warps,
-        // writing its part, merging the row): units of at most kUnitKeys keys, short enough that
-        // there are about 7 units per 4 SMs, and never below 256 keys. Sparse rows are short runs
-        // of selected blocks: whole rows up to 1024 keys per unit (no merge) beat finer splits.
-        chunk = std::min<int64_t>(kUnitKeys, total * 4 / std::max<int64_t>(1, 7 * (int64_t)P->num_sms));
+        // writing its part, merging the row): units of at most kUnitKeys keys (twice that for head
+        // dims above 128, whose CTAs hold fewer tiles in flight), short enough that there are about
+        // 7 units per 4 SMs, and never below 256 keys. Sparse rows are short runs of selected
+        // blocks: whole rows up to 1024 keys per unit (no merge) beat finer splits.
+        const int64_t unit_keys = (k.d > 128 || k.dv > 128) ? 2 * kUnitKeys : kUnitKeys;
+        chunk = std::min<int64_t>(unit_keys, total * 4 / std::max<int64_t>(1, 7 * (int64_t)P->num_sms));
         chunk = std::max<int64_t>(((chunk + 63) / 64) * 64, k.sparse_bs > 0 ? 1024 : 256);
     }
 
