@@ -15,7 +15,8 @@
 //
 // Top-K. One CTA per (query, KV head) row sorts (score, index) pairs packed into 64-bit keys
 // (descending score, then ascending index) with a bitonic sort in shared memory, keeps the first
-// k and sorts their indices ascending.
+// k and sorts their indices ascending; rows of at most 256 blocks with k <= 32 take a warp each
+// and pick the same k keys by k rounds of a warp minimum.
 #include "device_common.cuh"
 
 namespace pa {
@@ -296,6 +297,58 @@ __global__ void __launch_bounds__(kTopkThreads)
     for (int i = threadIdx.x; i < width; i += blockDim.x) out[i] = i < k ? (int32_t)keys[i] : -1;
 }
 
+// The same selection for rows of at most 256 blocks and k <= 32, a warp per row: each lane holds
+// the rank keys of blocks lane, lane + 32, ...; k rounds each take the smallest key of the warp
+// (the next block in the order above) and retire it, lane r keeping the r-th pick; the picks are
+// then written in ascending block order (a pick's place = the number of smaller picks).
+constexpr int kTopkWarpRows = 8;   // rows (warps) per CTA
+constexpr int kTopkWarpKeys = 8;   // keys per lane: rows of up to 256 blocks
+
+__global__ void __launch_bounds__(kTopkWarpRows * 32)
+    topk_warp_kernel(const float* __restrict__ scores, int32_t sw, int32_t* __restrict__ sel, int32_t width,
+                     const SeqInfo* __restrict__ seqs, const int32_t* __restrict__ q2seq, int32_t hkv, int32_t bs,
+                     int32_t topk, int64_t rows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kTopkWarpRows + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const SeqInfo si = seqs[q2seq[row / hkv]];
+    const int nb = (si.L + bs - 1) / bs;
+    const int k = (topk == 0 || topk >= nb) ? nb : topk;
+    int32_t* out = sel + row * width;
+    if (k == nb) {  // every block: no ranking needed
+        for (int i = lane; i < width; i += 32) out[i] = i < nb ? i : -1;
+        return;
+    }
+    const float* sc = scores + row * sw;
+    unsigned long long key[kTopkWarpKeys];
+#pragma unroll
+    for (int j = 0; j < kTopkWarpKeys; ++j) {
+        const int i = lane + 32 * j;
+        key[j] = i < nb ? rank_key(sc[i], i) : ~0ull;
+    }
+    int mine = -1;  // lane r: the r-th pick
+    for (int r = 0; r < k; ++r) {
+        unsigned long long m = key[0];
+#pragma unroll
+        for (int j = 1; j < kTopkWarpKeys; ++j) m = key[j] < m ? key[j] : m;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, m, o);
+            m = other < m ? other : m;
+        }
+        const int idx = (int)(uint32_t)m;
+        if (lane == r) mine = idx;
+        const bool owner = lane == (idx & 31);
+        const int slot = idx >> 5;
+#pragma unroll
+        for (int j = 0; j < kTopkWarpKeys; ++j) key[j] = (owner && j == slot) ? ~0ull : key[j];
+    }
+    int place = 0;
+    for (int r = 0; r < k; ++r) place += __shfl_sync(0xffffffffu, mine, r) < mine;
+    if (lane < k) out[place] = mine;
+    for (int i = k + lane; i < width; i += 32) out[i] = -1;
+}
+
 // Caller selection -> checked, compacted selection [Nq, Hkv, wout]: entries in [0, nb_s) that
 // are not repeats, in their original order, then -1. A bad entry records code 64 in the error
 // word and is dropped. A repeat is found through a bitmap of the row's blocks in shared memory.
@@ -495,6 +548,12 @@ cudaError_t launch_sparse_topk(const float* scores, int32_t sw, int32_t* sel, in
                                const int32_t* q2seq, int32_t hkv, int32_t block_size, int32_t topk,
                                int32_t nb_max, int64_t num_queries, cudaStream_t st) {
     if (num_queries == 0) return cudaSuccess;
+    if (nb_max <= 32 * kTopkWarpKeys && topk <= 32) {
+        const int64_t rows = num_queries * hkv;
+        topk_warp_kernel<<<(unsigned)((rows + kTopkWarpRows - 1) / kTopkWarpRows), kTopkWarpRows * 32, 0, st>>>(
+            scores, sw, sel, width, seqs, q2seq, hkv, block_size, topk, rows);
+        return cudaGetLastError();
+    }
     int n = 1;
     while (n < nb_max) n <<= 1;
     const size_t smem = (size_t)n * sizeof(unsigned long long);

@@ -124,6 +124,12 @@ def sparse_cases():
         # rows of 80 bytes: the proxy pass's scalar kernel
         ("bf16_d40_scalar_proxy", W.make_gqa("sp7", 68, [150, 77], [1, 2], 4, 2, 40, 40, 16, torch.bfloat16),
          16, 2),
+        # more than 256 blocks in a row, and k above 32: the top-K kernel's shared-memory sort (the
+        # other cases take its warp-per-row form)
+        ("bf16_313_blocks_sorted_topk", W.make_gqa("sp10", 72, [5000, 300], [1, 1], 8, 2, 64, 64, 16,
+                                                   torch.bfloat16), 16, 5),
+        ("bf16_k40_sorted_topk", W.make_gqa("sp11", 73, [3000, 800], [1, 1], 8, 2, 128, 128, 16, torch.bfloat16),
+         32, 40),
     ]
 
 
