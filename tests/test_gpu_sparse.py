@@ -130,6 +130,12 @@ def sparse_cases():
                                                    torch.bfloat16), 16, 5),
         ("bf16_k40_sorted_topk", W.make_gqa("sp11", 73, [3000, 800], [1, 1], 8, 2, 128, 128, 16, torch.bfloat16),
          32, 40),
+        # 256-key blocks: eight 32-key pieces per KV head in the tensor-core proxy pass; 2048-key
+        # blocks: beyond its 1024 keys, so the CUDA-core slot kernel scores them
+        ("bf16_bs256_mma_proxy", W.make_gqa("sp12", 74, [3000, 700, 90], [1, 1, 1], 16, 4, 128, 128, 16,
+                                            torch.bfloat16), 256, 3),
+        ("bf16_bs2048_slot_proxy", W.make_gqa("sp13", 75, [5000, 300], [1, 1], 8, 2, 128, 128, 64, torch.bfloat16),
+         2048, 1),
     ]
 
 
