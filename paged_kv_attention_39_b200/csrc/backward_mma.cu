@@ -101,10 +101,11 @@ cudaError_t bwd_launch_d(const BwdParams2& p, int num_key_units, int num_row_uni
                                                                    static_cast<const T*>(p.dout), p.drow, rows, D);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // dK/dV (then the ordered pass) on the caller's stream and dQ on a side stream, so that the
-    // second kernel's CTAs fill the SMs the first one's last wave leaves idle; both only read
-    // what the Drow kernel and the caller wrote. The side stream forks from and joins back into
-    // the caller's stream through events, so the call stays stream-ordered (and capturable).
+    // dQ on a side stream and dK/dV (then the ordered pass) on the caller's stream, so that each
+    // kernel's CTAs fill the SMs the other one's last wave leaves idle; both only read what the
+    // Drow kernel and the caller wrote. dQ is issued first (its CTAs start first; measured about
+    // 2 % faster than the other order). The side stream forks from and joins back into the
+    // caller's stream through events, so the call stays stream-ordered (and capturable).
     const bool fork = num_key_units > 0 && num_row_units > 0;
     std::unique_lock<std::mutex> lk(side_mutex(), std::defer_lock);
     SideStream* side = nullptr;
@@ -116,16 +117,16 @@ cudaError_t bwd_launch_d(const BwdParams2& p, int num_key_units, int num_row_uni
         if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
         if (e != cudaSuccess) return e;
     }
-    if (num_key_units > 0)
+    if (num_row_units > 0)
+        e = launch_backward_tc_dq(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, num_row_units,
+                                  rows / p.hq, fork ? side->stream : st);
+    if (e == cudaSuccess && num_key_units > 0)
         e = launch_backward_tc_dkdv(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, num_key_units,
                                     rows / p.hq, st);
     if (e == cudaSuccess && num_sums > 0) {
         bwd_ordered_kernel<D><<<dim3((num_sums + 3) / 4, p.hkv), 128, 0, st>>>(p, num_sums, backward_tc_key_tile());
         e = cudaGetLastError();
     }
-    if (e == cudaSuccess && num_row_units > 0)
-        e = launch_backward_tc_dq(p, std::is_same<T, __nv_bfloat16>::value ? PA_BF16 : PA_F16, num_row_units,
-                                  rows / p.hq, fork ? side->stream : st);
     if (fork) {  // joined on every path, so that a capture on the caller's stream never ends unjoined
         cudaError_t j = cudaEventRecord(side->join, side->stream);
         if (j == cudaSuccess) j = cudaStreamWaitEvent(st, side->join, 0);
