@@ -792,19 +792,45 @@ pa_status run_forward(pa_plan* P, const Call& c, cudaStream_t st) {
         p.merge_ctr = P->merge_ctr;
     }
     if (ev) PA_CUDA_TRY(cudaEventRecord(ev[0], st));
-    if (S->n_tc > 0) {
-        ++launches;
-        kernels |= PA_KERNEL_DECODE_TC;
-        p.units = S->tc_units;
-        p.num_units = S->n_tc;
-        e = pa::launch_decode_mma(p, c.dtype, S->tc_rows_max, st);
-        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "decode kernel launch failed: %s", cudaGetErrorString(e));
-    }
-    if (S->n_pre > 0) {
-        ++launches;
-        kernels |= PA_KERNEL_PREFILL_TC;
-        e = pa::launch_prefill_tc(p, c.dtype, P->num_pages, st);
-        if (e != cudaSuccess) return fail(PA_ERR_CUDA, "prefill kernel launch failed: %s", cudaGetErrorString(e));
+    {
+        // Decode rows beside prefill chunks: the persistent prefill kernel on the caller's stream,
+        // then the decode kernel on the library's side stream (forked and joined through events),
+        // so that decode CTAs take the SMs the prefill CTAs leave as they finish (C4: 3-4 % faster
+        // than the two in series).
+        const bool fork = S->n_tc > 0 && S->n_pre > 0;
+        std::unique_lock<std::mutex> side_lock(pa::side_mutex(), std::defer_lock);
+        pa::SideStream* side = nullptr;
+        if (fork) {
+            side_lock.lock();
+            e = pa::side_stream(&side);
+            if (e == cudaSuccess) e = cudaEventRecord(side->fork, st);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+            if (e != cudaSuccess) return fail(PA_ERR_CUDA, "side stream fork failed: %s", cudaGetErrorString(e));
+        }
+        const char* what = nullptr;
+        if (S->n_pre > 0) {
+            ++launches;
+            kernels |= PA_KERNEL_PREFILL_TC;
+            e = pa::launch_prefill_tc(p, c.dtype, P->num_pages, st);
+            if (e != cudaSuccess) what = "prefill kernel launch";
+        }
+        if (!what && S->n_tc > 0) {
+            ++launches;
+            kernels |= PA_KERNEL_DECODE_TC;
+            p.units = S->tc_units;
+            p.num_units = S->n_tc;
+            e = pa::launch_decode_mma(p, c.dtype, S->tc_rows_max, fork ? side->stream : st);
+            if (e != cudaSuccess) what = "decode kernel launch";
+        }
+        if (fork) {  // joined on every path, so that a capture on the caller's stream never ends unjoined
+            cudaError_t j = cudaEventRecord(side->join, side->stream);
+            if (j == cudaSuccess) j = cudaStreamWaitEvent(st, side->join, 0);
+            if (!what && j != cudaSuccess) {
+                e = j;
+                what = "side stream join";
+            }
+        }
+        if (what) return fail(PA_ERR_CUDA, "%s failed: %s", what, cudaGetErrorString(e));
     }
     if (S->n_mla > 0) {
         ++launches;

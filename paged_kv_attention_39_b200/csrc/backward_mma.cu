@@ -57,14 +57,6 @@ __global__ void __launch_bounds__(128) bwd_ordered_kernel(const BwdParams2 p, in
 }
 
 // ---------------------------------------------------------------------------------------------
-namespace {
-
-// A non-blocking side stream of the library per device, with the two events of a fork/join.
-struct SideStream {
-    cudaStream_t stream = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-};
-
 std::mutex& side_mutex() {
     static std::mutex m;
     return m;
@@ -92,6 +84,8 @@ cudaError_t side_stream(SideStream** out) {
     *out = &s;
     return cudaSuccess;
 }
+
+namespace {
 
 template <typename T, int D>
 cudaError_t bwd_launch_d(const BwdParams2& p, int num_key_units, int num_row_units, int64_t rows, int num_sums,

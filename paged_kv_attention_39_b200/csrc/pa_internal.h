@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "pa.h"
 
 namespace pa {
@@ -228,5 +230,17 @@ pa_status validated_gqa_view(pa_plan* P, const void* q, const void* k, const voi
 // Thread-local error message of the C ABI (pa_last_error_message).
 pa_status set_error(pa_status st, const char* fmt, ...);
 pa_status clear_error();
+
+// A non-blocking side stream of the library per device, with the two events of a fork/join: work
+// that can run beside the caller's stream forks from it (an event recorded there) and joins back
+// (an event recorded on the side stream that the caller's stream waits for), so a call stays
+// stream-ordered and capturable. side_stream() is called with side_mutex() held, which also
+// keeps each fork/join pair together.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex& side_mutex();
+cudaError_t side_stream(SideStream** out);
 
 }  // namespace pa

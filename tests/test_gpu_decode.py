@@ -246,7 +246,8 @@ def test_plan_reuse_and_workspace_growth(orc):
 
 def test_forward_replayed_from_a_cuda_graph(orc):
     """pa_forward on decode rows (parts merged by the decode kernel's last CTA) and a prefill chunk
-    (two launches), captured into a CUDA graph after a first call has built the plan's work list
+    (two launches, the decode kernel on the library's side stream, forked from and joined back into
+    the captured stream), captured into a CUDA graph after a first call has built the plan's work list
     and workspace, then replayed with three other sets of queries written into the captured input
     buffer: every replay matches the oracle on its own queries (the merge counters are back at
     zero after each replay)."""
