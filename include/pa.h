@@ -165,7 +165,9 @@ typedef struct pa_forward_options {
  * with stream-ordered allocation on `stream`; calls on one plan must therefore be ordered
  * (one stream, or explicit events). The first call with a new head configuration builds and
  * uploads that configuration's work list once (also available as pa_plan_prepare); make it
- * before capturing the stream into a CUDA graph.
+ * before capturing the stream into a CUDA graph. A batch with both decode rows and prefill chunks
+ * runs its decode kernel on a stream of the library forked from `stream` and joined back into it
+ * through events, so the call stays ordered on `stream` (and capturable with it).
  * Inputs must be finite; non-finite values propagate (ruDNN contract).
  */
 pa_status pa_forward(pa_plan* plan, const void* q, const void* k_cache, const void* v_cache,
